@@ -1,0 +1,218 @@
+"""CPU oracle for the ConvRot W4A8 codebook linear forward (numpy front end).
+
+TEST INFRASTRUCTURE ONLY.  This package may be imported only by ``tests/``,
+``__graft_entry__.smoke()`` and the CPU-baseline / reference legs of
+``bench.py``.  The CUDA library and its Python binding never import it, and
+it imports nothing from them.
+
+Every function is a thin marshalling wrapper over the scalar C definitions
+in ``cr_oracle.c`` (which carry the citations and the readings).  Arrays are
+numpy; bf16 values travel as their uint16 bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib() -> ctypes.CDLL:
+    """Load (building first if needed) the oracle shared library."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.build()
+            L = ctypes.CDLL(path)
+            P = ctypes.c_void_p
+            i64 = ctypes.c_int64
+            L.or_fp8_e4m3fn_to_f32.argtypes = [ctypes.c_uint8]
+            L.or_fp8_e4m3fn_to_f32.restype = ctypes.c_float
+            L.or_bf16_to_f32.argtypes = [ctypes.c_uint16]
+            L.or_bf16_to_f32.restype = ctypes.c_float
+            L.or_f32_to_bf16_rne.argtypes = [ctypes.c_float]
+            L.or_f32_to_bf16_rne.restype = ctypes.c_uint16
+            L.or_unpack_codes.argtypes = [P, i64, i64, P]
+            L.or_unpack_codes.restype = None
+            L.or_decode_one.argtypes = [ctypes.c_float, ctypes.c_float]
+            L.or_decode_one.restype = ctypes.c_int8
+            L.or_decode_w8.argtypes = [P, P, P, i64, i64, P]
+            L.or_decode_w8.restype = None
+            L.or_hadamard_dense.argtypes = [ctypes.c_int, P]
+            L.or_hadamard_dense.restype = ctypes.c_int
+            L.or_rotate_rows.argtypes = [P, i64, i64, P]
+            L.or_rotate_rows.restype = ctypes.c_int
+            L.or_act_quant_rows.argtypes = [P, i64, i64, i64, ctypes.c_int, P, P]
+            L.or_act_quant_rows.restype = ctypes.c_int
+            L.or_gemm_s32_rows.argtypes = [P, P, i64, i64, i64, i64, P]
+            L.or_gemm_s32_rows.restype = ctypes.c_int
+            L.or_epilogue.argtypes = [P, P, P, P, i64, i64, ctypes.c_int, P]
+            L.or_epilogue.restype = None
+            _lib = L
+    return _lib
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=dtype))
+
+
+# ---------------------------------------------------------------- scalars
+
+def fp8_e4m3fn_to_f32(byte: int) -> float:
+    return float(lib().or_fp8_e4m3fn_to_f32(int(byte)))
+
+
+def bf16_to_f32(bits: int) -> float:
+    return float(lib().or_bf16_to_f32(int(bits)))
+
+
+def f32_to_bf16(values) -> np.ndarray:
+    """fp32 array -> bf16 bit patterns (round to nearest even)."""
+    v = _c(values, np.float32).reshape(-1)
+    L = lib()
+    out = np.empty(v.shape, dtype=np.uint16)
+    for i, f in enumerate(v.tolist()):
+        out[i] = L.or_f32_to_bf16_rne(ctypes.c_float(f))
+    return out.reshape(np.shape(values))
+
+
+def decode_one(cb_value: float, srel_value: float) -> int:
+    return int(lib().or_decode_one(ctypes.c_float(cb_value), ctypes.c_float(srel_value)))
+
+
+# ---------------------------------------------------------------- arrays
+
+def unpack_codes(qdata) -> np.ndarray:
+    """Packed codes [N, K/2] (int8 or uint8) -> codes [N, K] uint8 in 0..15."""
+    q = _c(np.asarray(qdata).view(np.uint8), np.uint8)
+    n, kh = q.shape
+    out = np.empty((n, 2 * kh), dtype=np.uint8)
+    lib().or_unpack_codes(_p(q), n, kh, _p(out))
+    return out
+
+
+def decode_w8(qdata, srel, codebook) -> np.ndarray:
+    """Packed codes [N, K/2], fp8 group scales [N, K/16], codebook[16] -> int8 [N, K]."""
+    q = _c(np.asarray(qdata).view(np.uint8), np.uint8)
+    s = _c(np.asarray(srel).view(np.uint8), np.uint8)
+    cb = _c(codebook, np.float32)
+    n, kh = q.shape
+    k = 2 * kh
+    if s.shape != (n, k // 16) or cb.shape != (16,):
+        raise ValueError("decode_w8: shape mismatch")
+    out = np.empty((n, k), dtype=np.int8)
+    lib().or_decode_w8(_p(q), _p(s), _p(cb), n, k, _p(out))
+    return out
+
+
+def hadamard_dense(size: int) -> np.ndarray:
+    """The normalised regular Hadamard of the given power-of-4 size, fp64."""
+    out = np.empty((size, size), dtype=np.float64)
+    rc = lib().or_hadamard_dense(int(size), _p(out))
+    if rc != 0:
+        raise ValueError(f"hadamard size {size} is not a power of 4")
+    return out
+
+
+def rotate_rows(x_bf16) -> np.ndarray:
+    """bf16 bits [M, K] -> fp32 [M, K], block-256 rotated."""
+    x = _c(x_bf16, np.uint16)
+    m, k = x.shape
+    out = np.empty((m, k), dtype=np.float32)
+    if lib().or_rotate_rows(_p(x), m, k, _p(out)) != 0:
+        raise ValueError("rotate_rows: K must be a positive multiple of 256")
+    return out
+
+
+def act_quant(r, mp: Optional[int] = None, qmax: int = 127):
+    """Rotated fp32 rows [M, K] -> (xq int8 [MP, K], xs fp32 [MP])."""
+    r = _c(r, np.float32)
+    m, k = r.shape
+    mp = m if mp is None else int(mp)
+    xq = np.empty((mp, k), dtype=np.int8)
+    xs = np.empty((mp,), dtype=np.float32)
+    if lib().or_act_quant_rows(_p(r), m, k, mp, int(qmax), _p(xq), _p(xs)) != 0:
+        raise ValueError("act_quant: need MP >= M and 1 <= qmax <= 127")
+    return xq, xs
+
+
+def rotate_quant_act(x_bf16, mp: Optional[int] = None, qmax: int = 127):
+    return act_quant(rotate_rows(x_bf16), mp, qmax)
+
+
+def gemm_s32(xq, w8, threads: int = 1) -> np.ndarray:
+    """acc[m, n] = sum_k xq[m, k] * w8[n, k], int32 (exact; int64 inside)."""
+    xq = _c(xq, np.int8)
+    w8 = _c(w8, np.int8)
+    m, k = xq.shape
+    n = w8.shape[0]
+    if w8.shape[1] != k:
+        raise ValueError("gemm_s32: K mismatch")
+    acc = np.empty((m, n), dtype=np.int32)
+    L = lib()
+    threads = max(1, min(int(threads), m)) if m else 1
+    bounds = [m * t // threads for t in range(threads + 1)]
+    rcs = [0] * threads
+
+    def run(t):
+        rcs[t] = L.or_gemm_s32_rows(_p(xq), _p(w8), bounds[t], bounds[t + 1], n, k, _p(acc))
+
+    if threads == 1:
+        run(0)
+    else:
+        ts = [threading.Thread(target=run, args=(t,)) for t in range(threads)]
+        for t in ts:
+            t.start()
+        for t in ts:
+            t.join()
+    if any(rcs):
+        raise OverflowError("gemm_s32: accumulator left the int32 range")
+    return acc
+
+
+def epilogue(acc, xs, ws, bias=None, out: str = "bf16") -> np.ndarray:
+    """int32 [M, N] -> bf16 bits (uint16) or fp32 [M, N]."""
+    acc = _c(acc, np.int32)
+    m, n = acc.shape
+    xs = _c(xs, np.float32)[:m]
+    ws = _c(ws, np.float32)
+    b = None if bias is None else _c(bias, np.float32)
+    if out == "bf16":
+        res = np.empty((m, n), dtype=np.uint16)
+        flag = 1
+    elif out == "f32":
+        res = np.empty((m, n), dtype=np.float32)
+        flag = 0
+    else:
+        raise ValueError(out)
+    lib().or_epilogue(_p(acc), _p(xs), _p(ws), _p(b), m, n, flag, _p(res))
+    return res
+
+
+def linear(x_bf16, qdata, srel, codebook, s_channel, bias=None, qmax: int = 127,
+           out: str = "bf16", threads: int = 1) -> dict:
+    """The whole forward: rotate + quantise x, decode W, contract, epilogue.
+
+    Returns every intermediate: xq, xs, w8, acc, y.
+    """
+    xq, xs = rotate_quant_act(x_bf16, None, qmax)
+    w8 = decode_w8(qdata, srel, codebook)
+    acc = gemm_s32(xq, w8, threads)
+    y = epilogue(acc, xs, s_channel, bias, out)
+    return {"xq": xq, "xs": xs, "w8": w8, "acc": acc, "y": y}
+
+
+def mp_for(m: int) -> int:
+    """[CR] _gemv_mp: the decode GEMV's padded row count, next power of two (1,2,4,8)."""
+    return 1 << max(0, (int(m) - 1).bit_length())

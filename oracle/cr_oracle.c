@@ -1,0 +1,339 @@
+/*
+ * cr_oracle.c -- plain, slow, scalar CPU oracle for the ConvRot W4A8 codebook
+ * linear layer forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The CUDA library never
+ * links, includes or calls it, and it shares no source with the CUDA library.
+ *
+ * Build: gcc -std=c11 -O2 -ffp-contract=off -fno-fast-math -fPIC -shared
+ * (oracle/build.py).  FP contraction is off so every float expression below
+ * rounds exactly where it is written; x86-64 evaluates float in float
+ * (FLT_EVAL_METHOD == 0) under the default round-to-nearest-even mode, and
+ * subnormals are kept (no flush-to-zero).
+ *
+ * Sources (page title, then section):
+ *   [CR]  ai-toolkit convrot_w4a8_quant.py -- module docstring (storage
+ *         formula, buffers), FIXED_CODEBOOK, W4A8_SAT, _pack_codes /
+ *         _unpack_codes, unpack_w4a8_eager, w4a8_gemv_kernel (int32
+ *         multiply-accumulate and epilogue), w4a8_act_quant_kernel, _gemv_mp,
+ *         _w4a8_linear_ste_op (unpack -> act quant -> _int_mm -> epilogue),
+ *         dequantize_w4a8.
+ *   [H3]  h3-rs src/weights.rs -- hadamard(), rotate_activation().
+ *
+ * Every function restates one definition.  Where the pages leave a detail
+ * open (the fp32 summation order of the rotation, NaN handling, the
+ * epilogue's multiply order) the reading taken is stated at the function.
+ *
+ * Parity status: every function here is pinned by a CPU test against the
+ * pages' statements, closed forms, library routines or brute force
+ * (tests/test_oracle_pins.py).  The quality of the quantised layer against
+ * the unquantised weight is not a parity target and is not pinned.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------
+ * fp8 e4m3fn -> fp32.  [CR] w4a8_gemv_kernel and _fp8_rep8 reinterpret the
+ * scale byte as float8e4nv.  e4m3fn: 1 sign bit, 4 exponent bits (bias 7),
+ * 3 mantissa bits, no infinities, S.1111.111 is NaN.  Exact in fp32.
+ * ------------------------------------------------------------------------ */
+float or_fp8_e4m3fn_to_f32(uint8_t byte)
+{
+    int sign = (byte >> 7) & 1;
+    int e = (byte >> 3) & 0xF;
+    int m = byte & 0x7;
+    double v;
+    if (e == 0xF && m == 0x7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);        /* subnormal: (m/8) * 2^(1-7) */
+    else
+        v = ldexp(1.0 + m / 8.0, e - 7); /* normal: (1 + m/8) * 2^(e-7) */
+    return (float)(sign ? -v : v);
+}
+
+/* ------------------------------------------------------------------------
+ * bf16 <-> fp32.  bf16 is the top half of an fp32, so widening is exact.
+ * Narrowing rounds to nearest, ties to even.  NaN stays a quiet NaN.
+ * ------------------------------------------------------------------------ */
+float or_bf16_to_f32(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+uint16_t or_f32_to_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if (isnan(f))
+        return (uint16_t)(((u >> 16) & 0x8000u) | 0x7FC0u);
+    /* Round the low 16 bits away: add 0x7FFF, plus 1 when the kept lsb is odd
+     * (so an exact half goes to the even neighbour), then truncate. */
+    uint32_t keep_lsb = (u >> 16) & 1u;
+    u += 0x7FFFu + keep_lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/* ------------------------------------------------------------------------
+ * Packed codes.  [CR] _pack_codes / _unpack_codes: byte j of a row holds
+ * column 2j in its low nibble and column 2j+1 in its high nibble.
+ * qdata [N, KH] bytes -> codes [N, 2*KH] (values 0..15).
+ * ------------------------------------------------------------------------ */
+void or_unpack_codes(const uint8_t *qdata, int64_t N, int64_t KH, uint8_t *codes)
+{
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t j = 0; j < KH; ++j) {
+            uint8_t b = qdata[n * KH + j];
+            codes[n * 2 * KH + 2 * j] = b & 0xF;
+            codes[n * 2 * KH + 2 * j + 1] = (b >> 4) & 0xF;
+        }
+}
+
+/* ------------------------------------------------------------------------
+ * One weight onto the int8 grid.  [CR] module docstring (storage formula),
+ * unpack_w4a8_eager and W4A8_SAT = True: p = codebook[code] * s_rel in fp32,
+ * then round to nearest even and saturate to [-128, 127] (the kernels' single
+ * saturating round-to-nearest-even conversion).  The docstring's
+ * clamp(-127, 127) is the W4A8_SAT = False variant, which the kernels do not
+ * run.  Reading: a NaN product maps to 0, as that saturating conversion does.
+ * ------------------------------------------------------------------------ */
+int8_t or_decode_one(float cb_value, float srel_value)
+{
+    float p = cb_value * srel_value;
+    if (isnan(p))
+        return 0;
+    float r = rintf(p); /* default rounding mode: nearest, ties to even */
+    if (r < -128.0f)
+        r = -128.0f;
+    if (r > 127.0f)
+        r = 127.0f;
+    return (int8_t)r;
+}
+
+/* [CR] unpack_w4a8_eager with group size 16: qdata [N, K/2] packed codes,
+ * srel [N, K/16] fp8 e4m3fn bytes, codebook[16] fp32 -> w8 [N, K] int8. */
+void or_decode_w8(const uint8_t *qdata, const uint8_t *srel, const float *codebook,
+                  int64_t N, int64_t K, int8_t *w8)
+{
+    const int64_t KH = K / 2, KG = K / 16;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t b = qdata[n * KH + k / 2];
+            int code = (k % 2 == 0) ? (b & 0xF) : ((b >> 4) & 0xF);
+            float s = or_fp8_e4m3fn_to_f32(srel[n * KG + k / 16]);
+            w8[n * K + k] = or_decode_one(codebook[code], s);
+        }
+}
+
+/* ------------------------------------------------------------------------
+ * Dense regular Hadamard.  [H3] hadamard(): start from the 4x4 regular
+ * Hadamard h4 (all ones except -1 on the anti-diagonal); each step replaces
+ * H_n by H_4n with H_4n[4i+a][4j+b] = H_n[i][j] * h4[a][b]; stop at `size`
+ * (which must be a power of 4) and divide every entry by sqrt(size).
+ * Built in fp64.  Returns 0, or -1 if size is not a power of 4.
+ * ------------------------------------------------------------------------ */
+static const double OR_H4[4][4] = {
+    {1, 1, 1, -1},
+    {1, 1, -1, 1},
+    {1, -1, 1, 1},
+    {-1, 1, 1, 1},
+};
+
+int or_hadamard_dense(int size, double *H /* [size][size], row-major */)
+{
+    int n = 4;
+    int p = 4;
+    while (p < size)
+        p *= 4;
+    if (p != size)
+        return -1; /* not a power of 4 (the page bails out the same way) */
+    double *cur = (double *)malloc(sizeof(double) * (size_t)size * (size_t)size);
+    double *nxt = (double *)malloc(sizeof(double) * (size_t)size * (size_t)size);
+    if (!cur || !nxt) {
+        free(cur);
+        free(nxt);
+        return -2;
+    }
+    for (int a = 0; a < 4; ++a)
+        for (int b = 0; b < 4; ++b)
+            cur[a * 4 + b] = OR_H4[a][b];
+    while (n < size) {
+        int n4 = 4 * n;
+        for (int i = 0; i < n; ++i)
+            for (int j = 0; j < n; ++j)
+                for (int a = 0; a < 4; ++a)
+                    for (int b = 0; b < 4; ++b)
+                        nxt[(int64_t)(4 * i + a) * n4 + (4 * j + b)] =
+                            cur[(int64_t)i * n + j] * OR_H4[a][b];
+        double *t = cur;
+        cur = nxt;
+        nxt = t;
+        n = n4;
+    }
+    if (n != size) {
+        free(cur);
+        free(nxt);
+        return -1;
+    }
+    double norm = sqrt((double)size);
+    for (int64_t i = 0; i < (int64_t)size * size; ++i)
+        H[i] = cur[i] / norm;
+    free(cur);
+    free(nxt);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Block-256 rotation of one activation row, in fp32.
+ *
+ * Definition: r[b*256 : (b+1)*256] = x[b*256 : (b+1)*256] @ H_256 with
+ * H_256 = (h4 (x) h4 (x) h4 (x) h4) / 16 ([H3] hadamard, rotate_activation:
+ * the row is cut into blocks of the rotation size and each block is
+ * multiplied by H).  Because H_256 is a Kronecker power, x @ H_256 applies
+ * h4 along each base-4 digit of the index within the block (index
+ * i = 64*d3 + 16*d2 + 4*d1 + d0).
+ *
+ * Reading (the pages fix neither the precision nor the order of the fp32
+ * sums): the bf16 inputs are widened exactly to fp32 and never rounded to
+ * bf16 again.  The digits are processed in the order d0, d1, d2, d3 (index
+ * strides 1, 4, 16, 64).  For one quadruple (v0, v1, v2, v3) along a digit,
+ * output a is  S - 2*v[3-a]  with  S = (v0 + v1) + (v2 + v3),  which equals
+ * sum_b h4[a][b]*v[b] because row a of h4 is all ones except -1 at column
+ * 3-a.  2*v is exact, so S - 2*v rounds once.  After the four digits every
+ * value is multiplied by 1/16 (exact unless the result is subnormal).
+ * ------------------------------------------------------------------------ */
+static void or_rotate_block256(float *v /* 256 values, in place */)
+{
+    static const int strides[4] = {1, 4, 16, 64};
+    for (int t = 0; t < 4; ++t) {
+        int s = strides[t];
+        for (int i = 0; i < 256; ++i) {
+            if ((i / s) % 4 != 0)
+                continue; /* i is the first element of its quadruple */
+            float q[4] = {v[i], v[i + s], v[i + 2 * s], v[i + 3 * s]};
+            float S = (q[0] + q[1]) + (q[2] + q[3]);
+            for (int a = 0; a < 4; ++a) {
+                float twice = 2.0f * q[3 - a];
+                v[i + a * s] = S - twice;
+            }
+        }
+    }
+    for (int i = 0; i < 256; ++i)
+        v[i] = v[i] * 0.0625f;
+}
+
+/* x [M, K] bf16 bits -> r [M, K] fp32 rotated.  K must be a multiple of 256.
+ * Returns 0, or -1 on a bad K. */
+int or_rotate_rows(const uint16_t *x, int64_t M, int64_t K, float *r)
+{
+    if (K <= 0 || K % 256 != 0)
+        return -1;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t b = 0; b < K / 256; ++b) {
+            float *blk = r + m * K + b * 256;
+            for (int i = 0; i < 256; ++i)
+                blk[i] = or_bf16_to_f32(x[m * K + b * 256 + i]);
+            or_rotate_block256(blk);
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Per-token symmetric int8 quantisation.  [CR] w4a8_act_quant_kernel:
+ *   amax  = max_k |r[m,k]|               (exact under any order)
+ *   scale = amax > 0 ? amax / qmax : 1   (fp32 division)
+ *   q     = clamp(rint(r / scale), -qmax, qmax)
+ * into exactly MP rows: rows m >= M get q = 0 and scale = 1 ([CR] "rows >= M:
+ * zeros, scale 1").  Reading: the prefill quantiser (_int8_act_quant_padded,
+ * not on the pages) is the same arithmetic, which the pages state when they
+ * call the decode GEMV bit-identical to the _int_mm path.  qmax is the
+ * module's act_qmax; the default reading is 127.
+ *
+ * The max follows C fmaxf (a NaN operand is ignored); the activations are
+ * expected finite, and no further NaN rule is defined.
+ * ------------------------------------------------------------------------ */
+int or_act_quant_rows(const float *r, int64_t M, int64_t K, int64_t MP, int qmax,
+                      int8_t *xq, float *xs)
+{
+    if (MP < M || qmax < 1 || qmax > 127)
+        return -1;
+    for (int64_t m = 0; m < MP; ++m) {
+        if (m >= M) {
+            for (int64_t k = 0; k < K; ++k)
+                xq[m * K + k] = 0;
+            xs[m] = 1.0f;
+            continue;
+        }
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k)
+            amax = fmaxf(amax, fabsf(r[m * K + k]));
+        float scale = (amax > 0.0f) ? amax / (float)qmax : 1.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float q = rintf(r[m * K + k] / scale);
+            if (q < (float)-qmax)
+                q = (float)-qmax;
+            if (q > (float)qmax)
+                q = (float)qmax;
+            xq[m * K + k] = (int8_t)q;
+        }
+        xs[m] = scale;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * int8 x int8 -> int32 contraction.  [CR] _w4a8_linear_ste_op
+ * (torch._int_mm(aq, w8.t())) and w4a8_gemv_kernel (int32 multiply-
+ * accumulate, exact and order independent):
+ *   acc[m, n] = sum_k xq[m, k] * w8[n, k].
+ * Summed in int64; returns -1 if any result leaves the int32 range (it cannot
+ * for |xq| <= 127, |w8| <= 128 and K <= 132104).  Rows [m0, m1) only, so a
+ * caller may split the work.
+ * ------------------------------------------------------------------------ */
+int or_gemm_s32_rows(const int8_t *xq, const int8_t *w8, int64_t m0, int64_t m1,
+                     int64_t N, int64_t K, int32_t *acc /* [M, N], rows m0..m1 */)
+{
+    int bad = 0;
+    for (int64_t m = m0; m < m1; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t s = 0;
+            for (int64_t k = 0; k < K; ++k)
+                s += (int64_t)xq[m * K + k] * (int64_t)w8[n * K + k];
+            if (s > INT32_MAX || s < INT32_MIN)
+                bad = 1;
+            acc[m * N + n] = (int32_t)s;
+        }
+    return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Epilogue.  [CR] w4a8_gemv_kernel epilogue: out = float(acc) * (xs[m] *
+ * ws[n]) (+ bias[n]), then cast to the output dtype.  Reading: exactly that
+ * parenthesisation, each operation rounded on its own (no fused multiply-add),
+ * bias added last; the prefill epilogue (_int8_epilogue, not on the pages) is
+ * the same formula, since the pages call the two paths bit-identical.
+ * out_bf16 != 0: out is bf16 bits [M, N] (round to nearest even); else fp32.
+ * bias may be NULL.
+ * ------------------------------------------------------------------------ */
+void or_epilogue(const int32_t *acc, const float *xs, const float *ws, const float *bias,
+                 int64_t M, int64_t N, int out_bf16, void *out)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            float t = (float)acc[m * N + n]; /* int32 -> fp32, nearest even */
+            float sc = xs[m] * ws[n];
+            float y = t * sc;
+            if (bias)
+                y = y + bias[n];
+            if (out_bf16)
+                ((uint16_t *)out)[m * N + n] = or_f32_to_bf16_rne(y);
+            else
+                ((float *)out)[m * N + n] = y;
+        }
+}

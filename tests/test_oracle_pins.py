@@ -1,0 +1,370 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks an oracle function against something other than the
+oracle itself: hand-worked values from the pages (tests/golden/*.txt, each
+with its citation), closed forms, library routines (torch's fp8/bf16 casts,
+numpy's kron/matmul), invariants and brute force.  No GPU is used.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from w4a8_codebook_quantized_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+H4 = np.array([[1, 1, 1, -1], [1, 1, -1, 1], [1, -1, 1, 1], [-1, 1, 1, 1]], dtype=np.float64)
+U32 = 2.0 ** -24  # unit roundoff of fp32
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                yield line.split()
+
+
+def _bf16(values64):
+    t = torch.from_numpy(np.asarray(values64, dtype=np.float64)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _bf16_to_f64(bits):
+    return torch.from_numpy(np.asarray(bits, dtype=np.uint16).view(np.int16)).view(torch.bfloat16).double().numpy()
+
+
+def _dense_h(size):
+    h = np.ones((1, 1))
+    while h.shape[0] < size:
+        h = np.kron(h, H4)
+    return h / math.sqrt(size)
+
+
+# ---------------------------------------------------------------- fp8 / bf16
+
+def test_fp8_spot_values():
+    for byte, val in _rows("fp8_spot.txt"):
+        got = oracle.fp8_e4m3fn_to_f32(int(byte, 16))
+        if val == "nan":
+            assert math.isnan(got)
+        else:
+            assert got == float(val) and math.copysign(1, got) == math.copysign(1, float(val)), byte
+
+
+def test_fp8_exhaustive_vs_torch():
+    ref = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    for b in range(256):
+        got = oracle.fp8_e4m3fn_to_f32(b)
+        if math.isnan(ref[b]):
+            assert math.isnan(got)
+        else:
+            assert got == ref[b], hex(b)
+
+
+def test_bf16_widen_exhaustive_vs_torch():
+    bits = np.arange(0, 65536, 97, dtype=np.uint32).astype(np.uint16)
+    ref = _bf16_to_f64(bits)
+    for b, r in zip(bits.tolist(), ref.tolist()):
+        got = oracle.bf16_to_f32(b)
+        assert (math.isnan(got) and math.isnan(r)) or got == r
+
+
+def test_bf16_round_nearest_even_vs_torch():
+    rng = np.random.default_rng(0)
+    v = np.concatenate([
+        rng.standard_normal(4000).astype(np.float32),
+        (rng.standard_normal(1000) * 1e-39).astype(np.float32),  # subnormals
+        np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 3.3895e38, 3.4e38, np.inf, -np.inf,
+                  0.0, -0.0, 2 ** -133, 65504.0], dtype=np.float32),
+    ])
+    got = oracle.f32_to_bf16(v)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, ref)
+    assert oracle.f32_to_bf16(np.array([np.nan], np.float32))[0] & 0x7FFF > 0x7F80
+
+
+# ---------------------------------------------------------------- packing
+
+def test_unpack_worked_examples():
+    for byte, even, odd in _rows("unpack_example.txt"):
+        codes = oracle.unpack_codes(np.array([[int(byte, 16)]], dtype=np.uint8))
+        assert codes.tolist() == [[int(even), int(odd)]], byte
+
+
+def test_unpack_is_a_bijection_of_bytes():
+    q = np.arange(256, dtype=np.uint8).reshape(1, 256)
+    codes = oracle.unpack_codes(q).reshape(256, 2)
+    assert codes.min() == 0 and codes.max() == 15
+    pairs = {tuple(p) for p in codes.tolist()}
+    assert len(pairs) == 256
+    # row/column placement: byte j of row n fills columns 2j and 2j+1 of row n
+    q2 = np.array([[0x21, 0x43], [0x65, 0x87]], dtype=np.uint8)
+    assert oracle.unpack_codes(q2).tolist() == [[1, 2, 3, 4], [5, 6, 7, 8]]
+
+
+# ---------------------------------------------------------------- decode
+
+def test_decode_exhaustive_vs_torch_eager():
+    """All 256 scale bytes x 16 codes against the eager definition evaluated
+    with torch ops (codebook[code] * s_rel, round half even, clamp [-128, 127])."""
+    cb = inputs.codebook()
+    srel = np.repeat(np.arange(256, dtype=np.uint8), 1).reshape(256, 1)
+    # one row per scale byte, 16 columns = codes 0..15 (8 bytes: pairs (0,1),(2,3)..)
+    qdata = np.tile(np.array([0x10, 0x32, 0x54, 0x76, 0x98, 0xBA, 0xDC, 0xFE], dtype=np.uint8), (256, 1))
+    w8 = oracle.decode_w8(qdata, srel, cb)
+    s = torch.from_numpy(srel.reshape(-1).copy()).view(torch.float8_e4m3fn).float()
+    vals = torch.from_numpy(cb)[None, :] * s[:, None]
+    ref = vals.round().clamp(-128, 127)
+    finite = ~torch.isnan(vals)
+    assert np.array_equal(w8[finite.numpy()], ref[finite].to(torch.int8).numpy())
+    # reading: NaN scale bytes (0x7F, 0xFF) decode to 0
+    assert (w8[[0x7F, 0xFF]] == 0).all()
+
+
+def test_decode_ties_with_uniform_codebook():
+    cb = np.arange(-8, 8, dtype=np.float32)  # attach_ default codebook
+    for row in _rows("decode_ties_arange.txt"):
+        byte, expect = int(row[0], 16), [int(v) for v in row[1:]]
+        qdata = np.array([[0x10, 0x32, 0x54, 0x76, 0x98, 0xBA, 0xDC, 0xFE]], dtype=np.uint8)
+        w8 = oracle.decode_w8(qdata, np.array([[byte]], dtype=np.uint8), cb)
+        assert w8[0].tolist() == expect, hex(byte)
+
+
+def test_decode_saturation():
+    cb = inputs.codebook()
+    for byte, code, expect in _rows("decode_saturation.txt"):
+        c = int(code)
+        qdata = np.zeros((1, 8), dtype=np.uint8)
+        qdata[0, 0] = c  # column 0 = low nibble of byte 0
+        w8 = oracle.decode_w8(qdata, np.array([[int(byte, 16)]], dtype=np.uint8), cb)
+        assert int(w8[0, 0]) == int(expect), (byte, code)
+
+
+def test_decode_group_layout():
+    """Column k uses scale byte k // 16 of its own row."""
+    cb = np.arange(-8, 8, dtype=np.float32)
+    qdata = np.full((2, 16), 0x99, dtype=np.uint8)  # every code = 9 -> level 1
+    srel = np.array([[0x38, 0x40], [0x48, 0x50]], dtype=np.uint8)  # 1, 2, 4, 8
+    w8 = oracle.decode_w8(qdata, srel, cb)
+    assert (w8[0, :16] == 1).all() and (w8[0, 16:] == 2).all()
+    assert (w8[1, :16] == 4).all() and (w8[1, 16:] == 8).all()
+
+
+# ---------------------------------------------------------------- Hadamard
+
+def test_hadamard_dense_definition():
+    for size in (4, 16, 64, 256):
+        H = oracle.hadamard_dense(size)
+        assert np.array_equal(H, _dense_h(size)), size  # np.kron of the page's h4
+        S = H * math.sqrt(size)
+        assert set(np.unique(S).tolist()) == {-1.0, 1.0}
+        assert np.array_equal(S @ S.T, size * np.eye(size))  # orthogonal
+        assert np.array_equal(H, H.T)  # symmetric
+        assert np.array_equal(S.sum(axis=1), np.full(size, math.sqrt(size)))  # regular: constant row sums
+        assert np.allclose(H @ H, np.eye(size), atol=1e-12)  # its own inverse
+    for bad in (8, 128, 512):
+        with pytest.raises(ValueError):
+            oracle.hadamard_dense(bad)
+
+
+# ---------------------------------------------------------------- rotation
+
+def test_rotation_exact_on_small_integers():
+    rng = np.random.default_rng(1)
+    x = rng.integers(-8, 9, size=(5, 512)).astype(np.float64)
+    got = oracle.rotate_rows(_bf16(x)).astype(np.float64)
+    H = _dense_h(256)
+    ref = np.concatenate([x[:, :256] @ H, x[:, 256:] @ H], axis=1)
+    assert np.array_equal(got, ref)
+
+
+def test_rotation_error_bound_random():
+    """|fp32 butterfly - exact| <= 12 u * sum|x_block| / 16: four digit stages,
+    three roundings each, |h4| all ones (standard forward error bound)."""
+    x_bits = inputs.activations(16, 1024, seed=11)
+    x = _bf16_to_f64(x_bits)
+    got = oracle.rotate_rows(x_bits).astype(np.float64)
+    H = _dense_h(256)
+    for b in range(4):
+        blk = slice(256 * b, 256 * (b + 1))
+        exact = x[:, blk] @ H
+        bound = 12 * U32 * 1.001 * np.abs(x[:, blk]).sum(axis=1, keepdims=True) / 16
+        assert (np.abs(got[:, blk] - exact) <= bound).all()
+
+
+def test_rotation_is_an_involution():
+    x_bits = inputs.activations(4, 512, seed=12)
+    r = oracle.rotate_rows(x_bits)
+    # feed the (exactly bf16-representable) integers through twice
+    x = np.round(_bf16_to_f64(x_bits) * 4)  # small integers
+    xi = _bf16(x)
+    rr = oracle.rotate_rows(_bf16(oracle.rotate_rows(xi).astype(np.float64)))
+    assert np.allclose(rr, x, atol=1e-2 * np.abs(x).max())
+    assert r.shape == (4, 512)
+
+
+def test_rotation_identity_in_exact_arithmetic():
+    """x W^T = (x H)(W H)^T, checked in int64 through 16H on integer data."""
+    rng = np.random.default_rng(2)
+    for K in (256, 512):
+        x = rng.integers(-3, 4, size=(3, K)).astype(np.float64)
+        W = rng.integers(-3, 4, size=(5, K)).astype(np.float64)
+        rx = oracle.rotate_rows(_bf16(x)).astype(np.float64) * 16  # x (16 H): integers
+        rw = oracle.rotate_rows(_bf16(W)).astype(np.float64) * 16
+        assert np.array_equal(rx, np.round(rx)) and np.array_equal(rw, np.round(rw))
+        lhs = rx.astype(np.int64) @ rw.astype(np.int64).T
+        assert np.array_equal(lhs, 256 * (x.astype(np.int64) @ W.astype(np.int64).T))
+
+
+def test_rotation_rejects_bad_k():
+    with pytest.raises(ValueError):
+        oracle.rotate_rows(np.zeros((1, 128), np.uint16))
+
+
+# ---------------------------------------------------------------- act quant
+
+def test_act_quant_properties():
+    x_bits = inputs.activations(8, 2048, seed=13)
+    r = oracle.rotate_rows(x_bits)
+    for qmax in (127, 7):
+        xq, xs = oracle.act_quant(r, 8, qmax)
+        amax = np.abs(r).max(axis=1)
+        assert np.array_equal(xs, (amax / np.float32(qmax)).astype(np.float32))
+        assert np.abs(xq.astype(np.int32)).max() <= qmax
+        for m in range(8):
+            k = int(np.argmax(np.abs(r[m])))
+            assert int(xq[m, k]) == int(np.sign(r[m, k])) * qmax
+        err = np.abs(xq.astype(np.float64) * xs[:, None].astype(np.float64) - r.astype(np.float64))
+        assert (err <= xs[:, None] * (0.5 + 1e-5)).all()
+        # away from exact ties, q is the fp64 nearest integer of r / s
+        t = r.astype(np.float64) / xs[:, None]
+        away = np.abs(np.abs(t - np.floor(t)) - 0.5) > 1e-4
+        assert np.array_equal(xq[away], np.rint(t[away]).astype(np.int8))
+
+
+def test_act_quant_zero_row_and_padding():
+    r = np.zeros((3, 256), np.float32)
+    r[1, 5] = -3.0
+    xq, xs = oracle.act_quant(r, 8, 127)
+    assert xs[0] == 1.0 and (xq[0] == 0).all()
+    assert xs[1] == np.float32(3.0) / np.float32(127) and xq[1, 5] == -127
+    assert (xq[3:] == 0).all() and (xs[3:] == 1.0).all()
+    with pytest.raises(ValueError):
+        oracle.act_quant(r, 2, 127)
+
+
+def test_mp_padding_rule():
+    assert [oracle.mp_for(m) for m in range(1, 9)] == [1, 2, 4, 4, 8, 8, 8, 8]
+
+
+# ---------------------------------------------------------------- contraction
+
+def test_gemm_brute_force_tiny():
+    rng = np.random.default_rng(3)
+    for (M, N, K) in [(1, 1, 256), (3, 5, 256), (2, 7, 512), (4, 3, 768)]:
+        xq = rng.integers(-127, 128, size=(M, K)).astype(np.int8)
+        w8 = rng.integers(-128, 128, size=(N, K)).astype(np.int8)
+        ref = xq.astype(np.int64) @ w8.astype(np.int64).T
+        got = oracle.gemm_s32(xq, w8)
+        assert np.array_equal(got, ref)
+        assert np.array_equal(oracle.gemm_s32(xq, w8, threads=3), ref)
+
+
+def test_gemm_extreme_operands_and_overflow():
+    K = 12288
+    xq = np.full((2, K), -127, np.int8)
+    w8 = np.full((1, K), -128, np.int8)
+    assert oracle.gemm_s32(xq, w8)[0, 0] == 127 * 128 * K
+    K = 132352  # first multiple of 256 beyond the int32-safe depth 132104
+    with pytest.raises(OverflowError):
+        oracle.gemm_s32(np.full((1, K), -127, np.int8), np.full((1, K), -128, np.int8))
+
+
+# ---------------------------------------------------------------- epilogue
+
+def test_epilogue_hand_values():
+    for acc, xs, ws, bias, kind, expect in _rows("epilogue_hand.txt"):
+        b = None if bias == "none" else np.array([float(bias)], np.float32)
+        out = oracle.epilogue(np.array([[int(acc)]], np.int32), np.array([float(xs)], np.float32),
+                              np.array([float(ws)], np.float32), b, kind)
+        if kind == "bf16":
+            assert int(out[0, 0]) == int(expect, 16), (acc, xs)
+        else:
+            assert float(out[0, 0]) == float(expect), (acc, xs)
+
+
+def test_epilogue_random_vs_fp64():
+    rng = np.random.default_rng(4)
+    acc = rng.integers(-2 ** 30, 2 ** 30, size=(6, 40)).astype(np.int32)
+    xs = rng.uniform(1e-3, 1, size=6).astype(np.float32)
+    ws = rng.uniform(1e-4, 5e-4, size=40).astype(np.float32)
+    bias = rng.normal(size=40).astype(np.float32)
+    y = oracle.epilogue(acc, xs, ws, bias, "f32").astype(np.float64)
+    ref = acc.astype(np.float64) * (xs[:, None].astype(np.float64) * ws[None, :]) + bias
+    assert (np.abs(y - ref) <= 4 * U32 * (np.abs(ref) + np.abs(bias)) + 1e-30).all()
+    yb = oracle.epilogue(acc, xs, ws, None, "bf16")
+    refb = torch.from_numpy(oracle.epilogue(acc, xs, ws, None, "f32")).to(torch.bfloat16)
+    assert np.array_equal(yb, refb.view(torch.int16).numpy().view(np.uint16))
+
+
+# ---------------------------------------------------------------- whole layer
+
+def _dequantized_weight(layer):
+    """ai-toolkit convrot_w4a8_quant.py, dequantize_w4a8: rotate(w8 * s_channel),
+    with the int8 grid from torch's eager decode and a dense np.kron Hadamard."""
+    codes = torch.from_numpy(oracle.unpack_codes(layer.qdata).astype(np.int64))
+    s = torch.from_numpy(layer.srel.copy()).view(torch.float8_e4m3fn).float()
+    vals = torch.from_numpy(layer.codebook)[codes].view(layer.N, -1, 16) * s.unsqueeze(-1)
+    w8 = vals.view(layer.N, -1).round().clamp(-128, 127).double().numpy()
+    w_rot = w8 * layer.s_channel.astype(np.float64)[:, None]
+    H = _dense_h(256)
+    K = layer.K
+    return np.concatenate([w_rot[:, b:b + 256] @ H for b in range(0, K, 256)], axis=1), w8
+
+
+def test_linear_exact_one_hot_case():
+    """x = 127 * (row j of H): the rotation gives exactly 127 e_j, the scale is 1
+    and the layer output is 127 * w8[n, j] * s_channel[n]."""
+    layer = inputs.layer(24, 512, seed=5)
+    H = _dense_h(256)
+    x = np.zeros((3, 512))
+    js = [0, 77, 300]
+    for i, j in enumerate(js):
+        b = (j // 256) * 256
+        x[i, b:b + 256] = 127 * H[j % 256]
+    res = oracle.linear(_bf16(x), layer.qdata, layer.srel, layer.codebook, layer.s_channel, out="f32")
+    assert (res["xs"] == 1.0).all()
+    for i, j in enumerate(js):
+        e = np.zeros(512, np.int8)
+        e[j] = 127
+        assert np.array_equal(res["xq"][i], e)
+    Wd, w8 = _dequantized_weight(layer)
+    ref = _bf16_to_f64(_bf16(x)) @ Wd.T  # fp64, independent path
+    for i, j in enumerate(js):
+        exact = (np.float32(127 * w8[:, j]) * layer.s_channel).astype(np.float32)
+        assert np.array_equal(res["y"][i], exact)
+        assert np.allclose(res["y"][i], ref[i], rtol=1e-6, atol=1e-9)
+
+
+def test_linear_random_within_quantisation_bound():
+    """The whole chain against x @ dequantize_w4a8(W)^T in fp64: the only
+    error allowed is the activation rounding (|q s - r| <= s/2), the fp32
+    rotation error and the fp32 epilogue rounding."""
+    layer = inputs.layer(40, 768, seed=6)
+    x_bits = inputs.activations(5, 768, seed=6)
+    res = oracle.linear(x_bits, layer.qdata, layer.srel, layer.codebook, layer.s_channel, out="f32")
+    Wd, w8 = _dequantized_weight(layer)
+    x = _bf16_to_f64(x_bits)
+    ref = x @ Wd.T
+    xs = res["xs"].astype(np.float64)
+    absx = np.abs(x).reshape(5, 3, 256).sum(axis=2)  # per block L1
+    rot_err = np.repeat(12 * U32 * 1.001 * absx / 16, 256, axis=1)  # per element
+    act_err = xs[:, None] * (0.5 + 1e-5) + rot_err
+    bound = (act_err @ np.abs(w8).T) * layer.s_channel[None, :] + 4 * U32 * np.abs(ref) + 1e-12
+    assert (np.abs(res["y"] - ref) <= bound).all()
+    # and a plausible slip (a dropped outlier channel) would break it
+    assert np.abs(res["y"] - ref).max() < 0.05 * np.abs(ref).max()
