@@ -1,0 +1,519 @@
+#!/usr/bin/env python
+"""Benchmark of the ConvRot W4A8 codebook linear forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one pass of the whole hot path over one batch: rotate + quantise
+the activations, then the fused decode GEMV (M <= 8) or decode + tcgen05
+GEMM (M > 8), epilogue included.  The default workload is the decode batch
+M = 8, N = K = 4096; the metric is the weight bytes the layer streams
+(4.5 bits per weight + per-channel scales + codebook) per second.  A
+second block ("prefill") reports the M = 2048, N = K = 4096 prefill step in
+int8 TOPS.
+
+Timing: inputs live in HBM before the timed region; R rotating copies of the
+layer and activations (more bytes than the 126 MB L2) are cycled so every
+step streams its weights from HBM; the K timed steps are one CUDA-graph
+replay bracketed by CUDA events on the capturing stream, with a barrier and a
+synchronize on both sides; multi-GPU runs report the max over ranks.  SM
+clocks and throttle reasons are sampled through NVML during the timed region.
+
+Under torchrun every rank runs its own replica of the layer on its own batch
+(weak scaling, no data-path collective); the only collectives are the
+barrier and the max over ranks of the timings.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "W4A8 GEMV weight GB/s & % HBM roofline (M≤8); prefill int8 TOPS & % peak"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 vs 2.25 PFLOP/s)
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="c2_decode_m8_4k")
+    p.add_argument("--prefill-workload", default="c3_prefill_2k_4k")
+    p.add_argument("--no-prefill", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def weight_bytes(N, K):
+    """Algorithmic weight traffic of one decode pass: packed codes (K/2 per
+    row), fp8 group scales (K/16 per row), fp32 channel scales, fp32 codebook."""
+    return N * (K // 2) + N * (K // 16) + 4 * N + 64
+
+
+def gemv_launch_bytes(M, N, K):
+    """Algorithmic bytes of one GEMV launch: the weight stream, the int8
+    activation rows and scales it reads, and the bf16 output it writes."""
+    return weight_bytes(N, K) + M * K + 4 * M + 2 * M * N
+
+
+def prior_traffic(kernel_tag):
+    """DRAM bytes per launch recorded from an ncu capture of the current kernel
+    (profiles/<tag>.traffic), or None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel_tag}.traffic")
+    try:
+        with open(path) as f:
+            for line in f:
+                if line.startswith("dram_bytes_per_launch:"):
+                    return float(line.split(":", 1)[1])
+    except OSError:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, index: int, period: float = 0.002):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            self.h = nv.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.ok = True
+            self._sample()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception:
+            self.ok = False
+        return self
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        names = {
+            "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+            "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+            "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+        }
+        for k, bit in names.items():
+            if r & bit:
+                self.reasons.add(k)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- our arm
+
+class Sets:
+    """R rotating device copies of one workload (layer + activations)."""
+
+    def __init__(self, case, rank, min_bytes=int(1.25 * L2_BYTES)):
+        import torch
+
+        import w4a8_codebook_quantized_b200 as cr
+        from w4a8_codebook_quantized_b200 import inputs
+        self.case = case
+        M, N, K = case.M, case.N, case.K
+        per_set = weight_bytes(N, K) + 2 * M * K
+        self.R = max(2, int(math.ceil(min_bytes / per_set)))
+        layer = inputs.layer(N, K, case.seed + 1000 * rank)
+        x = inputs.activations(M, K, case.seed + 1000 * rank, case.dist)
+        q = torch.from_numpy(layer.qdata).cuda()
+        s = torch.from_numpy(layer.srel).cuda()
+        self.cb = torch.from_numpy(layer.codebook).cuda()
+        ws = torch.from_numpy(layer.s_channel).cuda()
+        xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+        self.q = [q.clone() for _ in range(self.R)]
+        self.s = [s.clone() for _ in range(self.R)]
+        self.ws = [ws.clone() for _ in range(self.R)]
+        self.x = [xd.clone() for _ in range(self.R)]
+        self.rows = cr.gemv_rows(M) if M <= cr.CR_GEMV_MAX_M else M
+        self.xq = [torch.empty(self.rows, K, dtype=torch.int8, device="cuda") for _ in range(self.R)]
+        self.xs = [torch.empty(self.rows, dtype=torch.float32, device="cuda") for _ in range(self.R)]
+        self.out = [torch.empty(M, N, dtype=torch.bfloat16, device="cuda") for _ in range(self.R)]
+        self.x_host = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+        self.out_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+
+    def step(self, i):
+        import w4a8_codebook_quantized_b200 as cr
+        r = i % self.R
+        cr.cr_w4a8_linear(self.x[r], self.q[r], self.s[r], self.cb, self.ws[r], out=self.out[r],
+                          xq_work=self.xq[r], xs_work=self.xs[r])
+
+    def contraction_only(self, i):
+        """The dominant kernel alone: the GEMV (M <= 8) on prepared activations."""
+        import w4a8_codebook_quantized_b200 as cr
+        r = i % self.R
+        M = self.case.M
+        cr.cr_w4a8_gemv(self.xq[r], self.xs[r], self.q[r], self.s[r], self.cb, self.ws[r], m=M, out=self.out[r])
+
+    def e2e_step(self, i):
+        """Through the public API with host buffers: H2D of x, forward, D2H of y."""
+        import w4a8_codebook_quantized_b200 as cr
+        r = i % self.R
+        self.x[r].copy_(self.x_host, non_blocking=True)
+        cr.cr_w4a8_linear(self.x[r], self.q[r], self.s[r], self.cb, self.ws[r], out=self.out[r],
+                          xq_work=self.xq[r], xs_work=self.xs[r])
+        self.out_host.copy_(self.out[r], non_blocking=True)
+
+
+def graph_time(fn, steps, warmup, world, sampler_index=None):
+    """Capture `steps` calls of fn(i) in one CUDA graph, replay it once after a
+    `warmup`-call warm graph; return (seconds of the timed replay, clocks)."""
+    import torch
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(max(1, warmup)):
+            fn(i)
+    stream.synchronize()
+    gw = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gw, stream=stream):
+        for i in range(max(1, warmup)):
+            fn(i)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            fn(i)
+    with torch.cuda.stream(stream):
+        gw.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(sampler_index if sampler_index is not None else torch.cuda.current_device())
+    with clocks:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    secs = e0.elapsed_time(e1) / 1000.0
+    del g, gw
+    return secs, clocks.summary()
+
+
+def eager_time(fn, steps, warmup, world):
+    import torch
+    stream = torch.cuda.current_stream()
+    for i in range(max(1, warmup)):
+        fn(i)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(steps):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return e0.elapsed_time(e1) / 1000.0
+
+
+def cpu_baseline(case, seconds):
+    """The oracle, as it stands, on the host: full forward passes of the
+    workload, single-threaded, repeated for about `seconds`."""
+    import oracle
+    from w4a8_codebook_quantized_b200 import inputs
+    layer = inputs.layer(case.N, case.K, case.seed)
+    M = case.M
+    rows = M
+    if M > 64:  # prefill-size batches: a row sample (rows are independent)
+        rows = 16
+    x = inputs.activations(rows, case.K, case.seed, case.dist)
+    oracle.lib()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.linear(x, layer.qdata, layer.srel, layer.codebook, layer.s_channel, threads=1)
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    el = time.perf_counter() - t0
+    per_pass = el / n
+    if M <= 8:
+        value = weight_bytes(case.N, case.K) / per_pass / 1e9
+        unit, sample = "GB/s", f"{n} full forward passes of the workload (M={M}, N={case.N}, K={case.K})"
+    else:
+        value = 2.0 * rows * case.N * case.K / per_pass / 1e12
+        unit, sample = "TOPS", f"{n} passes over {rows} of {M} token rows (N={case.N}, K={case.K})"
+    return {"value": value, "unit": unit, "cores": 1, "kind": "oracle", "sample": sample,
+            "seconds": round(el, 3)}
+
+
+def run_ours(args):
+    import torch
+
+    import w4a8_codebook_quantized_b200 as cr
+    from w4a8_codebook_quantized_b200 import inputs
+    world, rank, local = dist_setup(args)
+    torch.cuda.set_device(local)
+    cr.lib()
+    pk = peaks()
+    case = inputs.CASES[args.workload]
+    if case.M > 8:
+        raise SystemExit("the headline workload must be a decode batch (M <= 8)")
+    M, N, K = case.M, case.N, case.K
+    sets = Sets(case, rank)
+
+    # headline: the whole step (rotate+quant launch + GEMV launch), graph-replayed
+    secs, clocks = graph_time(sets.step, args.steps, args.warmup, world, local)
+    secs = max_over_ranks(secs, world)
+    wb = weight_bytes(N, K)
+    value = world * wb * args.steps / secs / 1e9
+
+    # the dominant kernel alone (GEMV), for the roofline
+    ksecs, _ = graph_time(sets.contraction_only, args.steps, args.warmup, world, local)
+    ksecs = max_over_ranks(ksecs, world)
+    per_launch = ksecs / args.steps
+    achieved = gemv_launch_bytes(M, N, K) / per_launch / 1e9
+    traffic = prior_traffic("gemv_kernel_c2")
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
+                "kernel": "cr::gv::gemv_kernel", "peak_source": f"{pk['source']} (hbm_gbs)",
+                "algorithmic_bytes_per_launch": gemv_launch_bytes(M, N, K),
+                "us_per_launch": round(per_launch * 1e6, 3)}
+
+    # end to end through the public API with host buffers
+    esecs = eager_time(sets.e2e_step, args.steps, args.warmup, world)
+    esecs = max_over_ranks(esecs, world)
+    e2e = {"value": round(world * wb * args.steps / esecs / 1e9, 2), "unit": "GB/s",
+           "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N,
+           "ms_per_step": round(esecs / args.steps * 1e3, 5)}
+
+    prefill = None
+    if not args.no_prefill:
+        prefill = run_prefill(args, world, rank, local, pk)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(case, args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
+        "config": {"workload": f"{case.name}: decode batch M={M}, N={N}, K={K}, rot 256, group 16, seed {case.seed}",
+                   "path": "cr_w4a8_linear = rotate+quant kernel + fused decode GEMV kernel",
+                   "l2": f"rotating {sets.R} copies of layer+activations ({sets.R * (wb + 2 * M * K) / 2**20:.0f} MiB > 126 MiB L2)",
+                   "timing": "one CUDA-graph replay of K steps, CUDA events on the capture stream",
+                   "parallelism": f"replica x{world}"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps,
+        "clocks": clocks, "prefill": prefill,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_prefill(args, world, rank, local, pk):
+    """The prefill step (rotate+quant, decode transient, tcgen05 GEMM), eager."""
+    import torch
+
+    import w4a8_codebook_quantized_b200 as cr
+    from w4a8_codebook_quantized_b200 import inputs
+    case = inputs.CASES[args.prefill_workload]
+    M, N, K = case.M, case.N, case.K
+    layer = inputs.layer(N, K, case.seed + 1000 * rank)
+    x = inputs.activations(M, K, case.seed + 1000 * rank, case.dist)
+    q = torch.from_numpy(layer.qdata).cuda()
+    s = torch.from_numpy(layer.srel).cuda()
+    cb = torch.from_numpy(layer.codebook).cuda()
+    ws = torch.from_numpy(layer.s_channel).cuda()
+    xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+    xs = torch.empty(M, dtype=torch.float32, device="cuda")
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    steps = max(3, min(args.steps, 50))
+
+    def step(i):
+        cr.cr_w4a8_linear(xd, q, s, cb, ws, out=out, xq_work=xq, xs_work=xs)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    # per-step timing with an L2 flush between steps (outside the events)
+    stream = torch.cuda.current_stream()
+    times = []
+    kt = []
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        cr.cr_rotate_quant_act(xd, M, 127, xq=xq, xs=xs)
+        e1.record(stream)
+        cr.cr_w4a8_gemm(xq, xs, q, s, cb, ws, out=out)
+        e2.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e2) / 1000.0)
+        kt.append(e1.elapsed_time(e2) / 1000.0)
+    t = max_over_ranks(statistics.median(times), world)
+    tg = max_over_ranks(statistics.median(kt), world)
+    ops = 2.0 * M * N * K
+    peak_tops = pk["bf16_tflops"] * INT8_OVER_BF16
+    achieved = ops / tg / 1e12
+    return {"workload": f"{case.name}: prefill M={M}, N={N}, K={K}", "value": round(world * ops / t / 1e12, 2),
+            "unit": "TOPS", "ms_per_step": round(t * 1e3, 4), "steps": steps,
+            "l2": "256 MiB write between steps, outside the timed events",
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_tops, 1),
+                         "unit": "TOPS", "frac": round(achieved / peak_tops, 4), "traffic": None,
+                         "kernel": "cr_w4a8_gemm call (decode-to-int8 transient + tcgen05 GEMM)",
+                         "peak_source": f"{pk['source']} bf16_tflops x {INT8_OVER_BF16} (nominal int8/bf16 ratio)",
+                         "us_per_call": round(tg * 1e6, 2)}}
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The oracle (plain CPU C) timed as the reference arm on the same workload."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from w4a8_codebook_quantized_b200 import inputs
+    case = inputs.CASES[args.workload]
+    M, N, K = case.M, case.N, case.K
+    layer = inputs.layer(N, K, case.seed)
+    x = inputs.activations(M, K, case.seed, case.dist)
+    oracle.lib()
+    # one step = one full forward pass, or a row sample of the layer when K
+    # full passes would not finish in about two minutes
+    t0 = time.perf_counter()
+    oracle.linear(x, layer.qdata, layer.srel, layer.codebook, layer.s_channel, threads=1)
+    one = time.perf_counter() - t0
+    budget = 120.0
+    frac = 1.0
+    if one * (args.steps + args.warmup) > budget:
+        frac = max(1.0 / 64, budget / (one * (args.steps + args.warmup)))
+    rows = max(16, int(N * frac) // 16 * 16)
+    sub = inputs.Layer(layer.qdata[:rows], layer.srel[:rows], layer.s_channel[:rows], layer.codebook)
+    for _ in range(args.warmup):
+        oracle.linear(x, sub.qdata, sub.srel, sub.codebook, sub.s_channel, threads=1)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.linear(x, sub.qdata, sub.srel, sub.codebook, sub.s_channel, threads=1)
+    el = time.perf_counter() - t0
+    wb = weight_bytes(rows, K)
+    value = wb * args.steps / el / 1e9
+    sample = (f"each step: full forward of M={M}, K={K} over {rows} of the {N} output rows "
+              f"({'whole layer' if rows == N else 'row sample'})")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
+            "config": {"workload": f"{case.name}: decode batch M={M}, N={N}, K={K}, rot 256, group 16",
+                       "parallelism": "host CPU, 1 thread"},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,208 @@
+/*
+ * cr_w4a8.h -- C ABI of the ConvRot W4A8 codebook linear layer forward on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The layer (ai-toolkit convrot_w4a8_quant.py, module docstring) stores a
+ * linear weight W [N out, K in] that was rotated by a block regular Hadamard
+ * (block R = 256) as 4-bit codebook indices with one fp8 e4m3fn relative
+ * scale per group of G = 16 columns and one fp32 scale per output channel:
+ *
+ *   w_int8[n, k] = sat_s8(rne(codebook[code[n, k]] * s_rel[n, k / 16]))
+ *   W_rot[n, k]  = w_int8[n, k] * s_channel[n]
+ *
+ * The forward rotates each activation row block-wise by the same Hadamard,
+ * quantises it per token to int8, contracts int8 x int8 -> int32 and rescales
+ * by the per-token and per-channel scales:
+ *
+ *   y[m, n] = bf16( float(sum_k xq[m, k] * w_int8[n, k]) * (xs[m] * s_channel[n]) [+ bias[n]] )
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * - Pointers are DEVICE pointers unless stated otherwise; the caller owns all
+ *   memory.  Every call is asynchronous on `stream` (NULL = the legacy default
+ *   stream) and returns as soon as the work is queued.
+ * - Arrays are dense and row-major, with exactly the shapes given.
+ * - Every pointer must be 16-byte aligned (CR_ERR_ALIGNMENT otherwise).
+ * - Sizes are int64_t.  M == 0 or N == 0 is an empty problem: CR_OK, nothing
+ *   is launched.  Negative sizes give CR_ERR_INVALID_ARG.
+ * - K must be a positive multiple of 256 (the rotation block; it implies the
+ *   group size 16) and at most CR_MAX_K (CR_ERR_UNSUPPORTED otherwise).
+ * - Arguments are validated before anything is launched; a failed validation
+ *   launches nothing and leaves every output untouched.  Launch failures
+ *   return CR_ERR_CUDA.  Nothing falls back to another implementation.
+ * - Values are not validated: activations must be finite and small enough
+ *   that a block sum of four of them does not overflow fp32 (|x| <= 2^124);
+ *   for other values the outputs are unspecified, but no call faults.
+ * - Calls that read a buffer another call on another stream is writing race,
+ *   as with any CUDA kernel.
+ */
+#ifndef CR_W4A8_H
+#define CR_W4A8_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (the same handle type, declared without the CUDA headers). */
+typedef struct CUstream_st *cr_stream_t;
+
+typedef enum {
+    CR_OK = 0,
+    CR_ERR_INVALID_ARG = 1,  /* null pointer, negative size, MP < M, act_qmax outside 1..127 */
+    CR_ERR_UNSUPPORTED = 2,  /* K not a positive multiple of 256, K > CR_MAX_K, GEMV with M > 8 */
+    CR_ERR_ALIGNMENT = 3,    /* a pointer is not 16-byte aligned */
+    CR_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    CR_ERR_TIMEOUT = 5,      /* a kernel gave up waiting on its own pipeline (see cr_check_device_error) */
+    CR_ERR_NO_DEVICE = 6     /* no sm_100 device is current */
+} cr_status;
+
+typedef enum {
+    CR_OUT_BF16 = 0, /* output elements are bf16, rounded to nearest even */
+    CR_OUT_F32 = 1   /* output elements are fp32 */
+} cr_out_dtype;
+
+/* Largest supported K: keeps |acc| <= 127 * 128 * K inside int32
+ * (ai-toolkit convrot_w4a8_quant.py, w4a8_gemv_kernel: int32 accumulation). */
+#define CR_MAX_K 131072
+/* Rotation block and group size (ai-toolkit convrot_w4a8_quant.py,
+ * ConvRotW4A8Quantizer.__init__ defaults rot_size=256, group_size=16). */
+#define CR_ROT 256
+#define CR_GROUP 16
+/* Largest M the decode GEMV takes (ai-toolkit convrot_w4a8_quant.py,
+ * W4A8_GEMV_MAX_M). */
+#define CR_GEMV_MAX_M 8
+
+/* Static, NUL-terminated description of a status code.  Host only. */
+const char *cr_status_string(cr_status s);
+
+/*
+ * (1) Rotate + per-token int8 quantisation of the activations.
+ *
+ * Defined by: ai-toolkit convrot_w4a8_quant.py, prepare_act (rotate, then
+ * quantise the rows once) and w4a8_act_quant_kernel (per-row symmetric int8
+ * quant into exactly MP rows); the rotation is h3-rs src/weights.rs,
+ * hadamard() / rotate_activation(): each 256-column block of a row times
+ * H_256 = (h4 (x) h4 (x) h4 (x) h4) / 16.
+ *
+ *   r      = x rotated block-wise, in fp32 from the exact bf16 inputs, digit
+ *            stages in the order stride 1, 4, 16, 64; per quadruple
+ *            out[a] = ((v0 + v1) + (v2 + v3)) - 2 * v[3 - a]; then * 1/16
+ *   xs[m]  = max_k |r[m, k]| / act_qmax   (1.0 if that max is 0)
+ *   xq[m,k]= clamp(rint(r[m, k] / xs[m]), -act_qmax, act_qmax)
+ *   rows M <= m < MP:  xq = 0, xs = 1
+ *
+ * x   [M, K]  bf16 (bit patterns), read only.
+ * xq  [MP, K] int8, written.     xs [MP] fp32, written.
+ * MP >= M (the decode GEMV pads to the next power of two; prefill passes MP = M).
+ * act_qmax in 1..127 (the layer uses 127).
+ */
+cr_status cr_rotate_quant_act(const uint16_t *x, int64_t M, int64_t K, int64_t MP,
+                              int act_qmax, int8_t *xq, float *xs, cr_stream_t stream);
+
+/*
+ * (2) Decode the packed codes onto the int8 grid.
+ *
+ * Defined by: ai-toolkit convrot_w4a8_quant.py, module docstring storage
+ * formula, unpack_w4a8_eager and w4a8_unpack_kernel with W4A8_SAT = True:
+ *   w8[n, k] = sat_s8(rne(codebook[code(n, k)] * fp8(srel[n, k / 16])))
+ * where code(n, 2j) is the low nibble and code(n, 2j+1) the high nibble of
+ * qdata[n, j], the product is one fp32 multiply, rne rounds to nearest even
+ * and sat_s8 saturates to [-128, 127] (a NaN product gives 0).
+ *
+ * qdata    [N, K/2]  packed codes, read only.
+ * srel     [N, K/16] fp8 e4m3fn scale bytes, read only.
+ * codebook [16]      fp32 levels, read only.
+ * w8       [N, K]    int8, written.
+ */
+cr_status cr_w4a8_decode_int8(const uint8_t *qdata, const uint8_t *srel, const float *codebook,
+                              int64_t N, int64_t K, int8_t *w8, cr_stream_t stream);
+
+/*
+ * (3) Prefill forward for any M: decode + int8 tensor-core contraction +
+ * epilogue.
+ *
+ * Defined by: ai-toolkit convrot_w4a8_quant.py, _w4a8_linear_ste_op (decode
+ * the codes, quantise the activations, torch._int_mm(aq, w8.t()), then
+ * _int8_epilogue) with the epilogue of w4a8_gemv_kernel:
+ *   acc[m, n] = sum_k xq[m, k] * w8[n, k]          (exact int32)
+ *   out[m, n] = float(acc) * (xs[m] * s_channel[n]) [+ bias[n]], each op
+ *               rounded on its own, then cast to out_dtype.
+ *
+ * xq        [M, K] int8 and xs [M] fp32: the output of cr_rotate_quant_act.
+ * qdata, srel, codebook: as in cr_w4a8_decode_int8.
+ * s_channel [N] fp32.   bias [N] fp32, or NULL for no bias.
+ * out       [M, N] bf16 or fp32 per out_dtype, written.
+ * acc_out   [M, N] int32, or NULL: when given, the raw accumulators are
+ *           written too (a parity/debug output).
+ */
+cr_status cr_w4a8_gemm(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                       const float *codebook, const float *s_channel, const float *bias,
+                       int64_t M, int64_t N, int64_t K, cr_out_dtype out_dtype, void *out,
+                       int32_t *acc_out, cr_stream_t stream);
+
+/*
+ * (4) Decode forward for 1 <= M <= 8: a fused GEMV that streams the packed
+ * codes, the fp8 group scales and the codebook (4.5 bits per weight) and
+ * never materialises the int8 weight.
+ *
+ * Defined by: ai-toolkit convrot_w4a8_quant.py, w4a8_gemv_kernel and
+ * gemv_prepared.  Same arguments and the same results as cr_w4a8_gemm,
+ * bit for bit (int32 accumulation is exact and order independent, and both
+ * share the epilogue).  xq needs only its first M rows.  M > 8 gives
+ * CR_ERR_UNSUPPORTED.
+ */
+cr_status cr_w4a8_gemv(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                       const float *codebook, const float *s_channel, const float *bias,
+                       int64_t M, int64_t N, int64_t K, cr_out_dtype out_dtype, void *out,
+                       int32_t *acc_out, cr_stream_t stream);
+
+/*
+ * (5) The epilogue alone, on an int32 accumulator.
+ *
+ * Defined by: ai-toolkit convrot_w4a8_quant.py, w4a8_gemv_kernel epilogue
+ * (and _int8_epilogue, called with the same arguments by the prefill op):
+ *   out[m, n] = float(acc[m, n]) * (xs[m] * s_channel[n]) [+ bias[n]]
+ *
+ * acc [M, N] int32, xs [M] fp32, s_channel [N] fp32, bias [N] fp32 or NULL;
+ * out [M, N] bf16 or fp32, written.
+ */
+cr_status cr_epilogue(const int32_t *acc, const float *xs, const float *s_channel, const float *bias,
+                      int64_t M, int64_t N, cr_out_dtype out_dtype, void *out, cr_stream_t stream);
+
+/*
+ * (6) The whole layer forward in one call: (1), then (4) when M <= 8, else (3).
+ *
+ * Defined by: ai-toolkit convrot_w4a8_quant.py, ConvRotW4A8Quantizer.forward
+ * (decode GEMV when gemv_ok, otherwise the prefill op).
+ *
+ * x [M, K] bf16 bits; weights as in (3); out [M, N].
+ * xq_work [max(M, MP), K] int8 and xs_work [max(M, MP)] fp32 are caller-owned
+ * scratch for the quantised activations, where MP is the next power of two
+ * of M when M <= 8 and M otherwise; their contents on return are the
+ * quantised activations.
+ */
+cr_status cr_w4a8_linear(const uint16_t *x, const uint8_t *qdata, const uint8_t *srel,
+                         const float *codebook, const float *s_channel, const float *bias,
+                         int64_t M, int64_t N, int64_t K, int act_qmax, cr_out_dtype out_dtype,
+                         void *out, int8_t *xq_work, float *xs_work, cr_stream_t stream);
+
+/*
+ * Waits for `stream`, then reads and clears the library's device error word,
+ * which a kernel sets when one of its bounded pipeline waits runs out (the
+ * kernel then abandons its tile and exits; its outputs are unspecified).
+ * Returns CR_OK, CR_ERR_TIMEOUT, or CR_ERR_CUDA if the wait itself failed.
+ * This is the one synchronising call in the library.
+ */
+cr_status cr_check_device_error(cr_stream_t stream);
+
+/* Library version, e.g. "0.1.0".  Host only. */
+const char *cr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CR_W4A8_H */

@@ -1,0 +1,134 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the
+header declares, and rejects bad arguments before touching any device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import w4a8_codebook_quantized_b200 as cr
+from w4a8_codebook_quantized_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "cr_w4a8.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return cr.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(cr_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv", "cr_epilogue",
+              "cr_w4a8_linear", "cr_status_string", "cr_check_device_error", "cr_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+    out = os.popen(f"nm -D --defined-only {cr.library_path()}").read()
+    exported = set(re.findall(r" T (cr_\w+)", out))
+    assert set(_declared()) <= exported
+    # nothing else leaks out under the cr_ prefix
+    assert exported == set(_declared())
+
+
+def test_library_is_built_for_sm100a_only():
+    out = os.popen(f"cuobjdump --list-elf {cr.library_path()} 2>&1").read()
+    assert "sm_100a" in out
+    assert not re.search(r"sm_(?!100a)\d+", out)
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert cr.cr_status_string(s)
+    assert cr.cr_status_string(99) == "unknown status"
+    assert cr.cr_version().count(".") == 2
+
+
+P = ctypes.c_void_p
+A16 = 0x10000  # a 16-byte aligned stand-in address; never dereferenced on these paths
+MIS = 0x10008  # 8-byte aligned only
+
+
+def test_rotate_quant_validation(L):
+    f = L.cr_rotate_quant_act
+    assert f(A16, -1, 256, 1, 127, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, 2, 256, 1, 127, A16, A16, None) == cr.CR_ERR_INVALID_ARG      # MP < M
+    assert f(A16, 1, 256, 1, 0, A16, A16, None) == cr.CR_ERR_INVALID_ARG        # qmax
+    assert f(A16, 1, 256, 1, 128, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, 1, 128, 1, 127, A16, A16, None) == cr.CR_ERR_UNSUPPORTED      # K % 256
+    assert f(A16, 1, 0, 1, 127, A16, A16, None) == cr.CR_ERR_UNSUPPORTED
+    assert f(A16, 1, 131072 + 256, 1, 127, A16, A16, None) == cr.CR_ERR_UNSUPPORTED
+    assert f(None, 1, 256, 1, 127, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(MIS, 1, 256, 1, 127, A16, A16, None) == cr.CR_ERR_ALIGNMENT
+    assert f(A16, 1, 256, 1, 127, MIS, A16, None) == cr.CR_ERR_ALIGNMENT
+    assert f(None, 0, 256, 0, 127, None, None, None) == cr.CR_OK                # empty
+
+
+def test_decode_validation(L):
+    f = L.cr_w4a8_decode_int8
+    assert f(A16, A16, A16, -1, 256, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, A16, A16, 4, 272, A16, None) == cr.CR_ERR_UNSUPPORTED
+    assert f(None, A16, A16, 4, 256, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, MIS, A16, 4, 256, A16, None) == cr.CR_ERR_ALIGNMENT
+    assert f(None, None, None, 0, 256, None, None) == cr.CR_OK
+
+
+@pytest.mark.parametrize("name", ["cr_w4a8_gemm", "cr_w4a8_gemv"])
+def test_contraction_validation(L, name):
+    f = getattr(L, name)
+    ok = [A16] * 7
+
+    def call(M=4, N=8, K=256, dtype=0, ptrs=None, out=A16, acc=None):
+        p = ptrs or ok
+        return f(*p, M, N, K, dtype, out, acc, None)
+
+    assert call(M=-1) == cr.CR_ERR_INVALID_ARG
+    assert call(dtype=7) == cr.CR_ERR_INVALID_ARG
+    assert call(K=320) == cr.CR_ERR_UNSUPPORTED
+    assert call(out=None) == cr.CR_ERR_INVALID_ARG
+    bad = list(ok)
+    bad[3] = MIS
+    assert call(ptrs=bad) == cr.CR_ERR_ALIGNMENT
+    nob = list(ok)
+    nob[6] = None  # bias is optional: fine
+    assert call(ptrs=nob, M=0) == cr.CR_OK
+    assert call(acc=MIS) == cr.CR_ERR_ALIGNMENT
+    assert call(M=0) == cr.CR_OK and call(N=0) == cr.CR_OK
+    if name == "cr_w4a8_gemv":
+        assert call(M=9) == cr.CR_ERR_UNSUPPORTED
+
+
+def test_epilogue_and_linear_validation(L):
+    assert L.cr_epilogue(A16, A16, A16, None, -1, 4, 0, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert L.cr_epilogue(A16, A16, A16, None, 2, 4, 3, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert L.cr_epilogue(A16, MIS, A16, None, 2, 4, 0, A16, None) == cr.CR_ERR_ALIGNMENT
+    assert L.cr_epilogue(None, None, None, None, 0, 4, 0, None, None) == cr.CR_OK
+    f = L.cr_w4a8_linear
+    assert f(A16, A16, A16, A16, A16, None, 2, 8, 256, 0, 0, A16, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, A16, A16, A16, A16, None, 2, 8, 384, 127, 0, A16, A16, A16, None) == cr.CR_ERR_UNSUPPORTED
+    assert f(None, A16, A16, A16, A16, None, 2, 8, 256, 127, 0, A16, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(MIS, A16, A16, A16, A16, None, 2, 8, 256, 127, 0, A16, A16, A16, None) == cr.CR_ERR_ALIGNMENT
+
+
+def test_valid_call_without_a_gpu_fails_loudly(L):
+    """On a machine with no usable sm_100 device a well-formed call reports
+    CR_ERR_NO_DEVICE instead of computing anything anywhere else."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert L.cr_w4a8_decode_int8(A16, A16, A16, 4, 256, A16, None) == cr.CR_ERR_NO_DEVICE
+    assert L.cr_check_device_error(None) == cr.CR_ERR_NO_DEVICE
+    with pytest.raises(ValueError):
+        cr.cr_w4a8_decode_int8(torch.zeros(4, 128, dtype=torch.uint8), torch.zeros(4, 16, dtype=torch.uint8),
+                               torch.zeros(16))

@@ -1,0 +1,197 @@
+"""GPU parity: every entry point of the C ABI against the CPU oracle, element
+by element, on seeded inputs.  Integer stages (unpack/decode, int8
+activations, scales, int32 accumulators) must be bit-exact; outputs meet the
+normwise tolerance and are also checked bit for bit."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import w4a8_codebook_quantized_b200 as cr
+from w4a8_codebook_quantized_b200 import inputs
+
+from gpu_util import Guarded, assert_output_close, bf16_dev, dev, host
+
+pytestmark = pytest.mark.gpu
+
+THREADS = max(1, min(32, os.cpu_count() or 1))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    cr.lib()
+    yield
+    cr.cr_check_device_error()
+
+
+def _layer_dev(layer):
+    return (dev(layer.qdata), dev(layer.srel), dev(layer.codebook), dev(layer.s_channel),
+            None if layer.bias is None else dev(layer.bias))
+
+
+# ---------------------------------------------------------------- decode
+
+def test_decode_exhaustive_scale_bytes_and_codes():
+    """All 256 scale bytes x 16 codes (NaN bytes included) through the kernel."""
+    N, K = 256, 256
+    q = np.tile(np.array([0x10, 0x32, 0x54, 0x76, 0x98, 0xBA, 0xDC, 0xFE], np.uint8), (N, K // 16))
+    s = np.repeat(np.arange(256, dtype=np.uint8)[:, None], K // 16, axis=1)
+    for cb in (inputs.codebook(), np.arange(-8, 8, dtype=np.float32),
+               np.linspace(-300, 300, 16).astype(np.float32)):
+        w8 = cr.cr_w4a8_decode_int8(dev(q), dev(s), dev(cb))
+        assert np.array_equal(host(w8), oracle.decode_w8(q, s, cb))
+
+
+@pytest.mark.parametrize("N,K,seed", [(1, 256, 0), (37, 512, 1), (1000, 1024, 2), (4096, 4096, 3)])
+def test_decode_random_layers(N, K, seed):
+    layer = inputs.layer(N, K, seed)
+    out = Guarded((N, K), torch.int8)
+    cr.cr_w4a8_decode_int8(dev(layer.qdata), dev(layer.srel), dev(layer.codebook), w8=out.tensor)
+    torch.cuda.synchronize()
+    assert out.intact()
+    assert np.array_equal(host(out.tensor), oracle.decode_w8(layer.qdata, layer.srel, layer.codebook))
+
+
+# ---------------------------------------------------------------- rotate + quantise
+
+def _rq_case(M, K, seed, mp=None, qmax=127, dist="outliers"):
+    x = inputs.activations(M, K, seed, dist)
+    MP = M if mp is None else mp
+    xq_g = Guarded((MP, K), torch.int8)
+    xs_g = Guarded((MP,), torch.float32)
+    cr.cr_rotate_quant_act(bf16_dev(x), MP, qmax, xq=xq_g.tensor, xs=xs_g.tensor)
+    torch.cuda.synchronize()
+    assert xq_g.intact() and xs_g.intact()
+    xq_r, xs_r = oracle.rotate_quant_act(x, MP, qmax)
+    assert np.array_equal(host(xs_g.tensor).view(np.uint32), xs_r.view(np.uint32))
+    assert np.array_equal(host(xq_g.tensor), xq_r)
+
+
+@pytest.mark.parametrize("M,K,MP", [(1, 256, 1), (3, 1024, 4), (8, 4096, 8), (5, 4096, 8), (2, 8192, 2),
+                                    (4, 12288, 4), (2, 16384, 2), (2, 20480, 2), (1, 65536, 1), (33, 768, 33)])
+def test_rotate_quant_shapes(M, K, MP):
+    _rq_case(M, K, seed=M * 1000 + K, mp=MP)
+
+
+def test_rotate_quant_other_qmax_and_gelu_inputs():
+    _rq_case(6, 2048, 7, qmax=7)
+    _rq_case(4, 12288, 8, dist="gelu")
+
+
+def test_rotate_quant_degenerate_rows():
+    """Zero rows (scale 1), subnormal-only rows, huge rows, a one-hot row."""
+    K = 512
+    rows = np.zeros((5, K), np.float64)
+    rows[1, :7] = 2.0 ** -130
+    rows[2] = np.linspace(-2.0 ** 100, 2.0 ** 100, K)
+    rows[3, 300] = -1.0
+    rows[4] = 1.0
+    x = torch.from_numpy(rows).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    xq, xs = cr.cr_rotate_quant_act(bf16_dev(x), 8, 127)
+    xq_r, xs_r = oracle.rotate_quant_act(x, 8, 127)
+    assert np.array_equal(host(xs).view(np.uint32), xs_r.view(np.uint32))
+    assert np.array_equal(host(xq), xq_r)
+    assert host(xs)[0] == 1.0 and (host(xq)[0] == 0).all()
+
+
+# ---------------------------------------------------------------- epilogue
+
+@pytest.mark.parametrize("M,N,with_bias,kind", [(1, 8, False, "bf16"), (7, 1000, True, "bf16"),
+                                                (64, 4096, False, "f32"), (3, 37, True, "f32"),
+                                                (5, 6, True, "bf16")])
+def test_epilogue(M, N, with_bias, kind):
+    rng = np.random.default_rng(M * N)
+    acc = rng.integers(-2 ** 28, 2 ** 28, size=(M, N)).astype(np.int32)
+    acc[0, 0] = 16777217
+    xs = rng.uniform(1e-3, 0.2, size=M).astype(np.float32)
+    ws = rng.uniform(1e-4, 5e-4, size=N).astype(np.float32)
+    bias = rng.normal(size=N).astype(np.float32) if with_bias else None
+    dt = torch.bfloat16 if kind == "bf16" else torch.float32
+    out = Guarded((M, N), dt)
+    cr.cr_epilogue(dev(acc), dev(xs), dev(ws), None if bias is None else dev(bias), out=out.tensor)
+    torch.cuda.synchronize()
+    assert out.intact()
+    assert_output_close(host(out.tensor), oracle.epilogue(acc, xs, ws, bias, kind), kind)
+
+
+# ---------------------------------------------------------------- contraction
+
+def _contraction_case(fn, M, N, K, seed, kind="bf16", with_bias=False, dist="outliers"):
+    layer = inputs.layer(N, K, seed, with_bias=with_bias)
+    x = inputs.activations(M, K, seed, dist)
+    xq_r, xs_r = oracle.rotate_quant_act(x, None, 127)
+    w8 = oracle.decode_w8(layer.qdata, layer.srel, layer.codebook)
+    acc_r = oracle.gemm_s32(xq_r, w8, THREADS)
+    y_r = oracle.epilogue(acc_r, xs_r, layer.s_channel, layer.bias, kind)
+    q, s, cb, ws, b = _layer_dev(layer)
+    dt = torch.bfloat16 if kind == "bf16" else torch.float32
+    out = Guarded((M, N), dt)
+    acc = Guarded((M, N), torch.int32)
+    fn(dev(xq_r), dev(xs_r), q, s, cb, ws, b, out=out.tensor, acc_out=acc.tensor)
+    torch.cuda.synchronize()
+    assert out.intact() and acc.intact()
+    assert np.array_equal(host(acc.tensor), acc_r)
+    assert_output_close(host(out.tensor), y_r, kind)
+    # and without the optional accumulator output
+    out2 = fn(dev(xq_r), dev(xs_r), q, s, cb, ws, b, out_dtype=dt)
+    assert np.array_equal(host(out2), host(out.tensor))
+    return host(acc.tensor), host(out.tensor)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 16, 256), (1, 1024, 1024), (2, 1000, 512), (3, 17, 768), (4, 4096, 1024),
+                                   (8, 4096, 4096), (5, 2048, 2048), (8, 256, 12288), (6, 33, 8192)])
+def test_gemv(M, N, K):
+    _contraction_case(cr.cr_w4a8_gemv, M, N, K, seed=M + N + K)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 256, 256), (8, 256, 512), (100, 300, 1024), (128, 256, 256),
+                                   (129, 257, 256), (300, 1000, 1024), (256, 4096, 2048), (2048, 512, 4096),
+                                   (17, 17, 768), (640, 1536, 1280)])
+def test_gemm(M, N, K):
+    _contraction_case(cr.cr_w4a8_gemm, M, N, K, seed=M + N + K)
+
+
+@pytest.mark.parametrize("kind,with_bias", [("f32", False), ("f32", True), ("bf16", True)])
+def test_output_kinds_and_bias(kind, with_bias):
+    _contraction_case(cr.cr_w4a8_gemv, 3, 520, 1024, 11, kind, with_bias)
+    _contraction_case(cr.cr_w4a8_gemm, 200, 520, 1024, 12, kind, with_bias)
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_gemv_equals_gemm_bitwise(M):
+    """The pages call the decode GEMV bit-identical to the _int_mm path."""
+    N, K = 768, 2048
+    layer = inputs.layer(N, K, 40 + M)
+    x = bf16_dev(inputs.activations(M, K, 40 + M))
+    xq, xs = cr.cr_rotate_quant_act(x, cr.gemv_rows(M), 127)
+    q, s, cb, ws, b = _layer_dev(layer)
+    o1, a1 = cr.cr_w4a8_gemv(xq, xs, q, s, cb, ws, m=M, acc_out=True)
+    o2, a2 = cr.cr_w4a8_gemm(xq, xs, q, s, cb, ws, m=M, acc_out=True)
+    assert torch.equal(a1, a2) and torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 512, 1024), (8, 1024, 4096), (5, 300, 512), (96, 640, 2048)])
+def test_linear_end_to_end(M, N, K):
+    layer = inputs.layer(N, K, 7 * M)
+    x = inputs.activations(M, K, 7 * M)
+    ref = oracle.linear(x, layer.qdata, layer.srel, layer.codebook, layer.s_channel, threads=THREADS)
+    q, s, cb, ws, b = _layer_dev(layer)
+    y = cr.cr_w4a8_linear(bf16_dev(x), q, s, cb, ws)
+    assert_output_close(host(y), ref["y"], "bf16")
+
+
+def test_empty_problems_launch_nothing():
+    layer = inputs.layer(16, 256, 1)
+    q, s, cb, ws, b = _layer_dev(layer)
+    xq = torch.empty(0, 256, dtype=torch.int8, device="cuda")
+    xs = torch.empty(0, dtype=torch.float32, device="cuda")
+    assert cr.cr_w4a8_gemm(xq, xs, q, s, cb, ws).shape == (0, 16)
+    assert cr.cr_w4a8_gemv(xq, xs, q, s, cb, ws).shape == (0, 16)
+
+
+def test_no_device_error_pending():
+    cr.cr_check_device_error()

@@ -1,0 +1,283 @@
+"""ConvRot W4A8 codebook linear layer forward on NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over the C ABI in ``include/cr_w4a8.h``
+(``libcr_w4a8.so``, built in-tree by ``w4a8_codebook_quantized_b200.build``).
+The functions carry the C names and only marshal arguments: they take torch
+CUDA tensors, pass their device pointers and the current CUDA stream, and
+raise ``CrError`` on a non-OK status.  All arithmetic runs in the library's
+kernels; there is no other implementation to fall back to, and a missing
+library or GPU raises.
+
+Storage of one layer (ai-toolkit convrot_w4a8_quant.py, module docstring):
+    qdata     uint8/int8 [N, K/2]   packed 4-bit codes, even column = low nibble
+    srel      uint8      [N, K/16]  fp8 e4m3fn group scales (byte view)
+    s_channel float32    [N]        per-output-channel scale
+    codebook  float32    [16]       codebook levels
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+__all__ = [
+    "CrError", "lib", "library_path",
+    "cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv",
+    "cr_epilogue", "cr_w4a8_linear", "cr_check_device_error", "cr_status_string", "cr_version",
+    "gemv_rows",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libcr_w4a8.so")
+
+CR_OK, CR_ERR_INVALID_ARG, CR_ERR_UNSUPPORTED, CR_ERR_ALIGNMENT, CR_ERR_CUDA, CR_ERR_TIMEOUT, CR_ERR_NO_DEVICE = range(7)
+CR_OUT_BF16, CR_OUT_F32 = 0, 1
+CR_GEMV_MAX_M = 8
+
+_lib = None
+_lock = threading.Lock()
+
+
+class CrError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {cr_status_string(status)} (status {status})")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library with typed entry points (the raw C ABI)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise ImportError(
+                    f"{_LIB_PATH} is missing: build it with `python -m w4a8_codebook_quantized_b200.build`")
+            L = ctypes.CDLL(_LIB_PATH)
+            P, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+            L.cr_status_string.argtypes = [i32]
+            L.cr_status_string.restype = ctypes.c_char_p
+            L.cr_version.argtypes = []
+            L.cr_version.restype = ctypes.c_char_p
+            L.cr_rotate_quant_act.argtypes = [P, i64, i64, i64, i32, P, P, P]
+            L.cr_w4a8_decode_int8.argtypes = [P, P, P, i64, i64, P, P]
+            contraction = [P, P, P, P, P, P, P, i64, i64, i64, i32, P, P, P]
+            L.cr_w4a8_gemm.argtypes = contraction
+            L.cr_w4a8_gemv.argtypes = contraction
+            L.cr_epilogue.argtypes = [P, P, P, P, i64, i64, i32, P, P]
+            L.cr_w4a8_linear.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P, P, P]
+            L.cr_check_device_error.argtypes = [P]
+            for name in ("cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv",
+                         "cr_epilogue", "cr_w4a8_linear", "cr_check_device_error"):
+                getattr(L, name).restype = i32
+            _lib = L
+    return _lib
+
+
+def cr_status_string(status: int) -> str:
+    return lib().cr_status_string(int(status)).decode()
+
+
+def cr_version() -> str:
+    return lib().cr_version().decode()
+
+
+# ---------------------------------------------------------------- marshalling
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need(t, name, dtypes, ndim=None, shape=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {tuple(t.shape)}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+def _check(status: int, where: str) -> None:
+    if status != CR_OK:
+        raise CrError(status, where)
+
+
+def _out_code(dtype) -> int:
+    torch = _torch()
+    if dtype == torch.bfloat16:
+        return CR_OUT_BF16
+    if dtype == torch.float32:
+        return CR_OUT_F32
+    raise TypeError(f"out dtype must be bfloat16 or float32, got {dtype}")
+
+
+def gemv_rows(m: int) -> int:
+    """Rows of the decode GEMV's padded activation operand: next power of two
+    of M (ai-toolkit convrot_w4a8_quant.py, _gemv_mp)."""
+    return 1 << max(0, (int(m) - 1).bit_length())
+
+
+def _layer(qdata, srel, codebook, s_channel, bias):
+    torch = _torch()
+    _need(qdata, "qdata", (torch.uint8, torch.int8), 2)
+    N, KH = qdata.shape
+    K = 2 * KH
+    _need(srel, "srel", (torch.uint8, torch.float8_e4m3fn), shape=(N, K // 16))
+    _need(codebook, "codebook", (torch.float32,), shape=(16,))
+    _need(s_channel, "s_channel", (torch.float32,), shape=(N,))
+    if bias is not None:
+        _need(bias, "bias", (torch.float32,), shape=(N,))
+    return N, K
+
+
+# ---------------------------------------------------------------- entry points
+
+def cr_rotate_quant_act(x, mp: Optional[int] = None, act_qmax: int = 127, xq=None, xs=None,
+                        stream=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
+    """x bf16 [M, K] -> (xq int8 [MP, K], xs fp32 [MP]); rows >= M are 0 / 1."""
+    torch = _torch()
+    _need(x, "x", (torch.bfloat16,), 2)
+    M, K = x.shape
+    MP = M if mp is None else int(mp)
+    if xq is None:
+        xq = torch.empty(MP, K, dtype=torch.int8, device=x.device)
+    if xs is None:
+        xs = torch.empty(MP, dtype=torch.float32, device=x.device)
+    _need(xq, "xq", (torch.int8,), shape=(MP, K))
+    _need(xs, "xs", (torch.float32,), shape=(MP,))
+    _check(lib().cr_rotate_quant_act(_ptr(x), M, K, MP, int(act_qmax), _ptr(xq), _ptr(xs), _stream(stream)),
+           "cr_rotate_quant_act")
+    return xq, xs
+
+
+def cr_w4a8_decode_int8(qdata, srel, codebook, w8=None, stream=None):
+    """Packed codes -> the int8 grid w8 [N, K]."""
+    torch = _torch()
+    _need(qdata, "qdata", (torch.uint8, torch.int8), 2)
+    N, K = qdata.shape[0], qdata.shape[1] * 2
+    _need(srel, "srel", (torch.uint8, torch.float8_e4m3fn), shape=(N, K // 16))
+    _need(codebook, "codebook", (torch.float32,), shape=(16,))
+    if w8 is None:
+        w8 = torch.empty(N, K, dtype=torch.int8, device=qdata.device)
+    _need(w8, "w8", (torch.int8,), shape=(N, K))
+    _check(lib().cr_w4a8_decode_int8(_ptr(qdata), _ptr(srel), _ptr(codebook), N, K, _ptr(w8), _stream(stream)),
+           "cr_w4a8_decode_int8")
+    return w8
+
+
+def _contraction(fn_name, xq, xs, qdata, srel, codebook, s_channel, bias, m, out_dtype, out, acc_out, stream):
+    torch = _torch()
+    N, K = _layer(qdata, srel, codebook, s_channel, bias)
+    _need(xq, "xq", (torch.int8,), 2)
+    _need(xs, "xs", (torch.float32,), 1)
+    M = xq.shape[0] if m is None else int(m)
+    if xq.shape[1] != K or xq.shape[0] < M or xs.shape[0] < M:
+        raise ValueError(f"xq {tuple(xq.shape)} / xs {tuple(xs.shape)} do not match M={M}, K={K}")
+    code = _out_code(out_dtype if out is None else out.dtype)
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=xq.device)
+    _need(out, "out", (torch.bfloat16, torch.float32), shape=(M, N))
+    if acc_out is True:
+        acc_out = torch.empty(M, N, dtype=torch.int32, device=xq.device)
+    if acc_out is not None and acc_out is not False:
+        _need(acc_out, "acc_out", (torch.int32,), shape=(M, N))
+    else:
+        acc_out = None
+    fn = getattr(lib(), fn_name)
+    _check(fn(_ptr(xq), _ptr(xs), _ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), _ptr(bias),
+              M, N, K, code, _ptr(out), _ptr(acc_out), _stream(stream)), fn_name)
+    return (out, acc_out) if acc_out is not None else out
+
+
+def cr_w4a8_gemm(xq, xs, qdata, srel, codebook, s_channel, bias=None, m: Optional[int] = None,
+                 out_dtype=None, out=None, acc_out=None, stream=None):
+    """Prefill forward on quantised activations.  acc_out=True also returns the
+    int32 accumulators (out, acc)."""
+    torch = _torch()
+    return _contraction("cr_w4a8_gemm", xq, xs, qdata, srel, codebook, s_channel, bias, m,
+                        out_dtype or torch.bfloat16, out, acc_out, stream)
+
+
+def cr_w4a8_gemv(xq, xs, qdata, srel, codebook, s_channel, bias=None, m: Optional[int] = None,
+                 out_dtype=None, out=None, acc_out=None, stream=None):
+    """Decode forward (M <= 8) on quantised activations; bitwise equal to cr_w4a8_gemm."""
+    torch = _torch()
+    return _contraction("cr_w4a8_gemv", xq, xs, qdata, srel, codebook, s_channel, bias, m,
+                        out_dtype or torch.bfloat16, out, acc_out, stream)
+
+
+def cr_epilogue(acc, xs, s_channel, bias=None, out_dtype=None, out=None, stream=None):
+    torch = _torch()
+    _need(acc, "acc", (torch.int32,), 2)
+    M, N = acc.shape
+    _need(xs, "xs", (torch.float32,), 1)
+    _need(s_channel, "s_channel", (torch.float32,), shape=(N,))
+    if bias is not None:
+        _need(bias, "bias", (torch.float32,), shape=(N,))
+    out_dtype = out_dtype or torch.bfloat16
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=acc.device)
+    _need(out, "out", (torch.bfloat16, torch.float32), shape=(M, N))
+    if xs.shape[0] < M:
+        raise ValueError("xs has fewer than M rows")
+    _check(lib().cr_epilogue(_ptr(acc), _ptr(xs), _ptr(s_channel), _ptr(bias), M, N, _out_code(out.dtype),
+                             _ptr(out), _stream(stream)), "cr_epilogue")
+    return out
+
+
+def cr_w4a8_linear(x, qdata, srel, codebook, s_channel, bias=None, act_qmax: int = 127, out_dtype=None,
+                   out=None, xq_work=None, xs_work=None, stream=None):
+    """The whole layer forward: rotate + quantise x, then the decode GEMV when
+    M <= 8, else the prefill GEMM."""
+    torch = _torch()
+    _need(x, "x", (torch.bfloat16,), 2)
+    M, K = x.shape
+    N, Kw = _layer(qdata, srel, codebook, s_channel, bias)
+    if Kw != K:
+        raise ValueError(f"x has K={K}, the layer K={Kw}")
+    rows = gemv_rows(M) if 1 <= M <= CR_GEMV_MAX_M else M
+    if xq_work is None:
+        xq_work = torch.empty(rows, K, dtype=torch.int8, device=x.device)
+    if xs_work is None:
+        xs_work = torch.empty(rows, dtype=torch.float32, device=x.device)
+    if xq_work.shape[0] < rows or xs_work.shape[0] < rows:
+        raise ValueError(f"work buffers need {rows} rows")
+    _need(xq_work, "xq_work", (torch.int8,), 2)
+    _need(xs_work, "xs_work", (torch.float32,), 1)
+    out_dtype = out_dtype or torch.bfloat16
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=x.device)
+    _need(out, "out", (torch.bfloat16, torch.float32), shape=(M, N))
+    _check(lib().cr_w4a8_linear(_ptr(x), _ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), _ptr(bias),
+                                M, N, K, int(act_qmax), _out_code(out.dtype), _ptr(out), _ptr(xq_work),
+                                _ptr(xs_work), _stream(stream)), "cr_w4a8_linear")
+    return out
+
+
+def cr_check_device_error(stream=None) -> None:
+    """Synchronise the stream and raise CrError if a kernel's bounded wait ran out."""
+    _check(lib().cr_check_device_error(_stream(stream)), "cr_check_device_error")

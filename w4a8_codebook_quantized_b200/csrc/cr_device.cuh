@@ -1,0 +1,348 @@
+// cr_device.cuh -- device helpers shared by the sm_100a kernels of the ConvRot
+// W4A8 codebook linear layer: fp8 scale decode, the per-CTA int8-grid lookup
+// table, nibble decode by byte permutes, the epilogue, the library error word,
+// and thin PTX wrappers for mbarriers, TMA, tcgen05 and TMEM.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "cr_w4a8.h"
+
+namespace cr {
+
+// Set by a kernel whose bounded pipeline wait ran out; read and cleared by
+// cr_check_device_error().  One per device (module-scope __device__ variable;
+// the library is a single translation unit, so it is defined here).
+__device__ int g_device_error = 0;
+
+enum : int { kErrTimeout = 1 };
+
+// ---------------------------------------------------------------- fp8 scales
+
+// fp8 e4m3fn byte -> fp32, exact.  Format (ai-toolkit convrot_w4a8_quant.py,
+// w4a8_gemv_kernel: the s_rel byte is read as float8e4nv): sign, 4 exponent
+// bits with bias 7, 3 mantissa bits, no infinities, S.1111.111 is NaN.
+// Normal values are rebuilt as fp32 bit fields (exponent e - 7 + 127 = e + 120,
+// mantissa in the top three fraction bits); subnormals are m * 2^-9.
+__device__ __forceinline__ float fp8e4m3fn_to_float(uint32_t b)
+{
+    const uint32_t sign = (b & 0x80u) << 24;
+    const uint32_t e = (b >> 3) & 0xFu;
+    const uint32_t m = b & 0x7u;
+    if (e == 0xFu && m == 0x7u)
+        return __uint_as_float(0x7FC00000u | sign);
+    float mag = (e == 0u) ? __fmul_rn((float)m, 0.001953125f)
+                          : __uint_as_float(((e + 120u) << 23) | (m << 20));
+    return __uint_as_float(__float_as_uint(mag) | sign);
+}
+
+// Round to nearest even and saturate to [-128, 127] in one conversion; NaN -> 0
+// (ai-toolkit convrot_w4a8_quant.py, _sat_s8 / W4A8_SAT).
+__device__ __forceinline__ int32_t sat_s8_rne(float v)
+{
+    int32_t r;
+    asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(r) : "f"(v));
+    return r;
+}
+
+// ---------------------------------------------------------------- int8-grid LUT
+//
+// The decoded weight depends only on (scale byte, code): w8 = sat_s8(rne(cb[code]
+// * fp8(s))).  A CTA tabulates all 256 x 16 values once; entry s is one uint4
+// whose 16 bytes are the levels of codes 0..15 (x: codes 0-3, y: 4-7, z: 8-11,
+// w: 12-15).
+__device__ __forceinline__ uint4 lut_entry(uint32_t s, const float *cb /* 16, any memory */)
+{
+    const float sv = fp8e4m3fn_to_float(s);
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int32_t l = sat_s8_rne(__fmul_rn(cb[4 * q + j], sv));
+            word |= ((uint32_t)l & 0xFFu) << (8 * j);
+        }
+        w[q] = word;
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// PTX prmt in its default mode: selector nibble i = {sign-replicate bit, 3-bit
+// source byte index} for output byte i; source bytes 0-3 from a, 4-7 from b.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
+{
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Decode 8 packed codes (one 32-bit word: nibble i = code of column base + i,
+// which is the storage order: even column in the low nibble) through the level
+// table T of their group.  Returns the int8 grid values of columns 0-3 in w0
+// and 4-7 in w1 (byte i of w0 = column i).
+//
+// Byte permutes do the table lookup: the low three bits of each code select
+// among levels 0-7 (T.x:T.y) and among levels 8-15 (T.z:T.w); bit 3 picks one
+// of the two.  The bit-3 byte mask comes from prmt's sign-replicate mode
+// applied to the code word and the code word shifted left by 4, whose bytes
+// carry code bit 3 in their sign bit.
+__device__ __forceinline__ void decode8(uint32_t c, const uint4 &T, uint32_t &w0, uint32_t &w1)
+{
+    const uint32_t s7 = c & 0x77777777u;
+    const uint32_t s7h = s7 >> 16;
+    const uint32_t lo0 = prmt(T.x, T.y, s7);
+    const uint32_t hi0 = prmt(T.z, T.w, s7);
+    const uint32_t lo1 = prmt(T.x, T.y, s7h);
+    const uint32_t hi1 = prmt(T.z, T.w, s7h);
+    const uint32_t c4 = c << 4;
+    // output byte i <- sign of: (c4 byte 0), (c byte 0), (c4 byte 1), (c byte 1)
+    const uint32_t m0 = prmt(c4, c, 0xD9C8u);
+    // ... and for codes 4-7: (c4 byte 2), (c byte 2), (c4 byte 3), (c byte 3)
+    const uint32_t m1 = prmt(c4, c, 0xFBEAu);
+    w0 = (hi0 & m0) | (lo0 & ~m0);
+    w1 = (hi1 & m1) | (lo1 & ~m1);
+}
+
+// ---------------------------------------------------------------- epilogue
+//
+// ai-toolkit convrot_w4a8_quant.py, w4a8_gemv_kernel epilogue:
+// float(acc) * (xs * ws) [+ bias], each operation rounded on its own.
+__device__ __forceinline__ float epilogue_value(int32_t acc, float xs, float ws, const float *bias,
+                                                int64_t n)
+{
+    float y = __fmul_rn(__int2float_rn(acc), __fmul_rn(xs, ws));
+    if (bias != nullptr)
+        y = __fadd_rn(y, bias[n]);
+    return y;
+}
+
+__device__ __forceinline__ uint16_t to_bf16_bits(float y)
+{
+    return __bfloat16_as_ushort(__float2bfloat16_rn(y));
+}
+
+// ---------------------------------------------------------------- loads
+
+// 16-byte streaming load that bypasses L1 (weights are read once).
+__device__ __forceinline__ uint4 ldg_stream16(const void *p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------- mbarrier
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Bounded wait for the phase with the given parity to complete.  Gives up
+// after `limit_ns` of wall time, or as soon as *abort is set by another warp
+// of the CTA; on giving up it sets *abort and the device error word and
+// returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                  uint64_t limit_ns = 2000000000ull)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((it & 63u) == 0u) {
+            if (*abort)
+                return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                *abort = 1;
+                atomicExch(&g_device_error, kErrTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+// The same bounded wait, taken by a whole warp: every lane polls, and the
+// outcome is the same in all lanes (warp-collective instructions follow it).
+__device__ __forceinline__ bool mbar_wait_bounded_warp(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                                       uint64_t limit_ns = 2000000000ull)
+{
+    if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity)))
+        return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (__all_sync(0xFFFFFFFFu, mbar_try_wait(bar, parity)))
+            return true;
+        if ((it & 63u) == 0u) {
+            int give_up = 0;
+            if ((threadIdx.x & 31) == 0) {
+                if (*abort) {
+                    give_up = 1;
+                } else if (globaltimer_ns() - t0 > limit_ns) {
+                    *abort = 1;
+                    atomicExch(&g_device_error, kErrTimeout);
+                    give_up = 1;
+                }
+            }
+            if (__shfl_sync(0xFFFFFFFFu, give_up, 0))
+                return false;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- TMA
+
+__device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, int32_t x, int32_t y, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const void *tmap)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
+}
+
+// ---------------------------------------------------------------- tcgen05 / TMEM
+
+__device__ __forceinline__ void tmem_alloc(uint32_t *smem_result, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(smem_result)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Arrive on an mbarrier once every tcgen05 operation this thread issued so far
+// has completed.
+__device__ __forceinline__ void tc_commit(uint64_t *bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+// D[tmem] (+)= A[smem] x B[smem]^T, int8 x int8 -> int32.
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 consecutive 32-bit TMEM columns of this warp's 32 lanes -> 32 registers.
+__device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait()
+{
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major operand tile stored in the
+// 128-byte-swizzled canonical layout: rows of 128 bytes, 8-row atoms of 1024
+// bytes stacked along the row dimension (stride-dimension byte offset 1024).
+// Fields: start address >> 4 in bits 0-13, leading byte offset >> 4 in 16-29
+// (unused for swizzled K-major tiles; set to 1), stride byte offset >> 4 in
+// 32-45, descriptor version 1 in bits 46-47, swizzle mode 2 (128 B) in 61-63.
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;
+    d |= (uint64_t)(1024u >> 4) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)2u << 61;
+    return d;
+}
+
+// Instruction descriptor for kind::i8: s32 accumulator, signed A and B, both
+// K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N)
+{
+    return (2u << 4)                        // D format: s32
+           | (1u << 7)                      // A: signed 8-bit
+           | (1u << 10)                     // B: signed 8-bit
+           | ((uint32_t)(N >> 3) << 17)     // N / 8
+           | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
+}  // namespace cr

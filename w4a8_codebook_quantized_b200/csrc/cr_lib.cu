@@ -1,0 +1,358 @@
+// cr_lib.cu -- the C ABI of the ConvRot W4A8 codebook linear forward
+// (include/cr_w4a8.h): argument validation, per-device state, TMA
+// descriptors, and the launches of the sm_100a kernels.
+//
+// Built as one translation unit (the kernels are header files) into
+// libcr_w4a8.so with nvcc -gencode arch=compute_100a,code=sm_100a.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstdint>
+#include <mutex>
+
+#include "cr_w4a8.h"
+#include "cr_device.cuh"
+#include "k_elementwise.cuh"
+#include "k_gemm.cuh"
+#include "k_gemv.cuh"
+#include "k_rotquant.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool probed = false;
+    bool usable = false;
+    int num_sms = 0;
+    cudaMemPool_t pool = nullptr;  // stream-ordered pool for the prefill weight transient
+    bool gemm_attr_set = false;
+};
+
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mutex;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode_tiled = nullptr;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cr_status check_k(int64_t K)
+{
+    if (K <= 0 || K % CR_ROT != 0 || K > CR_MAX_K)
+        return CR_ERR_UNSUPPORTED;
+    return CR_OK;
+}
+
+// The current device's state, probing it once.  Fails with CR_ERR_NO_DEVICE
+// when there is no usable sm_100 device.
+cr_status current_device(DeviceState **out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return CR_ERR_NO_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceState &d = g_dev[dev];
+    if (!d.probed) {
+        d.probed = true;
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return CR_ERR_NO_DEVICE;
+        }
+        d.usable = (major == 10 && minor == 0);
+        d.num_sms = sms;
+        if (d.usable) {
+            cudaMemPoolProps props = {};
+            props.allocType = cudaMemAllocationTypePinned;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            if (cudaMemPoolCreate(&d.pool, &props) != cudaSuccess) {
+                cudaGetLastError();
+                d.usable = false;
+            } else {
+                uint64_t keep = UINT64_MAX;
+                cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
+            }
+        }
+        if (d.usable && g_encode_tiled == nullptr) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr) {
+                cudaGetLastError();
+                d.usable = false;
+            } else {
+                g_encode_tiled = reinterpret_cast<EncodeTiledFn>(fn);
+            }
+        }
+    }
+    if (!d.usable)
+        return CR_ERR_NO_DEVICE;
+    *out = &d;
+    return CR_OK;
+}
+
+cr_status launched(cudaError_t e)
+{
+    if (e != cudaSuccess)
+        return CR_ERR_CUDA;
+    return CR_OK;
+}
+
+// 2-D int8 tensor map over a row-major [rows, inner] matrix, box
+// [box_rows, 128 bytes], 128-byte swizzle; out-of-range rows read as zero.
+bool make_tmap_i8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows, uint32_t box_rows)
+{
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner};
+    const cuuint32_t box[2] = {128u, box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
+                                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Shared validation of the contraction entry points.
+cr_status check_contraction(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                            const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N,
+                            int64_t K, cr_out_dtype out_dtype, void *out, int32_t *acc_out)
+{
+    if (M < 0 || N < 0 || K < 0)
+        return CR_ERR_INVALID_ARG;
+    if (out_dtype != CR_OUT_BF16 && out_dtype != CR_OUT_F32)
+        return CR_ERR_INVALID_ARG;
+    const cr_status k = check_k(K);
+    if (k != CR_OK)
+        return k;
+    if (M > INT_MAX || N > INT_MAX)
+        return CR_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0)
+        return CR_OK;
+    if (!xq || !xs || !qdata || !srel || !codebook || !s_channel || !out)
+        return CR_ERR_INVALID_ARG;
+    if (!aligned16(xq) || !aligned16(xs) || !aligned16(qdata) || !aligned16(srel) || !aligned16(codebook) ||
+        !aligned16(s_channel) || !aligned16(out) || (bias && !aligned16(bias)) || (acc_out && !aligned16(acc_out)))
+        return CR_ERR_ALIGNMENT;
+    return CR_OK;
+}
+
+cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                   const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K,
+                   cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream)
+{
+    using namespace cr;
+    if (!d.gemm_attr_set) {
+        if (cudaFuncSetAttribute(gm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gm::kSmemBytes) != cudaSuccess) {
+            cudaGetLastError();
+            return CR_ERR_CUDA;
+        }
+        d.gemm_attr_set = true;
+    }
+    // The int8 grid of the weight, decoded once per call into a transient
+    // from the library's stream-ordered pool.
+    int8_t *w8 = nullptr;
+    if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&w8), (size_t)(N * K), d.pool, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return CR_ERR_CUDA;
+    }
+    cr_status st = launched(ew::launch_decode(qdata, srel, codebook, N, K, w8, d.num_sms, stream));
+    CUtensorMap ta, tb;
+    if (st == CR_OK && (!make_tmap_i8(&ta, xq, (uint64_t)K, (uint64_t)M, (uint32_t)gm::BM) ||
+                        !make_tmap_i8(&tb, w8, (uint64_t)K, (uint64_t)N, (uint32_t)gm::BN)))
+        st = CR_ERR_CUDA;
+    if (st == CR_OK) {
+        const int64_t tiles = ((M + gm::BM - 1) / gm::BM) * ((N + gm::BN - 1) / gm::BN);
+        const int grid = (int)(tiles < d.num_sms ? tiles : d.num_sms);
+        const int out_f32 = out_dtype == CR_OUT_F32;
+        const int vec_ok = out_f32 ? (N % 4 == 0) : (N % 8 == 0);
+        gm::gemm_kernel<<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(ta, tb, xs, s_channel, bias, (int)M, (int)N,
+                                                                         (int)K, out_f32, vec_ok, out, acc_out);
+        st = launched(cudaGetLastError());
+    }
+    if (cudaFreeAsync(w8, stream) != cudaSuccess) {
+        cudaGetLastError();
+        if (st == CR_OK)
+            st = CR_ERR_CUDA;
+    }
+    return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *cr_status_string(cr_status s)
+{
+    switch (s) {
+    case CR_OK: return "ok";
+    case CR_ERR_INVALID_ARG: return "invalid argument";
+    case CR_ERR_UNSUPPORTED: return "unsupported shape";
+    case CR_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case CR_ERR_CUDA: return "CUDA runtime or launch failure";
+    case CR_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case CR_ERR_NO_DEVICE: return "no usable sm_100 device";
+    }
+    return "unknown status";
+}
+
+const char *cr_version(void) { return "0.1.0"; }
+
+cr_status cr_rotate_quant_act(const uint16_t *x, int64_t M, int64_t K, int64_t MP, int act_qmax, int8_t *xq, float *xs,
+                              cr_stream_t stream)
+{
+    if (M < 0 || K < 0 || MP < M || act_qmax < 1 || act_qmax > 127)
+        return CR_ERR_INVALID_ARG;
+    const cr_status k = check_k(K);
+    if (k != CR_OK)
+        return k;
+    if (MP > INT_MAX)
+        return CR_ERR_UNSUPPORTED;
+    if (MP == 0)
+        return CR_OK;
+    if ((M > 0 && !x) || !xq || !xs)
+        return CR_ERR_INVALID_ARG;
+    if ((x && !aligned16(x)) || !aligned16(xq) || !aligned16(xs))
+        return CR_ERR_ALIGNMENT;
+    DeviceState *d = nullptr;
+    const cr_status ds = current_device(&d);
+    if (ds != CR_OK)
+        return ds;
+    return launched(cr::rq::launch(x, M, K, MP, act_qmax, xq, xs, stream));
+}
+
+cr_status cr_w4a8_decode_int8(const uint8_t *qdata, const uint8_t *srel, const float *codebook, int64_t N, int64_t K,
+                              int8_t *w8, cr_stream_t stream)
+{
+    if (N < 0 || K < 0)
+        return CR_ERR_INVALID_ARG;
+    const cr_status k = check_k(K);
+    if (k != CR_OK)
+        return k;
+    if (N == 0)
+        return CR_OK;
+    if (!qdata || !srel || !codebook || !w8)
+        return CR_ERR_INVALID_ARG;
+    if (!aligned16(qdata) || !aligned16(srel) || !aligned16(codebook) || !aligned16(w8))
+        return CR_ERR_ALIGNMENT;
+    DeviceState *d = nullptr;
+    const cr_status ds = current_device(&d);
+    if (ds != CR_OK)
+        return ds;
+    return launched(cr::ew::launch_decode(qdata, srel, codebook, N, K, w8, d->num_sms, stream));
+}
+
+cr_status cr_w4a8_gemm(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                       const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N,
+                       int64_t K, cr_out_dtype out_dtype, void *out, int32_t *acc_out, cr_stream_t stream)
+{
+    cr_status st = check_contraction(xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, acc_out);
+    if (st != CR_OK || M == 0 || N == 0)
+        return st;
+    DeviceState *d = nullptr;
+    st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    return run_gemm(*d, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, acc_out, stream);
+}
+
+cr_status cr_w4a8_gemv(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                       const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N,
+                       int64_t K, cr_out_dtype out_dtype, void *out, int32_t *acc_out, cr_stream_t stream)
+{
+    if (M > CR_GEMV_MAX_M)
+        return CR_ERR_UNSUPPORTED;
+    cr_status st = check_contraction(xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, acc_out);
+    if (st != CR_OK || M == 0 || N == 0)
+        return st;
+    DeviceState *d = nullptr;
+    st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    return launched(cr::gv::launch(xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K,
+                                   out_dtype == CR_OUT_F32, out, acc_out, stream));
+}
+
+cr_status cr_epilogue(const int32_t *acc, const float *xs, const float *s_channel, const float *bias, int64_t M,
+                      int64_t N, cr_out_dtype out_dtype, void *out, cr_stream_t stream)
+{
+    if (M < 0 || N < 0 || (out_dtype != CR_OUT_BF16 && out_dtype != CR_OUT_F32))
+        return CR_ERR_INVALID_ARG;
+    if (M == 0 || N == 0)
+        return CR_OK;
+    if (!acc || !xs || !s_channel || !out)
+        return CR_ERR_INVALID_ARG;
+    if (!aligned16(acc) || !aligned16(xs) || !aligned16(s_channel) || !aligned16(out) || (bias && !aligned16(bias)))
+        return CR_ERR_ALIGNMENT;
+    DeviceState *d = nullptr;
+    const cr_status ds = current_device(&d);
+    if (ds != CR_OK)
+        return ds;
+    return launched(cr::ew::launch_epilogue(acc, xs, s_channel, bias, M, N, out_dtype == CR_OUT_F32, out, d->num_sms,
+                                            stream));
+}
+
+cr_status cr_w4a8_linear(const uint16_t *x, const uint8_t *qdata, const uint8_t *srel, const float *codebook,
+                         const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K, int act_qmax,
+                         cr_out_dtype out_dtype, void *out, int8_t *xq_work, float *xs_work, cr_stream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0 || act_qmax < 1 || act_qmax > 127)
+        return CR_ERR_INVALID_ARG;
+    int64_t MP = M;
+    if (M >= 1 && M <= CR_GEMV_MAX_M) {
+        MP = 1;
+        while (MP < M)
+            MP <<= 1;
+    }
+    cr_status st = check_contraction(xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype,
+                                      out, nullptr);
+    if (st != CR_OK || M == 0 || N == 0)
+        return st;
+    if (!x)
+        return CR_ERR_INVALID_ARG;
+    if (!aligned16(x))
+        return CR_ERR_ALIGNMENT;
+    DeviceState *d = nullptr;
+    st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    st = launched(cr::rq::launch(x, M, K, MP, act_qmax, xq_work, xs_work, stream));
+    if (st != CR_OK)
+        return st;
+    if (M <= CR_GEMV_MAX_M)
+        return launched(cr::gv::launch(xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K,
+                                       out_dtype == CR_OUT_F32, out, nullptr, stream));
+    return run_gemm(*d, xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, nullptr,
+                    stream);
+}
+
+cr_status cr_check_device_error(cr_stream_t stream)
+{
+    DeviceState *d = nullptr;
+    const cr_status ds = current_device(&d);
+    if (ds != CR_OK)
+        return ds;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) {
+        cudaGetLastError();
+        return CR_ERR_CUDA;
+    }
+    int v = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&v, cr::g_device_error, sizeof(int)) != cudaSuccess ||
+        cudaMemcpyToSymbol(cr::g_device_error, &zero, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return CR_ERR_CUDA;
+    }
+    return v ? CR_ERR_TIMEOUT : CR_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,124 @@
+// k_elementwise.cuh -- the two bandwidth-bound stand-alone kernels: decode of
+// the packed codes onto the int8 grid, and the epilogue on an int32
+// accumulator.
+#pragma once
+
+#include "cr_device.cuh"
+
+namespace cr {
+namespace ew {
+
+constexpr int kThreads = 256;
+
+// ai-toolkit convrot_w4a8_quant.py, unpack_w4a8_eager / w4a8_unpack_kernel:
+// w8[n, k] = sat_s8(rne(codebook[code] * fp8(srel[n, k/16]))).
+//
+// One thread decodes one 16-byte chunk of packed codes (32 weights, two
+// groups): a streaming 16-byte load, the two group scale bytes, two lookups in
+// the CTA's level table, four byte-permute decodes and two 16-byte stores.
+// HBM traffic per weight: 0.5 + 1/16 bytes in, 1 byte out.
+__global__ void __launch_bounds__(kThreads) decode_int8_kernel(const uint8_t *__restrict__ qdata,
+                                                               const uint8_t *__restrict__ srel,
+                                                               const float *__restrict__ codebook, int64_t N,
+                                                               int64_t K, int8_t *__restrict__ w8)
+{
+    __shared__ uint4 lut[256];
+    __shared__ float cb[16];
+    if (threadIdx.x < 16)
+        cb[threadIdx.x] = codebook[threadIdx.x];
+    __syncthreads();
+    for (int s = threadIdx.x; s < 256; s += kThreads)
+        lut[s] = lut_entry((uint32_t)s, cb);
+    __syncthreads();
+
+    const int64_t chunks_per_row = K / 32;
+    const int64_t total = N * chunks_per_row;
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < total; i += stride) {
+        const int64_t n = i / chunks_per_row;
+        const int64_t j = i - n * chunks_per_row;
+        const uint4 c = ldg_stream16(qdata + n * (K / 2) + 16 * j);
+        const uint32_t sb = __ldg(reinterpret_cast<const uint16_t *>(srel + n * (K / 16) + 2 * j));
+        const uint4 T0 = lut[sb & 0xFFu];
+        const uint4 T1 = lut[sb >> 8];
+        uint4 o0, o1;
+        decode8(c.x, T0, o0.x, o0.y);
+        decode8(c.y, T0, o0.z, o0.w);
+        decode8(c.z, T1, o1.x, o1.y);
+        decode8(c.w, T1, o1.z, o1.w);
+        uint4 *dst = reinterpret_cast<uint4 *>(w8 + n * K + 32 * j);
+        dst[0] = o0;
+        dst[1] = o1;
+    }
+}
+
+inline cudaError_t launch_decode(const uint8_t *qdata, const uint8_t *srel, const float *codebook, int64_t N,
+                                 int64_t K, int8_t *w8, int num_sms, cudaStream_t stream)
+{
+    const int64_t total = N * (K / 32);
+    int64_t blocks = (total + kThreads - 1) / kThreads;
+    const int64_t cap = (int64_t)num_sms * 8;
+    if (blocks > cap)
+        blocks = cap;
+    decode_int8_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(qdata, srel, codebook, N, K, w8);
+    return cudaGetLastError();
+}
+
+// ai-toolkit convrot_w4a8_quant.py, w4a8_gemv_kernel epilogue, on a stored
+// int32 accumulator.  Four outputs per thread along a row when N % 4 == 0
+// (16-byte accumulator loads), one otherwise.
+__global__ void __launch_bounds__(kThreads) epilogue_kernel(const int32_t *__restrict__ acc,
+                                                            const float *__restrict__ xs,
+                                                            const float *__restrict__ ws,
+                                                            const float *__restrict__ bias, int64_t M, int64_t N,
+                                                            int out_f32, void *__restrict__ out)
+{
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    if ((N & 3) == 0) {
+        const int64_t total = M * N / 4;
+        for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < total; i += stride) {
+            const int64_t e = 4 * i;
+            const int64_t m = e / N, n = e - m * N;
+            const int4 a = __ldg(reinterpret_cast<const int4 *>(acc) + i);
+            const float xm = xs[m];
+            const float y0 = epilogue_value(a.x, xm, ws[n], bias, n);
+            const float y1 = epilogue_value(a.y, xm, ws[n + 1], bias, n + 1);
+            const float y2 = epilogue_value(a.z, xm, ws[n + 2], bias, n + 2);
+            const float y3 = epilogue_value(a.w, xm, ws[n + 3], bias, n + 3);
+            if (out_f32) {
+                reinterpret_cast<float4 *>(out)[i] = make_float4(y0, y1, y2, y3);
+            } else {
+                const uint32_t lo = (uint32_t)to_bf16_bits(y0) | ((uint32_t)to_bf16_bits(y1) << 16);
+                const uint32_t hi = (uint32_t)to_bf16_bits(y2) | ((uint32_t)to_bf16_bits(y3) << 16);
+                reinterpret_cast<uint2 *>(out)[i] = make_uint2(lo, hi);
+            }
+        }
+    } else {
+        const int64_t total = M * N;
+        for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < total; e += stride) {
+            const int64_t m = e / N, n = e - m * N;
+            const float y = epilogue_value(acc[e], xs[m], ws[n], bias, n);
+            if (out_f32)
+                reinterpret_cast<float *>(out)[e] = y;
+            else
+                reinterpret_cast<uint16_t *>(out)[e] = to_bf16_bits(y);
+        }
+    }
+}
+
+inline cudaError_t launch_epilogue(const int32_t *acc, const float *xs, const float *ws, const float *bias,
+                                   int64_t M, int64_t N, int out_f32, void *out, int num_sms, cudaStream_t stream)
+{
+    const int64_t work = ((N & 3) == 0) ? M * N / 4 : M * N;
+    int64_t blocks = (work + kThreads - 1) / kThreads;
+    const int64_t cap = (int64_t)num_sms * 8;
+    if (blocks > cap)
+        blocks = cap;
+    if (blocks < 1)
+        blocks = 1;
+    epilogue_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(acc, xs, ws, bias, M, N, out_f32, out);
+    return cudaGetLastError();
+}
+
+}  // namespace ew
+}  // namespace cr

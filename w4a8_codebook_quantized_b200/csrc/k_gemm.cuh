@@ -1,0 +1,262 @@
+// k_gemm.cuh -- prefill contraction on the 5th-generation tensor cores.
+//
+// What it computes (ai-toolkit convrot_w4a8_quant.py, _w4a8_linear_ste_op:
+// torch._int_mm(aq, w8.t()) followed by the epilogue):
+//   acc[m, n] = sum_k A[m, k] * B[n, k]   A = xq [M, K] int8, B = w8 [N, K] int8
+//   out[m, n] = float(acc) * (xs[m] * ws[n]) [+ bias[n]]
+//
+// B200 design: a persistent, warp-specialised kernel, one CTA per SM.
+//   warp 0      one thread issues TMA loads of 128-wide K slices of the A tile
+//               (128 rows) and the B tile (256 rows) into a 4-stage ring of
+//               128-byte-swizzled shared-memory buffers (48 KB per stage);
+//   warp 1      allocates 512 TMEM columns (two 128 x 256 int32 accumulators)
+//               and one thread issues tcgen05.mma kind::i8 (M 128, N 256, K 32,
+//               four per stage), releasing each stage with tcgen05.commit;
+//   warps 2-5   the epilogue: tcgen05.ld of 32 columns at a time, the
+//               per-token x per-channel fp32 rescale (+ bias), bf16 or fp32
+//               stores, then the TMEM buffer is handed back to the MMA warp,
+//               so the epilogue of tile i overlaps the MMAs of tile i + 1.
+// Every wait is bounded (a second or two); a wait that runs out sets the
+// library error word, every role stops, TMEM is freed and the kernel returns.
+// TMA zero-fills rows past M or N, so ragged edges need no special casing
+// except in the epilogue's stores.
+#pragma once
+
+#include <cuda.h>
+
+#include "cr_device.cuh"
+
+namespace cr {
+namespace gm {
+
+constexpr int BM = 128, BN = 256, BK = 128;  // BK in int8 elements = bytes
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK;              // 16 KB
+constexpr int kBBytes = BN * BK;              // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kTmemCols = 2 * BN;             // two accumulators
+constexpr int kThreads = 192;
+constexpr uint32_t kIdesc = idesc_i8(BM, BN);
+
+struct __align__(1024) Smem {
+    uint8_t stage[kStages][kStageBytes];  // A at +0, B at +kABytes; every buffer 1024-aligned
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t tmem_full[2];
+    uint64_t tmem_empty[2];
+    uint32_t tmem_base;
+    int abort;
+};
+
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + slack to align the base
+
+__device__ __forceinline__ void tile_coords(int tile, int tiles_n, int &tm, int &tn)
+{
+    tm = tile / tiles_n;
+    tn = tile - tm * tiles_n;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const float *__restrict__ xs, const float *__restrict__ ws, const float *__restrict__ bias, int M,
+                int N, int K, int out_f32, int vec_ok, void *__restrict__ out, int32_t *__restrict__ acc_out)
+{
+    extern __shared__ uint8_t smem_raw[];
+    Smem &sh = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles_m = (M + BM - 1) / BM, tiles_n = (N + BN - 1) / BN;
+    const int num_tiles = tiles_m * tiles_n;
+    const int kblocks = K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sh.tmem_full[b], 1);
+            mbar_init(&sh.tmem_empty[b], 4);
+        }
+        sh.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        tmem_alloc(&sh.tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+    volatile int *abort = &sh.abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&tmA);
+            prefetch_tmap(&tmB);
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued[kStages];
+            uint32_t issued_phase[kStages];
+            for (int s = 0; s < kStages; ++s)
+                issued[s] = 0, issued_phase[s] = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+                int tm, tn;
+                tile_coords(tile, tiles_n, tm, tn);
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sh.full[stage], kStageBytes);
+                    tma_load_2d(sh.stage[stage], &tmA, kb * BK, tm * BM, &sh.full[stage]);
+                    tma_load_2d(sh.stage[stage] + kABytes, &tmB, kb * BK, tn * BN, &sh.full[stage]);
+                    issued[stage] = 1;
+                    issued_phase[stage] = phase;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // Let copies already in flight land before the CTA goes away.
+                for (int s = 0; s < kStages; ++s)
+                    if (issued[s]) {
+                        volatile int no_abort = 0;
+                        mbar_wait_bounded(&sh.full[s], issued_phase[s], &no_abort, 20000000ull);
+                    }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int local = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++local) {
+                const int buf = local & 1;
+                const uint32_t use = (uint32_t)(local >> 1) & 1u;
+                if (!mbar_wait_bounded(&sh.tmem_empty[buf], use ^ 1u, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(buf * BN);
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait_bounded(&sh.full[stage], phase, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(sh.stage[stage]);
+                    const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 32; ++kk) {
+                        const uint64_t ad = sw128_kmajor_desc(a_addr + 32u * kk);
+                        const uint64_t bd = sw128_kmajor_desc(b_addr + 32u * kk);
+                        mma_i8(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(&sh.empty[stage]);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok)
+                    tc_commit(&sh.tmem_full[buf]);
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5)
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        int local = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
+            int tm, tn;
+            tile_coords(tile, tiles_n, tm, tn);
+            const int buf = local & 1;
+            const uint32_t use = (uint32_t)(local >> 1) & 1u;
+            if (!mbar_wait_bounded_warp(&sh.tmem_full[buf], use, abort))
+                break;
+            tc_fence_after();
+            const int row = tm * BM + 32 * q + lane;
+            const bool row_ok = row < M;
+            const float xm = row_ok ? xs[row] : 0.0f;
+            const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN);
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                uint32_t r[32];
+                __syncwarp();  // the TMEM load below is warp-collective
+                tmem_ld_32cols(tbase + (uint32_t)(32 * ch), r);
+                tmem_ld_wait();
+                const int col0 = tn * BN + 32 * ch;
+                const int64_t base = (int64_t)row * N + col0;
+                if (!row_ok || col0 >= N) {
+                    // nothing of this row/column chunk is in range
+                } else if (vec_ok && col0 + 32 <= N) {
+                    float y[32];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const float4 w4 = __ldg(reinterpret_cast<const float4 *>(ws + col0 + j));
+                        const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            y[j + u] = epilogue_value((int32_t)r[j + u], xm, wv[u], bias, col0 + j + u);
+                    }
+                    if (out_f32) {
+                        float4 *o = reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + base);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            o[j] = make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+                    } else {
+                        uint4 *o = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(out) + base);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint32_t p[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                p[u] = (uint32_t)to_bf16_bits(y[8 * j + 2 * u]) |
+                                       ((uint32_t)to_bf16_bits(y[8 * j + 2 * u + 1]) << 16);
+                            o[j] = make_uint4(p[0], p[1], p[2], p[3]);
+                        }
+                    }
+                    if (acc_out != nullptr) {
+                        uint4 *o = reinterpret_cast<uint4 *>(acc_out + base);
+#pragma unroll
+                        for (int j = 0; j < 8; ++j)
+                            o[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+                    }
+                } else {
+                    for (int j = 0; j < 32 && col0 + j < N; ++j) {
+                        const int n = col0 + j;
+                        const float y = epilogue_value((int32_t)r[j], xm, ws[n], bias, n);
+                        if (out_f32)
+                            reinterpret_cast<float *>(out)[base + j] = y;
+                        else
+                            reinterpret_cast<uint16_t *>(out)[base + j] = to_bf16_bits(y);
+                        if (acc_out != nullptr)
+                            acc_out[base + j] = (int32_t)r[j];
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&sh.tmem_empty[buf]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace gm
+}  // namespace cr

@@ -1,0 +1,213 @@
+// k_rotquant.cuh -- block-256 regular-Hadamard rotation of bf16 activation
+// rows fused with per-token symmetric int8 quantisation.
+//
+// What it computes (ai-toolkit convrot_w4a8_quant.py, prepare_act and
+// w4a8_act_quant_kernel; h3-rs src/weights.rs, hadamard / rotate_activation):
+// each 256-column block of a row is multiplied by H_256 = h4^(x4) / 16, the
+// row's absolute maximum gives the scale amax / qmax, and every value is
+// rounded to nearest even after the division and clamped to +-qmax.  Rows
+// M..MP-1 are the decode GEMV's padding: zeros with scale 1.
+//
+// fp32 order (the pages leave it open; this order is the layer's definition
+// here): the bf16 inputs widen exactly; the four base-4 digits of the index
+// within the block are processed in the order stride 1, 4, 16, 64; one
+// quadruple (v0, v1, v2, v3) along a digit becomes S - 2 v[3-a] with
+// S = (v0 + v1) + (v2 + v3); the result is scaled by 1/16.
+//
+// Layout: one CTA of 256 threads per row.  A half-warp (16 lanes) owns one
+// 256-element block, viewed as a 16 x 16 matrix with element 16a + b: lane L
+// first holds row a = L (16 contiguous bf16, two 16-byte loads), applies the
+// stride-1 and stride-4 digits in registers, transposes through shared memory
+// so that it holds column b = L, applies the stride-16 and stride-64 digits in
+// registers, and keeps the 16 fp32 results in registers until the row's
+// maximum is known.  The quantised bytes go back to row order through a
+// second, byte-wide shared-memory transpose and leave as one 16-byte store per
+// lane.  HBM traffic is the algorithmic minimum: 2 bytes read and 1 written
+// per element.  Rows with K > 4096 * kMaxBlocksInRegs are handled by a
+// second pass that recomputes the rotation instead of holding it.
+#pragma once
+
+#include "cr_device.cuh"
+
+namespace cr {
+namespace rq {
+
+constexpr int kThreads = 256;
+constexpr int kHalfWarps = kThreads / 16;  // blocks of 256 in flight per CTA
+constexpr int kMaxBlocksInRegs = 4;        // per half-warp: K <= 16384 stays in registers
+
+// One digit of the rotation on a quadruple (row a of h4 is all ones except
+// -1 at column 3 - a).  2v is exact, so fma(-2, v, S) is S - 2v rounded once.
+__device__ __forceinline__ void h4_quad(float &a0, float &a1, float &a2, float &a3)
+{
+    const float S = __fadd_rn(__fadd_rn(a0, a1), __fadd_rn(a2, a3));
+    const float y0 = __fmaf_rn(-2.0f, a3, S);
+    const float y1 = __fmaf_rn(-2.0f, a2, S);
+    const float y2 = __fmaf_rn(-2.0f, a1, S);
+    const float y3 = __fmaf_rn(-2.0f, a0, S);
+    a0 = y0;
+    a1 = y1;
+    a2 = y2;
+    a3 = y3;
+}
+
+// Rotate one 256-element block.  On return lane L of the half-warp holds
+// v[a] = rotated element 16a + L (a = 0..15).  `tr` is this half-warp's
+// 16 x 17 fp32 transpose buffer.
+__device__ __forceinline__ void rotate_block(const uint16_t *__restrict__ blk, int L, float *tr, unsigned hmask,
+                                             float (&v)[16])
+{
+    const uint4 *src = reinterpret_cast<const uint4 *>(blk + 16 * L);
+    const uint4 p0 = __ldg(src);
+    const uint4 p1 = __ldg(src + 1);
+    const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);             // element 2i: low half
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);  // element 2i+1: high half
+    }
+    // stride 1 (digit d0 = b % 4), then stride 4 (digit d1 = b / 4)
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        h4_quad(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        h4_quad(v[q], v[q + 4], v[q + 8], v[q + 12]);
+    // transpose: row L out, column L in (row pitch 17 words: conflict-free)
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        tr[L * 17 + i] = v[i];
+    __syncwarp(hmask);
+#pragma unroll
+    for (int a = 0; a < 16; ++a)
+        v[a] = tr[a * 17 + L];
+    __syncwarp(hmask);
+    // stride 16 (digit d2 = a % 4), then stride 64 (digit d3 = a / 4)
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        h4_quad(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        h4_quad(v[q], v[q + 4], v[q + 8], v[q + 12]);
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        v[i] = __fmul_rn(v[i], 0.0625f);
+}
+
+// Quantise this lane's 16 column values of block b and store them in row order.
+__device__ __forceinline__ void quantise_store(const float (&v)[16], float scale, float fq, int L, uint8_t *tb,
+                                               unsigned hmask, int8_t *__restrict__ dst_block)
+{
+#pragma unroll
+    for (int a = 0; a < 16; ++a) {
+        float q = rintf(__fdiv_rn(v[a], scale));
+        q = fminf(fmaxf(q, -fq), fq);
+        tb[16 * a + L] = (uint8_t)(int8_t)__float2int_rn(q);
+    }
+    __syncwarp(hmask);
+    const uint4 o = *reinterpret_cast<const uint4 *>(tb + 16 * L);
+    *reinterpret_cast<uint4 *>(dst_block + 16 * L) = o;
+    __syncwarp(hmask);
+}
+
+template <int J, bool kRecompute>
+__global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
+                                                            int qmax, int8_t *__restrict__ xq,
+                                                            float *__restrict__ xs)
+{
+    __shared__ float tr_all[kHalfWarps][16 * 17];
+    __shared__ __align__(16) uint8_t tb_all[kHalfWarps][272];
+    __shared__ float warp_max[kThreads / 32];
+
+    const int tid = threadIdx.x;
+    const int hw = tid >> 4, L = tid & 15, warp = tid >> 5, lane = tid & 31;
+    const unsigned hmask = 0xFFFFu << (16 * (hw & 1));
+    const int64_t m = blockIdx.x;
+    const int NB = (int)(K / 256);
+    int8_t *__restrict__ qrow = xq + m * K;
+
+    if (m >= M) {  // padding row of the decode GEMV operand
+        for (int64_t c = tid; c < K / 16; c += kThreads)
+            reinterpret_cast<uint4 *>(qrow)[c] = make_uint4(0u, 0u, 0u, 0u);
+        if (tid == 0)
+            xs[m] = 1.0f;
+        return;
+    }
+
+    const uint16_t *__restrict__ xrow = x + m * K;
+    float *tr = tr_all[hw];
+    uint8_t *tb = tb_all[hw];
+    float amax = 0.0f;
+    float v[kRecompute ? 1 : J][16];
+
+    if (!kRecompute) {
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int b = hw + kHalfWarps * j;
+            if (b < NB) {
+                rotate_block(xrow + 256 * b, L, tr, hmask, v[j]);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    amax = fmaxf(amax, fabsf(v[j][i]));
+            }
+        }
+    } else {
+        for (int b = hw; b < NB; b += kHalfWarps) {
+            rotate_block(xrow + 256 * b, L, tr, hmask, v[0]);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                amax = fmaxf(amax, fabsf(v[0][i]));
+        }
+    }
+
+    // row maximum (exact in any order)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+    if (lane == 0)
+        warp_max[warp] = amax;
+    __syncthreads();
+    float rmax = warp_max[0];
+#pragma unroll
+    for (int w = 1; w < kThreads / 32; ++w)
+        rmax = fmaxf(rmax, warp_max[w]);
+    const float fq = (float)qmax;
+    const float scale = (rmax > 0.0f) ? __fdiv_rn(rmax, fq) : 1.0f;
+
+    if (!kRecompute) {
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int b = hw + kHalfWarps * j;
+            if (b < NB)
+                quantise_store(v[j], scale, fq, L, tb, hmask, qrow + 256 * b);
+        }
+    } else {
+        for (int b = hw; b < NB; b += kHalfWarps) {
+            rotate_block(xrow + 256 * b, L, tr, hmask, v[0]);
+            quantise_store(v[0], scale, fq, L, tb, hmask, qrow + 256 * b);
+        }
+    }
+    if (tid == 0)
+        xs[m] = scale;
+}
+
+inline cudaError_t launch(const uint16_t *x, int64_t M, int64_t K, int64_t MP, int qmax, int8_t *xq, float *xs,
+                          cudaStream_t stream)
+{
+    const dim3 grid((unsigned)MP), block(kThreads);
+    const int64_t per_hw = (K / 256 + kHalfWarps - 1) / kHalfWarps;  // blocks per half-warp
+    if (per_hw <= 1)
+        rotquant_kernel<1, false><<<grid, block, 0, stream>>>(x, M, K, qmax, xq, xs);
+    else if (per_hw == 2)
+        rotquant_kernel<2, false><<<grid, block, 0, stream>>>(x, M, K, qmax, xq, xs);
+    else if (per_hw == 3)
+        rotquant_kernel<3, false><<<grid, block, 0, stream>>>(x, M, K, qmax, xq, xs);
+    else if (per_hw == 4)
+        rotquant_kernel<4, false><<<grid, block, 0, stream>>>(x, M, K, qmax, xq, xs);
+    else
+        rotquant_kernel<1, true><<<grid, block, 0, stream>>>(x, M, K, qmax, xq, xs);
+    return cudaGetLastError();
+}
+
+}  // namespace rq
+}  // namespace cr
