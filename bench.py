@@ -166,7 +166,9 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- distributed
 
-def dist_setup(args):
+def dist_setup(backend: str = "nccl"):
+    """Join the torchrun process group (one process per GPU) when WORLD_SIZE > 1.
+    Returns (world, rank, local_rank)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -175,9 +177,11 @@ def dist_setup(args):
 
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
     return world, rank, local
 
 
@@ -188,13 +192,26 @@ def barrier(world):
 
 
 def max_over_ranks(value: float, world: int) -> float:
+    """The slowest rank's timing: every multi-GPU number is the max over ranks."""
     if world == 1:
         return value
     import torch
     import torch.distributed as dist
-    t = torch.tensor([value], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate_value(bytes_per_step_per_rank: float, steps: int, world: int, max_seconds: float) -> float:
+    """Whole-job throughput in GB/s: every rank streams its own replica's
+    weights each step (weak scaling), divided by the slowest rank's time."""
+    return world * bytes_per_step_per_rank * steps / max_seconds / 1e9
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own layer and batch (independent replicas)."""
+    return seed + 1000 * rank
 
 
 # ---------------------------------------------------------------- our arm
@@ -211,8 +228,8 @@ class Sets:
         M, N, K = case.M, case.N, case.K
         per_set = weight_bytes(N, K) + 2 * M * K
         self.R = max(2, int(math.ceil(min_bytes / per_set)))
-        layer = inputs.layer(N, K, case.seed + 1000 * rank)
-        x = inputs.activations(M, K, case.seed + 1000 * rank, case.dist)
+        layer = inputs.layer(N, K, rank_seed(case.seed, rank))
+        x = inputs.activations(M, K, rank_seed(case.seed, rank), case.dist)
         q = torch.from_numpy(layer.qdata).cuda()
         s = torch.from_numpy(layer.srel).cuda()
         self.cb = torch.from_numpy(layer.codebook).cuda()
@@ -341,7 +358,7 @@ def run_ours(args):
 
     import w4a8_codebook_quantized_b200 as cr
     from w4a8_codebook_quantized_b200 import inputs
-    world, rank, local = dist_setup(args)
+    world, rank, local = dist_setup()
     torch.cuda.set_device(local)
     cr.lib()
     pk = peaks()
@@ -355,7 +372,7 @@ def run_ours(args):
     secs, clocks = graph_time(sets.step, args.steps, args.warmup, world, local)
     secs = max_over_ranks(secs, world)
     wb = weight_bytes(N, K)
-    value = world * wb * args.steps / secs / 1e9
+    value = aggregate_value(wb, args.steps, world, secs)
 
     # the dominant kernel alone (GEMV), for the roofline
     ksecs, _ = graph_time(sets.contraction_only, args.steps, args.warmup, world, local)
@@ -372,7 +389,7 @@ def run_ours(args):
     # end to end through the public API with host buffers
     esecs = eager_time(sets.e2e_step, args.steps, args.warmup, world)
     esecs = max_over_ranks(esecs, world)
-    e2e = {"value": round(world * wb * args.steps / esecs / 1e9, 2), "unit": "GB/s",
+    e2e = {"value": round(aggregate_value(wb, args.steps, world, esecs), 2), "unit": "GB/s",
            "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N,
            "ms_per_step": round(esecs / args.steps * 1e3, 5)}
 
@@ -411,8 +428,8 @@ def run_prefill(args, world, rank, local, pk):
     from w4a8_codebook_quantized_b200 import inputs
     case = inputs.CASES[args.prefill_workload]
     M, N, K = case.M, case.N, case.K
-    layer = inputs.layer(N, K, case.seed + 1000 * rank)
-    x = inputs.activations(M, K, case.seed + 1000 * rank, case.dist)
+    layer = inputs.layer(N, K, rank_seed(case.seed, rank))
+    x = inputs.activations(M, K, rank_seed(case.seed, rank), case.dist)
     q = torch.from_numpy(layer.qdata).cuda()
     s = torch.from_numpy(layer.srel).cuda()
     cb = torch.from_numpy(layer.codebook).cuda()

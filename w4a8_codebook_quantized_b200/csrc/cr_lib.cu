@@ -330,7 +330,7 @@ cr_status cr_w4a8_linear(const uint16_t *x, const uint8_t *qdata, const uint8_t 
         return st;
     if (M <= CR_GEMV_MAX_M)
         return launched(cr::gv::launch(xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K,
-                                       out_dtype == CR_OUT_F32, out, nullptr, stream));
+                                       out_dtype == CR_OUT_F32, out, nullptr, stream, /*pdl=*/true));
     return run_gemm(*d, xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, nullptr,
                     stream);
 }

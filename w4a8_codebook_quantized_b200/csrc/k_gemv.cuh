@@ -79,11 +79,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint4 A[kBatch], B[kBatch], X0[kBatch], X1[kBatch];
     uint32_t SA[kBatch], SB[kBatch];
 
-    auto issue = [&](int i0) {
+    // Weight loads (codes + group scales) and activation loads are issued
+    // separately: the weights do not depend on the activation kernel, so they
+    // can be in flight before griddepcontrol.wait.
+    auto issue_w = [&](int i0) {
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             const int i = i0 + u;
-            A[u] = B[u] = X0[u] = X1[u] = z4;
+            A[u] = B[u] = z4;
             SA[u] = SB[u] = 0u;
             if (i < cnt) {
                 const int64_t s = warp + (int64_t)kWarps * i;
@@ -95,17 +98,25 @@ __global__ void __launch_bounds__(kThreads, 2)
                     B[u] = ldg_stream16(pb + 64 * s);
                     SB[u] = __ldg(reinterpret_cast<const uint16_t *>(psb + 8 * s));
                 }
-                if (vx) {
-                    X0[u] = __ldg(reinterpret_cast<const uint4 *>(px + 128 * s));
-                    X1[u] = __ldg(reinterpret_cast<const uint4 *>(px + 128 * s + 16));
-                }
+            }
+        }
+    };
+    auto issue_x = [&](int i0) {
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int i = i0 + u;
+            X0[u] = X1[u] = z4;
+            if (i < cnt && vx) {
+                const int64_t s = warp + (int64_t)kWarps * i;
+                X0[u] = *reinterpret_cast<const uint4 *>(px + 128 * s);
+                X1[u] = *reinterpret_cast<const uint4 *>(px + 128 * s + 16);
             }
         }
     };
 
-    // First loads go out before the table is built, so its cost hides under
-    // the memory latency.
-    issue(0);
+    // The first weight loads go out before the table is built, so its cost
+    // hides under the memory latency.
+    issue_w(0);
 
     if (tid < 16)
         cbs[tid] = codebook[tid];
@@ -118,11 +129,18 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncthreads();
 
+    // When launched as a programmatic dependent of the activation kernel, wait
+    // here for its results (a no-op otherwise).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    issue_x(0);
+
     int32_t c[4] = {0, 0, 0, 0};
     const int copy = lane & 7;
     for (int i0 = 0; i0 < cnt; i0 += kBatch) {
-        if (i0 > 0)
-            issue(i0);
+        if (i0 > 0) {
+            issue_w(i0);
+            issue_x(i0);
+        }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
             if (i0 + u < cnt) {
@@ -172,14 +190,25 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 }
 
+// pdl: launch as a programmatic dependent of the previous kernel in the
+// stream (the activation kernel), so the weight stream starts early.
 inline cudaError_t launch(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
                           const float *codebook, const float *ws, const float *bias, int64_t M, int64_t N, int64_t K,
-                          int out_f32, void *out, int32_t *acc_out, cudaStream_t stream)
+                          int out_f32, void *out, int32_t *acc_out, cudaStream_t stream, bool pdl = false)
 {
     const int64_t blocks = (N + kRows - 1) / kRows;
-    gemv_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(xq, xs, qdata, srel, codebook, ws, bias, (int)M, N, K,
-                                                           out_f32, out, acc_out);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, gemv_kernel, xq, xs, qdata, srel, codebook, ws, bias, (int)M, N, K, out_f32, out,
+                              acc_out);
 }
 
 }  // namespace gv

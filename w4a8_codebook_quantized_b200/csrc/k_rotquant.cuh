@@ -119,6 +119,10 @@ __global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__re
     __shared__ __align__(16) uint8_t tb_all[kHalfWarps][272];
     __shared__ float warp_max[kThreads / 32];
 
+    // Let a programmatic dependent (the decode GEMV) start its weight stream
+    // now; it waits for this grid's results before it reads them.
+    asm volatile("griddepcontrol.launch_dependents;" :::);
+
     const int tid = threadIdx.x;
     const int hw = tid >> 4, L = tid & 15, warp = tid >> 5, lane = tid & 31;
     const unsigned hmask = 0xFFFFu << (16 * (hw & 1));
