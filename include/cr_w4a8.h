@@ -30,9 +30,9 @@
  * - Arguments are validated before anything is launched; a failed validation
  *   launches nothing and leaves every output untouched.  Launch failures
  *   return CR_ERR_CUDA.  Nothing falls back to another implementation.
- * - Values are not validated: activations must be finite and small enough
- *   that a block sum of four of them does not overflow fp32 (|x| <= 2^124);
- *   for other values the outputs are unspecified, but no call faults.
+ * - Values are not validated: activations must be finite with |x| < 2^119,
+ *   so that no partial sum of the block rotation (at most 256 |x|) overflows
+ *   fp32; for other values the outputs are unspecified, but no call faults.
  * - Calls that read a buffer another call on another stream is writing race,
  *   as with any CUDA kernel.
  */

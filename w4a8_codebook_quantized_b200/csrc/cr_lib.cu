@@ -28,6 +28,7 @@ struct DeviceState {
     int num_sms = 0;
     cudaMemPool_t pool = nullptr;  // stream-ordered pool for the prefill weight transient
     bool gemm_attr_set = false;
+    bool gemv_attr_set = false;
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -39,6 +40,23 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_
 EncodeTiledFn g_encode_tiled = nullptr;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The driver's tensor-map encoder, looked up once through the runtime (no
+// link against libcuda).  Called with g_mutex held.
+bool have_encode_tiled()
+{
+    if (g_encode_tiled != nullptr)
+        return true;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr) {
+        cudaGetLastError();
+        return false;
+    }
+    g_encode_tiled = reinterpret_cast<EncodeTiledFn>(fn);
+    return true;
+}
 
 cr_status check_k(int64_t K)
 {
@@ -82,17 +100,8 @@ cr_status current_device(DeviceState **out)
                 cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
             }
         }
-        if (d.usable && g_encode_tiled == nullptr) {
-            void *fn = nullptr;
-            cudaDriverEntryPointQueryResult q;
-            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-                q != cudaDriverEntryPointSuccess || fn == nullptr) {
-                cudaGetLastError();
-                d.usable = false;
-            } else {
-                g_encode_tiled = reinterpret_cast<EncodeTiledFn>(fn);
-            }
-        }
+        if (d.usable && !have_encode_tiled())
+            d.usable = false;
     }
     if (!d.usable)
         return CR_ERR_NO_DEVICE;
@@ -119,6 +128,61 @@ bool make_tmap_i8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t r
                                       box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// 2-D tensor map, no swizzle: a row-major [rows, inner] array of `esize`-byte
+// elements with the given row pitch in bytes, box [box_rows, box_inner].
+bool make_tmap_plain(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, uint64_t inner, uint64_t rows,
+                     uint64_t pitch, uint32_t box_inner, uint32_t box_rows)
+{
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {pitch};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = g_encode_tiled(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
+                                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// The decode GEMV: tensor maps over the packed codes (as 32-bit words, one
+// 512-byte row slice per stage row) and the scale bytes, a persistent grid of
+// two CTAs per SM, optionally as a programmatic dependent of the previous
+// kernel on the stream.
+cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const uint8_t *qdata,
+                   const uint8_t *srel, const float *codebook, const float *s_channel, const float *bias, int64_t M,
+                   int64_t N, int64_t K, cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream,
+                   bool pdl)
+{
+    using namespace cr;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(gv::gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gv::kSmemBytes) != cudaSuccess) {
+            cudaGetLastError();
+            return CR_ERR_CUDA;
+        }
+        attr_set = true;
+    }
+    CUtensorMap tc, ts;
+    if (!make_tmap_plain(&tc, qdata, CU_TENSOR_MAP_DATA_TYPE_UINT32, (uint64_t)(K / 8), (uint64_t)N,
+                         (uint64_t)(K / 2), gv::kChunk / 8, gv::kRows) ||
+        !make_tmap_plain(&ts, srel, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)(K / 16), (uint64_t)N,
+                         (uint64_t)(K / 16), gv::kChunk / 16, gv::kRows))
+        return CR_ERR_CUDA;
+    const int64_t tiles = (N + gv::kRows - 1) / gv::kRows;
+    const int64_t grid = tiles < 2 * (int64_t)num_sms ? tiles : 2 * (int64_t)num_sms;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(gv::kThreads);
+    cfg.dynamicSmemBytes = gv::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return launched(cudaLaunchKernelEx(&cfg, gv::gemv_kernel, tc, ts, xq, xs, codebook, s_channel, bias, (int)M,
+                                       (int)N, (int)K, out_dtype == CR_OUT_F32 ? 1 : 0, out, acc_out));
 }
 
 // Shared validation of the contraction entry points.
@@ -278,8 +342,8 @@ cr_status cr_w4a8_gemv(const int8_t *xq, const float *xs, const uint8_t *qdata, 
     st = current_device(&d);
     if (st != CR_OK)
         return st;
-    return launched(cr::gv::launch(xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K,
-                                   out_dtype == CR_OUT_F32, out, acc_out, stream));
+    return run_gemv(d->num_sms, d->gemv_attr_set, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K,
+                    out_dtype, out, acc_out, stream, false);
 }
 
 cr_status cr_epilogue(const int32_t *acc, const float *xs, const float *s_channel, const float *bias, int64_t M,
@@ -329,8 +393,8 @@ cr_status cr_w4a8_linear(const uint16_t *x, const uint8_t *qdata, const uint8_t 
     if (st != CR_OK)
         return st;
     if (M <= CR_GEMV_MAX_M)
-        return launched(cr::gv::launch(xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K,
-                                       out_dtype == CR_OUT_F32, out, nullptr, stream, /*pdl=*/true));
+        return run_gemv(d->num_sms, d->gemv_attr_set, xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M,
+                        N, K, out_dtype, out, nullptr, stream, /*pdl=*/true);
     return run_gemm(*d, xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, nullptr,
                     stream);
 }

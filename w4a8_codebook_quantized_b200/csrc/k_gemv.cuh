@@ -6,39 +6,60 @@
 // costs 4.5 bits of HBM traffic and is never materialised.  The int32 sums
 // are exact, so the result equals the prefill path bit for bit.
 //
-// B200 design.  The page's kernel multiply-accumulates with int32 IMAD in
-// registers.  Here the decoded int8 weights stay in registers too, but the
-// dot products go to the warp-level int8 tensor-core instruction
-// (mma.sync m16n8k32, A = 16 weight rows x 32 k, B = 32 k x 8 tokens), fed
-// directly from registers: no shared-memory round trip, and the ALU budget
-// per weight drops to the decode itself (about 1.4 instructions), which
-// keeps the kernel memory-bound at M = 8.  (The tcgen05 path would need the
-// operands in shared memory; at 8 tokens the tensor work is negligible.)
-//
-// Since the sum runs over k, any permutation of k is allowed as long as A and
-// B use the same one.  Thread (g = lane / 4, t = lane % 4) loads 16 contiguous
-// bytes (32 codes) of weight rows g and g + 8 for k in [128 s + 32 t, +32) of
-// slice s, and the matching 32 activation bytes of token g; code word i
-// (columns 8i..8i+7) feeds MMA i: its first four columns go to the fragment
-// slots of logical k = 4t..4t+3, its last four to 16+4t..16+4t+3.
-//
-// The level table (16 int8 levels per fp8 scale byte) is replicated 8 times
-// with copy c living in bank group c; lane l reads copy l % 8, so the eight
-// lanes of each quarter-warp phase of a 16-byte shared load never conflict.
-//
-// Grid: one CTA (8 warps) per 16 output rows; the warps split the K slices
-// (s = warp, warp + 8, ...) and the int32 partial sums meet in shared memory.
+// B200 design.
+//  * Streaming: a persistent grid (two CTAs per SM).  In each CTA one
+//    producer warp moves 16-row x 1024-column tiles of the packed codes
+//    (8 KB) and their group scales (1 KB) into a 6-stage shared-memory ring
+//    with 2-D TMA copies; eight consumer warps decode and contract each stage
+//    while the following ones are in flight.  Bytes in flight are set by the
+//    ring, not by registers, which keeps HBM busy.
+//  * Decode: a per-CTA table of the 16 int8 levels of every fp8 scale byte
+//    (exact: the decoded value depends only on the pair), replicated 8 times
+//    with copy c in bank group c so that a quarter-warp's 16-byte lookups
+//    never conflict; byte permutes turn 8 packed codes into 8 int8 levels.
+//  * Contraction: the page's kernel uses int32 IMAD in registers; here the
+//    decoded weights go straight from registers into the warp-level int8
+//    tensor-core instruction (mma.sync m16n8k32: A = 16 weight rows x 32 k,
+//    B = 32 k x 8 tokens), so the ALU only pays for the decode.  Since the sum
+//    runs over k, any permutation of k is allowed as long as A and B use the
+//    same one: thread (g = lane / 4, t = lane % 4) takes the 16 contiguous
+//    bytes (32 codes) of rows g and g + 8 at k = 128 w + 32 t of its warp's
+//    slice w, and the matching 32 activation bytes of token g; code word i
+//    (columns 8i..8i+7) feeds MMA i, its first four columns in the fragment
+//    slots of logical k = 4t..4t+3 and its last four in 16+4t..16+4t+3.
+//  * The int32 partial sums of the eight warps meet in shared memory; the
+//    fused epilogue writes the 16 x M outputs of the row tile.
+//  * When launched as a programmatic dependent of the activation kernel, the
+//    weight stream and the table build start before that kernel finishes;
+//    the consumers wait for it (griddepcontrol.wait) before reading xq / xs.
 #pragma once
+
+#include <cuda.h>
 
 #include "cr_device.cuh"
 
 namespace cr {
 namespace gv {
 
-constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
-constexpr int kRows = 16;   // output rows per CTA
-constexpr int kBatch = 4;   // slices whose loads are in flight together per warp
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kRows = 16;                            // output rows per tile
+constexpr int kChunk = 1024;                         // k per stage
+constexpr int kStages = 6;
+constexpr int kCodeBytes = kRows * kChunk / 2;       // 8 KB
+constexpr int kSrelBytes = kRows * kChunk / 16;      // 1 KB
+
+struct __align__(1024) Smem {
+    uint8_t codes[kStages][kCodeBytes];  // row r of a stage at r * 512 bytes
+    uint8_t srel[kStages][kSrelBytes];   // row r of a stage at r * 64 bytes
+    uint4 lut8[256 * 8];                 // lut8[s * 8 + c]: copy c of the levels of scale byte s
+    int32_t red[kConsumerWarps][kRows][8];
+    float cb[16];
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    int abort;
+};
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 
 __device__ __forceinline__ void mma_s8(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                        uint32_t b0, uint32_t b1)
@@ -50,165 +71,161 @@ __device__ __forceinline__ void mma_s8(int32_t (&c)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 __global__ void __launch_bounds__(kThreads, 2)
-    gemv_kernel(const int8_t *__restrict__ xq, const float *__restrict__ xs, const uint8_t *__restrict__ qdata,
-                const uint8_t *__restrict__ srel, const float *__restrict__ codebook,
-                const float *__restrict__ ws, const float *__restrict__ bias, int M, int64_t N, int64_t K,
-                int out_f32, void *__restrict__ out, int32_t *__restrict__ acc_out)
+    gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_srel,
+                const int8_t *__restrict__ xq, const float *__restrict__ xs, const float *__restrict__ codebook,
+                const float *__restrict__ ws, const float *__restrict__ bias, int M, int N, int K, int out_f32,
+                void *__restrict__ out, int32_t *__restrict__ acc_out)
 {
-    __shared__ uint4 lut8[256 * 8];  // lut8[s * 8 + c]: copy c of entry s
-    __shared__ int32_t red[kWarps][kRows][8];
-    __shared__ float cbs[16];
+    extern __shared__ uint8_t smem_raw[];
+    Smem &sh = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int64_t n0 = (int64_t)blockIdx.x * kRows;
-    const int64_t KH = K >> 1, KG = K >> 4;
-    const int nslice = (int)(K >> 7);
-    const int cnt = (nslice > warp) ? (nslice - warp + kWarps - 1) / kWarps : 0;
+    const int ntiles = (N + kRows - 1) / kRows;
+    const int nchunks = (K + kChunk - 1) / kChunk;
 
-    const int64_t ra = n0 + g, rb = n0 + g + 8;
-    const bool va = ra < N, vb = rb < N, vx = g < M;
-    const uint8_t *pa = qdata + ra * KH + 16 * t;
-    const uint8_t *pb = qdata + rb * KH + 16 * t;
-    const uint8_t *psa = srel + ra * KG + 2 * t;
-    const uint8_t *psb = srel + rb * KG + 2 * t;
-    const int8_t *px = xq + (int64_t)g * K + 32 * t;
-    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-
-    uint4 A[kBatch], B[kBatch], X0[kBatch], X1[kBatch];
-    uint32_t SA[kBatch], SB[kBatch];
-
-    // Weight loads (codes + group scales) and activation loads are issued
-    // separately: the weights do not depend on the activation kernel, so they
-    // can be in flight before griddepcontrol.wait.
-    auto issue_w = [&](int i0) {
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int i = i0 + u;
-            A[u] = B[u] = z4;
-            SA[u] = SB[u] = 0u;
-            if (i < cnt) {
-                const int64_t s = warp + (int64_t)kWarps * i;
-                if (va) {
-                    A[u] = ldg_stream16(pa + 64 * s);
-                    SA[u] = __ldg(reinterpret_cast<const uint16_t *>(psa + 8 * s));
-                }
-                if (vb) {
-                    B[u] = ldg_stream16(pb + 64 * s);
-                    SB[u] = __ldg(reinterpret_cast<const uint16_t *>(psb + 8 * s));
-                }
-            }
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.empty[s], kConsumerWarps);
         }
-    };
-    auto issue_x = [&](int i0) {
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            const int i = i0 + u;
-            X0[u] = X1[u] = z4;
-            if (i < cnt && vx) {
-                const int64_t s = warp + (int64_t)kWarps * i;
-                X0[u] = *reinterpret_cast<const uint4 *>(px + 128 * s);
-                X1[u] = *reinterpret_cast<const uint4 *>(px + 128 * s + 16);
-            }
-        }
-    };
-
-    // The first weight loads go out before the table is built, so its cost
-    // hides under the memory latency.
-    issue_w(0);
-
+        sh.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
     if (tid < 16)
-        cbs[tid] = codebook[tid];
+        sh.cb[tid] = codebook[tid];
     __syncthreads();
-    {
-        const uint4 e = lut_entry((uint32_t)tid, cbs);
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-            lut8[tid * 8 + ((r + tid) & 7)] = e;
-    }
-    __syncthreads();
+    volatile int *abort = &sh.abort;
 
-    // When launched as a programmatic dependent of the activation kernel, wait
-    // here for its results (a no-op otherwise).
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    issue_x(0);
-
-    int32_t c[4] = {0, 0, 0, 0};
-    const int copy = lane & 7;
-    for (int i0 = 0; i0 < cnt; i0 += kBatch) {
-        if (i0 > 0) {
-            issue_w(i0);
-            issue_x(i0);
-        }
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-            if (i0 + u < cnt) {
-                const uint4 TA0 = lut8[(SA[u] & 0xFFu) * 8 + copy];
-                const uint4 TA1 = lut8[(SA[u] >> 8) * 8 + copy];
-                const uint4 TB0 = lut8[(SB[u] & 0xFFu) * 8 + copy];
-                const uint4 TB1 = lut8[(SB[u] >> 8) * 8 + copy];
-                uint32_t a0, a1, a2, a3;
-                decode8(A[u].x, TA0, a0, a2);
-                decode8(B[u].x, TB0, a1, a3);
-                mma_s8(c, a0, a1, a2, a3, X0[u].x, X0[u].y);
-                decode8(A[u].y, TA0, a0, a2);
-                decode8(B[u].y, TB0, a1, a3);
-                mma_s8(c, a0, a1, a2, a3, X0[u].z, X0[u].w);
-                decode8(A[u].z, TA1, a0, a2);
-                decode8(B[u].z, TB1, a1, a3);
-                mma_s8(c, a0, a1, a2, a3, X1[u].x, X1[u].y);
-                decode8(A[u].w, TA1, a0, a2);
-                decode8(B[u].w, TB1, a1, a3);
-                mma_s8(c, a0, a1, a2, a3, X1[u].z, X1[u].w);
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tm_codes);
+            prefetch_tmap(&tm_srel);
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued[kStages];
+            uint32_t issued_phase[kStages];
+            for (int s = 0; s < kStages; ++s)
+                issued[s] = 0, issued_phase[s] = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
+                for (int c = 0; c < nchunks; ++c) {
+                    if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&sh.full[stage], kCodeBytes + kSrelBytes);
+                    tma_load_2d(sh.codes[stage], &tm_codes, c * (kChunk / 8), tile * kRows, &sh.full[stage]);
+                    tma_load_2d(sh.srel[stage], &tm_srel, c * (kChunk / 16), tile * kRows, &sh.full[stage]);
+                    issued[stage] = 1;
+                    issued_phase[stage] = phase;
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                for (int s = 0; s < kStages; ++s)
+                    if (issued[s]) {
+                        volatile int no_abort = 0;
+                        mbar_wait_bounded(&sh.full[s], issued_phase[s], &no_abort, 20000000ull);
+                    }
             }
         }
-    }
-
-    // C fragment: c0 (row g, token 2t), c1 (g, 2t+1), c2 (g+8, 2t), c3 (g+8, 2t+1)
-    red[warp][g][2 * t] = c[0];
-    red[warp][g][2 * t + 1] = c[1];
-    red[warp][g + 8][2 * t] = c[2];
-    red[warp][g + 8][2 * t + 1] = c[3];
-    __syncthreads();
-    if (tid < kRows * 8) {
-        const int r = tid >> 3, m = tid & 7;
-        int32_t acc = 0;
+    } else {
+        // ------------------------------------------------ consumers
+        {
+            const uint4 e = lut_entry((uint32_t)tid, sh.cb);
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w)
-            acc += red[w][r][m];
-        const int64_t n = n0 + r;
-        if (m < M && n < N) {
-            const float y = epilogue_value(acc, xs[m], ws[n], bias, n);
-            if (out_f32)
-                reinterpret_cast<float *>(out)[(int64_t)m * N + n] = y;
-            else
-                reinterpret_cast<uint16_t *>(out)[(int64_t)m * N + n] = to_bf16_bits(y);
-            if (acc_out != nullptr)
-                acc_out[(int64_t)m * N + n] = acc;
+            for (int r = 0; r < 8; ++r)
+                sh.lut8[tid * 8 + ((r + tid) & 7)] = e;
+        }
+        consumer_sync();
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+
+        const int g = lane >> 2, t = lane & 3;
+        const int copy = lane & 7;
+        const bool vx = g < M;
+        const int8_t *px = xq + (int64_t)g * K + 128 * warp + 32 * t;
+        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            int32_t c[4] = {0, 0, 0, 0};
+            for (int ch = 0; ch < nchunks; ++ch) {
+                const bool active = ch * kChunk + 128 * warp < K;  // this warp's slice exists
+                uint4 X0 = z4, X1 = z4;
+                if (active && vx) {
+                    X0 = *reinterpret_cast<const uint4 *>(px + (int64_t)ch * kChunk);
+                    X1 = *reinterpret_cast<const uint4 *>(px + (int64_t)ch * kChunk + 16);
+                }
+                const bool ok = mbar_wait_bounded_warp(&sh.full[stage], phase, abort);
+                if (ok && active) {
+                    const uint8_t *cs = sh.codes[stage] + 64 * warp + 16 * t;
+                    const uint4 A = *reinterpret_cast<const uint4 *>(cs + 512 * g);
+                    const uint4 B = *reinterpret_cast<const uint4 *>(cs + 512 * (g + 8));
+                    const uint8_t *ss = sh.srel[stage] + 8 * warp + 2 * t;
+                    const uint32_t SA = *reinterpret_cast<const uint16_t *>(ss + 64 * g);
+                    const uint32_t SB = *reinterpret_cast<const uint16_t *>(ss + 64 * (g + 8));
+                    const uint4 TA0 = sh.lut8[(SA & 0xFFu) * 8 + copy];
+                    const uint4 TA1 = sh.lut8[(SA >> 8) * 8 + copy];
+                    const uint4 TB0 = sh.lut8[(SB & 0xFFu) * 8 + copy];
+                    const uint4 TB1 = sh.lut8[(SB >> 8) * 8 + copy];
+                    uint32_t a0, a1, a2, a3;
+                    decode8(A.x, TA0, a0, a2);
+                    decode8(B.x, TB0, a1, a3);
+                    mma_s8(c, a0, a1, a2, a3, X0.x, X0.y);
+                    decode8(A.y, TA0, a0, a2);
+                    decode8(B.y, TB0, a1, a3);
+                    mma_s8(c, a0, a1, a2, a3, X0.z, X0.w);
+                    decode8(A.z, TA1, a0, a2);
+                    decode8(B.z, TB1, a1, a3);
+                    mma_s8(c, a0, a1, a2, a3, X1.x, X1.y);
+                    decode8(A.w, TA1, a0, a2);
+                    decode8(B.w, TB1, a1, a3);
+                    mma_s8(c, a0, a1, a2, a3, X1.z, X1.w);
+                }
+                __syncwarp();
+                if (ok && lane == 0)
+                    mbar_arrive(&sh.empty[stage]);
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            // C fragment: c0 (row g, token 2t), c1 (g, 2t+1), c2 (g+8, 2t), c3 (g+8, 2t+1)
+            sh.red[warp][g][2 * t] = c[0];
+            sh.red[warp][g][2 * t + 1] = c[1];
+            sh.red[warp][g + 8][2 * t] = c[2];
+            sh.red[warp][g + 8][2 * t + 1] = c[3];
+            consumer_sync();
+            if (tid < kRows * 8) {
+                const int r = tid >> 3, m = tid & 7;
+                int32_t acc = 0;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w)
+                    acc += sh.red[w][r][m];
+                const int n = tile * kRows + r;
+                if (m < M && n < N && !*abort) {
+                    const float y = epilogue_value(acc, xs[m], ws[n], bias, n);
+                    const int64_t o = (int64_t)m * N + n;
+                    if (out_f32)
+                        reinterpret_cast<float *>(out)[o] = y;
+                    else
+                        reinterpret_cast<uint16_t *>(out)[o] = to_bf16_bits(y);
+                    if (acc_out != nullptr)
+                        acc_out[o] = acc;
+                }
+            }
+            consumer_sync();
         }
     }
-}
-
-// pdl: launch as a programmatic dependent of the previous kernel in the
-// stream (the activation kernel), so the weight stream starts early.
-inline cudaError_t launch(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
-                          const float *codebook, const float *ws, const float *bias, int64_t M, int64_t N, int64_t K,
-                          int out_f32, void *out, int32_t *acc_out, cudaStream_t stream, bool pdl = false)
-{
-    const int64_t blocks = (N + kRows - 1) / kRows;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)blocks);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, gemv_kernel, xq, xs, qdata, srel, codebook, ws, bias, (int)M, N, K, out_f32, out,
-                              acc_out);
+    __syncthreads();
 }
 
 }  // namespace gv

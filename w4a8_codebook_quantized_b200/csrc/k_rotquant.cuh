@@ -53,7 +53,7 @@ __device__ __forceinline__ void h4_quad(float &a0, float &a1, float &a2, float &
 
 // Rotate one 256-element block.  On return lane L of the half-warp holds
 // v[a] = rotated element 16a + L (a = 0..15).  `tr` is this half-warp's
-// 16 x 17 fp32 transpose buffer.
+// 16 x 16 fp32 transpose buffer (16-byte aligned).
 __device__ __forceinline__ void rotate_block(const uint16_t *__restrict__ blk, int L, float *tr, unsigned hmask,
                                              float (&v)[16])
 {
@@ -73,14 +73,20 @@ __device__ __forceinline__ void rotate_block(const uint16_t *__restrict__ blk, i
 #pragma unroll
     for (int q = 0; q < 4; ++q)
         h4_quad(v[q], v[q + 4], v[q + 8], v[q + 12]);
-    // transpose: row L out, column L in (row pitch 17 words: conflict-free)
+    // Transpose through shared memory: row L goes out as four 16-byte stores,
+    // column L comes back as 16 scalar loads.  Chunk c of row a lives at chunk
+    // position c ^ ((a >> 1) & 3), which makes both sides conflict-free.
+    {
+        float4 *rowp = reinterpret_cast<float4 *>(tr + 16 * L);
+        const int sw = (L >> 1) & 3;
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-        tr[L * 17 + i] = v[i];
+        for (int c = 0; c < 4; ++c)
+            rowp[c ^ sw] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+    }
     __syncwarp(hmask);
 #pragma unroll
     for (int a = 0; a < 16; ++a)
-        v[a] = tr[a * 17 + L];
+        v[a] = tr[16 * a + 4 * ((L >> 2) ^ ((a >> 1) & 3)) + (L & 3)];
     __syncwarp(hmask);
     // stride 16 (digit d2 = a % 4), then stride 64 (digit d3 = a / 4)
 #pragma unroll
@@ -94,16 +100,36 @@ __device__ __forceinline__ void rotate_block(const uint16_t *__restrict__ blk, i
         v[i] = __fmul_rn(v[i], 0.0625f);
 }
 
+// rint(r / s) clamped to +-qmax, without a per-element division.
+//
+// inv = 1/s rounded once per row.  When s is a normal fp32 and |r| <= amax,
+// t = r * inv differs from the correctly rounded quotient v = r / s by at most
+// 3 * 2^-24 * |r / s| <= 3 * 2^-24 * 128 < 2^-15.  So unless t lies within 2^-15
+// of a half-integer, t and v round to the same integer and neither is a tie;
+// in that rare case the quotient is computed exactly and rounded.  Adding
+// 1.5 * 2^23 rounds t to an integer (nearest even) in the low mantissa bits
+// (valid for |t| < 2^22), which also yields the integer without a conversion.
+// `exact_only` (a subnormal s) takes the exact path for every element.
+__device__ __forceinline__ int32_t quantise_one(float r, float s, float inv, int32_t qmax, bool exact_only)
+{
+    const float kMagic = 12582912.0f;  // 1.5 * 2^23
+    const float t = __fmul_rn(r, inv);
+    const float tm = __fadd_rn(t, kMagic);
+    const float rt = __fsub_rn(tm, kMagic);
+    int32_t q = __float_as_int(tm) - 0x4B400000;
+    if (exact_only || fabsf(__fsub_rn(t, rt)) >= 0.499969482421875f)  // within 2^-15 of k + 1/2
+        q = __float2int_rn(__fdiv_rn(r, s));
+    return min(max(q, -qmax), qmax);
+}
+
 // Quantise this lane's 16 column values of block b and store them in row order.
-__device__ __forceinline__ void quantise_store(const float (&v)[16], float scale, float fq, int L, uint8_t *tb,
-                                               unsigned hmask, int8_t *__restrict__ dst_block)
+__device__ __forceinline__ void quantise_store(const float (&v)[16], float scale, float inv, int32_t qmax,
+                                               bool exact_only, int L, uint8_t *tb, unsigned hmask,
+                                               int8_t *__restrict__ dst_block)
 {
 #pragma unroll
-    for (int a = 0; a < 16; ++a) {
-        float q = rintf(__fdiv_rn(v[a], scale));
-        q = fminf(fmaxf(q, -fq), fq);
-        tb[16 * a + L] = (uint8_t)(int8_t)__float2int_rn(q);
-    }
+    for (int a = 0; a < 16; ++a)
+        tb[16 * a + L] = (uint8_t)quantise_one(v[a], scale, inv, qmax, exact_only);
     __syncwarp(hmask);
     const uint4 o = *reinterpret_cast<const uint4 *>(tb + 16 * L);
     *reinterpret_cast<uint4 *>(dst_block + 16 * L) = o;
@@ -115,7 +141,9 @@ __global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__re
                                                             int qmax, int8_t *__restrict__ xq,
                                                             float *__restrict__ xs)
 {
-    __shared__ float tr_all[kHalfWarps][16 * 17];
+    // half-warp buffers 16 floats apart in bank space: the two halves of a warp
+    // never touch the same bank in one transpose step
+    __shared__ __align__(16) float tr_all[kHalfWarps][16 * 16 + 16];
     __shared__ __align__(16) uint8_t tb_all[kHalfWarps][272];
     __shared__ float warp_max[kThreads / 32];
 
@@ -175,20 +203,21 @@ __global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__re
 #pragma unroll
     for (int w = 1; w < kThreads / 32; ++w)
         rmax = fmaxf(rmax, warp_max[w]);
-    const float fq = (float)qmax;
-    const float scale = (rmax > 0.0f) ? __fdiv_rn(rmax, fq) : 1.0f;
+    const float scale = (rmax > 0.0f) ? __fdiv_rn(rmax, (float)qmax) : 1.0f;
+    const float inv = __frcp_rn(scale);
+    const bool exact_only = scale < 1.17549435e-38f;  // subnormal scale: 1/s may be inexact or overflow
 
     if (!kRecompute) {
 #pragma unroll
         for (int j = 0; j < J; ++j) {
             const int b = hw + kHalfWarps * j;
             if (b < NB)
-                quantise_store(v[j], scale, fq, L, tb, hmask, qrow + 256 * b);
+                quantise_store(v[j], scale, inv, qmax, exact_only, L, tb, hmask, qrow + 256 * b);
         }
     } else {
         for (int b = hw; b < NB; b += kHalfWarps) {
             rotate_block(xrow + 256 * b, L, tr, hmask, v[0]);
-            quantise_store(v[0], scale, fq, L, tb, hmask, qrow + 256 * b);
+            quantise_store(v[0], scale, inv, qmax, exact_only, L, tb, hmask, qrow + 256 * b);
         }
     }
     if (tid == 0)
