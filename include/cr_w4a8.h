@@ -190,6 +190,37 @@ cr_status cr_w4a8_linear(const uint16_t *x, const uint8_t *qdata, const uint8_t 
                          void *out, int8_t *xq_work, float *xs_work, cr_stream_t stream);
 
 /*
+ * (7) The decode forward (1 <= M <= 8) without any allocation.
+ *
+ * The pages have no counterpart of this entry point; it exists for callers
+ * that cannot allocate device memory at the time of the call and so cannot
+ * supply the scratch buffers cr_w4a8_linear needs: code running while a CUDA
+ * graph is being captured (cudaMalloc may not be called then), serving loops
+ * whose device memory is owned by their own allocator, and real-time paths
+ * that cannot afford the synchronisation an allocation can imply.
+ *
+ * It computes exactly what cr_w4a8_linear computes for M <= 8 (rotate +
+ * quantise, then the decode GEMV), with the quantised activations kept in a
+ * scratch array that the library reserves statically on every device that
+ * loads it (CR_NOALLOC_SCRATCH_BYTES, held until the process exits).  The
+ * caller still passes x, the layer and out, as for cr_w4a8_linear.
+ *
+ * Limits: 1 <= M <= 8 and K <= CR_MAX_K, so the padded activations
+ * (next power of two of M rows x K bytes) always fit; M > 8 returns
+ * CR_ERR_UNSUPPORTED.  It calls no allocation routine.
+ * The first call on a device looks up the scratch array's device address;
+ * make that first call before any stream capture on that device.
+ * Every call on a device shares the one scratch array, so calls whose
+ * kernels overlap on the GPU (different streams, or concurrent host threads)
+ * race and give undefined results; serialise them on one stream.
+ */
+#define CR_NOALLOC_SCRATCH_BYTES (CR_GEMV_MAX_M * CR_MAX_K + 256)
+cr_status cr_w4a8_linear_decode_noalloc(const uint16_t *x, const uint8_t *qdata, const uint8_t *srel,
+                                        const float *codebook, const float *s_channel, const float *bias,
+                                        int64_t M, int64_t N, int64_t K, int act_qmax, cr_out_dtype out_dtype,
+                                        void *out, cr_stream_t stream);
+
+/*
  * Waits for `stream`, then reads and clears the library's device error word,
  * which a kernel sets when one of its bounded pipeline waits runs out (the
  * kernel then abandons its tile and exits; its outputs are unspecified).

@@ -24,7 +24,8 @@ from typing import Optional, Tuple
 __all__ = [
     "CrError", "lib", "library_path",
     "cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv",
-    "cr_epilogue", "cr_w4a8_linear", "cr_check_device_error", "cr_status_string", "cr_version",
+    "cr_epilogue", "cr_w4a8_linear", "cr_w4a8_linear_decode_noalloc", "cr_check_device_error",
+    "cr_status_string", "cr_version",
     "gemv_rows",
 ]
 
@@ -71,8 +72,10 @@ def lib() -> ctypes.CDLL:
             L.cr_epilogue.argtypes = [P, P, P, P, i64, i64, i32, P, P]
             L.cr_w4a8_linear.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P, P, P]
             L.cr_check_device_error.argtypes = [P]
+            L.cr_w4a8_linear_decode_noalloc.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P]
             for name in ("cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv",
-                         "cr_epilogue", "cr_w4a8_linear", "cr_check_device_error"):
+                         "cr_epilogue", "cr_w4a8_linear", "cr_check_device_error",
+                         "cr_w4a8_linear_decode_noalloc"):
                 getattr(L, name).restype = i32
             _lib = L
     return _lib
@@ -275,6 +278,30 @@ def cr_w4a8_linear(x, qdata, srel, codebook, s_channel, bias=None, act_qmax: int
     _check(lib().cr_w4a8_linear(_ptr(x), _ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), _ptr(bias),
                                 M, N, K, int(act_qmax), _out_code(out.dtype), _ptr(out), _ptr(xq_work),
                                 _ptr(xs_work), _stream(stream)), "cr_w4a8_linear")
+    return out
+
+
+def cr_w4a8_linear_decode_noalloc(x, qdata, srel, codebook, s_channel, bias=None, act_qmax: int = 127,
+                                  out_dtype=None, out=None, stream=None):
+    """The decode forward (M <= 8) for callers that cannot allocate device
+    memory during the call (e.g. while a CUDA graph is being captured): the
+    quantised activations live in a small scratch array the library reserves
+    statically per device.  Pass `out` to allocate nothing at all.  Calls that
+    overlap on the GPU share that scratch and race; make the first call on a
+    device before any stream capture."""
+    torch = _torch()
+    _need(x, "x", (torch.bfloat16,), 2)
+    M, K = x.shape
+    N, Kw = _layer(qdata, srel, codebook, s_channel, bias)
+    if Kw != K:
+        raise ValueError(f"x has K={K}, the layer K={Kw}")
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype or torch.bfloat16, device=x.device)
+    _need(out, "out", (torch.bfloat16, torch.float32), shape=(M, N))
+    _check(lib().cr_w4a8_linear_decode_noalloc(_ptr(x), _ptr(qdata), _ptr(srel), _ptr(codebook),
+                                               _ptr(s_channel), _ptr(bias), M, N, K, int(act_qmax),
+                                               _out_code(out.dtype), _ptr(out), _stream(stream)),
+           "cr_w4a8_linear_decode_noalloc")
     return out
 
 

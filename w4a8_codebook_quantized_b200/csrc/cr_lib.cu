@@ -399,6 +399,105 @@ cr_status cr_w4a8_linear(const uint16_t *x, const uint8_t *qdata, const uint8_t 
                     stream);
 }
 
+// ---------------------------------------------------------------- decode forward without allocation
+//
+// The scratch of cr_w4a8_linear_decode_noalloc: the padded int8 activations
+// (at most 8 rows of K <= CR_MAX_K bytes) at offset 0 and their 8 fp32 scales
+// at offset CR_GEMV_MAX_M * CR_MAX_K.  One array per device, reserved when the
+// module loads on that device.  In host code `g_noalloc_scratch` is only a
+// host-side stand-in for the symbol: its device address is looked up once per
+// device with cudaGetSymbolAddress and that address is what the kernels get.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[CR_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+struct NoallocState {
+    bool ready = false;
+    uint8_t *scratch = nullptr;  // device address of g_noalloc_scratch on this device
+    int num_sms = 0;
+    bool gemv_attr_set = false;
+};
+NoallocState g_noalloc[kMaxDevices];
+
+// Once per device, with that device current: check it is an sm_100 part,
+// look up the scratch array's device address, the SM count and the tensor-map
+// encoder.  Allocates nothing.
+cr_status noalloc_scratch(NoallocState **out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return CR_ERR_NO_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(g_mutex);
+    NoallocState &s = g_noalloc[dev];
+    if (!s.ready) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return CR_ERR_NO_DEVICE;
+        }
+        if (major != 10 || minor != 0)
+            return CR_ERR_NO_DEVICE;
+        if (cudaDeviceGetAttribute(&s.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return CR_ERR_NO_DEVICE;
+        }
+        if (!have_encode_tiled())
+            return CR_ERR_NO_DEVICE;
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return CR_ERR_CUDA;
+        }
+        s.scratch = static_cast<uint8_t *>(p);
+        s.ready = true;
+    }
+    *out = &s;
+    return CR_OK;
+}
+}  // namespace
+
+cr_status cr_w4a8_linear_decode_noalloc(const uint16_t *x, const uint8_t *qdata, const uint8_t *srel,
+                                        const float *codebook, const float *s_channel, const float *bias,
+                                        int64_t M, int64_t N, int64_t K, int act_qmax, cr_out_dtype out_dtype,
+                                        void *out, cr_stream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0 || act_qmax < 1 || act_qmax > 127 ||
+        (out_dtype != CR_OUT_BF16 && out_dtype != CR_OUT_F32))
+        return CR_ERR_INVALID_ARG;
+    const cr_status k = check_k(K);
+    if (k != CR_OK)
+        return k;
+    if (M > CR_GEMV_MAX_M)
+        return CR_ERR_UNSUPPORTED;  // the padded activations would not fit the static scratch
+    if (M == 0 || N == 0)
+        return CR_OK;
+    int64_t MP = 1;
+    while (MP < M)
+        MP <<= 1;
+    if (MP * K > (int64_t)CR_GEMV_MAX_M * CR_MAX_K)
+        return CR_ERR_UNSUPPORTED;
+    if (!x || !qdata || !srel || !codebook || !s_channel || !out)
+        return CR_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(qdata) || !aligned16(srel) || !aligned16(codebook) || !aligned16(s_channel) ||
+        !aligned16(out) || (bias && !aligned16(bias)))
+        return CR_ERR_ALIGNMENT;
+    NoallocState *ns = nullptr;
+    const cr_status ss = noalloc_scratch(&ns);
+    if (ss != CR_OK)
+        return ss;
+    int8_t *xq = reinterpret_cast<int8_t *>(ns->scratch);
+    float *xs = reinterpret_cast<float *>(ns->scratch + (size_t)CR_GEMV_MAX_M * CR_MAX_K);
+    // The activation kernel rewrites every scratch byte the GEMV reads (rows
+    // M..MP-1 as zeros with scale 1), so nothing left by an earlier call leaks in.
+    cr_status st = launched(cr::rq::launch(x, M, K, MP, act_qmax, xq, xs, stream));
+    if (st != CR_OK)
+        return st;
+    return run_gemv(ns->num_sms, ns->gemv_attr_set, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K,
+                    out_dtype, out, nullptr, stream, /*pdl=*/true);
+}
+
 cr_status cr_check_device_error(cr_stream_t stream)
 {
     DeviceState *d = nullptr;
