@@ -124,6 +124,14 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float y)
     return __bfloat16_as_ushort(__float2bfloat16_rn(y));
 }
 
+// Two values to a pair of bf16 (round to nearest even) in one conversion:
+// lo in bits 0-15, hi in bits 16-31.
+__device__ __forceinline__ uint32_t to_bf16x2_bits(float lo, float hi)
+{
+    const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&p);
+}
+
 // ---------------------------------------------------------------- loads
 
 // 16-byte streaming load that bypasses L1 (weights are read once).
@@ -248,6 +256,32 @@ __device__ __forceinline__ void prefetch_tmap(const void *tmap)
 {
     asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");
 }
+
+// Bulk tensor store of one box from shared memory (shared::cta source), in
+// the calling thread's bulk-async group.  Out-of-range parts of the box are
+// not written.
+__device__ __forceinline__ void tma_store_2d(const void *tmap, int32_t x, int32_t y, const void *smem_src)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(tmap), "r"(x),
+                 "r"(y), "r"(smem_u32(smem_src))
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until at most N committed bulk groups still read their shared-memory source.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read()
+{
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+
+// Wait until every committed bulk group has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Make this thread's generic-proxy shared-memory writes visible to the async
+// proxy (TMA) before a bulk copy reads them.
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ---------------------------------------------------------------- tcgen05 / TMEM
 

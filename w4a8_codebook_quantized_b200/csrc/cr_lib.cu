@@ -146,7 +146,7 @@ bool make_tmap_plain(CUtensorMap *map, const void *base, CUtensorMapDataType dty
 }
 
 // The decode GEMV: tensor maps over the packed codes (as 32-bit words, one
-// 512-byte row slice per stage row) and the scale bytes, a persistent grid of
+// row slice of a stage per box row) and the scale bytes, a persistent grid of
 // two CTAs per SM, optionally as a programmatic dependent of the previous
 // kernel on the stream.
 cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const uint8_t *qdata,
@@ -155,9 +155,10 @@ cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *x
                    bool pdl)
 {
     using namespace cr;
+    using C = gv::Prod;
     if (!attr_set) {
-        if (cudaFuncSetAttribute(gv::gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gv::kSmemBytes) != cudaSuccess) {
+        if (cudaFuncSetAttribute(gv::gemv_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)C::kSmemBytes) != cudaSuccess) {
             cudaGetLastError();
             return CR_ERR_CUDA;
         }
@@ -165,23 +166,23 @@ cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *x
     }
     CUtensorMap tc, ts;
     if (!make_tmap_plain(&tc, qdata, CU_TENSOR_MAP_DATA_TYPE_UINT32, (uint64_t)(K / 8), (uint64_t)N,
-                         (uint64_t)(K / 2), gv::kChunk / 8, gv::kRows) ||
+                         (uint64_t)(K / 2), C::kChunk / 8, gv::kRows) ||
         !make_tmap_plain(&ts, srel, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)(K / 16), (uint64_t)N,
-                         (uint64_t)(K / 16), gv::kChunk / 16, gv::kRows))
+                         (uint64_t)(K / 16), C::kChunk / 16, gv::kRows))
         return CR_ERR_CUDA;
     const int64_t tiles = (N + gv::kRows - 1) / gv::kRows;
     const int64_t grid = tiles < 2 * (int64_t)num_sms ? tiles : 2 * (int64_t)num_sms;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(gv::kThreads);
-    cfg.dynamicSmemBytes = gv::kSmemBytes;
+    cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return launched(cudaLaunchKernelEx(&cfg, gv::gemv_kernel, tc, ts, xq, xs, codebook, s_channel, bias, (int)M,
+    return launched(cudaLaunchKernelEx(&cfg, gv::gemv_kernel<C>, tc, ts, xq, xs, codebook, s_channel, bias, (int)M,
                                        (int)N, (int)K, out_dtype == CR_OUT_F32 ? 1 : 0, out, acc_out));
 }
 
@@ -230,17 +231,34 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
         return CR_ERR_CUDA;
     }
     cr_status st = launched(ew::launch_decode(qdata, srel, codebook, N, K, w8, d.num_sms, stream));
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, to;
+    const int out_f32 = out_dtype == CR_OUT_F32;
+    const int vec_ok = out_f32 ? (N % 4 == 0) : (N % 8 == 0);
+    // Output through TMA bulk stores when rows are 16-byte multiples and the
+    // int32 accumulators are not requested: 32-row x 128-byte boxes, 128B swizzle.
+    const int tma_out = vec_ok && acc_out == nullptr;
     if (st == CR_OK && (!make_tmap_i8(&ta, xq, (uint64_t)K, (uint64_t)M, (uint32_t)gm::BM) ||
                         !make_tmap_i8(&tb, w8, (uint64_t)K, (uint64_t)N, (uint32_t)gm::BN)))
         st = CR_ERR_CUDA;
     if (st == CR_OK) {
+        to = ta;  // placeholder when the output does not go through TMA
+        if (tma_out) {
+            const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+            const cuuint64_t strides[1] = {(cuuint64_t)N * (out_f32 ? 4u : 2u)};
+            const cuuint32_t box[2] = {out_f32 ? 32u : 64u, 32u};
+            const cuuint32_t estr[2] = {1u, 1u};
+            if (g_encode_tiled(&to, out_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out,
+                               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                st = CR_ERR_CUDA;
+        }
+    }
+    if (st == CR_OK) {
         const int64_t tiles = ((M + gm::BM - 1) / gm::BM) * ((N + gm::BN - 1) / gm::BN);
         const int grid = (int)(tiles < d.num_sms ? tiles : d.num_sms);
-        const int out_f32 = out_dtype == CR_OUT_F32;
-        const int vec_ok = out_f32 ? (N % 4 == 0) : (N % 8 == 0);
-        gm::gemm_kernel<<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(ta, tb, xs, s_channel, bias, (int)M, (int)N,
-                                                                         (int)K, out_f32, vec_ok, out, acc_out);
+        gm::gemm_kernel<<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(ta, tb, to, xs, s_channel, bias, (int)M,
+                                                                         (int)N, (int)K, out_f32, vec_ok, tma_out, out,
+                                                                         acc_out);
         st = launched(cudaGetLastError());
     }
     if (cudaFreeAsync(w8, stream) != cudaSuccess) {

@@ -38,8 +38,13 @@ constexpr int kTmemCols = 2 * BN;             // two accumulators
 constexpr int kThreads = 192;
 constexpr uint32_t kIdesc = idesc_i8(BM, BN);
 
+constexpr int kEpiBytes = 32 * 128;  // one epilogue store unit: 32 rows x 128 bytes
+
 struct __align__(1024) Smem {
     uint8_t stage[kStages][kStageBytes];  // A at +0, B at +kABytes; every buffer 1024-aligned
+    uint8_t epi[4][kEpiBytes];            // per epilogue warp, one 128B-swizzled staging unit
+    float wsb[2][BN];                     // per-tile channel scales (double-buffered by tile parity)
+    float biasb[2][BN];                   // per-tile bias
     uint64_t full[kStages];
     uint64_t empty[kStages];
     uint64_t tmem_full[2];
@@ -58,8 +63,9 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_n, int &tm, int 
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const float *__restrict__ xs, const float *__restrict__ ws, const float *__restrict__ bias, int M,
-                int N, int K, int out_f32, int vec_ok, void *__restrict__ out, int32_t *__restrict__ acc_out)
+                const __grid_constant__ CUtensorMap tmOut, const float *__restrict__ xs,
+                const float *__restrict__ ws, const float *__restrict__ bias, int M, int N, int K, int out_f32,
+                int vec_ok, int tma_out, void *__restrict__ out, int32_t *__restrict__ acc_out)
 {
     extern __shared__ uint8_t smem_raw[];
     Smem &sh = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -174,80 +180,169 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------ epilogue (warps 2..5)
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        // Warp q owns TMEM lanes 32q..32q+31 = rows 32q.. of the tile.
+        // Per tile: the 128 epilogue threads stage the tile's channel scales
+        // (and bias) in shared memory before waiting for the accumulator, so
+        // that latency hides under the MMAs.  The accumulator is read 32
+        // columns at a time, the next chunk's TMEM load in flight while the
+        // current one is converted.  Fast path (tma_out): each 128-byte column
+        // unit (64 bf16 or 32 fp32 columns) of the warp's 32 rows goes into a
+        // 128B-swizzled staging buffer (16-byte chunk c of row r at chunk
+        // c ^ (r % 8): conflict-free) and leaves with one TMA bulk store.  Otherwise (int32 accumulators requested, or rows
+        // not 16-byte multiples) each thread stores its own row.
+        // The loop never exits early: after an abort every warp still reaches
+        // the same named barriers, skipping the work.
+        const int q = warp & 3;
+        const int et = threadIdx.x - 64;  // 0..127 among the epilogue threads
         int local = 0;
+        uint32_t units_issued = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++local) {
             int tm, tn;
             tile_coords(tile, tiles_n, tm, tn);
             const int buf = local & 1;
             const uint32_t use = (uint32_t)(local >> 1) & 1u;
-            if (!mbar_wait_bounded_warp(&sh.tmem_full[buf], use, abort))
-                break;
+            for (int j = et; j < BN; j += 128) {
+                const int n = tn * BN + j;
+                sh.wsb[buf][j] = n < N ? ws[n] : 0.0f;
+                sh.biasb[buf][j] = (bias != nullptr && n < N) ? bias[n] : 0.0f;
+            }
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+            const bool ok = mbar_wait_bounded_warp(&sh.tmem_full[buf], use, abort);
+            if (!ok)
+                continue;
             tc_fence_after();
             const int row = tm * BM + 32 * q + lane;
             const bool row_ok = row < M;
             const float xm = row_ok ? xs[row] : 0.0f;
             const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN);
-            for (int ch = 0; ch < BN / 32; ++ch) {
-                uint32_t r[32];
-                __syncwarp();  // the TMEM load below is warp-collective
-                tmem_ld_32cols(tbase + (uint32_t)(32 * ch), r);
-                tmem_ld_wait();
-                const int col0 = tn * BN + 32 * ch;
-                const int64_t base = (int64_t)row * N + col0;
-                if (!row_ok || col0 >= N) {
-                    // nothing of this row/column chunk is in range
-                } else if (vec_ok && col0 + 32 <= N) {
-                    float y[32];
+            const float *wsv = sh.wsb[buf];
+            const float *bsv = sh.biasb[buf];
+            const bool has_bias = bias != nullptr;
+            // 32 accumulators of columns [c0, c0 + 32) of the tile -> 32 fp32 or 16 bf16x2 words
+            auto convert32 = [&](const uint32_t (&v)[32], int c0, uint32_t *dst) {
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        const float4 w4 = __ldg(reinterpret_cast<const float4 *>(ws + col0 + j));
-                        const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 w4 = *reinterpret_cast<const float4 *>(wsv + c0 + j);
+                    const float4 b4 = *reinterpret_cast<const float4 *>(bsv + c0 + j);
+                    const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+                    const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+                    float y[4];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            y[j + u] = epilogue_value((int32_t)r[j + u], xm, wv[u], bias, col0 + j + u);
+                    for (int e = 0; e < 4; ++e) {
+                        y[e] = __fmul_rn(__int2float_rn((int32_t)v[j + e]), __fmul_rn(xm, wv[e]));
+                        if (has_bias)
+                            y[e] = __fadd_rn(y[e], bv[e]);
                     }
                     if (out_f32) {
-                        float4 *o = reinterpret_cast<float4 *>(reinterpret_cast<float *>(out) + base);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            o[j] = make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+                        for (int e = 0; e < 4; ++e)
+                            dst[j + e] = __float_as_uint(y[e]);
                     } else {
-                        uint4 *o = reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(out) + base);
+                        dst[j / 2] = to_bf16x2_bits(y[0], y[1]);
+                        dst[j / 2 + 1] = to_bf16x2_bits(y[2], y[3]);
+                    }
+                }
+            };
+            // one 128-byte unit of the warp's 32 rows -> staging buffer -> TMA bulk store
+            auto store_unit = [&](const uint32_t (&p)[32], int ucol0) {
+                if (units_issued >= 1) {
+                    if (lane == 0)
+                        bulk_wait_read<0>();  // the previous store has read the staging buffer
+                    __syncwarp();
+                }
+                uint8_t *stg = sh.epi[q];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint32_t p[4];
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(stg + lane * 128 + ((c ^ (lane & 7)) * 16)) =
+                        make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmOut, ucol0, tm * BM + 32 * q, stg);
+                    bulk_commit();
+                }
+                ++units_issued;
+            };
+            auto release_accumulator = [&]() {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&sh.tmem_empty[buf]);
+            };
+            uint32_t cur[32], nxt[32], packed[32];
+            __syncwarp();
+            tmem_ld_32cols(tbase, cur);
+            tmem_ld_wait();
+            if (tma_out && !out_f32) {
+                // units of 64 columns: two 32-column chunks each
+                for (int u = 0; u < BN / 64; ++u) {
+                    __syncwarp();
+                    tmem_ld_32cols(tbase + (uint32_t)(64 * u + 32), nxt);
+                    convert32(cur, 64 * u, packed);
+                    tmem_ld_wait();
+                    if (u + 1 < BN / 64) {
+                        __syncwarp();
+                        tmem_ld_32cols(tbase + (uint32_t)(64 * u + 64), cur);
+                    } else {
+                        release_accumulator();
+                    }
+                    convert32(nxt, 64 * u + 32, packed + 16);
+                    store_unit(packed, tn * BN + 64 * u);
+                    if (u + 1 < BN / 64)
+                        tmem_ld_wait();
+                }
+            } else if (tma_out) {
+                // units of 32 fp32 columns
+                for (int u = 0; u < BN / 32; ++u) {
+                    if (u + 1 < BN / 32) {
+                        __syncwarp();
+                        tmem_ld_32cols(tbase + (uint32_t)(32 * u + 32), nxt);
+                    } else {
+                        release_accumulator();
+                    }
+                    convert32(cur, 32 * u, packed);
+                    store_unit(packed, tn * BN + 32 * u);
+                    if (u + 1 < BN / 32) {
+                        tmem_ld_wait();
 #pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                p[u] = (uint32_t)to_bf16_bits(y[8 * j + 2 * u]) |
-                                       ((uint32_t)to_bf16_bits(y[8 * j + 2 * u + 1]) << 16);
-                            o[j] = make_uint4(p[0], p[1], p[2], p[3]);
+                        for (int j = 0; j < 32; ++j)
+                            cur[j] = nxt[j];
+                    }
+                }
+            } else {
+                for (int ch = 0; ch < BN / 32; ++ch) {
+                    if (ch + 1 < BN / 32) {
+                        __syncwarp();
+                        tmem_ld_32cols(tbase + (uint32_t)(32 * (ch + 1)), nxt);
+                    } else {
+                        release_accumulator();
+                    }
+                    const int col0 = tn * BN + 32 * ch;
+                    if (row_ok && col0 < N) {
+                        const int64_t base = (int64_t)row * N + col0;
+                        for (int j = 0; j < 32 && col0 + j < N; ++j) {
+                            const int n = col0 + j;
+                            const float y = epilogue_value((int32_t)cur[j], xm, ws[n], bias, n);
+                            if (out_f32)
+                                reinterpret_cast<float *>(out)[base + j] = y;
+                            else
+                                reinterpret_cast<uint16_t *>(out)[base + j] = to_bf16_bits(y);
+                            if (acc_out != nullptr)
+                                acc_out[base + j] = (int32_t)cur[j];
                         }
                     }
-                    if (acc_out != nullptr) {
-                        uint4 *o = reinterpret_cast<uint4 *>(acc_out + base);
+                    if (ch + 1 < BN / 32) {
+                        tmem_ld_wait();
 #pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            o[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-                    }
-                } else {
-                    for (int j = 0; j < 32 && col0 + j < N; ++j) {
-                        const int n = col0 + j;
-                        const float y = epilogue_value((int32_t)r[j], xm, ws[n], bias, n);
-                        if (out_f32)
-                            reinterpret_cast<float *>(out)[base + j] = y;
-                        else
-                            reinterpret_cast<uint16_t *>(out)[base + j] = to_bf16_bits(y);
-                        if (acc_out != nullptr)
-                            acc_out[base + j] = (int32_t)r[j];
+                        for (int j = 0; j < 32; ++j)
+                            cur[j] = nxt[j];
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&sh.tmem_empty[buf]);
         }
+        if (lane == 0)
+            bulk_wait_all();  // every output store has landed before the CTA exits
+        __syncwarp();
     }
 
     tc_fence_before();

@@ -8,10 +8,10 @@
 //
 // B200 design.
 //  * Streaming: a persistent grid (two CTAs per SM).  In each CTA one
-//    producer warp moves 16-row x 1024-column tiles of the packed codes
-//    (8 KB) and their group scales (1 KB) into a 6-stage shared-memory ring
-//    with 2-D TMA copies; eight consumer warps decode and contract each stage
-//    while the following ones are in flight.  Bytes in flight are set by the
+//    producer warp moves 16-row x 2048-column tiles of the packed codes
+//    (16 KB) and their group scales (2 KB) into a 4-stage shared-memory ring
+//    with 2-D TMA copies; eight consumer warps (two 128-column slices each)
+//    decode and contract each stage while the following ones are in flight.  Bytes in flight are set by the
 //    ring, not by registers, which keeps HBM busy.
 //  * Decode: a per-CTA table of the 16 int8 levels of every fp8 scale byte
 //    (exact: the decoded value depends only on the pair), replicated 8 times
@@ -44,22 +44,31 @@ namespace gv {
 constexpr int kConsumerWarps = 8;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kRows = 16;                            // output rows per tile
-constexpr int kChunk = 1024;                         // k per stage
-constexpr int kStages = 6;
-constexpr int kCodeBytes = kRows * kChunk / 2;       // 8 KB
-constexpr int kSrelBytes = kRows * kChunk / 16;      // 1 KB
 
-struct __align__(1024) Smem {
-    uint8_t codes[kStages][kCodeBytes];  // row r of a stage at r * 512 bytes
-    uint8_t srel[kStages][kSrelBytes];   // row r of a stage at r * 64 bytes
-    uint4 lut8[256 * 8];                 // lut8[s * 8 + c]: copy c of the levels of scale byte s
-    int32_t red[kConsumerWarps][kRows][8];
-    float cb[16];
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
-    int abort;
+// Shape of one pipeline stage: every consumer warp takes SLICES slices of 128
+// k per stage, so a stage covers CHUNK = 8 * SLICES * 128 columns of 16 rows.
+template <int SLICES, int STAGES>
+struct Cfg {
+    static constexpr int kSlices = SLICES;
+    static constexpr int kStages = STAGES;
+    static constexpr int kChunk = kConsumerWarps * SLICES * 128;
+    static constexpr int kCodeBytes = kRows * kChunk / 2;
+    static constexpr int kSrelBytes = kRows * kChunk / 16;
+    struct __align__(1024) Smem {
+        uint8_t codes[STAGES][kCodeBytes];  // row r of a stage at r * kChunk / 2 bytes
+        uint8_t srel[STAGES][kSrelBytes];   // row r of a stage at r * kChunk / 16 bytes
+        uint4 lut8[256 * 8];                // lut8[s * 8 + c]: copy c of the levels of scale byte s
+        int32_t red[kConsumerWarps][kRows][8];
+        float cb[16];
+        uint64_t full[STAGES];
+        uint64_t empty[STAGES];
+        int abort;
+    };
+    static constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 };
-constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+
+// The configuration the library launches.
+using Prod = Cfg<2, 4>;
 
 __device__ __forceinline__ void mma_s8(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                        uint32_t b0, uint32_t b1)
@@ -73,21 +82,53 @@ __device__ __forceinline__ void mma_s8(int32_t (&c)[4], uint32_t a0, uint32_t a1
 
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
+// One slice: 16 rows x 128 k of this stage against the token fragments X0, X1.
+__device__ __forceinline__ void slice_mma(const uint8_t *codes_row_g, const uint8_t *codes_row_g8,
+                                          const uint8_t *srel_row_g, const uint8_t *srel_row_g8, const uint4 *lut8,
+                                          int copy, const uint4 &X0, const uint4 &X1, int32_t (&c)[4],
+                                          int32_t (&d)[4])
+{
+    const uint4 A = *reinterpret_cast<const uint4 *>(codes_row_g);
+    const uint4 B = *reinterpret_cast<const uint4 *>(codes_row_g8);
+    const uint32_t SA = *reinterpret_cast<const uint16_t *>(srel_row_g);
+    const uint32_t SB = *reinterpret_cast<const uint16_t *>(srel_row_g8);
+    const uint4 TA0 = lut8[(SA & 0xFFu) * 8 + copy];
+    const uint4 TA1 = lut8[(SA >> 8) * 8 + copy];
+    const uint4 TB0 = lut8[(SB & 0xFFu) * 8 + copy];
+    const uint4 TB1 = lut8[(SB >> 8) * 8 + copy];
+    uint32_t a0, a1, a2, a3, e0, e1, e2, e3;
+    decode8(A.x, TA0, a0, a2);
+    decode8(B.x, TB0, a1, a3);
+    decode8(A.y, TA0, e0, e2);
+    decode8(B.y, TB0, e1, e3);
+    mma_s8(c, a0, a1, a2, a3, X0.x, X0.y);
+    mma_s8(d, e0, e1, e2, e3, X0.z, X0.w);
+    decode8(A.z, TA1, a0, a2);
+    decode8(B.z, TB1, a1, a3);
+    decode8(A.w, TA1, e0, e2);
+    decode8(B.w, TB1, e1, e3);
+    mma_s8(c, a0, a1, a2, a3, X1.x, X1.y);
+    mma_s8(d, e0, e1, e2, e3, X1.z, X1.w);
+}
+
+template <class C>
 __global__ void __launch_bounds__(kThreads, 2)
     gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_srel,
                 const int8_t *__restrict__ xq, const float *__restrict__ xs, const float *__restrict__ codebook,
                 const float *__restrict__ ws, const float *__restrict__ bias, int M, int N, int K, int out_f32,
                 void *__restrict__ out, int32_t *__restrict__ acc_out)
 {
+    constexpr int S = C::kSlices, STAGES = C::kStages, CHUNK = C::kChunk;
+    using Smem = typename C::Smem;
     extern __shared__ uint8_t smem_raw[];
     Smem &sh = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int ntiles = (N + kRows - 1) / kRows;
-    const int nchunks = (K + kChunk - 1) / kChunk;
+    const int nchunks = (K + CHUNK - 1) / CHUNK;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(&sh.full[s], 1);
             mbar_init(&sh.empty[s], kConsumerWarps);
         }
@@ -107,9 +148,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             prefetch_tmap(&tm_srel);
             int stage = 0;
             uint32_t phase = 0;
-            int issued[kStages];
-            uint32_t issued_phase[kStages];
-            for (int s = 0; s < kStages; ++s)
+            int issued[STAGES];
+            uint32_t issued_phase[STAGES];
+            for (int s = 0; s < STAGES; ++s)
                 issued[s] = 0, issued_phase[s] = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
@@ -118,19 +159,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&sh.full[stage], kCodeBytes + kSrelBytes);
-                    tma_load_2d(sh.codes[stage], &tm_codes, c * (kChunk / 8), tile * kRows, &sh.full[stage]);
-                    tma_load_2d(sh.srel[stage], &tm_srel, c * (kChunk / 16), tile * kRows, &sh.full[stage]);
+                    mbar_arrive_expect_tx(&sh.full[stage], C::kCodeBytes + C::kSrelBytes);
+                    tma_load_2d(sh.codes[stage], &tm_codes, c * (CHUNK / 8), tile * kRows, &sh.full[stage]);
+                    tma_load_2d(sh.srel[stage], &tm_srel, c * (CHUNK / 16), tile * kRows, &sh.full[stage]);
                     issued[stage] = 1;
                     issued_phase[stage] = phase;
-                    if (++stage == kStages) {
+                    if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
             }
             if (!ok) {
-                for (int s = 0; s < kStages; ++s)
+                for (int s = 0; s < STAGES; ++s)
                     if (issued[s]) {
                         volatile int no_abort = 0;
                         mbar_wait_bounded(&sh.full[s], issued_phase[s], &no_abort, 20000000ull);
@@ -151,53 +192,62 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int g = lane >> 2, t = lane & 3;
         const int copy = lane & 7;
         const bool vx = g < M;
+        // slice j of this warp in a stage: k offset 128 * (warp + 8 j) in the chunk
         const int8_t *px = xq + (int64_t)g * K + 128 * warp + 32 * t;
         const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+        // The activation fragments of a chunk do not depend on the row tile;
+        // the next chunk's are fetched (through L1/L2) while the current one
+        // is computed, in the order the chunks are consumed.
+        auto fetch_x = [&](int ch, uint4 (&X)[S][2]) {
+#pragma unroll
+            for (int j = 0; j < S; ++j) {
+                X[j][0] = X[j][1] = z4;
+                const int k0 = ch * CHUNK + 128 * (warp + 8 * j);
+                if (vx && k0 < K) {
+                    X[j][0] = *reinterpret_cast<const uint4 *>(px + (int64_t)ch * CHUNK + 1024 * j);
+                    X[j][1] = *reinterpret_cast<const uint4 *>(px + (int64_t)ch * CHUNK + 1024 * j + 16);
+                }
+            }
+        };
+        uint4 Xc[S][2], Xn[S][2];
+        fetch_x(0, Xn);
+        int xch = 0;  // chunk index of Xn
         int stage = 0;
         uint32_t phase = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            int32_t c[4] = {0, 0, 0, 0};
+            // two accumulators break the dependency chain between the MMAs of a slice
+            int32_t c[4] = {0, 0, 0, 0}, d[4] = {0, 0, 0, 0};
             for (int ch = 0; ch < nchunks; ++ch) {
-                const bool active = ch * kChunk + 128 * warp < K;  // this warp's slice exists
-                uint4 X0 = z4, X1 = z4;
-                if (active && vx) {
-                    X0 = *reinterpret_cast<const uint4 *>(px + (int64_t)ch * kChunk);
-                    X1 = *reinterpret_cast<const uint4 *>(px + (int64_t)ch * kChunk + 16);
-                }
+#pragma unroll
+                for (int j = 0; j < S; ++j)
+                    Xc[j][0] = Xn[j][0], Xc[j][1] = Xn[j][1];
+                if (++xch == nchunks)
+                    xch = 0;
+                fetch_x(xch, Xn);
                 const bool ok = mbar_wait_bounded_warp(&sh.full[stage], phase, abort);
-                if (ok && active) {
-                    const uint8_t *cs = sh.codes[stage] + 64 * warp + 16 * t;
-                    const uint4 A = *reinterpret_cast<const uint4 *>(cs + 512 * g);
-                    const uint4 B = *reinterpret_cast<const uint4 *>(cs + 512 * (g + 8));
-                    const uint8_t *ss = sh.srel[stage] + 8 * warp + 2 * t;
-                    const uint32_t SA = *reinterpret_cast<const uint16_t *>(ss + 64 * g);
-                    const uint32_t SB = *reinterpret_cast<const uint16_t *>(ss + 64 * (g + 8));
-                    const uint4 TA0 = sh.lut8[(SA & 0xFFu) * 8 + copy];
-                    const uint4 TA1 = sh.lut8[(SA >> 8) * 8 + copy];
-                    const uint4 TB0 = sh.lut8[(SB & 0xFFu) * 8 + copy];
-                    const uint4 TB1 = sh.lut8[(SB >> 8) * 8 + copy];
-                    uint32_t a0, a1, a2, a3;
-                    decode8(A.x, TA0, a0, a2);
-                    decode8(B.x, TB0, a1, a3);
-                    mma_s8(c, a0, a1, a2, a3, X0.x, X0.y);
-                    decode8(A.y, TA0, a0, a2);
-                    decode8(B.y, TB0, a1, a3);
-                    mma_s8(c, a0, a1, a2, a3, X0.z, X0.w);
-                    decode8(A.z, TA1, a0, a2);
-                    decode8(B.z, TB1, a1, a3);
-                    mma_s8(c, a0, a1, a2, a3, X1.x, X1.y);
-                    decode8(A.w, TA1, a0, a2);
-                    decode8(B.w, TB1, a1, a3);
-                    mma_s8(c, a0, a1, a2, a3, X1.z, X1.w);
+                if (ok) {
+#pragma unroll
+                    for (int j = 0; j < S; ++j) {
+                        const int sl = warp + 8 * j;
+                        if (ch * CHUNK + 128 * sl < K) {
+                            const uint8_t *cs = sh.codes[stage] + 64 * sl + 16 * t;
+                            const uint8_t *ss = sh.srel[stage] + 8 * sl + 2 * t;
+                            slice_mma(cs + (CHUNK / 2) * g, cs + (CHUNK / 2) * (g + 8), ss + (CHUNK / 16) * g,
+                                      ss + (CHUNK / 16) * (g + 8), sh.lut8, copy, Xc[j][0], Xc[j][1], c, d);
+                        }
+                    }
                 }
                 __syncwarp();
                 if (ok && lane == 0)
                     mbar_arrive(&sh.empty[stage]);
-                if (++stage == kStages) {
+                if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1u;
                 }
             }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                c[i] += d[i];
             // C fragment: c0 (row g, token 2t), c1 (g, 2t+1), c2 (g+8, 2t), c3 (g+8, 2t+1)
             sh.red[warp][g][2 * t] = c[0];
             sh.red[warp][g][2 * t + 1] = c[1];

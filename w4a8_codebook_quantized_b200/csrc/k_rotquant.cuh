@@ -52,7 +52,7 @@ __device__ __forceinline__ void h4_quad(float &a0, float &a1, float &a2, float &
 }
 
 // Rotate one 256-element block.  On return lane L of the half-warp holds
-// v[a] = rotated element 16a + L (a = 0..15).  `tr` is this half-warp's
+// v[a] = 16 x rotated element 16a + L (a = 0..15).  `tr` is this half-warp's
 // 16 x 16 fp32 transpose buffer (16-byte aligned).
 __device__ __forceinline__ void rotate_block(const uint16_t *__restrict__ blk, int L, float *tr, unsigned hmask,
                                              float (&v)[16])
@@ -84,9 +84,15 @@ __device__ __forceinline__ void rotate_block(const uint16_t *__restrict__ blk, i
             rowp[c ^ sw] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
     }
     __syncwarp(hmask);
+    {
+        const float *base[4];
 #pragma unroll
-    for (int a = 0; a < 16; ++a)
-        v[a] = tr[16 * a + 4 * ((L >> 2) ^ ((a >> 1) & 3)) + (L & 3)];
+        for (int k = 0; k < 4; ++k)
+            base[k] = tr + 4 * ((L >> 2) ^ k) + (L & 3);
+#pragma unroll
+        for (int a = 0; a < 16; ++a)
+            v[a] = base[(a >> 1) & 3][16 * a];
+    }
     __syncwarp(hmask);
     // stride 16 (digit d2 = a % 4), then stride 64 (digit d3 = a / 4)
 #pragma unroll
@@ -95,41 +101,60 @@ __device__ __forceinline__ void rotate_block(const uint16_t *__restrict__ blk, i
 #pragma unroll
     for (int q = 0; q < 4; ++q)
         h4_quad(v[q], v[q + 4], v[q + 8], v[q + 12]);
-#pragma unroll
-    for (int i = 0; i < 16; ++i)
-        v[i] = __fmul_rn(v[i], 0.0625f);
+    // The final 1/16 is not applied here: v holds R = 16 r.  Scaling by a power
+    // of two commutes with rounding away from subnormals, so the quantiser
+    // works on R with the scale multiplied by 16 and gets the same integers
+    // (rows whose values reach the subnormal range take an exact path that
+    // applies the 1/16 per element).
 }
 
-// rint(r / s) clamped to +-qmax, without a per-element division.
+// Quantise this lane's 16 column values of one block and store them in row
+// order.  v holds R = 16 r (see rotate_block); scale is s, the row's scale.
 //
-// inv = 1/s rounded once per row.  When s is a normal fp32 and |r| <= amax,
-// t = r * inv differs from the correctly rounded quotient v = r / s by at most
-// 3 * 2^-24 * |r / s| <= 3 * 2^-24 * 128 < 2^-15.  So unless t lies within 2^-15
-// of a half-integer, t and v round to the same integer and neither is a tie;
-// in that rare case the quotient is computed exactly and rounded.  Adding
-// 1.5 * 2^23 rounds t to an integer (nearest even) in the low mantissa bits
-// (valid for |t| < 2^22), which also yields the integer without a conversion.
-// `exact_only` (a subnormal s) takes the exact path for every element.
-__device__ __forceinline__ int32_t quantise_one(float r, float s, float inv, int32_t qmax, bool exact_only)
-{
-    const float kMagic = 12582912.0f;  // 1.5 * 2^23
-    const float t = __fmul_rn(r, inv);
-    const float tm = __fadd_rn(t, kMagic);
-    const float rt = __fsub_rn(tm, kMagic);
-    int32_t q = __float_as_int(tm) - 0x4B400000;
-    if (exact_only || fabsf(__fsub_rn(t, rt)) >= 0.499969482421875f)  // within 2^-15 of k + 1/2
-        q = __float2int_rn(__fdiv_rn(r, s));
-    return min(max(q, -qmax), qmax);
-}
-
-// Quantise this lane's 16 column values of block b and store them in row order.
-__device__ __forceinline__ void quantise_store(const float (&v)[16], float scale, float inv, int32_t qmax,
-                                               bool exact_only, int L, uint8_t *tb, unsigned hmask,
+// Fast path (any row whose max |r| >= 2^-100): q = rint(r / s) without a
+// per-element division.  inv16 = (1/s rounded) / 16, so t = R * inv16 equals
+// r * (1/s rounded) rounded; it differs from the correctly rounded quotient
+// v = r / s by at most 3 * 2^-24 * |r / s| <= 3 * 2^-24 * 128 < 2^-15.  Unless t
+// lies within 2^-15 of a half-integer, t and v round to the same integer and
+// neither is a tie; those rare elements are redone with the exact quotient
+// R / (16 s).  Adding 1.5 * 2^23 rounds t to an integer (nearest even) in the
+// low mantissa bits, whose low byte is the two's-complement int8 result.  No
+// clamp is needed: |t| <= qmax + 2^-15 cannot round past qmax.
+//
+// Exact path (a row of tiny values, max |r| < 2^-100): r = R / 16 rounded per
+// element (it may be subnormal), q = rint(r / s) with the division, clamped.
+__device__ __forceinline__ void quantise_store(const float (&v)[16], float scale, float inv16, int32_t qmax,
+                                               bool exact_row, int L, uint8_t *tb, unsigned hmask,
                                                int8_t *__restrict__ dst_block)
 {
+    const float kMagic = 12582912.0f;  // 1.5 * 2^23
+    if (!exact_row) {
+        uint32_t near = 0;
 #pragma unroll
-    for (int a = 0; a < 16; ++a)
-        tb[16 * a + L] = (uint8_t)quantise_one(v[a], scale, inv, qmax, exact_only);
+        for (int a = 0; a < 16; ++a) {
+            const float t = __fmul_rn(v[a], inv16);
+            const float tm = __fadd_rn(t, kMagic);
+            const float d = __fsub_rn(t, __fsub_rn(tm, kMagic));
+            near |= (fabsf(d) >= 0.499969482421875f ? 1u : 0u) << a;  // within 2^-15 of k + 1/2
+            tb[16 * a + L] = (uint8_t)__float_as_uint(tm);
+        }
+        if (near) {
+            const float s16 = __fmul_rn(scale, 16.0f);
+#pragma unroll
+            for (int a = 0; a < 16; ++a)
+                if ((near >> a) & 1u) {
+                    const int32_t q = __float2int_rn(__fdiv_rn(v[a], s16));
+                    tb[16 * a + L] = (uint8_t)min(max(q, -qmax), qmax);
+                }
+        }
+    } else {
+#pragma unroll
+        for (int a = 0; a < 16; ++a) {
+            const float r = __fmul_rn(v[a], 0.0625f);
+            const int32_t q = __float2int_rn(__fdiv_rn(r, scale));
+            tb[16 * a + L] = (uint8_t)min(max(q, -qmax), qmax);
+        }
+    }
     __syncwarp(hmask);
     const uint4 o = *reinterpret_cast<const uint4 *>(tb + 16 * L);
     *reinterpret_cast<uint4 *>(dst_block + 16 * L) = o;
@@ -203,21 +228,24 @@ __global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__re
 #pragma unroll
     for (int w = 1; w < kThreads / 32; ++w)
         rmax = fmaxf(rmax, warp_max[w]);
-    const float scale = (rmax > 0.0f) ? __fdiv_rn(rmax, (float)qmax) : 1.0f;
-    const float inv = __frcp_rn(scale);
-    const bool exact_only = scale < 1.17549435e-38f;  // subnormal scale: 1/s may be inexact or overflow
+    // rmax is max |R| = 16 max |r|; the row maximum of r is rmax / 16 rounded
+    // (rounding is monotonic, so that is also the max of the rounded r).
+    const float rowmax = __fmul_rn(rmax, 0.0625f);
+    const float scale = (rowmax > 0.0f) ? __fdiv_rn(rowmax, (float)qmax) : 1.0f;
+    const bool exact_row = rowmax > 0.0f && rowmax < 7.8886091e-31f;  // max |r| < 2^-100
+    const float inv16 = __fmul_rn(__frcp_rn(scale), 0.0625f);
 
     if (!kRecompute) {
 #pragma unroll
         for (int j = 0; j < J; ++j) {
             const int b = hw + kHalfWarps * j;
             if (b < NB)
-                quantise_store(v[j], scale, inv, qmax, exact_only, L, tb, hmask, qrow + 256 * b);
+                quantise_store(v[j], scale, inv16, qmax, exact_row, L, tb, hmask, qrow + 256 * b);
         }
     } else {
         for (int b = hw; b < NB; b += kHalfWarps) {
             rotate_block(xrow + 256 * b, L, tr, hmask, v[0]);
-            quantise_store(v[0], scale, inv, qmax, exact_only, L, tb, hmask, qrow + 256 * b);
+            quantise_store(v[0], scale, inv16, qmax, exact_row, L, tb, hmask, qrow + 256 * b);
         }
     }
     if (tid == 0)
