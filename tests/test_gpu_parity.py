@@ -155,6 +155,14 @@ def test_gemm(M, N, K):
     _contraction_case(cr.cr_w4a8_gemm, M, N, K, seed=M + N + K)
 
 
+@pytest.mark.parametrize("M,N,K", [(2048, 4096, 512), (2000, 4000, 768), (4096, 2560, 256), (1100, 9000, 256),
+                                   (4352, 2304, 512)])
+def test_gemm_cta_pairs(M, N, K):
+    """Shapes with at least one 256 x 256 tile per SM pair take the CTA-pair
+    tcgen05 kernel (M = 256 per pair); ragged M and N included."""
+    _contraction_case(cr.cr_w4a8_gemm, M, N, K, seed=M + N + K, with_bias=(K == 768))
+
+
 @pytest.mark.parametrize("kind,with_bias", [("f32", False), ("f32", True), ("bf16", True)])
 def test_output_kinds_and_bias(kind, with_bias):
     _contraction_case(cr.cr_w4a8_gemv, 3, 520, 1024, 11, kind, with_bias)

@@ -28,6 +28,7 @@ struct DeviceState {
     int num_sms = 0;
     cudaMemPool_t pool = nullptr;  // stream-ordered pool for the prefill weight transient
     bool gemm_attr_set = false;
+    bool gemm_pair_attr_set = false;
     bool gemv_attr_set = false;
 };
 
@@ -147,7 +148,7 @@ bool make_tmap_plain(CUtensorMap *map, const void *base, CUtensorMapDataType dty
 
 // The decode GEMV: tensor maps over the packed codes (as 32-bit words, one
 // row slice of a stage per box row) and the scale bytes, a persistent grid of
-// two CTAs per SM, optionally as a programmatic dependent of the previous
+// as many CTAs as fit on the SMs, optionally as a programmatic dependent of the previous
 // kernel on the stream.
 cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const uint8_t *qdata,
                    const uint8_t *srel, const float *codebook, const float *s_channel, const float *bias, int64_t M,
@@ -166,12 +167,13 @@ cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *x
     }
     CUtensorMap tc, ts;
     if (!make_tmap_plain(&tc, qdata, CU_TENSOR_MAP_DATA_TYPE_UINT32, (uint64_t)(K / 8), (uint64_t)N,
-                         (uint64_t)(K / 2), C::kChunk / 8, gv::kRows) ||
+                         (uint64_t)(K / 2), C::kChunk / 8, C::kRows) ||
         !make_tmap_plain(&ts, srel, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)(K / 16), (uint64_t)N,
-                         (uint64_t)(K / 16), C::kChunk / 16, gv::kRows))
+                         (uint64_t)(K / 16), C::kChunk / 16, C::kRows))
         return CR_ERR_CUDA;
-    const int64_t tiles = (N + gv::kRows - 1) / gv::kRows;
-    const int64_t grid = tiles < 2 * (int64_t)num_sms ? tiles : 2 * (int64_t)num_sms;
+    const int64_t tiles = (N + C::kRows - 1) / C::kRows;
+    const int64_t slots = (int64_t)C::kMinBlocks * num_sms;
+    const int64_t grid = tiles < slots ? tiles : slots;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(gv::kThreads);
@@ -253,7 +255,41 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
                 st = CR_ERR_CUDA;
         }
     }
-    if (st == CR_OK) {
+    // 256 x 256 tiles on CTA pairs when there is at least one per SM pair;
+    // otherwise 128 x 256 tiles on single CTAs.
+    const int64_t pair_tiles = ((M + 255) / 256) * ((N + gm::BN - 1) / gm::BN);
+    const bool use_pair = pair_tiles >= d.num_sms / 2;
+    if (st == CR_OK && use_pair) {
+        CUtensorMap tb_half;
+        if (!d.gemm_pair_attr_set) {
+            if (cudaFuncSetAttribute(gm::gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)gm::pair::kSmemBytes) != cudaSuccess) {
+                cudaGetLastError();
+                st = CR_ERR_CUDA;
+            } else {
+                d.gemm_pair_attr_set = true;
+            }
+        }
+        if (st == CR_OK && !make_tmap_i8(&tb_half, w8, (uint64_t)K, (uint64_t)N, 128u))
+            st = CR_ERR_CUDA;
+        if (st == CR_OK) {
+            const int64_t pairs = pair_tiles < d.num_sms / 2 ? pair_tiles : d.num_sms / 2;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)(2 * pairs));
+            cfg.blockDim = dim3(gm::kThreads);
+            cfg.dynamicSmemBytes = gm::pair::kSmemBytes;
+            cfg.stream = stream;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            st = launched(cudaLaunchKernelEx(&cfg, gm::gemm_pair_kernel, ta, tb_half, to, xs, s_channel, bias, (int)M,
+                                             (int)N, (int)K, out_f32, vec_ok, tma_out, out, acc_out));
+        }
+    } else if (st == CR_OK) {
         const int64_t tiles = ((M + gm::BM - 1) / gm::BM) * ((N + gm::BN - 1) / gm::BN);
         const int grid = (int)(tiles < d.num_sms ? tiles : d.num_sms);
         gm::gemm_kernel<<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(ta, tb, to, xs, s_channel, bias, (int)M,

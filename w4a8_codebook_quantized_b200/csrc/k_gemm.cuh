@@ -61,6 +61,141 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_n, int &tm, int 
     tn = tile - tm * tiles_n;
 }
 
+// Epilogue of one 128 x 256 accumulator tile for one warp: its 32 TMEM lanes
+// are rows row0 + lane; `tbase` addresses lane 0 of the warp's quarter at the
+// tile's first column; the output columns are col_base + [0, 256).  Fast path
+// (tma_out): 128-byte column units (64 bf16 or 32 fp32 columns) go through the
+// 128B-swizzled staging buffer `stage_buf` (16-byte chunk c of row r at chunk
+// c ^ (r % 8): conflict-free) and one TMA bulk store each; the next 32-column
+// TMEM load is in flight while the current chunk is converted.  Otherwise each
+// thread stores its own row.  release() hands the accumulator back once every
+// column is in registers.
+template <class Release>
+__device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row0, int col_base, int lane, float xm, bool row_ok,
+                                              const float *wsv, const float *bsv, bool has_bias, int M, int N,
+                                              int out_f32, int tma_out, const CUtensorMap *tmOut, uint8_t *stage_buf,
+                                              uint32_t &units_issued, void *__restrict__ out,
+                                              int32_t *__restrict__ acc_out, const float *__restrict__ ws,
+                                              const float *__restrict__ bias, Release release)
+{
+    const int row = row0 + lane;
+    // 32 accumulators of columns [c0, c0 + 32) of the tile -> 32 fp32 or 16 bf16x2 words
+    auto convert32 = [&](const uint32_t (&v)[32], int c0, uint32_t *dst) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+            const float4 w4 = *reinterpret_cast<const float4 *>(wsv + c0 + j);
+            const float4 b4 = *reinterpret_cast<const float4 *>(bsv + c0 + j);
+            const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+            const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+            float y[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                y[e] = __fmul_rn(__int2float_rn((int32_t)v[j + e]), __fmul_rn(xm, wv[e]));
+                if (has_bias)
+                    y[e] = __fadd_rn(y[e], bv[e]);
+            }
+            if (out_f32) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    dst[j + e] = __float_as_uint(y[e]);
+            } else {
+                dst[j / 2] = to_bf16x2_bits(y[0], y[1]);
+                dst[j / 2 + 1] = to_bf16x2_bits(y[2], y[3]);
+            }
+        }
+    };
+    // one 128-byte unit of the warp's 32 rows -> staging buffer -> TMA bulk store
+    auto store_unit = [&](const uint32_t (&p)[32], int ucol0) {
+        if (units_issued >= 1) {
+            if (lane == 0)
+                bulk_wait_read<0>();  // the previous store has read the staging buffer
+            __syncwarp();
+        }
+        uint8_t *stg = stage_buf;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4 *>(stg + lane * 128 + ((c ^ (lane & 7)) * 16)) =
+                make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmOut, ucol0, row0, stg);
+            bulk_commit();
+        }
+        ++units_issued;
+    };
+    uint32_t cur[32], nxt[32], packed[32];
+    __syncwarp();
+    tmem_ld_32cols(tbase, cur);
+    tmem_ld_wait();
+    if (tma_out && !out_f32) {
+        // units of 64 columns: two 32-column chunks each
+        for (int u = 0; u < BN / 64; ++u) {
+            __syncwarp();
+            tmem_ld_32cols(tbase + (uint32_t)(64 * u + 32), nxt);
+            convert32(cur, 64 * u, packed);
+            tmem_ld_wait();
+            if (u + 1 < BN / 64) {
+                __syncwarp();
+                tmem_ld_32cols(tbase + (uint32_t)(64 * u + 64), cur);
+            } else {
+                release();
+            }
+            convert32(nxt, 64 * u + 32, packed + 16);
+            store_unit(packed, col_base + 64 * u);
+            if (u + 1 < BN / 64)
+                tmem_ld_wait();
+        }
+    } else if (tma_out) {
+        // units of 32 fp32 columns
+        for (int u = 0; u < BN / 32; ++u) {
+            if (u + 1 < BN / 32) {
+                __syncwarp();
+                tmem_ld_32cols(tbase + (uint32_t)(32 * u + 32), nxt);
+            } else {
+                release();
+            }
+            convert32(cur, 32 * u, packed);
+            store_unit(packed, col_base + 32 * u);
+            if (u + 1 < BN / 32) {
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    cur[j] = nxt[j];
+            }
+        }
+    } else {
+        for (int ch = 0; ch < BN / 32; ++ch) {
+            if (ch + 1 < BN / 32) {
+                __syncwarp();
+                tmem_ld_32cols(tbase + (uint32_t)(32 * (ch + 1)), nxt);
+            } else {
+                release();
+            }
+            const int col0 = col_base + 32 * ch;
+            if (row_ok && col0 < N) {
+                const int64_t base = (int64_t)row * N + col0;
+                for (int j = 0; j < 32 && col0 + j < N; ++j) {
+                    const int n = col0 + j;
+                    const float y = epilogue_value((int32_t)cur[j], xm, ws[n], bias, n);
+                    if (out_f32)
+                        reinterpret_cast<float *>(out)[base + j] = y;
+                    else
+                        reinterpret_cast<uint16_t *>(out)[base + j] = to_bf16_bits(y);
+                    if (acc_out != nullptr)
+                        acc_out[base + j] = (int32_t)cur[j];
+                }
+            }
+            if (ch + 1 < BN / 32) {
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    cur[j] = nxt[j];
+            }
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmOut, const float *__restrict__ xs,
@@ -215,130 +350,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool row_ok = row < M;
             const float xm = row_ok ? xs[row] : 0.0f;
             const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN);
-            const float *wsv = sh.wsb[buf];
-            const float *bsv = sh.biasb[buf];
-            const bool has_bias = bias != nullptr;
-            // 32 accumulators of columns [c0, c0 + 32) of the tile -> 32 fp32 or 16 bf16x2 words
-            auto convert32 = [&](const uint32_t (&v)[32], int c0, uint32_t *dst) {
-#pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const float4 w4 = *reinterpret_cast<const float4 *>(wsv + c0 + j);
-                    const float4 b4 = *reinterpret_cast<const float4 *>(bsv + c0 + j);
-                    const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
-                    const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
-                    float y[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        y[e] = __fmul_rn(__int2float_rn((int32_t)v[j + e]), __fmul_rn(xm, wv[e]));
-                        if (has_bias)
-                            y[e] = __fadd_rn(y[e], bv[e]);
-                    }
-                    if (out_f32) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            dst[j + e] = __float_as_uint(y[e]);
-                    } else {
-                        dst[j / 2] = to_bf16x2_bits(y[0], y[1]);
-                        dst[j / 2 + 1] = to_bf16x2_bits(y[2], y[3]);
-                    }
-                }
-            };
-            // one 128-byte unit of the warp's 32 rows -> staging buffer -> TMA bulk store
-            auto store_unit = [&](const uint32_t (&p)[32], int ucol0) {
-                if (units_issued >= 1) {
-                    if (lane == 0)
-                        bulk_wait_read<0>();  // the previous store has read the staging buffer
-                    __syncwarp();
-                }
-                uint8_t *stg = sh.epi[q];
-#pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4 *>(stg + lane * 128 + ((c ^ (lane & 7)) * 16)) =
-                        make_uint4(p[4 * c], p[4 * c + 1], p[4 * c + 2], p[4 * c + 3]);
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmOut, ucol0, tm * BM + 32 * q, stg);
-                    bulk_commit();
-                }
-                ++units_issued;
-            };
-            auto release_accumulator = [&]() {
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&sh.tmem_empty[buf]);
-            };
-            uint32_t cur[32], nxt[32], packed[32];
-            __syncwarp();
-            tmem_ld_32cols(tbase, cur);
-            tmem_ld_wait();
-            if (tma_out && !out_f32) {
-                // units of 64 columns: two 32-column chunks each
-                for (int u = 0; u < BN / 64; ++u) {
-                    __syncwarp();
-                    tmem_ld_32cols(tbase + (uint32_t)(64 * u + 32), nxt);
-                    convert32(cur, 64 * u, packed);
-                    tmem_ld_wait();
-                    if (u + 1 < BN / 64) {
-                        __syncwarp();
-                        tmem_ld_32cols(tbase + (uint32_t)(64 * u + 64), cur);
-                    } else {
-                        release_accumulator();
-                    }
-                    convert32(nxt, 64 * u + 32, packed + 16);
-                    store_unit(packed, tn * BN + 64 * u);
-                    if (u + 1 < BN / 64)
-                        tmem_ld_wait();
-                }
-            } else if (tma_out) {
-                // units of 32 fp32 columns
-                for (int u = 0; u < BN / 32; ++u) {
-                    if (u + 1 < BN / 32) {
-                        __syncwarp();
-                        tmem_ld_32cols(tbase + (uint32_t)(32 * u + 32), nxt);
-                    } else {
-                        release_accumulator();
-                    }
-                    convert32(cur, 32 * u, packed);
-                    store_unit(packed, tn * BN + 32 * u);
-                    if (u + 1 < BN / 32) {
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            cur[j] = nxt[j];
-                    }
-                }
-            } else {
-                for (int ch = 0; ch < BN / 32; ++ch) {
-                    if (ch + 1 < BN / 32) {
-                        __syncwarp();
-                        tmem_ld_32cols(tbase + (uint32_t)(32 * (ch + 1)), nxt);
-                    } else {
-                        release_accumulator();
-                    }
-                    const int col0 = tn * BN + 32 * ch;
-                    if (row_ok && col0 < N) {
-                        const int64_t base = (int64_t)row * N + col0;
-                        for (int j = 0; j < 32 && col0 + j < N; ++j) {
-                            const int n = col0 + j;
-                            const float y = epilogue_value((int32_t)cur[j], xm, ws[n], bias, n);
-                            if (out_f32)
-                                reinterpret_cast<float *>(out)[base + j] = y;
-                            else
-                                reinterpret_cast<uint16_t *>(out)[base + j] = to_bf16_bits(y);
-                            if (acc_out != nullptr)
-                                acc_out[base + j] = (int32_t)cur[j];
-                        }
-                    }
-                    if (ch + 1 < BN / 32) {
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            cur[j] = nxt[j];
-                    }
-                }
-            }
+            epilogue_tile(tbase, tm * BM + 32 * q, tn * BN, lane, xm, row_ok, sh.wsb[buf], sh.biasb[buf],
+                          bias != nullptr, M, N, out_f32, tma_out, &tmOut, sh.epi[q], units_issued, out, acc_out, ws,
+                          bias, [&]() {
+                              tc_fence_before();
+                              __syncwarp();
+                              if (lane == 0)
+                                  mbar_arrive(&sh.tmem_empty[buf]);
+                          });
         }
         if (lane == 0)
             bulk_wait_all();  // every output store has landed before the CTA exits
@@ -350,6 +369,222 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+
+// ---------------------------------------------------------------- CTA-pair variant
+//
+// For problems with at least one 256 x 256 tile per SM pair: a cluster of two
+// CTAs computes a 256 x 256 tile with tcgen05.mma.cta_group::2 (M = 256,
+// N = 256, K = 32).  Each CTA loads only its own 128 rows of A and its own 128
+// rows of B (no multicast loads), so every SM moves 32 KB instead of 48 KB per
+// 128-wide K slice for the same MMA work; each CTA's TMEM receives its 128 rows
+// of the accumulator.  The leader (rank 0) issues the MMAs; both CTAs' TMA
+// copies signal the leader's "full" barrier; the leader's commits are sent to
+// both CTAs' "empty" and "tmem_full" barriers; both CTAs' epilogue warps
+// release the accumulator on the leader's "tmem_empty" barrier.
+namespace pair {
+constexpr int kStages = 6;
+constexpr int kHalfBytes = 128 * BK;           // 16 KB: one CTA's half of A or of B
+constexpr int kStageBytes = 2 * kHalfBytes;    // A half at +0, B half at +16 KB
+constexpr uint32_t kIdesc = idesc_i8(256, BN);
+
+struct __align__(1024) Smem {
+    uint8_t stage[kStages][kStageBytes];
+    uint8_t epi[4][kEpiBytes];
+    float wsb[2][BN];
+    float biasb[2][BN];
+    uint64_t full[kStages];       // leader: both CTAs' bytes of a stage
+    uint64_t empty[kStages];      // each CTA: its stage may be refilled
+    uint64_t tmem_full[2];        // each CTA: its accumulator rows are complete
+    uint64_t tmem_empty[2];       // leader: both CTAs' epilogues released the accumulator
+    uint32_t tmem_base;
+    int abort;
+};
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
+}  // namespace pair
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmOut, const float *__restrict__ xs,
+                     const float *__restrict__ ws, const float *__restrict__ bias, int M, int N, int K, int out_f32,
+                     int vec_ok, int tma_out, void *__restrict__ out, int32_t *__restrict__ acc_out)
+{
+    extern __shared__ uint8_t smem_raw[];
+    pair::Smem &sh = *reinterpret_cast<pair::Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int npairs = gridDim.x >> 1, pair_id = blockIdx.x >> 1;
+    const int tiles_m = (M + 255) / 256, tiles_n = (N + BN - 1) / BN;
+    const int num_tiles = tiles_m * tiles_n;
+    const int kblocks = K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < pair::kStages; ++s) {
+            mbar_init(&sh.full[s], 1);
+            mbar_init(&sh.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sh.tmem_full[b], 1);
+            mbar_init(&sh.tmem_empty[b], 8);
+        }
+        sh.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&sh.tmem_base, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();  // both CTAs' barriers exist before anyone signals them
+    tc_fence_after();
+    const uint32_t tmem = sh.tmem_base;
+    volatile int *abort = &sh.abort;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            prefetch_tmap(&tmA);
+            prefetch_tmap(&tmB);
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued[pair::kStages];
+            uint32_t issued_phase[pair::kStages];
+            for (int s = 0; s < pair::kStages; ++s)
+                issued[s] = 0, issued_phase[s] = 0;
+            bool ok = true;
+            for (int tile = pair_id; ok && tile < num_tiles; tile += npairs) {
+                int tm, tn;
+                tile_coords(tile, tiles_n, tm, tn);
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t full_leader = mapa_shared(smem_u32(&sh.full[stage]), 0);
+                    if (leader)
+                        mbar_arrive_expect_tx(&sh.full[stage], 2 * pair::kStageBytes);
+                    tma_load_2d_pair(sh.stage[stage], &tmA, kb * BK, tm * 256 + (int)rank * 128, full_leader);
+                    tma_load_2d_pair(sh.stage[stage] + pair::kHalfBytes, &tmB, kb * BK, tn * BN + (int)rank * 128,
+                                     full_leader);
+                    issued[stage] = 1;
+                    issued_phase[stage] = phase;
+                    if (++stage == pair::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                // let copies in flight land before the CTAs go away: the leader
+                // waits on its barriers (bounded); the partner, whose copies
+                // signal the leader, waits a fixed 100 us
+                if (leader) {
+                    for (int s = 0; s < pair::kStages; ++s)
+                        if (issued[s]) {
+                            volatile int no_abort = 0;
+                            mbar_wait_bounded(&sh.full[s], issued_phase[s], &no_abort, 20000000ull);
+                        }
+                } else {
+                    const uint64_t t0 = globaltimer_ns();
+                    while (globaltimer_ns() - t0 < 100000ull) {
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader only)
+        if (leader && lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int local = 0;
+            bool ok = true;
+            const uint32_t peer = 1;
+            for (int tile = pair_id; ok && tile < num_tiles; tile += npairs, ++local) {
+                const int buf = local & 1;
+                const uint32_t use = (uint32_t)(local >> 1) & 1u;
+                if (!mbar_wait_bounded(&sh.tmem_empty[buf], use ^ 1u, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(buf * BN);
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait_bounded(&sh.full[stage], phase, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(sh.stage[stage]);
+                    const uint32_t b_addr = a_addr + pair::kHalfBytes;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 32; ++kk)
+                        mma_i8_pair(d, sw128_kmajor_desc(a_addr + 32u * kk), sw128_kmajor_desc(b_addr + 32u * kk),
+                                    pair::kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                    const uint32_t e = smem_u32(&sh.empty[stage]);
+                    tc_commit_pair(mapa_shared(e, 0));
+                    tc_commit_pair(mapa_shared(e, peer));
+                    if (++stage == pair::kStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok) {
+                    const uint32_t f = smem_u32(&sh.tmem_full[buf]);
+                    tc_commit_pair(mapa_shared(f, 0));
+                    tc_commit_pair(mapa_shared(f, peer));
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
+        const int q = warp & 3;
+        const int et = threadIdx.x - 64;
+        int local = 0;
+        uint32_t units_issued = 0;
+        for (int tile = pair_id; tile < num_tiles; tile += npairs, ++local) {
+            int tm, tn;
+            tile_coords(tile, tiles_n, tm, tn);
+            const int buf = local & 1;
+            const uint32_t use = (uint32_t)(local >> 1) & 1u;
+            for (int j = et; j < BN; j += 128) {
+                const int n = tn * BN + j;
+                sh.wsb[buf][j] = n < N ? ws[n] : 0.0f;
+                sh.biasb[buf][j] = (bias != nullptr && n < N) ? bias[n] : 0.0f;
+            }
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+            const bool ok = mbar_wait_bounded_warp(&sh.tmem_full[buf], use, abort);
+            if (!ok)
+                continue;
+            tc_fence_after();
+            const int row0 = tm * 256 + (int)rank * 128 + 32 * q;
+            const bool row_ok = row0 + lane < M;
+            const float xm = row_ok ? xs[row0 + lane] : 0.0f;
+            const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN);
+            const uint32_t release_addr = mapa_shared(smem_u32(&sh.tmem_empty[buf]), 0);
+            epilogue_tile(tbase, row0, tn * BN, lane, xm, row_ok, sh.wsb[buf], sh.biasb[buf], bias != nullptr, M,
+                          N, out_f32, tma_out, &tmOut, sh.epi[q], units_issued, out, acc_out, ws, bias, [&]() {
+                              tc_fence_before();
+                              __syncwarp();
+                              if (lane == 0)
+                                  mbar_arrive_cluster(release_addr);
+                          });
+        }
+        if (lane == 0)
+            bulk_wait_all();
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // no CTA leaves while its partner may still signal it
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, kTmemCols);
     }
 }
 

@@ -7,11 +7,11 @@
 // are exact, so the result equals the prefill path bit for bit.
 //
 // B200 design.
-//  * Streaming: a persistent grid (two CTAs per SM).  In each CTA one
-//    producer warp moves 16-row x 2048-column tiles of the packed codes
-//    (16 KB) and their group scales (2 KB) into a 4-stage shared-memory ring
-//    with 2-D TMA copies; eight consumer warps (two 128-column slices each)
-//    decode and contract each stage while the following ones are in flight.  Bytes in flight are set by the
+//  * Streaming: a persistent grid (several CTAs per SM).  In each CTA one
+//    producer warp moves tiles of 16 weight rows x 1024 columns of the packed
+//    codes (8 KB) and their group scales (1 KB) into a ring of shared-memory
+//    stages with 2-D TMA copies; eight consumer warps decode and contract each
+//    stage while the following ones are in flight.  Bytes in flight are set by the
 //    ring, not by registers, which keeps HBM busy.
 //  * Decode: a per-CTA table of the 16 int8 levels of every fp8 scale byte
 //    (exact: the decoded value depends only on the pair), replicated 8 times
@@ -43,14 +43,18 @@ namespace gv {
 
 constexpr int kConsumerWarps = 8;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
-constexpr int kRows = 16;                            // output rows per tile
 
-// Shape of one pipeline stage: every consumer warp takes SLICES slices of 128
-// k per stage, so a stage covers CHUNK = 8 * SLICES * 128 columns of 16 rows.
-template <int SLICES, int STAGES>
+// Shape of the pipeline.  A tile is RG groups of 16 weight rows; every
+// consumer warp takes SLICES slices of 128 k per stage, so a stage covers
+// CHUNK = 8 * SLICES * 128 columns of the tile's 16 RG rows.  MINB is the
+// number of CTAs the kernel is compiled to fit on one SM.
+template <int RG, int SLICES, int STAGES, int MINB>
 struct Cfg {
+    static constexpr int kRG = RG;
+    static constexpr int kRows = 16 * RG;
     static constexpr int kSlices = SLICES;
     static constexpr int kStages = STAGES;
+    static constexpr int kMinBlocks = MINB;
     static constexpr int kChunk = kConsumerWarps * SLICES * 128;
     static constexpr int kCodeBytes = kRows * kChunk / 2;
     static constexpr int kSrelBytes = kRows * kChunk / 16;
@@ -68,7 +72,7 @@ struct Cfg {
 };
 
 // The configuration the library launches.
-using Prod = Cfg<2, 4>;
+using Prod = Cfg<1, 1, 4, 3>;
 
 __device__ __forceinline__ void mma_s8(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                        uint32_t b0, uint32_t b1)
@@ -82,20 +86,19 @@ __device__ __forceinline__ void mma_s8(int32_t (&c)[4], uint32_t a0, uint32_t a1
 
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
-// One slice: 16 rows x 128 k of this stage against the token fragments X0, X1.
-__device__ __forceinline__ void slice_mma(const uint8_t *codes_row_g, const uint8_t *codes_row_g8,
-                                          const uint8_t *srel_row_g, const uint8_t *srel_row_g8, const uint4 *lut8,
-                                          int copy, const uint4 &X0, const uint4 &X1, int32_t (&c)[4],
-                                          int32_t (&d)[4])
+// One slice of one 16-row group: rows g and g + 8 (relative to the group) x
+// 128 k of this stage against the token fragments X0, X1.  `lutc` already
+// points at this lane's table copy; entry s is lutc[8 s].
+__device__ __forceinline__ void slice_mma(const uint8_t *codes_g, const uint8_t *codes_g8, const uint8_t *srel_g,
+                                          const uint8_t *srel_g8, const uint4 *lutc, const uint4 &X0,
+                                          const uint4 &X1, int32_t (&c)[4], int32_t (&d)[4])
 {
-    const uint4 A = *reinterpret_cast<const uint4 *>(codes_row_g);
-    const uint4 B = *reinterpret_cast<const uint4 *>(codes_row_g8);
-    const uint32_t SA = *reinterpret_cast<const uint16_t *>(srel_row_g);
-    const uint32_t SB = *reinterpret_cast<const uint16_t *>(srel_row_g8);
-    const uint4 TA0 = lut8[(SA & 0xFFu) * 8 + copy];
-    const uint4 TA1 = lut8[(SA >> 8) * 8 + copy];
-    const uint4 TB0 = lut8[(SB & 0xFFu) * 8 + copy];
-    const uint4 TB1 = lut8[(SB >> 8) * 8 + copy];
+    const uint4 A = *reinterpret_cast<const uint4 *>(codes_g);
+    const uint4 B = *reinterpret_cast<const uint4 *>(codes_g8);
+    const uint4 TA0 = lutc[8 * (uint32_t)srel_g[0]];
+    const uint4 TA1 = lutc[8 * (uint32_t)srel_g[1]];
+    const uint4 TB0 = lutc[8 * (uint32_t)srel_g8[0]];
+    const uint4 TB1 = lutc[8 * (uint32_t)srel_g8[1]];
     uint32_t a0, a1, a2, a3, e0, e1, e2, e3;
     decode8(A.x, TA0, a0, a2);
     decode8(B.x, TB0, a1, a3);
@@ -112,19 +115,19 @@ __device__ __forceinline__ void slice_mma(const uint8_t *codes_row_g, const uint
 }
 
 template <class C>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, C::kMinBlocks)
     gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_srel,
                 const int8_t *__restrict__ xq, const float *__restrict__ xs, const float *__restrict__ codebook,
                 const float *__restrict__ ws, const float *__restrict__ bias, int M, int N, int K, int out_f32,
                 void *__restrict__ out, int32_t *__restrict__ acc_out)
 {
-    constexpr int S = C::kSlices, STAGES = C::kStages, CHUNK = C::kChunk;
+    constexpr int RG = C::kRG, ROWS = C::kRows, S = C::kSlices, STAGES = C::kStages, CHUNK = C::kChunk;
     using Smem = typename C::Smem;
     extern __shared__ uint8_t smem_raw[];
     Smem &sh = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int ntiles = (N + kRows - 1) / kRows;
+    const int ntiles = (N + ROWS - 1) / ROWS;
     const int nchunks = (K + CHUNK - 1) / CHUNK;
 
     if (tid == 0) {
@@ -160,8 +163,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                         break;
                     }
                     mbar_arrive_expect_tx(&sh.full[stage], C::kCodeBytes + C::kSrelBytes);
-                    tma_load_2d(sh.codes[stage], &tm_codes, c * (CHUNK / 8), tile * kRows, &sh.full[stage]);
-                    tma_load_2d(sh.srel[stage], &tm_srel, c * (CHUNK / 16), tile * kRows, &sh.full[stage]);
+                    tma_load_2d(sh.codes[stage], &tm_codes, c * (CHUNK / 8), tile * ROWS, &sh.full[stage]);
+                    tma_load_2d(sh.srel[stage], &tm_srel, c * (CHUNK / 16), tile * ROWS, &sh.full[stage]);
                     issued[stage] = 1;
                     issued_phase[stage] = phase;
                     if (++stage == STAGES) {
@@ -190,14 +193,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         asm volatile("griddepcontrol.wait;" ::: "memory");
 
         const int g = lane >> 2, t = lane & 3;
-        const int copy = lane & 7;
+        const uint4 *lutc = sh.lut8 + (lane & 7);
         const bool vx = g < M;
         // slice j of this warp in a stage: k offset 128 * (warp + 8 j) in the chunk
         const int8_t *px = xq + (int64_t)g * K + 128 * warp + 32 * t;
         const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
         // The activation fragments of a chunk do not depend on the row tile;
         // the next chunk's are fetched (through L1/L2) while the current one
-        // is computed, in the order the chunks are consumed.
+        // is computed.  Two register sets alternate with the chunk parity.
         auto fetch_x = [&](int ch, uint4 (&X)[S][2]) {
 #pragma unroll
             for (int j = 0; j < S; ++j) {
@@ -209,58 +212,79 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
             }
         };
-        uint4 Xc[S][2], Xn[S][2];
-        fetch_x(0, Xn);
-        int xch = 0;  // chunk index of Xn
+        uint4 XA[S][2], XB[S][2];
         int stage = 0;
         uint32_t phase = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            // two accumulators break the dependency chain between the MMAs of a slice
-            int32_t c[4] = {0, 0, 0, 0}, d[4] = {0, 0, 0, 0};
-            for (int ch = 0; ch < nchunks; ++ch) {
+        // consume one stage: all slices of this warp, all row groups
+        auto consume = [&](int ch, const uint4 (&X)[S][2], int32_t (&c)[RG][4], int32_t (&d)[RG][4]) {
+            const bool ok = mbar_wait_bounded_warp(&sh.full[stage], phase, abort);
+            if (ok) {
 #pragma unroll
-                for (int j = 0; j < S; ++j)
-                    Xc[j][0] = Xn[j][0], Xc[j][1] = Xn[j][1];
-                if (++xch == nchunks)
-                    xch = 0;
-                fetch_x(xch, Xn);
-                const bool ok = mbar_wait_bounded_warp(&sh.full[stage], phase, abort);
-                if (ok) {
+                for (int j = 0; j < S; ++j) {
+                    const int sl = warp + 8 * j;
+                    if (ch * CHUNK + 128 * sl < K) {
+                        const uint8_t *cs = sh.codes[stage] + 64 * sl + 16 * t + (CHUNK / 2) * g;
+                        const uint8_t *ss = sh.srel[stage] + 8 * sl + 2 * t + (CHUNK / 16) * g;
 #pragma unroll
-                    for (int j = 0; j < S; ++j) {
-                        const int sl = warp + 8 * j;
-                        if (ch * CHUNK + 128 * sl < K) {
-                            const uint8_t *cs = sh.codes[stage] + 64 * sl + 16 * t;
-                            const uint8_t *ss = sh.srel[stage] + 8 * sl + 2 * t;
-                            slice_mma(cs + (CHUNK / 2) * g, cs + (CHUNK / 2) * (g + 8), ss + (CHUNK / 16) * g,
-                                      ss + (CHUNK / 16) * (g + 8), sh.lut8, copy, Xc[j][0], Xc[j][1], c, d);
-                        }
+                        for (int rg = 0; rg < RG; ++rg)
+                            slice_mma(cs + (CHUNK / 2) * 16 * rg, cs + (CHUNK / 2) * (16 * rg + 8),
+                                      ss + (CHUNK / 16) * 16 * rg, ss + (CHUNK / 16) * (16 * rg + 8), lutc,
+                                      X[j][0], X[j][1], c[rg], d[rg]);
                     }
                 }
-                __syncwarp();
-                if (ok && lane == 0)
-                    mbar_arrive(&sh.empty[stage]);
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
+            }
+            __syncwarp();
+            if (ok && lane == 0)
+                mbar_arrive(&sh.empty[stage]);
+            if (++stage == STAGES) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        };
+        fetch_x(0, XA);
+        int xnext = nchunks > 1 ? 1 : 0;  // chunk whose fragments are fetched next
+        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+            // two accumulators per row group break the dependency chain between MMAs
+            int32_t c[RG][4], d[RG][4];
+#pragma unroll
+            for (int rg = 0; rg < RG; ++rg)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    c[rg][i] = d[rg][i] = 0;
+            // chunks in pairs: XA holds the even chunk's fragments, XB the odd one's
+            for (int ch = 0; ch < nchunks; ch += 2) {
+                fetch_x(xnext, XB);
+                if (++xnext == nchunks)
+                    xnext = 0;
+                consume(ch, XA, c, d);
+                if (ch + 1 < nchunks) {
+                    fetch_x(xnext, XA);
+                    if (++xnext == nchunks)
+                        xnext = 0;
+                    consume(ch + 1, XB, c, d);
+                } else {
+                    // odd chunk count: XB holds the next tile's chunk 0
+#pragma unroll
+                    for (int j = 0; j < S; ++j)
+                        XA[j][0] = XB[j][0], XA[j][1] = XB[j][1];
                 }
             }
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                c[i] += d[i];
-            // C fragment: c0 (row g, token 2t), c1 (g, 2t+1), c2 (g+8, 2t), c3 (g+8, 2t+1)
-            sh.red[warp][g][2 * t] = c[0];
-            sh.red[warp][g][2 * t + 1] = c[1];
-            sh.red[warp][g + 8][2 * t] = c[2];
-            sh.red[warp][g + 8][2 * t + 1] = c[3];
+            for (int rg = 0; rg < RG; ++rg) {
+                // C fragment: c0 (row g, token 2t), c1 (g, 2t+1), c2 (g+8, 2t), c3 (g+8, 2t+1)
+                sh.red[warp][16 * rg + g][2 * t] = c[rg][0] + d[rg][0];
+                sh.red[warp][16 * rg + g][2 * t + 1] = c[rg][1] + d[rg][1];
+                sh.red[warp][16 * rg + g + 8][2 * t] = c[rg][2] + d[rg][2];
+                sh.red[warp][16 * rg + g + 8][2 * t + 1] = c[rg][3] + d[rg][3];
+            }
             consumer_sync();
-            if (tid < kRows * 8) {
-                const int r = tid >> 3, m = tid & 7;
+            for (int e = tid; e < ROWS * 8; e += 256) {
+                const int r = e >> 3, m = e & 7;
                 int32_t acc = 0;
 #pragma unroll
                 for (int w = 0; w < kConsumerWarps; ++w)
                     acc += sh.red[w][r][m];
-                const int n = tile * kRows + r;
+                const int n = tile * ROWS + r;
                 if (m < M && n < N && !*abort) {
                     const float y = epilogue_value(acc, xs[m], ws[n], bias, n);
                     const int64_t o = (int64_t)m * N + n;
