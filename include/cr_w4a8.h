@@ -35,6 +35,18 @@
  *   fp32; for other values the outputs are unspecified, but no call faults.
  * - Calls that read a buffer another call on another stream is writing race,
  *   as with any CUDA kernel.
+ * - Overlapped launches.  cr_rotate_quant_act, cr_w4a8_gemv, cr_w4a8_linear
+ *   (decode path) and cr_w4a8_linear_decode_noalloc launch their kernels as
+ *   programmatic dependents of the previous kernel on the stream, and those
+ *   kernels allow the next kernel to launch early.  Stream order still holds
+ *   for every activation, scale and output buffer: each kernel waits for its
+ *   predecessor to complete before it reads a result of it or writes a
+ *   buffer that the predecessor may read.  The decode GEMV alone starts
+ *   reading the layer (qdata, srel, codebook) before that wait, so the layer
+ *   must not be written by a kernel that itself allows early launch of its
+ *   dependents (griddepcontrol.launch_dependents / PDL) and immediately
+ *   precedes the GEMV on the stream; a kernel that does not, and every copy
+ *   or memset, orders as usual.
  */
 #ifndef CR_W4A8_H
 #define CR_W4A8_H

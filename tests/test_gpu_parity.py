@@ -203,3 +203,35 @@ def test_empty_problems_launch_nothing():
 
 def test_no_device_error_pending():
     cr.cr_check_device_error()
+
+
+def test_gemv_back_to_back_and_two_streams():
+    """Chained launches (each may start before the previous one ends) and
+    launches in flight on two streams at once give the oracle's outputs;
+    runs that share a row tile hand their partial sums over exactly."""
+    cases = [(8, 4096, 4096, 61), (3, 2000, 1280, 62), (1, 8192, 2048, 63)]
+    ref, dev_in = [], []
+    for M, N, K, seed in cases:
+        layer = inputs.layer(N, K, seed)
+        x = inputs.activations(M, K, seed)
+        xq_r, xs_r = oracle.rotate_quant_act(x, cr.gemv_rows(M), 127)
+        w8 = oracle.decode_w8(layer.qdata, layer.srel, layer.codebook)
+        acc_r = oracle.gemm_s32(xq_r[:M], w8, THREADS)
+        ref.append(acc_r)
+        dev_in.append((dev(xq_r), dev(xs_r)) + _layer_dev(layer) + (M,))
+    # back to back on one stream, the same buffers every time
+    for (xq, xs, q, s, cb, ws, b, M), acc_r in zip(dev_in, ref):
+        outs = [cr.cr_w4a8_gemv(xq, xs, q, s, cb, ws, m=M, acc_out=True)[1] for _ in range(6)]
+        for a in outs:
+            assert np.array_equal(host(a), acc_r)
+    # interleaved on two streams
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    got = []
+    for rep in range(4):
+        for i, (xq, xs, q, s, cb, ws, b, M) in enumerate(dev_in):
+            st = streams[(i + rep) % 2]
+            with torch.cuda.stream(st):
+                got.append((i, cr.cr_w4a8_gemv(xq, xs, q, s, cb, ws, m=M, acc_out=True)[1]))
+    torch.cuda.synchronize()
+    for i, a in got:
+        assert np.array_equal(host(a), ref[i])

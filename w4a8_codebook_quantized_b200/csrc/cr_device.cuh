@@ -161,6 +161,15 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
     asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Arrive without release ordering.  For a consumer handing a ring stage back
+// after every value it read from the stage has been used in registers: no
+// ordering of its other (global) memory operations is needed, and a release
+// arrive would wait for this thread's outstanding prefetch loads.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes)
 {
     asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
@@ -242,6 +251,29 @@ __device__ __forceinline__ bool mbar_wait_bounded_warp(uint64_t *bar, uint32_t p
 }
 
 // ---------------------------------------------------------------- TMA
+
+// The dynamic shared-memory buffer rounded up to a 1024-byte boundary (the
+// alignment the 128-byte-swizzled TMA layouts need).  The padding is added to
+// the __shared__ array itself rather than to an integer copy of its address,
+// so the result stays in the shared state space and its reads compile to
+// shared-memory loads instead of generic ones.
+template <class T>
+__device__ __forceinline__ T &smem_aligned_1024(uint8_t *smem_raw)
+{
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    return *reinterpret_cast<T *>(smem_raw + pad);
+}
+
+// 3-D tiled bulk tensor load into this CTA's shared memory.
+__device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, int32_t x, int32_t y, int32_t z,
+                                            uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+            smem_u32(smem_dst)),
+        "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
 
 __device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, int32_t x, int32_t y, uint64_t *bar)
 {

@@ -131,25 +131,29 @@ bool make_tmap_i8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t r
     return r == CUDA_SUCCESS;
 }
 
-// 2-D tensor map, no swizzle: a row-major [rows, inner] array of `esize`-byte
-// elements with the given row pitch in bytes, box [box_rows, box_inner].
-bool make_tmap_plain(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, uint64_t inner, uint64_t rows,
-                     uint64_t pitch, uint32_t box_inner, uint32_t box_rows)
+// 3-D tensor map, no swizzle or the 128-byte swizzle, over `base` with the
+// given dims (innermost first), the byte strides of dims 1 and 2 and the box.
+// The strides need not increase: the maps below reorder a row-major array so
+// that a box lands in shared memory in the order the kernel reads it.
+bool make_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, const uint64_t (&dims)[3],
+                  const uint64_t (&strides)[2], const uint32_t (&box)[3], bool swizzle128)
 {
-    const cuuint64_t dims[2] = {inner, rows};
-    const cuuint64_t strides[1] = {pitch};
-    const cuuint32_t box[2] = {box_inner, box_rows};
-    const cuuint32_t estr[2] = {1u, 1u};
-    const CUresult r = g_encode_tiled(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr,
-                                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+    const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+    const cuuint64_t st[2] = {strides[0], strides[1]};
+    const cuuint32_t b[3] = {box[0], box[1], box[2]};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    const CUresult r = g_encode_tiled(map, dtype, 3, const_cast<void *>(base), d, st, b, estr,
+                                      CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                      swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-// The decode GEMV: tensor maps over the packed codes (as 32-bit words, one
-// row slice of a stage per box row) and the scale bytes, a persistent grid of
-// as many CTAs as fit on the SMs, optionally as a programmatic dependent of the previous
-// kernel on the stream.
+// The decode GEMV: three tensor maps that put a stage into shared memory as
+// codes [slice][row][64 B], scales [256-column block][row][16 B] and
+// activations [slice][token][128 B] (128-byte swizzle); a persistent grid of
+// as many CTAs as fit on the SMs, optionally as a programmatic dependent of
+// the previous kernel on the stream.
 cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const uint8_t *qdata,
                    const uint8_t *srel, const float *codebook, const float *s_channel, const float *bias, int64_t M,
                    int64_t N, int64_t K, cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream,
@@ -165,13 +169,18 @@ cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *x
         }
         attr_set = true;
     }
-    CUtensorMap tc, ts;
-    if (!make_tmap_plain(&tc, qdata, CU_TENSOR_MAP_DATA_TYPE_UINT32, (uint64_t)(K / 8), (uint64_t)N,
-                         (uint64_t)(K / 2), C::kChunk / 8, C::kRows) ||
-        !make_tmap_plain(&ts, srel, CU_TENSOR_MAP_DATA_TYPE_UINT8, (uint64_t)(K / 16), (uint64_t)N,
-                         (uint64_t)(K / 16), C::kChunk / 16, C::kRows))
+    CUtensorMap tc, ts, tx;
+    const uint64_t uK = (uint64_t)K, uN = (uint64_t)N, uM = (uint64_t)M;
+    if (!make_tmap_3d(&tc, qdata, CU_TENSOR_MAP_DATA_TYPE_UINT32, {16, uN, uK / gv::kSlice}, {uK / 2, 64},
+                      {16, (uint32_t)gv::kRows, (uint32_t)(gv::kChunk / gv::kSlice)}, false) ||
+        !make_tmap_3d(&ts, srel, CU_TENSOR_MAP_DATA_TYPE_UINT8, {16, uN, uK / 256}, {uK / 16, 16},
+                      {16, (uint32_t)gv::kRows, (uint32_t)(gv::kChunk / 256)}, false) ||
+        !make_tmap_3d(&tx, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, {(uint64_t)gv::kSlice, uM, uK / gv::kSlice},
+                      {uK, (uint64_t)gv::kSlice},
+                      {(uint32_t)gv::kSlice, (uint32_t)gv::kTokens, (uint32_t)(gv::kChunk / gv::kSlice)}, true))
         return CR_ERR_CUDA;
-    const int64_t tiles = (N + C::kRows - 1) / C::kRows;
+    // persistent grid: at most one wave, whole row tiles per CTA
+    const int64_t tiles = (N + gv::kRows - 1) / gv::kRows;
     const int64_t slots = (int64_t)C::kMinBlocks * num_sms;
     const int64_t grid = tiles < slots ? tiles : slots;
     cudaLaunchConfig_t cfg = {};
@@ -184,7 +193,7 @@ cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *x
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return launched(cudaLaunchKernelEx(&cfg, gv::gemv_kernel<C>, tc, ts, xq, xs, codebook, s_channel, bias, (int)M,
+    return launched(cudaLaunchKernelEx(&cfg, gv::gemv_kernel<C>, tc, ts, tx, xs, codebook, s_channel, bias, (int)M,
                                        (int)N, (int)K, out_dtype == CR_OUT_F32 ? 1 : 0, out, acc_out));
 }
 
@@ -397,7 +406,7 @@ cr_status cr_w4a8_gemv(const int8_t *xq, const float *xs, const uint8_t *qdata, 
     if (st != CR_OK)
         return st;
     return run_gemv(d->num_sms, d->gemv_attr_set, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K,
-                    out_dtype, out, acc_out, stream, false);
+                    out_dtype, out, acc_out, stream, /*pdl=*/true);
 }
 
 cr_status cr_epilogue(const int32_t *acc, const float *xs, const float *s_channel, const float *bias, int64_t M,

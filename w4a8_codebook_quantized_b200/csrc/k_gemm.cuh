@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 int vec_ok, int tma_out, void *__restrict__ out, int32_t *__restrict__ acc_out)
 {
     extern __shared__ uint8_t smem_raw[];
-    Smem &sh = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem &sh = smem_aligned_1024<Smem>(smem_raw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tiles_m = (M + BM - 1) / BM, tiles_n = (N + BN - 1) / BN;
@@ -412,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                      int vec_ok, int tma_out, void *__restrict__ out, int32_t *__restrict__ acc_out)
 {
     extern __shared__ uint8_t smem_raw[];
-    pair::Smem &sh = *reinterpret_cast<pair::Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    pair::Smem &sh = smem_aligned_1024<pair::Smem>(smem_raw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();

@@ -7,16 +7,25 @@
 // are exact, so the result equals the prefill path bit for bit.
 //
 // B200 design.
-//  * Streaming: a persistent grid (several CTAs per SM).  In each CTA one
-//    producer warp moves tiles of 16 weight rows x 1024 columns of the packed
-//    codes (8 KB) and their group scales (1 KB) into a ring of shared-memory
-//    stages with 2-D TMA copies; eight consumer warps decode and contract each
-//    stage while the following ones are in flight.  Bytes in flight are set by the
-//    ring, not by registers, which keeps HBM busy.
+//  * Streaming: a persistent grid (three CTAs per SM).  In each CTA one
+//    producer warp moves, per stage, the packed codes (16 weight rows x 1024
+//    columns, 8 KB), their group scales (1 KB) and the matching 1024 columns
+//    of the (at most 8) activation rows (8 KB) into a ring of shared-memory
+//    stages with 3-D TMA copies; eight consumer warps decode and contract each
+//    stage while the following ones are in flight; an epilogue warp reduces
+//    the consumers' partial sums and writes the outputs of a tile while the
+//    consumers already work on the next one.  Bytes in flight are set by the
+//    ring, not by registers, and the consumers issue no global memory
+//    accesses and take no CTA-wide barrier in the loop.
+//  * Shared-memory layouts chosen for conflict-free reads: the tensor maps
+//    order the box so that a stage holds the codes as [slice][row][64 B], the
+//    scales as [256-column block][row][16 B] and the activations as
+//    [slice][token][128 B] with the 128-byte swizzle; every quarter-warp
+//    request then touches 8 distinct 16-byte bank groups.
 //  * Decode: a per-CTA table of the 16 int8 levels of every fp8 scale byte
-//    (exact: the decoded value depends only on the pair), replicated 8 times
-//    with copy c in bank group c so that a quarter-warp's 16-byte lookups
-//    never conflict; byte permutes turn 8 packed codes into 8 int8 levels.
+//    (exact: the decoded value depends only on the pair), replicated so that
+//    the lanes of a quarter-warp mostly read distinct bank groups; byte
+//    permutes turn 8 packed codes into 8 int8 levels.
 //  * Contraction: the page's kernel uses int32 IMAD in registers; here the
 //    decoded weights go straight from registers into the warp-level int8
 //    tensor-core instruction (mma.sync m16n8k32: A = 16 weight rows x 32 k,
@@ -27,11 +36,11 @@
 //    slice w, and the matching 32 activation bytes of token g; code word i
 //    (columns 8i..8i+7) feeds MMA i, its first four columns in the fragment
 //    slots of logical k = 4t..4t+3 and its last four in 16+4t..16+4t+3.
-//  * The int32 partial sums of the eight warps meet in shared memory; the
-//    fused epilogue writes the 16 x M outputs of the row tile.
-//  * When launched as a programmatic dependent of the activation kernel, the
-//    weight stream and the table build start before that kernel finishes;
-//    the consumers wait for it (griddepcontrol.wait) before reading xq / xs.
+//  * Launch overlap: the kernel lets the next kernel on the stream launch at
+//    once, and it may itself start before the previous kernel ends (weight
+//    stream and table build first); the activation copies and every read of
+//    xq / xs and write of the outputs wait for that kernel
+//    (griddepcontrol.wait).
 #pragma once
 
 #include <cuda.h>
@@ -42,37 +51,45 @@ namespace cr {
 namespace gv {
 
 constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kProducerWarp = kConsumerWarps;       // TMA issue
+constexpr int kEpilogueWarp = kConsumerWarps + 1;   // reduction, split-tile hand-off, outputs
+constexpr int kThreads = (kConsumerWarps + 2) * 32;
+constexpr int kRows = 16;                            // weight rows of a tile (the MMA's M)
+constexpr int kSlice = 128;                          // columns per consumer warp per stage
+constexpr int kChunk = kConsumerWarps * kSlice;      // columns per stage
+constexpr int kTokens = 8;                           // activation rows of a stage (the MMA's N)
+constexpr int kCodeBytes = kRows * kChunk / 2;
+constexpr int kSrelBytes = kRows * kChunk / 16;
+constexpr int kXBytes = kTokens * kChunk;
+constexpr int kStageTx = kCodeBytes + kSrelBytes + kXBytes;
+constexpr int kRedBufs = 1;  // partial-sum mailboxes between the consumers and the epilogue warp
 
-// Shape of the pipeline.  A tile is RG groups of 16 weight rows; every
-// consumer warp takes SLICES slices of 128 k per stage, so a stage covers
-// CHUNK = 8 * SLICES * 128 columns of the tile's 16 RG rows.  MINB is the
-// number of CTAs the kernel is compiled to fit on one SM.
-template <int RG, int SLICES, int STAGES, int MINB>
+// Shape of the ring: STAGES stages, MINB CTAs per SM, COPIES copies of the
+// level table (8 copies make every quarter-warp lookup conflict-free, 4 leave
+// occasional two-way conflicts for half the shared memory).
+template <int STAGES, int MINB, int COPIES>
 struct Cfg {
-    static constexpr int kRG = RG;
-    static constexpr int kRows = 16 * RG;
-    static constexpr int kSlices = SLICES;
     static constexpr int kStages = STAGES;
     static constexpr int kMinBlocks = MINB;
-    static constexpr int kChunk = kConsumerWarps * SLICES * 128;
-    static constexpr int kCodeBytes = kRows * kChunk / 2;
-    static constexpr int kSrelBytes = kRows * kChunk / 16;
+    static constexpr int kCopies = COPIES;
     struct __align__(1024) Smem {
-        uint8_t codes[STAGES][kCodeBytes];  // row r of a stage at r * kChunk / 2 bytes
-        uint8_t srel[STAGES][kSrelBytes];   // row r of a stage at r * kChunk / 16 bytes
-        uint4 lut8[256 * 8];                // lut8[s * 8 + c]: copy c of the levels of scale byte s
-        int32_t red[kConsumerWarps][kRows][8];
+        uint8_t x[STAGES][kXBytes];          // [slice][token][128 B], 128-byte swizzle (1024-aligned)
+        uint8_t codes[STAGES][kCodeBytes];   // [slice][row][64 B]
+        uint8_t srel[STAGES][kSrelBytes];    // [256-column block][row][16 B]
+        uint4 lut[256 * COPIES];             // lut[s * COPIES + c]: copy c of the levels of scale byte s
+        int32_t red[kRedBufs][kConsumerWarps][kRows][8];  // per-warp partial sums
         float cb[16];
         uint64_t full[STAGES];
         uint64_t empty[STAGES];
+        uint64_t red_full[kRedBufs];   // the eight consumer warps have written red[b]
+        uint64_t red_empty[kRedBufs];  // the epilogue warp has read red[b]
         int abort;
     };
     static constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 };
 
 // The configuration the library launches.
-using Prod = Cfg<1, 1, 4, 3>;
+using Prod = Cfg<3, 3, 4>;
 
 __device__ __forceinline__ void mma_s8(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                        uint32_t b0, uint32_t b1)
@@ -86,54 +103,85 @@ __device__ __forceinline__ void mma_s8(int32_t (&c)[4], uint32_t a0, uint32_t a1
 
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
-// One slice of one 16-row group: rows g and g + 8 (relative to the group) x
-// 128 k of this stage against the token fragments X0, X1.  `lutc` already
-// points at this lane's table copy; entry s is lutc[8 s].
-__device__ __forceinline__ void slice_mma(const uint8_t *codes_g, const uint8_t *codes_g8, const uint8_t *srel_g,
-                                          const uint8_t *srel_g8, const uint4 *lutc, const uint4 &X0,
-                                          const uint4 &X1, int32_t (&c)[4], int32_t (&d)[4])
+// The operands of one stage for one thread: its activation fragments, the
+// 32 codes of rows g and g + 8, and the level tables of their two groups.
+struct Ops {
+    uint4 X0, X1, A, B, TA0, TA1, TB0, TB1;
+};
+
+// Fetch a stage's operands from shared memory.  `lutc` already points at this
+// lane's table copy; entry s is lutc[COPIES s].
+template <int COPIES>
+__device__ __forceinline__ void fetch_ops(Ops &o, const uint8_t *x0, const uint8_t *x1, const uint8_t *codes_g,
+                                          const uint8_t *srel_g, const uint4 *lutc)
 {
-    const uint4 A = *reinterpret_cast<const uint4 *>(codes_g);
-    const uint4 B = *reinterpret_cast<const uint4 *>(codes_g8);
-    const uint4 TA0 = lutc[8 * (uint32_t)srel_g[0]];
-    const uint4 TA1 = lutc[8 * (uint32_t)srel_g[1]];
-    const uint4 TB0 = lutc[8 * (uint32_t)srel_g8[0]];
-    const uint4 TB1 = lutc[8 * (uint32_t)srel_g8[1]];
-    uint32_t a0, a1, a2, a3, e0, e1, e2, e3;
-    decode8(A.x, TA0, a0, a2);
-    decode8(B.x, TB0, a1, a3);
-    decode8(A.y, TA0, e0, e2);
-    decode8(B.y, TB0, e1, e3);
-    mma_s8(c, a0, a1, a2, a3, X0.x, X0.y);
-    mma_s8(d, e0, e1, e2, e3, X0.z, X0.w);
-    decode8(A.z, TA1, a0, a2);
-    decode8(B.z, TB1, a1, a3);
-    decode8(A.w, TA1, e0, e2);
-    decode8(B.w, TB1, e1, e3);
-    mma_s8(c, a0, a1, a2, a3, X1.x, X1.y);
-    mma_s8(d, e0, e1, e2, e3, X1.z, X1.w);
+    o.X0 = *reinterpret_cast<const uint4 *>(x0);
+    o.X1 = *reinterpret_cast<const uint4 *>(x1);
+    o.A = *reinterpret_cast<const uint4 *>(codes_g);
+    o.B = *reinterpret_cast<const uint4 *>(codes_g + 8 * 64);
+    o.TA0 = lutc[COPIES * (uint32_t)srel_g[0]];
+    o.TA1 = lutc[COPIES * (uint32_t)srel_g[1]];
+    o.TB0 = lutc[COPIES * (uint32_t)srel_g[8 * 16]];
+    o.TB1 = lutc[COPIES * (uint32_t)srel_g[8 * 16 + 1]];
 }
 
+// One slice of the tile: rows g and g + 8 x 128 k against the token
+// fragments, into the two accumulators.
+__device__ __forceinline__ void slice_mma(const Ops &o, int32_t (&c)[4], int32_t (&d)[4])
+{
+    uint32_t a0, a1, a2, a3, e0, e1, e2, e3;
+    decode8(o.A.x, o.TA0, a0, a2);
+    decode8(o.B.x, o.TB0, a1, a3);
+    decode8(o.A.y, o.TA0, e0, e2);
+    decode8(o.B.y, o.TB0, e1, e3);
+    mma_s8(c, a0, a1, a2, a3, o.X0.x, o.X0.y);
+    mma_s8(d, e0, e1, e2, e3, o.X0.z, o.X0.w);
+    decode8(o.A.z, o.TA1, a0, a2);
+    decode8(o.B.z, o.TB1, a1, a3);
+    decode8(o.A.w, o.TA1, e0, e2);
+    decode8(o.B.w, o.TB1, e1, e3);
+    mma_s8(c, a0, a1, a2, a3, o.X1.x, o.X1.y);
+    mma_s8(d, e0, e1, e2, e3, o.X1.z, o.X1.w);
+}
+
+// tm_codes: the packed codes as 32-bit words, dims {16, N, K / 128}, strides
+//           {K / 2, 64} bytes, box {16, 16, 8}.
+// tm_srel:  the scale bytes, dims {16, N, K / 256}, strides {K / 16, 16}, box {16, 16, 4}.
+// tm_x:     xq, dims {128, M, K / 128}, strides {K, 128}, box {128, 8, 8}, 128-byte swizzle.
 template <class C>
 __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
     gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_srel,
-                const int8_t *__restrict__ xq, const float *__restrict__ xs, const float *__restrict__ codebook,
-                const float *__restrict__ ws, const float *__restrict__ bias, int M, int N, int K, int out_f32,
-                void *__restrict__ out, int32_t *__restrict__ acc_out)
+                const __grid_constant__ CUtensorMap tm_x, const float *__restrict__ xs,
+                const float *__restrict__ codebook, const float *__restrict__ ws, const float *__restrict__ bias,
+                int M, int N, int K, int out_f32, void *__restrict__ out, int32_t *__restrict__ acc_out)
 {
-    constexpr int RG = C::kRG, ROWS = C::kRows, S = C::kSlices, STAGES = C::kStages, CHUNK = C::kChunk;
+    constexpr int STAGES = C::kStages;
     using Smem = typename C::Smem;
     extern __shared__ uint8_t smem_raw[];
-    Smem &sh = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Smem &sh = smem_aligned_1024<Smem>(smem_raw);
+
+    // The next kernel on the stream may launch now: a GEMV of the next layer
+    // starts its weight stream in the SM slots this grid frees, and whatever
+    // it is waits (griddepcontrol.wait) for this grid before it reads any
+    // result or rewrites any input of it.
+    asm volatile("griddepcontrol.launch_dependents;" :::);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int ntiles = (N + ROWS - 1) / ROWS;
-    const int nchunks = (K + CHUNK - 1) / CHUNK;
+    const int ntiles = (N + kRows - 1) / kRows;
+    const int nchunks = (K + kChunk - 1) / kChunk;
+    // Persistent grid: this CTA takes row tiles blockIdx.x, + gridDim.x, ...,
+    // each as nchunks stages; `total` stages in all.
+    const int my_tiles = (int)blockIdx.x < ntiles ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int total = my_tiles * nchunks;
 
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&sh.full[s], 1);
             mbar_init(&sh.empty[s], kConsumerWarps);
+        }
+        for (int b = 0; b < kRedBufs; ++b) {
+            mbar_init(&sh.red_full[b], kConsumerWarps);
+            mbar_init(&sh.red_empty[b], 1);
         }
         sh.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -144,159 +192,155 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
     __syncthreads();
     volatile int *abort = &sh.abort;
 
-    if (warp == kConsumerWarps) {
+    if (warp == kProducerWarp) {
         // ------------------------------------------------ producer
         if (lane == 0) {
             prefetch_tmap(&tm_codes);
             prefetch_tmap(&tm_srel);
-            int stage = 0;
-            uint32_t phase = 0;
-            int issued[STAGES];
-            uint32_t issued_phase[STAGES];
-            for (int s = 0; s < STAGES; ++s)
-                issued[s] = 0, issued_phase[s] = 0;
+            prefetch_tmap(&tm_x);
+            auto weights = [&](int q, int s) {
+                const int i = q / nchunks, tile = (int)blockIdx.x + i * (int)gridDim.x, c = q - i * nchunks;
+                tma_load_3d(sh.codes[s], &tm_codes, 0, tile * kRows, c * (kChunk / kSlice), &sh.full[s]);
+                tma_load_3d(sh.srel[s], &tm_srel, 0, tile * kRows, c * (kChunk / 256), &sh.full[s]);
+            };
+            auto acts = [&](int q, int s) {
+                tma_load_3d(sh.x[s], &tm_x, 0, 0, (q % nchunks) * (kChunk / kSlice), &sh.full[s]);
+            };
+            // The first stages' weights go out before the activation kernel has
+            // finished; their activation copies follow the dependency wait.
+            const int pre = total < STAGES ? total : STAGES;
+            for (int q = 0; q < pre; ++q) {
+                mbar_arrive_expect_tx(&sh.full[q], kStageTx);
+                weights(q, q);
+            }
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            for (int q = 0; q < pre; ++q)
+                acts(q, q);
+            int issued_upto = pre;  // stages [0, issued_upto) of the run have been issued
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
-                for (int c = 0; c < nchunks; ++c) {
-                    if (!mbar_wait_bounded(&sh.empty[stage], phase ^ 1u, abort)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_expect_tx(&sh.full[stage], C::kCodeBytes + C::kSrelBytes);
-                    tma_load_2d(sh.codes[stage], &tm_codes, c * (CHUNK / 8), tile * ROWS, &sh.full[stage]);
-                    tma_load_2d(sh.srel[stage], &tm_srel, c * (CHUNK / 16), tile * ROWS, &sh.full[stage]);
-                    issued[stage] = 1;
-                    issued_phase[stage] = phase;
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+            for (int q = pre; q < total; ++q) {
+                const int s = q % STAGES;
+                const uint32_t ph = (uint32_t)(q / STAGES) & 1u;
+                if (!mbar_wait_bounded(&sh.empty[s], ph ^ 1u, abort)) {
+                    ok = false;
+                    issued_upto = q;
+                    break;
                 }
+                mbar_arrive_expect_tx(&sh.full[s], kStageTx);
+                weights(q, s);
+                acts(q, s);
             }
             if (!ok) {
-                for (int s = 0; s < STAGES; ++s)
-                    if (issued[s]) {
-                        volatile int no_abort = 0;
-                        mbar_wait_bounded(&sh.full[s], issued_phase[s], &no_abort, 20000000ull);
-                    }
+                // let the copies in flight land before the CTA exits
+                for (int q = issued_upto - STAGES < 0 ? 0 : issued_upto - STAGES; q < issued_upto; ++q) {
+                    volatile int no_abort = 0;
+                    mbar_wait_bounded(&sh.full[q % STAGES], (uint32_t)(q / STAGES) & 1u, &no_abort, 20000000ull);
+                }
             }
         }
-    } else {
+    } else if (warp < kConsumerWarps) {
         // ------------------------------------------------ consumers
         {
             const uint4 e = lut_entry((uint32_t)tid, sh.cb);
 #pragma unroll
-            for (int r = 0; r < 8; ++r)
-                sh.lut8[tid * 8 + ((r + tid) & 7)] = e;
+            for (int r = 0; r < C::kCopies; ++r)
+                sh.lut[tid * C::kCopies + ((r + tid) & (C::kCopies - 1))] = e;
         }
         consumer_sync();
-        asm volatile("griddepcontrol.wait;" ::: "memory");
+        // (the consumers read only shared memory: the activation copies
+        // already wait for the previous kernel in the producer)
 
-        const int g = lane >> 2, t = lane & 3;
-        const uint4 *lutc = sh.lut8 + (lane & 7);
-        const bool vx = g < M;
-        // slice j of this warp in a stage: k offset 128 * (warp + 8 j) in the chunk
-        const int8_t *px = xq + (int64_t)g * K + 128 * warp + 32 * t;
-        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-        // The activation fragments of a chunk do not depend on the row tile;
-        // the next chunk's are fetched (through L1/L2) while the current one
-        // is computed.  Two register sets alternate with the chunk parity.
-        auto fetch_x = [&](int ch, uint4 (&X)[S][2]) {
-#pragma unroll
-            for (int j = 0; j < S; ++j) {
-                X[j][0] = X[j][1] = z4;
-                const int k0 = ch * CHUNK + 128 * (warp + 8 * j);
-                if (vx && k0 < K) {
-                    X[j][0] = *reinterpret_cast<const uint4 *>(px + (int64_t)ch * CHUNK + 1024 * j);
-                    X[j][1] = *reinterpret_cast<const uint4 *>(px + (int64_t)ch * CHUNK + 1024 * j + 16);
-                }
-            }
-        };
-        uint4 XA[S][2], XB[S][2];
+        const int g = lane >> 2, t = lane & 3, sl = warp;
+        const uint4 *lutc = sh.lut + (lane & (C::kCopies - 1));
+        // this thread's offsets inside a stage
+        const int off_code = sl * (kRows * 64) + g * 64 + 16 * t;                       // row g; g + 8 at +512
+        const int off_srel = (sl >> 1) * (kRows * 16) + g * 16 + 8 * (sl & 1) + 2 * t;  // row g; g + 8 at +128
+        const int off_x0 = sl * (kTokens * 128) + g * 128 + 16 * ((2 * t) ^ g);
+        const int off_x1 = sl * (kTokens * 128) + g * 128 + 16 * ((2 * t + 1) ^ g);
         int stage = 0;
         uint32_t phase = 0;
-        // consume one stage: all slices of this warp, all row groups
-        auto consume = [&](int ch, const uint4 (&X)[S][2], int32_t (&c)[RG][4], int32_t (&d)[RG][4]) {
-            const bool ok = mbar_wait_bounded_warp(&sh.full[stage], phase, abort);
-            if (ok) {
-#pragma unroll
-                for (int j = 0; j < S; ++j) {
-                    const int sl = warp + 8 * j;
-                    if (ch * CHUNK + 128 * sl < K) {
-                        const uint8_t *cs = sh.codes[stage] + 64 * sl + 16 * t + (CHUNK / 2) * g;
-                        const uint8_t *ss = sh.srel[stage] + 8 * sl + 2 * t + (CHUNK / 16) * g;
-#pragma unroll
-                        for (int rg = 0; rg < RG; ++rg)
-                            slice_mma(cs + (CHUNK / 2) * 16 * rg, cs + (CHUNK / 2) * (16 * rg + 8),
-                                      ss + (CHUNK / 16) * 16 * rg, ss + (CHUNK / 16) * (16 * rg + 8), lutc,
-                                      X[j][0], X[j][1], c[rg], d[rg]);
-                    }
+        for (int seg = 0; seg < my_tiles; ++seg) {
+            // two accumulators break the dependency chain between MMAs
+            int32_t c[4] = {0, 0, 0, 0}, d[4] = {0, 0, 0, 0};
+            for (int ch = 0; ch < nchunks; ++ch) {
+                const bool ok = mbar_wait_bounded_warp(&sh.full[stage], phase, abort);
+                if (ok && ch * kChunk + kSlice * sl < K) {
+                    Ops o;
+                    fetch_ops<C::kCopies>(o, sh.x[stage] + off_x0, sh.x[stage] + off_x1,
+                                          sh.codes[stage] + off_code, sh.srel[stage] + off_srel, lutc);
+                    slice_mma(o, c, d);
                 }
+                __syncwarp();
+                if (ok && lane == 0)
+                    mbar_arrive_relaxed(&sh.empty[stage]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            // hand the partial sums to the epilogue warp and go on
+            const int rb = seg % kRedBufs;
+            const bool ok = mbar_wait_bounded_warp(&sh.red_empty[rb], ((uint32_t)(seg / kRedBufs) & 1u) ^ 1u, abort);
+            // C fragment: c0 (row g, token 2t), c1 (g, 2t+1), c2 (g+8, 2t), c3 (g+8, 2t+1)
+            sh.red[rb][warp][g][2 * t] = c[0] + d[0];
+            sh.red[rb][warp][g][2 * t + 1] = c[1] + d[1];
+            sh.red[rb][warp][g + 8][2 * t] = c[2] + d[2];
+            sh.red[rb][warp][g + 8][2 * t + 1] = c[3] + d[3];
+            __syncwarp();
+            if (ok && lane == 0)
+                mbar_arrive(&sh.red_full[rb]);
+        }
+    } else {
+        // ------------------------------------------------ epilogue warp
+        // Per tile: sum the eight warps' partials and write the outputs, while
+        // the consumers already decode the next tile.
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        for (int seg = 0; seg < my_tiles; ++seg) {
+            const int tile = (int)blockIdx.x + seg * (int)gridDim.x;
+            // this lane's outputs: e = lane + 32 u -> row e / 8, token e % 8
+            float exs[4], ews[4], eb[4];
+            bool live[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = lane + 32 * u, r = e >> 3, m = e & 7, n = tile * kRows + r;
+                live[u] = m < M && n < N;
+                exs[u] = live[u] ? xs[m] : 0.0f;
+                ews[u] = live[u] ? ws[n] : 0.0f;
+                eb[u] = (live[u] && bias != nullptr) ? bias[n] : 0.0f;
+            }
+            const int rb = seg % kRedBufs;
+            const bool ok = mbar_wait_bounded_warp(&sh.red_full[rb], (uint32_t)(seg / kRedBufs) & 1u, abort);
+            int32_t acc[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = lane + 32 * u;
+                int32_t v = 0;
+#pragma unroll
+                for (int w = 0; w < kConsumerWarps; ++w)
+                    v += sh.red[rb][w][e >> 3][e & 7];
+                acc[u] = v;
             }
             __syncwarp();
             if (ok && lane == 0)
-                mbar_arrive(&sh.empty[stage]);
-            if (++stage == STAGES) {
-                stage = 0;
-                phase ^= 1u;
-            }
-        };
-        fetch_x(0, XA);
-        int xnext = nchunks > 1 ? 1 : 0;  // chunk whose fragments are fetched next
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
-            // two accumulators per row group break the dependency chain between MMAs
-            int32_t c[RG][4], d[RG][4];
+                mbar_arrive(&sh.red_empty[rb]);
+            if (ok && !*abort) {
 #pragma unroll
-            for (int rg = 0; rg < RG; ++rg)
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    c[rg][i] = d[rg][i] = 0;
-            // chunks in pairs: XA holds the even chunk's fragments, XB the odd one's
-            for (int ch = 0; ch < nchunks; ch += 2) {
-                fetch_x(xnext, XB);
-                if (++xnext == nchunks)
-                    xnext = 0;
-                consume(ch, XA, c, d);
-                if (ch + 1 < nchunks) {
-                    fetch_x(xnext, XA);
-                    if (++xnext == nchunks)
-                        xnext = 0;
-                    consume(ch + 1, XB, c, d);
-                } else {
-                    // odd chunk count: XB holds the next tile's chunk 0
-#pragma unroll
-                    for (int j = 0; j < S; ++j)
-                        XA[j][0] = XB[j][0], XA[j][1] = XB[j][1];
-                }
-            }
-#pragma unroll
-            for (int rg = 0; rg < RG; ++rg) {
-                // C fragment: c0 (row g, token 2t), c1 (g, 2t+1), c2 (g+8, 2t), c3 (g+8, 2t+1)
-                sh.red[warp][16 * rg + g][2 * t] = c[rg][0] + d[rg][0];
-                sh.red[warp][16 * rg + g][2 * t + 1] = c[rg][1] + d[rg][1];
-                sh.red[warp][16 * rg + g + 8][2 * t] = c[rg][2] + d[rg][2];
-                sh.red[warp][16 * rg + g + 8][2 * t + 1] = c[rg][3] + d[rg][3];
-            }
-            consumer_sync();
-            for (int e = tid; e < ROWS * 8; e += 256) {
-                const int r = e >> 3, m = e & 7;
-                int32_t acc = 0;
-#pragma unroll
-                for (int w = 0; w < kConsumerWarps; ++w)
-                    acc += sh.red[w][r][m];
-                const int n = tile * ROWS + r;
-                if (m < M && n < N && !*abort) {
-                    const float y = epilogue_value(acc, xs[m], ws[n], bias, n);
+                for (int u = 0; u < 4; ++u) {
+                    if (!live[u])
+                        continue;
+                    const int e = lane + 32 * u, n = tile * kRows + (e >> 3), m = e & 7;
+                    float y = __fmul_rn(__int2float_rn(acc[u]), __fmul_rn(exs[u], ews[u]));
+                    if (bias != nullptr)
+                        y = __fadd_rn(y, eb[u]);
                     const int64_t o = (int64_t)m * N + n;
                     if (out_f32)
                         reinterpret_cast<float *>(out)[o] = y;
                     else
                         reinterpret_cast<uint16_t *>(out)[o] = to_bf16_bits(y);
                     if (acc_out != nullptr)
-                        acc_out[o] = acc;
+                        acc_out[o] = acc[u];
                 }
             }
-            consumer_sync();
         }
     }
     __syncthreads();

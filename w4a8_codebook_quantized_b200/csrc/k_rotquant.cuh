@@ -175,6 +175,11 @@ __global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__re
     // Let a programmatic dependent (the decode GEMV) start its weight stream
     // now; it waits for this grid's results before it reads them.
     asm volatile("griddepcontrol.launch_dependents;" :::);
+    // Launched as a programmatic dependent itself, this grid may be resident
+    // before the previous kernel on the stream has finished: x may still be
+    // in the making and xq / xs still being read, so nothing is touched
+    // before that kernel completes.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     const int tid = threadIdx.x;
     const int hw = tid >> 4, L = tid & 15, warp = tid >> 5, lane = tid & 31;
@@ -255,19 +260,25 @@ __global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__re
 inline cudaError_t launch(const uint16_t *x, int64_t M, int64_t K, int64_t MP, int qmax, int8_t *xq, float *xs,
                           cudaStream_t stream)
 {
-    const dim3 grid((unsigned)MP), block(kThreads);
     const int64_t per_hw = (K / 256 + kHalfWarps - 1) / kHalfWarps;  // blocks per half-warp
-    if (per_hw <= 1)
-        rotquant_kernel<1, false><<<grid, block, 0, stream>>>(x, M, K, qmax, xq, xs);
-    else if (per_hw == 2)
-        rotquant_kernel<2, false><<<grid, block, 0, stream>>>(x, M, K, qmax, xq, xs);
-    else if (per_hw == 3)
-        rotquant_kernel<3, false><<<grid, block, 0, stream>>>(x, M, K, qmax, xq, xs);
-    else if (per_hw == 4)
-        rotquant_kernel<4, false><<<grid, block, 0, stream>>>(x, M, K, qmax, xq, xs);
-    else
-        rotquant_kernel<1, true><<<grid, block, 0, stream>>>(x, M, K, qmax, xq, xs);
-    return cudaGetLastError();
+    void (*kern)(const uint16_t *, int64_t, int64_t, int, int8_t *, float *) =
+        per_hw <= 1   ? rotquant_kernel<1, false>
+        : per_hw == 2 ? rotquant_kernel<2, false>
+        : per_hw == 3 ? rotquant_kernel<3, false>
+        : per_hw == 4 ? rotquant_kernel<4, false>
+                      : rotquant_kernel<1, true>;
+    // a programmatic dependent of the previous kernel on the stream: its
+    // launch overlaps that kernel's tail, and the kernel waits for it
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)MP);
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, x, M, K, qmax, xq, xs);
 }
 
 }  // namespace rq
