@@ -264,6 +264,15 @@ __device__ __forceinline__ T &smem_aligned_1024(uint8_t *smem_raw)
     return *reinterpret_cast<T *>(smem_raw + pad);
 }
 
+// Prefetch of a 3-D tile into L2 (no shared memory, no completion to track;
+// out-of-range parts of the box are ignored).
+__device__ __forceinline__ void tma_prefetch_3d(const void *tmap, int32_t x, int32_t y, int32_t z)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(tmap), "r"(x), "r"(y),
+                 "r"(z)
+                 : "memory");
+}
+
 // 3-D tiled bulk tensor load into this CTA's shared memory.
 __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, int32_t x, int32_t y, int32_t z,
                                             uint64_t *bar)

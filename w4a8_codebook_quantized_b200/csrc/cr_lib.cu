@@ -179,8 +179,11 @@ cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *x
                       {uK, (uint64_t)gv::kSlice},
                       {(uint32_t)gv::kSlice, (uint32_t)gv::kTokens, (uint32_t)(gv::kChunk / gv::kSlice)}, true))
         return CR_ERR_CUDA;
-    // persistent grid: at most one wave, whole row tiles per CTA
     const int64_t tiles = (N + gv::kRows - 1) / gv::kRows;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    // persistent grid of several CTAs per SM, at most one wave
     const int64_t slots = (int64_t)C::kMinBlocks * num_sms;
     const int64_t grid = tiles < slots ? tiles : slots;
     cudaLaunchConfig_t cfg = {};
@@ -188,13 +191,11 @@ cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *x
     cfg.blockDim = dim3(gv::kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     return launched(cudaLaunchKernelEx(&cfg, gv::gemv_kernel<C>, tc, ts, tx, xs, codebook, s_channel, bias, (int)M,
-                                       (int)N, (int)K, out_dtype == CR_OUT_F32 ? 1 : 0, out, acc_out));
+                                       (int)N, (int)K, out_dtype == CR_OUT_F32 ? 1 : 0, out, acc_out,
+                                       (uint32_t)(C::kCopies * sizeof(uint4)), gv::kPrefetchAhead));
 }
 
 // Shared validation of the contraction entry points.

@@ -7,7 +7,7 @@
 // are exact, so the result equals the prefill path bit for bit.
 //
 // B200 design.
-//  * Streaming: a persistent grid (three CTAs per SM).  In each CTA one
+//  * Streaming: a persistent grid (two CTAs per SM).  In each CTA one
 //    producer warp moves, per stage, the packed codes (16 weight rows x 1024
 //    columns, 8 KB), their group scales (1 KB) and the matching 1024 columns
 //    of the (at most 8) activation rows (8 KB) into a ring of shared-memory
@@ -62,6 +62,7 @@ constexpr int kCodeBytes = kRows * kChunk / 2;
 constexpr int kSrelBytes = kRows * kChunk / 16;
 constexpr int kXBytes = kTokens * kChunk;
 constexpr int kStageTx = kCodeBytes + kSrelBytes + kXBytes;
+constexpr int kPrefetchAhead = 3;  // L2 prefetch distance of the weight stream, in stages
 constexpr int kRedBufs = 1;  // partial-sum mailboxes between the consumers and the epilogue warp
 
 // Shape of the ring: STAGES stages, MINB CTAs per SM, COPIES copies of the
@@ -89,7 +90,7 @@ struct Cfg {
 };
 
 // The configuration the library launches.
-using Prod = Cfg<3, 3, 4>;
+using Prod = Cfg<5, 2, 4>;
 
 __device__ __forceinline__ void mma_s8(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                        uint32_t b0, uint32_t b1)
@@ -109,20 +110,22 @@ struct Ops {
     uint4 X0, X1, A, B, TA0, TA1, TB0, TB1;
 };
 
-// Fetch a stage's operands from shared memory.  `lutc` already points at this
-// lane's table copy; entry s is lutc[COPIES s].
-template <int COPIES>
+// Fetch a stage's operands from shared memory.  `lutb` points at this lane's
+// copy of the level table; the entry of scale byte s sits s * lut_step bytes
+// further.  lut_step is a kernel argument rather than a constant so that the
+// address is one integer multiply-add, which issues on the FMA pipe and leaves
+// the ALU pipe, the decode's bottleneck, to the byte permutes.
 __device__ __forceinline__ void fetch_ops(Ops &o, const uint8_t *x0, const uint8_t *x1, const uint8_t *codes_g,
-                                          const uint8_t *srel_g, const uint4 *lutc)
+                                          const uint8_t *srel_g, const uint8_t *lutb, uint32_t lut_step)
 {
     o.X0 = *reinterpret_cast<const uint4 *>(x0);
     o.X1 = *reinterpret_cast<const uint4 *>(x1);
     o.A = *reinterpret_cast<const uint4 *>(codes_g);
     o.B = *reinterpret_cast<const uint4 *>(codes_g + 8 * 64);
-    o.TA0 = lutc[COPIES * (uint32_t)srel_g[0]];
-    o.TA1 = lutc[COPIES * (uint32_t)srel_g[1]];
-    o.TB0 = lutc[COPIES * (uint32_t)srel_g[8 * 16]];
-    o.TB1 = lutc[COPIES * (uint32_t)srel_g[8 * 16 + 1]];
+    o.TA0 = *reinterpret_cast<const uint4 *>(lutb + (uint32_t)srel_g[0] * lut_step);
+    o.TA1 = *reinterpret_cast<const uint4 *>(lutb + (uint32_t)srel_g[1] * lut_step);
+    o.TB0 = *reinterpret_cast<const uint4 *>(lutb + (uint32_t)srel_g[8 * 16] * lut_step);
+    o.TB1 = *reinterpret_cast<const uint4 *>(lutb + (uint32_t)srel_g[8 * 16 + 1] * lut_step);
 }
 
 // One slice of the tile: rows g and g + 8 x 128 k against the token
@@ -148,12 +151,15 @@ __device__ __forceinline__ void slice_mma(const Ops &o, int32_t (&c)[4], int32_t
 //           {K / 2, 64} bytes, box {16, 16, 8}.
 // tm_srel:  the scale bytes, dims {16, N, K / 256}, strides {K / 16, 16}, box {16, 16, 4}.
 // tm_x:     xq, dims {128, M, K / 128}, strides {K, 128}, box {128, 8, 8}, 128-byte swizzle.
+// lut_step: bytes between the table entries of consecutive scale bytes in one
+//           copy (kCopies * 16).  ahead: L2 prefetch distance in stages.
 template <class C>
 __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
     gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_srel,
                 const __grid_constant__ CUtensorMap tm_x, const float *__restrict__ xs,
                 const float *__restrict__ codebook, const float *__restrict__ ws, const float *__restrict__ bias,
-                int M, int N, int K, int out_f32, void *__restrict__ out, int32_t *__restrict__ acc_out)
+                int M, int N, int K, int out_f32, void *__restrict__ out, int32_t *__restrict__ acc_out,
+                uint32_t lut_step, int ahead)
 {
     constexpr int STAGES = C::kStages;
     using Smem = typename C::Smem;
@@ -203,6 +209,16 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
                 tma_load_3d(sh.codes[s], &tm_codes, 0, tile * kRows, c * (kChunk / kSlice), &sh.full[s]);
                 tma_load_3d(sh.srel[s], &tm_srel, 0, tile * kRows, c * (kChunk / 256), &sh.full[s]);
             };
+            // L2 prefetch of the weights of stage q: `ahead` stages of HBM reads
+            // in flight beyond the shared-memory ring, so that a refill of the
+            // ring usually finds its data in L2
+            auto prefetch = [&](int q) {
+                if (q < total) {
+                    const int i = q / nchunks, tile = (int)blockIdx.x + i * (int)gridDim.x, c = q - i * nchunks;
+                    tma_prefetch_3d(&tm_codes, 0, tile * kRows, c * (kChunk / kSlice));
+                    tma_prefetch_3d(&tm_srel, 0, tile * kRows, c * (kChunk / 256));
+                }
+            };
             auto acts = [&](int q, int s) {
                 tma_load_3d(sh.x[s], &tm_x, 0, 0, (q % nchunks) * (kChunk / kSlice), &sh.full[s]);
             };
@@ -213,6 +229,8 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
                 mbar_arrive_expect_tx(&sh.full[q], kStageTx);
                 weights(q, q);
             }
+            for (int q = pre; q < pre + ahead; ++q)
+                prefetch(q);
             asm volatile("griddepcontrol.wait;" ::: "memory");
             for (int q = 0; q < pre; ++q)
                 acts(q, q);
@@ -229,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
                 mbar_arrive_expect_tx(&sh.full[s], kStageTx);
                 weights(q, s);
                 acts(q, s);
+                prefetch(q + ahead);
             }
             if (!ok) {
                 // let the copies in flight land before the CTA exits
@@ -251,34 +270,16 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
         // already wait for the previous kernel in the producer)
 
         const int g = lane >> 2, t = lane & 3, sl = warp;
-        const uint4 *lutc = sh.lut + (lane & (C::kCopies - 1));
+        const uint8_t *lutb = reinterpret_cast<const uint8_t *>(sh.lut + (lane & (C::kCopies - 1)));
         // this thread's offsets inside a stage
         const int off_code = sl * (kRows * 64) + g * 64 + 16 * t;                       // row g; g + 8 at +512
         const int off_srel = (sl >> 1) * (kRows * 16) + g * 16 + 8 * (sl & 1) + 2 * t;  // row g; g + 8 at +128
         const int off_x0 = sl * (kTokens * 128) + g * 128 + 16 * ((2 * t) ^ g);
         const int off_x1 = sl * (kTokens * 128) + g * 128 + 16 * ((2 * t + 1) ^ g);
-        int stage = 0;
-        uint32_t phase = 0;
-        for (int seg = 0; seg < my_tiles; ++seg) {
-            // two accumulators break the dependency chain between MMAs
-            int32_t c[4] = {0, 0, 0, 0}, d[4] = {0, 0, 0, 0};
-            for (int ch = 0; ch < nchunks; ++ch) {
-                const bool ok = mbar_wait_bounded_warp(&sh.full[stage], phase, abort);
-                if (ok && ch * kChunk + kSlice * sl < K) {
-                    Ops o;
-                    fetch_ops<C::kCopies>(o, sh.x[stage] + off_x0, sh.x[stage] + off_x1,
-                                          sh.codes[stage] + off_code, sh.srel[stage] + off_srel, lutc);
-                    slice_mma(o, c, d);
-                }
-                __syncwarp();
-                if (ok && lane == 0)
-                    mbar_arrive_relaxed(&sh.empty[stage]);
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
-            }
-            // hand the partial sums to the epilogue warp and go on
+        // chunks in which this warp's slice lies inside K (K is a multiple of 256)
+        const int nvalid = (K - kSlice * sl + kChunk - 1) / kChunk;
+        // hand a tile's partial sums to the epilogue warp and go on
+        auto hand_off = [&](int seg, int32_t (&c)[4], int32_t (&d)[4]) {
             const int rb = seg % kRedBufs;
             const bool ok = mbar_wait_bounded_warp(&sh.red_empty[rb], ((uint32_t)(seg / kRedBufs) & 1u) ^ 1u, abort);
             // C fragment: c0 (row g, token 2t), c1 (g, 2t+1), c2 (g+8, 2t), c3 (g+8, 2t+1)
@@ -289,6 +290,38 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
             __syncwarp();
             if (ok && lane == 0)
                 mbar_arrive(&sh.red_full[rb]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                c[i] = d[i] = 0;
+        };
+        // two accumulators break the dependency chain between MMAs
+        int32_t c[4] = {0, 0, 0, 0}, d[4] = {0, 0, 0, 0};
+        int ch = 0, seg = 0;
+        // The ring is walked STAGES stages at a time with the stage index a
+        // compile-time constant, so every shared-memory address is a fixed
+        // offset from this thread's base registers.
+        for (int q0 = 0; q0 < total; q0 += STAGES) {
+            const uint32_t ph = (uint32_t)(q0 / STAGES) & 1u;
+#pragma unroll
+            for (int s = 0; s < STAGES; ++s) {
+                if (q0 + s < total) {
+                    const bool ok = mbar_wait_bounded_warp(&sh.full[s], ph, abort);
+                    if (ok && ch < nvalid) {
+                        Ops o;
+                        fetch_ops(o, sh.x[s] + off_x0, sh.x[s] + off_x1, sh.codes[s] + off_code,
+                                  sh.srel[s] + off_srel, lutb, lut_step);
+                        slice_mma(o, c, d);
+                    }
+                    __syncwarp();
+                    if (ok && lane == 0)
+                        mbar_arrive_relaxed(&sh.empty[s]);
+                    if (++ch == nchunks) {
+                        hand_off(seg, c, d);
+                        ch = 0;
+                        ++seg;
+                    }
+                }
+            }
         }
     } else {
         // ------------------------------------------------ epilogue warp
