@@ -85,18 +85,38 @@ def gemv_launch_bytes(M, N, K):
     return weight_bytes(N, K) + M * K + 4 * M + 2 * M * N
 
 
-def prior_traffic(kernel_tag):
+GEMV_SOURCES = ("k_gemv.cuh", "cr_device.cuh")
+
+
+def source_digest(files):
+    """Short digest of kernel sources, to tell whether recorded counters are
+    still those of the current kernel."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "w4a8_codebook_quantized_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def prior_traffic(kernel_tag, sources=GEMV_SOURCES):
     """DRAM bytes per launch recorded from an ncu capture of the current kernel
-    (profiles/<tag>.traffic), or None."""
+    (profiles/<tag>.traffic), or None when there is none or the kernel's
+    sources changed since it was taken."""
     path = os.path.join(ROOT, "profiles", f"{kernel_tag}.traffic")
+    value, digest = None, None
     try:
         with open(path) as f:
             for line in f:
                 if line.startswith("dram_bytes_per_launch:"):
-                    return float(line.split(":", 1)[1])
+                    value = float(line.split(":", 1)[1])
+                elif line.startswith("source_digest:"):
+                    digest = line.split(":", 1)[1].strip()
     except OSError:
-        pass
-    return None
+        return None
+    if digest != source_digest(sources):
+        return None
+    return value
 
 
 # ---------------------------------------------------------------- clocks
