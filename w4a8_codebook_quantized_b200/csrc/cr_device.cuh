@@ -416,15 +416,6 @@ __device__ __forceinline__ void cluster_sync()
 }
 
 // Arrive on an mbarrier given by a shared::cluster address (this CTA's or the peer's).
-// Arrive on an mbarrier of a CTA of this cluster with the default semantics
-// (release at CTA scope).  For writers of this CTA's shared memory that the
-// tensor cores will read: after fence.proxy.async.shared::cta, this orders the
-// writes before the arrive without a cluster-wide memory fence.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
-{
-    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");

@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <climits>
+#include <functional>
 #include <cstdint>
 #include <mutex>
 
@@ -15,7 +16,6 @@
 #include "cr_device.cuh"
 #include "k_elementwise.cuh"
 #include "k_gemm.cuh"
-#include "k_gemm_dec.cuh"
 #include "k_gemv.cuh"
 #include "k_rotquant.cuh"
 
@@ -30,8 +30,11 @@ struct DeviceState {
     cudaMemPool_t pool = nullptr;  // stream-ordered pool for the prefill weight transient
     bool gemm_attr_set = false;
     bool gemm_pair_attr_set = false;
-    bool gemm_dec_attr_set = false;
     bool gemv_attr_set = false;
+    // side stream and events on which cr_w4a8_linear's prefill path decodes
+    // the weight while the activations are rotated and quantised
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
 };
 
 DeviceState g_dev[kMaxDevices];
@@ -133,21 +136,6 @@ bool make_tmap_i8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t r
     return r == CUDA_SUCCESS;
 }
 
-// 2-D uint8 tensor map without swizzle: a row-major [rows, inner] byte array
-// with the given row pitch, box [box_rows, box_inner].
-bool make_tmap_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows, uint64_t pitch,
-                  uint32_t box_inner, uint32_t box_rows)
-{
-    const cuuint64_t dims[2] = {inner, rows};
-    const cuuint64_t strides[1] = {pitch};
-    const cuuint32_t box[2] = {box_inner, box_rows};
-    const cuuint32_t estr[2] = {1u, 1u};
-    const CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
-                                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 // 3-D tensor map, no swizzle or the 128-byte swizzle, over `base` with the
 // given dims (innermost first), the byte strides of dims 1 and 2 and the box.
 // The strides need not increase: the maps below reorder a row-major array so
@@ -239,71 +227,39 @@ cr_status check_contraction(const int8_t *xq, const float *xs, const uint8_t *qd
     return CR_OK;
 }
 
-// The output tensor map of the GEMMs' TMA bulk stores: 32-row x 128-byte
-// boxes, 128-byte swizzle.
-bool make_tmap_out(CUtensorMap *to, void *out, int64_t M, int64_t N, bool out_f32)
+// The side stream and fork/join events of a device, created on first use.
+cr_status side_stream(DeviceState &d)
 {
-    const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
-    const cuuint64_t strides[1] = {(cuuint64_t)N * (out_f32 ? 4u : 2u)};
-    const cuuint32_t box[2] = {out_f32 ? 32u : 64u, 32u};
-    const cuuint32_t estr[2] = {1u, 1u};
-    return g_encode_tiled(to, out_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dims,
-                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (d.side != nullptr)
+        return CR_OK;
+    cudaStream_t s = nullptr;
+    cudaEvent_t f = nullptr, j = nullptr;
+    if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&f, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&j, cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();
+        if (s)
+            cudaStreamDestroy(s);
+        if (f)
+            cudaEventDestroy(f);
+        return CR_ERR_CUDA;
+    }
+    d.side = s;
+    d.fork = f;
+    d.join = j;
+    return CR_OK;
 }
 
+// The prefill contraction.  When `activations` is given (cr_w4a8_linear), it
+// launches the activation kernel on `stream` while the weight decode runs on
+// the device's side stream (the two are independent); the GEMM waits for both.
 cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
                    const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K,
-                   cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream)
+                   cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream,
+                   const std::function<cr_status()> *activations = nullptr)
 {
     using namespace cr;
-    const int out_f32 = out_dtype == CR_OUT_F32;
-    const int vec_ok = out_f32 ? (N % 4 == 0) : (N % 8 == 0);
-    // Output through TMA bulk stores when rows are 16-byte multiples and the
-    // int32 accumulators are not requested.
-    const int tma_out = vec_ok && acc_out == nullptr;
-    CUtensorMap ta, to;
-    if (!make_tmap_i8(&ta, xq, (uint64_t)K, (uint64_t)M, (uint32_t)gm::BM))
-        return CR_ERR_CUDA;
-    to = ta;  // placeholder when the output does not go through TMA
-    if (tma_out && !make_tmap_out(&to, out, M, N, out_f32))
-        return CR_ERR_CUDA;
-
-    // At least one 256 x 256 tile per SM pair: CTA pairs with the weight decode
-    // fused into the pipeline.
-    const int64_t pair_tiles = ((M + 255) / 256) * ((N + gm::BN - 1) / gm::BN);
-    if (pair_tiles >= d.num_sms / 2) {
-        if (!d.gemm_dec_attr_set) {
-            if (cudaFuncSetAttribute(gd::gemm_dec_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)gd::kSmemBytes) != cudaSuccess) {
-                cudaGetLastError();
-                return CR_ERR_CUDA;
-            }
-            d.gemm_dec_attr_set = true;
-        }
-        CUtensorMap tq, ts;
-        if (!make_tmap_u8(&tq, qdata, (uint64_t)(K / 2), (uint64_t)N, (uint64_t)(K / 2), (uint32_t)(gm::BK / 2), 128u) ||
-            !make_tmap_u8(&ts, srel, (uint64_t)(K / 16), (uint64_t)N, (uint64_t)(K / 16), 16u, 128u))
-            return CR_ERR_CUDA;
-        const int64_t pairs = pair_tiles < d.num_sms / 2 ? pair_tiles : d.num_sms / 2;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(2 * pairs));
-        cfg.blockDim = dim3(gd::kThreads);
-        cfg.dynamicSmemBytes = gd::kSmemBytes;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        return launched(cudaLaunchKernelEx(&cfg, gd::gemm_dec_pair_kernel, ta, tq, ts, to, codebook, xs, s_channel,
-                                           bias, (int)M, (int)N, (int)K, out_f32, tma_out, out, acc_out));
-    }
-
-    // Otherwise 128 x 256 tiles on single CTAs, the weight decoded once per
-    // call into an int8 transient from the library's stream-ordered pool.
     if (!d.gemm_attr_set) {
         if (cudaFuncSetAttribute(gm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gm::kSmemBytes) != cudaSuccess) {
@@ -312,16 +268,93 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
         }
         d.gemm_attr_set = true;
     }
+    // The int8 grid of the weight, decoded once per call into a transient
+    // from the library's stream-ordered pool.
     int8_t *w8 = nullptr;
     if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&w8), (size_t)(N * K), d.pool, stream) != cudaSuccess) {
         cudaGetLastError();
         return CR_ERR_CUDA;
     }
-    cr_status st = launched(ew::launch_decode(qdata, srel, codebook, N, K, w8, d.num_sms, stream));
-    CUtensorMap tb;
-    if (st == CR_OK && !make_tmap_i8(&tb, w8, (uint64_t)K, (uint64_t)N, (uint32_t)gm::BN))
+    cr_status st = CR_OK;
+    if (activations != nullptr) {
+        st = side_stream(d);
+        if (st == CR_OK && (cudaEventRecord(d.fork, stream) != cudaSuccess ||
+                            cudaStreamWaitEvent(d.side, d.fork, 0) != cudaSuccess)) {
+            cudaGetLastError();
+            st = CR_ERR_CUDA;
+        }
+        if (st == CR_OK)
+            st = launched(ew::launch_decode(qdata, srel, codebook, N, K, w8, d.num_sms, d.side));
+        if (st == CR_OK && cudaEventRecord(d.join, d.side) != cudaSuccess) {
+            cudaGetLastError();
+            st = CR_ERR_CUDA;
+        }
+        if (st == CR_OK)
+            st = (*activations)();
+        if (st == CR_OK && cudaStreamWaitEvent(stream, d.join, 0) != cudaSuccess) {
+            cudaGetLastError();
+            st = CR_ERR_CUDA;
+        }
+    } else {
+        st = launched(ew::launch_decode(qdata, srel, codebook, N, K, w8, d.num_sms, stream));
+    }
+    CUtensorMap ta, tb, to;
+    const int out_f32 = out_dtype == CR_OUT_F32;
+    const int vec_ok = out_f32 ? (N % 4 == 0) : (N % 8 == 0);
+    // Output through TMA bulk stores when rows are 16-byte multiples and the
+    // int32 accumulators are not requested: 32-row x 128-byte boxes, 128B swizzle.
+    const int tma_out = vec_ok && acc_out == nullptr;
+    if (st == CR_OK && (!make_tmap_i8(&ta, xq, (uint64_t)K, (uint64_t)M, (uint32_t)gm::BM) ||
+                        !make_tmap_i8(&tb, w8, (uint64_t)K, (uint64_t)N, (uint32_t)gm::BN)))
         st = CR_ERR_CUDA;
     if (st == CR_OK) {
+        to = ta;  // placeholder when the output does not go through TMA
+        if (tma_out) {
+            const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
+            const cuuint64_t strides[1] = {(cuuint64_t)N * (out_f32 ? 4u : 2u)};
+            const cuuint32_t box[2] = {out_f32 ? 32u : 64u, 32u};
+            const cuuint32_t estr[2] = {1u, 1u};
+            if (g_encode_tiled(&to, out_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out,
+                               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                st = CR_ERR_CUDA;
+        }
+    }
+    // 256 x 256 tiles on CTA pairs when there is at least one per SM pair;
+    // otherwise 128 x 256 tiles on single CTAs.
+    const int64_t pair_tiles = ((M + 255) / 256) * ((N + gm::BN - 1) / gm::BN);
+    const bool use_pair = pair_tiles >= d.num_sms / 2;
+    if (st == CR_OK && use_pair) {
+        CUtensorMap tb_half;
+        if (!d.gemm_pair_attr_set) {
+            if (cudaFuncSetAttribute(gm::gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)gm::pair::kSmemBytes) != cudaSuccess) {
+                cudaGetLastError();
+                st = CR_ERR_CUDA;
+            } else {
+                d.gemm_pair_attr_set = true;
+            }
+        }
+        if (st == CR_OK && !make_tmap_i8(&tb_half, w8, (uint64_t)K, (uint64_t)N, 128u))
+            st = CR_ERR_CUDA;
+        if (st == CR_OK) {
+            const int64_t pairs = pair_tiles < d.num_sms / 2 ? pair_tiles : d.num_sms / 2;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)(2 * pairs));
+            cfg.blockDim = dim3(gm::kThreads);
+            cfg.dynamicSmemBytes = gm::pair::kSmemBytes;
+            cfg.stream = stream;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            st = launched(cudaLaunchKernelEx(&cfg, gm::gemm_pair_kernel, ta, tb_half, to, xs, s_channel, bias, (int)M,
+                                             (int)N, (int)K, out_f32, vec_ok, tma_out, out, acc_out));
+        }
+    } else if (st == CR_OK) {
         const int64_t tiles = ((M + gm::BM - 1) / gm::BM) * ((N + gm::BN - 1) / gm::BN);
         const int grid = (int)(tiles < d.num_sms ? tiles : d.num_sms);
         gm::gemm_kernel<<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(ta, tb, to, xs, s_channel, bias, (int)M,
@@ -475,14 +508,17 @@ cr_status cr_w4a8_linear(const uint16_t *x, const uint8_t *qdata, const uint8_t 
     st = current_device(&d);
     if (st != CR_OK)
         return st;
-    st = launched(cr::rq::launch(x, M, K, MP, act_qmax, xq_work, xs_work, stream));
+    auto activations = [&]() { return launched(cr::rq::launch(x, M, K, MP, act_qmax, xq_work, xs_work, stream)); };
+    if (M > CR_GEMV_MAX_M) {
+        const std::function<cr_status()> act = activations;
+        return run_gemm(*d, xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, nullptr,
+                        stream, &act);
+    }
+    st = activations();
     if (st != CR_OK)
         return st;
-    if (M <= CR_GEMV_MAX_M)
-        return run_gemv(d->num_sms, d->gemv_attr_set, xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M,
-                        N, K, out_dtype, out, nullptr, stream, /*pdl=*/true);
-    return run_gemm(*d, xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, nullptr,
-                    stream);
+    return run_gemv(d->num_sms, d->gemv_attr_set, xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K,
+                    out_dtype, out, nullptr, stream, /*pdl=*/true);
 }
 
 // ---------------------------------------------------------------- decode forward without allocation

@@ -13,42 +13,67 @@ constexpr int kThreads = 256;
 // ai-toolkit convrot_w4a8_quant.py, unpack_w4a8_eager / w4a8_unpack_kernel:
 // w8[n, k] = sat_s8(rne(codebook[code] * fp8(srel[n, k/16]))).
 //
-// One thread decodes one 16-byte chunk of packed codes (32 weights, two
-// groups): a streaming 16-byte load, the two group scale bytes, two lookups in
-// the CTA's level table, four byte-permute decodes and two 16-byte stores.
-// HBM traffic per weight: 0.5 + 1/16 bytes in, 1 byte out.
+// Grid-stride over 16-byte chunks of packed codes (32 weights, two groups).
+// Each thread issues the loads of kDecodeUnroll chunks (64 bytes of codes and their
+// scale bytes) before it decodes any, so that enough bytes are in flight to
+// keep HBM busy; per chunk two lookups in the CTA's level table (4 copies, the
+// copy chosen by lane, to spread a quarter-warp's lookups over bank groups),
+// four byte-permute decodes and two 16-byte stores.  HBM traffic per weight:
+// 0.5 + 1/16 bytes in, 1 byte out.
+constexpr int kDecodeUnroll = 4;
+constexpr int kDecodeLutCopies = 4;
+
 __global__ void __launch_bounds__(kThreads) decode_int8_kernel(const uint8_t *__restrict__ qdata,
                                                                const uint8_t *__restrict__ srel,
                                                                const float *__restrict__ codebook, int64_t N,
                                                                int64_t K, int8_t *__restrict__ w8)
 {
-    __shared__ uint4 lut[256];
+    __shared__ uint4 lut[256 * kDecodeLutCopies];
     __shared__ float cb[16];
     if (threadIdx.x < 16)
         cb[threadIdx.x] = codebook[threadIdx.x];
     __syncthreads();
-    for (int s = threadIdx.x; s < 256; s += kThreads)
-        lut[s] = lut_entry((uint32_t)s, cb);
+    for (int s = threadIdx.x; s < 256; s += kThreads) {
+        const uint4 e = lut_entry((uint32_t)s, cb);
+#pragma unroll
+        for (int c = 0; c < kDecodeLutCopies; ++c)
+            lut[s * kDecodeLutCopies + c] = e;
+    }
     __syncthreads();
 
+    const uint4 *lutc = lut + (threadIdx.x & (kDecodeLutCopies - 1));
     const int64_t chunks_per_row = K / 32;
     const int64_t total = N * chunks_per_row;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < total; i += stride) {
-        const int64_t n = i / chunks_per_row;
-        const int64_t j = i - n * chunks_per_row;
-        const uint4 c = ldg_stream16(qdata + n * (K / 2) + 16 * j);
-        const uint32_t sb = __ldg(reinterpret_cast<const uint16_t *>(srel + n * (K / 16) + 2 * j));
-        const uint4 T0 = lut[sb & 0xFFu];
-        const uint4 T1 = lut[sb >> 8];
-        uint4 o0, o1;
-        decode8(c.x, T0, o0.x, o0.y);
-        decode8(c.y, T0, o0.z, o0.w);
-        decode8(c.z, T1, o1.x, o1.y);
-        decode8(c.w, T1, o1.z, o1.w);
-        uint4 *dst = reinterpret_cast<uint4 *>(w8 + n * K + 32 * j);
-        dst[0] = o0;
-        dst[1] = o1;
+    for (int64_t i0 = (int64_t)blockIdx.x * kThreads + threadIdx.x; i0 < total; i0 += kDecodeUnroll * stride) {
+        uint4 c[kDecodeUnroll];
+        uint32_t sb[kDecodeUnroll];
+#pragma unroll
+        for (int u = 0; u < kDecodeUnroll; ++u) {
+            const int64_t i = i0 + u * stride;
+            if (i < total) {
+                const int64_t n = i / chunks_per_row;
+                const int64_t j = i - n * chunks_per_row;
+                c[u] = ldg_stream16(qdata + n * (K / 2) + 16 * j);
+                sb[u] = __ldg(reinterpret_cast<const uint16_t *>(srel + n * (K / 16) + 2 * j));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kDecodeUnroll; ++u) {
+            const int64_t i = i0 + u * stride;
+            if (i < total) {
+                const uint4 T0 = lutc[kDecodeLutCopies * (sb[u] & 0xFFu)];
+                const uint4 T1 = lutc[kDecodeLutCopies * (sb[u] >> 8)];
+                uint4 o0, o1;
+                decode8(c[u].x, T0, o0.x, o0.y);
+                decode8(c[u].y, T0, o0.z, o0.w);
+                decode8(c[u].z, T1, o1.x, o1.y);
+                decode8(c[u].w, T1, o1.z, o1.w);
+                uint4 *dst = reinterpret_cast<uint4 *>(w8 + 32 * i);  // rows are K bytes: chunk i starts at 32 i
+                dst[0] = o0;
+                dst[1] = o1;
+            }
+        }
     }
 }
 
@@ -56,7 +81,7 @@ inline cudaError_t launch_decode(const uint8_t *qdata, const uint8_t *srel, cons
                                  int64_t K, int8_t *w8, int num_sms, cudaStream_t stream)
 {
     const int64_t total = N * (K / 32);
-    int64_t blocks = (total + kThreads - 1) / kThreads;
+    int64_t blocks = (total + (int64_t)kThreads * kDecodeUnroll - 1) / ((int64_t)kThreads * kDecodeUnroll);
     const int64_t cap = (int64_t)num_sms * 8;
     if (blocks > cap)
         blocks = cap;
