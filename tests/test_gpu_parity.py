@@ -238,3 +238,21 @@ def test_gemv_back_to_back_and_two_streams():
     torch.cuda.synchronize()
     for i, a in got:
         assert np.array_equal(host(a), ref[i])
+
+
+@pytest.mark.parametrize("M", [3, 300])
+def test_w4a8_linear_layer_object(M):
+    """The prepared layer gives cr_w4a8_linear's outputs bit for bit and checks
+    its per-call arguments."""
+    N, K = 520, 1024
+    layer = inputs.layer(N, K, 90 + M, with_bias=True)
+    x = bf16_dev(inputs.activations(M, K, 90 + M))
+    q, s, cb, ws, b = _layer_dev(layer)
+    lin = cr.W4A8Linear(q, s, cb, ws, b)
+    y1 = lin(x)
+    y2 = cr.cr_w4a8_linear(x, q, s, cb, ws, b)
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    with pytest.raises(ValueError):
+        lin(bf16_dev(inputs.activations(M, 512, 1)))
+    with pytest.raises(ValueError):
+        lin(x, xq_work=torch.empty(cr.gemv_rows(M) if M <= 8 else M, K, dtype=torch.int8))  # host tensor

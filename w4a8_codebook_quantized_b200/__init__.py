@@ -22,6 +22,7 @@ import threading
 from typing import Optional, Tuple
 
 __all__ = [
+    "W4A8Linear",
     "CrError", "lib", "library_path",
     "cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv",
     "cr_epilogue", "cr_w4a8_linear", "cr_w4a8_linear_decode_noalloc", "cr_check_device_error",
@@ -103,6 +104,9 @@ def _ptr(t) -> Optional[int]:
 def _stream(stream) -> Optional[int]:
     torch = _torch()
     if stream is None:
+        raw = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+        if raw is not None:  # the current stream's handle without building a Stream object
+            return raw(torch.cuda.current_device())
         stream = torch.cuda.current_stream()
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
@@ -279,6 +283,50 @@ def cr_w4a8_linear(x, qdata, srel, codebook, s_channel, bias=None, act_qmax: int
                                 M, N, K, int(act_qmax), _out_code(out.dtype), _ptr(out), _ptr(xq_work),
                                 _ptr(xs_work), _stream(stream)), "cr_w4a8_linear")
     return out
+
+
+class W4A8Linear:
+    """A layer whose buffers are checked once, for repeated forwards.
+
+    Holds qdata, srel, codebook, s_channel (and bias) as given (no copies) and
+    their device pointers; forward() checks only the activations, the output
+    and the work buffers, then makes the cr_w4a8_linear call.  The caller must
+    not resize or free the layer's tensors while the object is in use."""
+
+    def __init__(self, qdata, srel, codebook, s_channel, bias=None, act_qmax: int = 127):
+        self.N, self.K = _layer(qdata, srel, codebook, s_channel, bias)
+        if not 1 <= int(act_qmax) <= 127:
+            raise ValueError("act_qmax must be in 1..127")
+        self.act_qmax = int(act_qmax)
+        self._tensors = (qdata, srel, codebook, s_channel, bias)  # keep them alive
+        self._ptrs = (_ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), _ptr(bias))
+        self._fn = lib().cr_w4a8_linear
+
+    def forward(self, x, out=None, xq_work=None, xs_work=None, stream=None):
+        torch = _torch()
+        _need(x, "x", (torch.bfloat16,), 2)
+        M, K = x.shape
+        if K != self.K:
+            raise ValueError(f"x has K={K}, the layer K={self.K}")
+        rows = gemv_rows(M) if 1 <= M <= CR_GEMV_MAX_M else M
+        if xq_work is None:
+            xq_work = torch.empty(rows, K, dtype=torch.int8, device=x.device)
+        elif not xq_work.is_cuda or xq_work.dtype != torch.int8 or xq_work.dim() != 2 or xq_work.shape[0] < rows \
+                or xq_work.shape[1] != K or not xq_work.is_contiguous():
+            raise ValueError(f"xq_work must be a contiguous CUDA int8 [>= {rows}, {K}] tensor")
+        if xs_work is None:
+            xs_work = torch.empty(rows, dtype=torch.float32, device=x.device)
+        elif not xs_work.is_cuda or xs_work.dtype != torch.float32 or xs_work.dim() != 1 or xs_work.shape[0] < rows:
+            raise ValueError(f"xs_work must be a CUDA float32 [>= {rows}] tensor")
+        if out is None:
+            out = torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
+        _need(out, "out", (torch.bfloat16, torch.float32), shape=(M, self.N))
+        q, s, cb, ws, b = self._ptrs
+        _check(self._fn(x.data_ptr(), q, s, cb, ws, b, M, self.N, K, self.act_qmax, _out_code(out.dtype),
+                        out.data_ptr(), xq_work.data_ptr(), xs_work.data_ptr(), _stream(stream)), "cr_w4a8_linear")
+        return out
+
+    __call__ = forward
 
 
 def cr_w4a8_linear_decode_noalloc(x, qdata, srel, codebook, s_channel, bias=None, act_qmax: int = 127,
