@@ -233,6 +233,50 @@ cr_status cr_w4a8_linear_decode_noalloc(const uint16_t *x, const uint8_t *qdata,
                                         void *out, cr_stream_t stream);
 
 /*
+ * (8) Several layers fed the same input, in one decode launch.
+ *
+ * Defined by: ai-toolkit convrot_w4a8_quant.py, w4a8_grouped_linear (layers
+ * that share the rotation share one rotate + quantise of x on the decode
+ * path) and gemv_prepared for each layer.  Here the layers' GEMVs are also one
+ * launch: their row tiles are numbered one after the other and spread over
+ * one persistent grid, so small layers (q/k/v, gate/up) share one ramp-up and
+ * one tail.  Every layer's outputs equal those of cr_w4a8_gemv on that layer,
+ * bit for bit.
+ *
+ * cr_w4a8_layer (all pointers device pointers, 16-byte aligned):
+ *   qdata [N, K/2], srel [N, K/16], s_channel [N], bias [N] or NULL,
+ *   out [M, N] (bf16 or fp32 as out_dtype), acc_out [M, N] int32 or NULL.
+ *   N >= 0 (N == 0: the layer produces nothing).
+ * All layers use the same K, the same codebook[16] (the one they were
+ * quantised with; the pages' fixed codebook) and the same activations.
+ * 1 <= num_layers <= CR_MAX_LAYERS, else CR_ERR_INVALID_ARG; `layers` is a
+ * host array, read during the call only.
+ */
+#define CR_MAX_LAYERS 4
+typedef struct {
+    const uint8_t *qdata;
+    const uint8_t *srel;
+    const float *s_channel;
+    const float *bias;
+    int64_t N;
+    void *out;
+    int32_t *acc_out;
+} cr_w4a8_layer;
+
+/* (8a) The grouped decode GEMV on quantised activations (xq [>= M, K] int8,
+ * xs [M] fp32), 1 <= M <= 8; M > 8 gives CR_ERR_UNSUPPORTED. */
+cr_status cr_w4a8_gemv_grouped(const int8_t *xq, const float *xs, const float *codebook, int64_t M, int64_t K,
+                               const cr_w4a8_layer *layers, int num_layers, cr_out_dtype out_dtype,
+                               cr_stream_t stream);
+
+/* (8b) The grouped layer forward: (1) once, then (8a) when M <= 8, or (3)
+ * for each layer when M > 8.  x, xq_work, xs_work as in (6); acc_out must be
+ * NULL in every layer (CR_ERR_INVALID_ARG otherwise). */
+cr_status cr_w4a8_linear_grouped(const uint16_t *x, const float *codebook, int64_t M, int64_t K,
+                                 const cr_w4a8_layer *layers, int num_layers, int act_qmax,
+                                 cr_out_dtype out_dtype, int8_t *xq_work, float *xs_work, cr_stream_t stream);
+
+/*
  * Waits for `stream`, then reads and clears the library's device error word,
  * which a kernel sets when one of its bounded pipeline waits runs out (the
  * kernel then abandons its tile and exits; its outputs are unspecified).

@@ -28,7 +28,8 @@ def _declared():
 def test_header_declares_the_boundary():
     names = _declared()
     for n in ("cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv", "cr_epilogue",
-              "cr_w4a8_linear", "cr_status_string", "cr_check_device_error", "cr_version"):
+              "cr_w4a8_linear", "cr_status_string", "cr_check_device_error", "cr_version",
+              "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped"):
         assert n in names
 
 
@@ -119,6 +120,42 @@ def test_epilogue_and_linear_validation(L):
     assert f(A16, A16, A16, A16, A16, None, 2, 8, 384, 127, 0, A16, A16, A16, None) == cr.CR_ERR_UNSUPPORTED
     assert f(None, A16, A16, A16, A16, None, 2, 8, 256, 127, 0, A16, A16, A16, None) == cr.CR_ERR_INVALID_ARG
     assert f(MIS, A16, A16, A16, A16, None, 2, 8, 256, 127, 0, A16, A16, A16, None) == cr.CR_ERR_ALIGNMENT
+
+
+def _layers(*specs):
+    """A cr_w4a8_layer array; each spec is a dict of field overrides."""
+    arr = (cr.CrLayer * max(1, len(specs)))()
+    for i, sp in enumerate(specs):
+        f = dict(qdata=A16, srel=A16, s_channel=A16, bias=None, N=8, out=A16, acc_out=None)
+        f.update(sp)
+        arr[i] = cr.CrLayer(**f)
+    return arr
+
+
+def test_grouped_validation(L):
+    g = L.cr_w4a8_gemv_grouped
+    two = _layers({}, {"N": 16})
+    assert g(A16, A16, A16, 4, 256, two, 0, 0, None) == cr.CR_ERR_INVALID_ARG            # no layers
+    assert g(A16, A16, A16, 4, 256, _layers(*[{}] * 5), 5, 0, None) == cr.CR_ERR_INVALID_ARG  # > CR_MAX_LAYERS
+    assert g(A16, A16, A16, 4, 256, None, 1, 0, None) == cr.CR_ERR_INVALID_ARG
+    assert g(A16, A16, A16, 9, 256, two, 2, 0, None) == cr.CR_ERR_UNSUPPORTED             # M > 8
+    assert g(A16, A16, A16, 4, 320, two, 2, 0, None) == cr.CR_ERR_UNSUPPORTED             # K % 256
+    assert g(A16, A16, A16, 4, 256, two, 2, 5, None) == cr.CR_ERR_INVALID_ARG             # out dtype
+    assert g(A16, A16, A16, 4, 256, _layers({}, {"srel": MIS}), 2, 0, None) == cr.CR_ERR_ALIGNMENT
+    assert g(A16, A16, A16, 4, 256, _layers({}, {"out": None}), 2, 0, None) == cr.CR_ERR_INVALID_ARG
+    assert g(A16, A16, A16, 4, 256, _layers({"N": -1}), 1, 0, None) == cr.CR_ERR_INVALID_ARG
+    assert g(A16, A16, MIS, 4, 256, two, 2, 0, None) == cr.CR_ERR_ALIGNMENT               # codebook
+    # empty layers may carry null pointers; an all-empty call or M == 0 does nothing
+    empty = _layers({"N": 0, "qdata": None, "srel": None, "s_channel": None, "out": None})
+    assert g(A16, A16, A16, 4, 256, empty, 1, 0, None) == cr.CR_OK
+    assert g(None, None, None, 0, 256, two, 2, 0, None) == cr.CR_OK
+    f = L.cr_w4a8_linear_grouped
+    assert f(A16, A16, 2, 256, two, 2, 0, 0, A16, A16, None) == cr.CR_ERR_INVALID_ARG       # act_qmax
+    assert f(A16, A16, 2, 256, _layers({"acc_out": A16}), 1, 127, 0, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(None, A16, 2, 256, two, 2, 127, 0, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(MIS, A16, 2, 256, two, 2, 127, 0, A16, A16, None) == cr.CR_ERR_ALIGNMENT
+    assert f(A16, A16, 2, 256, two, 2, 127, 0, MIS, A16, None) == cr.CR_ERR_ALIGNMENT
+    assert f(None, A16, 2, 256, empty, 1, 127, 0, None, None, None) == cr.CR_OK
 
 
 def test_valid_call_without_a_gpu_fails_loudly(L):

@@ -256,3 +256,68 @@ def test_w4a8_linear_layer_object(M):
         lin(bf16_dev(inputs.activations(M, 512, 1)))
     with pytest.raises(ValueError):
         lin(x, xq_work=torch.empty(cr.gemv_rows(M) if M <= 8 else M, K, dtype=torch.int8))  # host tensor
+
+
+# ---------------------------------------------------------------- grouped decode (several layers, one input)
+
+@pytest.mark.parametrize("M,K,Ns,bias", [(1, 1024, (512, 512, 512), False),      # q/k/v
+                                         (4, 2048, (2048, 512, 512), True),      # q and grouped k/v
+                                         (8, 1024, (2816, 2816), False),          # gate/up
+                                         (3, 768, (17, 0, 1000, 8), True),        # ragged and an empty layer
+                                         (2, 16384, (520, 1040), False)])         # activations streamed
+def test_gemv_grouped_matches_oracle_and_single_layers(M, K, Ns, bias):
+    """Each layer of a grouped call equals the oracle's contraction of that
+    layer (int32 bit-exact, bf16 within tolerance) and the single-layer
+    decode GEMV bit for bit."""
+    x = inputs.activations(M, K, 300 + M)
+    xq_r, xs_r = oracle.rotate_quant_act(x, None, 127)
+    xq, xs = dev(xq_r), dev(xs_r)
+    layers = [inputs.layer(N, K, 310 + i, with_bias=bias) if N else None for i, N in enumerate(Ns)]
+    cb = dev(inputs.codebook())
+    specs, guards = [], []
+    for ly, N in zip(layers, Ns):
+        if ly is None:
+            z = torch.empty(0, K // 2, dtype=torch.uint8, device="cuda")
+            specs.append((z, torch.empty(0, K // 16, dtype=torch.uint8, device="cuda"),
+                          torch.empty(0, device="cuda")))
+        else:
+            q, s, _, ws, b = _layer_dev(ly)
+            specs.append((q, s, ws, b))
+        guards.append(Guarded((M, N), torch.bfloat16))
+    outs, accs = cr.cr_w4a8_gemv_grouped(xq, xs, cb, specs, outs=[g.tensor for g in guards], acc_out=True)
+    torch.cuda.synchronize()
+    for (ly, N), go, acc, out in zip(zip(layers, Ns), guards, accs, outs):
+        assert go.intact()
+        if ly is None:
+            continue
+        w8 = oracle.decode_w8(ly.qdata, ly.srel, ly.codebook)
+        acc_r = oracle.gemm_s32(xq_r, w8, THREADS)
+        y_r = oracle.epilogue(acc_r, xs_r, ly.s_channel, ly.bias, "bf16")
+        assert np.array_equal(host(acc), acc_r)
+        assert_output_close(host(out), y_r, "bf16")
+        q, s, _, ws, b = _layer_dev(ly)
+        o1, a1 = cr.cr_w4a8_gemv(xq, xs, q, s, cb, ws, b, acc_out=True)
+        assert torch.equal(a1, acc) and torch.equal(o1.view(torch.int16), out.view(torch.int16))
+
+
+@pytest.mark.parametrize("M", [2, 7, 200])
+def test_linear_grouped_end_to_end(M):
+    """One rotate + quantise for all layers, then the grouped GEMV (M <= 8)
+    or a GEMM per layer; each output equals the single-layer forward."""
+    K, Ns = 1024, (768, 256, 256)
+    x = inputs.activations(M, K, 400 + M)
+    cb = dev(inputs.codebook())
+    layers = [inputs.layer(N, K, 410 + i, with_bias=(i == 0)) for i, N in enumerate(Ns)]
+    devs = [_layer_dev(ly) for ly in layers]
+    xd = bf16_dev(x)
+    outs = cr.cr_w4a8_linear_grouped(xd, cb, [(q, s, ws, b) for q, s, _, ws, b in devs])
+    for ly, (q, s, _, ws, b), y in zip(layers, devs, outs):
+        y1 = cr.cr_w4a8_linear(xd, q, s, cb, ws, b)
+        assert torch.equal(y1.view(torch.int16), y.view(torch.int16))
+        ref = oracle.linear(x, ly.qdata, ly.srel, ly.codebook, ly.s_channel, ly.bias, threads=THREADS)
+        assert_output_close(host(y), ref["y"], "bf16")
+    # fp32 outputs through the same call
+    outs32 = cr.cr_w4a8_linear_grouped(xd, cb, [(q, s, ws, b) for q, s, _, ws, b in devs], out_dtype=torch.float32)
+    for ly, y in zip(layers, outs32):
+        ref = oracle.linear(x, ly.qdata, ly.srel, ly.codebook, ly.s_channel, ly.bias, out="f32", threads=THREADS)
+        assert_output_close(host(y), ref["y"], "f32")

@@ -26,6 +26,7 @@ __all__ = [
     "CrError", "lib", "library_path",
     "cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv",
     "cr_epilogue", "cr_w4a8_linear", "cr_w4a8_linear_decode_noalloc", "cr_check_device_error",
+    "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped", "CrLayer",
     "cr_status_string", "cr_version",
     "gemv_rows",
 ]
@@ -36,6 +37,14 @@ _LIB_PATH = os.path.join(_PKG, "libcr_w4a8.so")
 CR_OK, CR_ERR_INVALID_ARG, CR_ERR_UNSUPPORTED, CR_ERR_ALIGNMENT, CR_ERR_CUDA, CR_ERR_TIMEOUT, CR_ERR_NO_DEVICE = range(7)
 CR_OUT_BF16, CR_OUT_F32 = 0, 1
 CR_GEMV_MAX_M = 8
+CR_MAX_LAYERS = 4
+
+
+class CrLayer(ctypes.Structure):
+    """cr_w4a8_layer: one layer of a grouped call (device pointers)."""
+    _fields_ = [("qdata", ctypes.c_void_p), ("srel", ctypes.c_void_p), ("s_channel", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("N", ctypes.c_int64), ("out", ctypes.c_void_p),
+                ("acc_out", ctypes.c_void_p)]
 
 _lib = None
 _lock = threading.Lock()
@@ -74,6 +83,9 @@ def lib() -> ctypes.CDLL:
             L.cr_w4a8_linear.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P, P, P]
             L.cr_check_device_error.argtypes = [P]
             L.cr_w4a8_linear_decode_noalloc.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P]
+            LP = ctypes.POINTER(CrLayer)
+            L.cr_w4a8_gemv_grouped.argtypes = [P, P, P, i64, i64, LP, i32, i32, P]
+            L.cr_w4a8_linear_grouped.argtypes = [P, P, i64, i64, LP, i32, i32, i32, P, P, P]
             for name in ("cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv",
                          "cr_epilogue", "cr_w4a8_linear", "cr_check_device_error",
                          "cr_w4a8_linear_decode_noalloc"):
@@ -351,6 +363,86 @@ def cr_w4a8_linear_decode_noalloc(x, qdata, srel, codebook, s_channel, bias=None
                                                _out_code(out.dtype), _ptr(out), _stream(stream)),
            "cr_w4a8_linear_decode_noalloc")
     return out
+
+
+def _grouped(layers, codebook, K, M, out_dtype, outs, acc_out, device):
+    """Check a list of (qdata, srel, s_channel[, bias]) layers that share K and
+    the codebook; allocate missing outputs; return the C array and the outputs."""
+    torch = _torch()
+    layers = list(layers)
+    if not 1 <= len(layers) <= CR_MAX_LAYERS:
+        raise ValueError(f"1..{CR_MAX_LAYERS} layers, got {len(layers)}")
+    if outs is not None and len(outs) != len(layers):
+        raise ValueError("one output per layer")
+    arr = (CrLayer * len(layers))()
+    res, accs = [], []
+    for i, ly in enumerate(layers):
+        qdata, srel, s_channel = ly[0], ly[1], ly[2]
+        bias = ly[3] if len(ly) > 3 else None
+        N, Kw = _layer(qdata, srel, codebook, s_channel, bias)
+        if Kw != K:
+            raise ValueError(f"layer {i} has K={Kw}, expected {K}")
+        out = None if outs is None else outs[i]
+        if out is None:
+            out = torch.empty(M, N, dtype=out_dtype, device=device)
+        _need(out, f"out[{i}]", (torch.bfloat16, torch.float32), shape=(M, N))
+        if out.dtype != out_dtype:
+            raise TypeError("all outputs of a grouped call have one dtype")
+        acc = None
+        if acc_out:
+            acc = torch.empty(M, N, dtype=torch.int32, device=device)
+        arr[i] = CrLayer(_ptr(qdata), _ptr(srel), _ptr(s_channel), _ptr(bias), N, _ptr(out), _ptr(acc))
+        res.append(out)
+        accs.append(acc)
+    return arr, res, accs
+
+
+def cr_w4a8_gemv_grouped(xq, xs, codebook, layers, m: Optional[int] = None, out_dtype=None, outs=None,
+                         acc_out: bool = False, stream=None):
+    """Decode GEMV of 1..4 layers on the same quantised activations in one
+    launch.  layers: (qdata, srel, s_channel[, bias]) per layer.  Returns the
+    list of outputs (and of int32 accumulators when acc_out=True); each equals
+    cr_w4a8_gemv on that layer bit for bit."""
+    torch = _torch()
+    _need(xq, "xq", (torch.int8,), 2)
+    _need(xs, "xs", (torch.float32,), 1)
+    M = xq.shape[0] if m is None else int(m)
+    K = xq.shape[1]
+    if xq.shape[0] < M or xs.shape[0] < M:
+        raise ValueError(f"xq {tuple(xq.shape)} / xs {tuple(xs.shape)} have fewer than M={M} rows")
+    if out_dtype is None:
+        out_dtype = outs[0].dtype if outs else torch.bfloat16
+    _out_code(out_dtype)
+    arr, res, accs = _grouped(layers, codebook, K, M, out_dtype, outs, acc_out, xq.device)
+    _check(lib().cr_w4a8_gemv_grouped(_ptr(xq), _ptr(xs), _ptr(codebook), M, K, arr, len(res),
+                                      _out_code(out_dtype), _stream(stream)), "cr_w4a8_gemv_grouped")
+    return (res, accs) if acc_out else res
+
+
+def cr_w4a8_linear_grouped(x, codebook, layers, act_qmax: int = 127, out_dtype=None, outs=None,
+                           xq_work=None, xs_work=None, stream=None):
+    """Forward of 1..4 layers fed the same x (q/k/v, gate/up): one rotate +
+    quantise, then one grouped decode GEMV (M <= 8) or a GEMM per layer."""
+    torch = _torch()
+    _need(x, "x", (torch.bfloat16,), 2)
+    M, K = x.shape
+    if out_dtype is None:
+        out_dtype = outs[0].dtype if outs else torch.bfloat16
+    _out_code(out_dtype)
+    arr, res, _ = _grouped(layers, codebook, K, M, out_dtype, outs, False, x.device)
+    rows = gemv_rows(M) if 1 <= M <= CR_GEMV_MAX_M else M
+    if xq_work is None:
+        xq_work = torch.empty(rows, K, dtype=torch.int8, device=x.device)
+    if xs_work is None:
+        xs_work = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _need(xq_work, "xq_work", (torch.int8,), 2)
+    _need(xs_work, "xs_work", (torch.float32,), 1)
+    if xq_work.shape[0] < rows or xq_work.shape[1] != K or xs_work.shape[0] < rows:
+        raise ValueError(f"work buffers need {rows} rows of K={K}")
+    _check(lib().cr_w4a8_linear_grouped(_ptr(x), _ptr(codebook), M, K, arr, len(res), int(act_qmax),
+                                        _out_code(out_dtype), _ptr(xq_work), _ptr(xs_work), _stream(stream)),
+           "cr_w4a8_linear_grouped")
+    return res
 
 
 def cr_check_device_error(stream=None) -> None:

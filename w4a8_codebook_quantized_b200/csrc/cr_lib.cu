@@ -10,6 +10,7 @@
 #include <climits>
 #include <functional>
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 
 #include "cr_w4a8.h"
@@ -154,15 +155,17 @@ bool make_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype,
     return r == CUDA_SUCCESS;
 }
 
-// The decode GEMV: three tensor maps that put a stage into shared memory as
-// codes [slice][row][64 B], scales [256-column block][row][16 B] and
-// activations [slice][token][128 B] (128-byte swizzle); a persistent grid of
-// as many CTAs as fit on the SMs, optionally as a programmatic dependent of
-// the previous kernel on the stream.
-cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const uint8_t *qdata,
-                   const uint8_t *srel, const float *codebook, const float *s_channel, const float *bias, int64_t M,
-                   int64_t N, int64_t K, cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream,
-                   bool pdl)
+// The decode GEMV over 1..CR_MAX_LAYERS layers that share the activations
+// and the codebook (layers[i].N may be 0).  Layer arguments are already
+// checked.  Tensor maps put a stage into shared memory as codes
+// [slice][row][64 B] and scales [256-column block][row][16 B] (one pair per
+// layer) and activations [slice][token][128 B] (128-byte swizzle); the row
+// tiles of all layers are numbered one after the other and run on a
+// persistent grid of as many CTAs as fit on the SMs, optionally as a
+// programmatic dependent of the previous kernel on the stream.
+cr_status run_gemv_layers(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const float *codebook,
+                          int64_t M, int64_t K, const cr_w4a8_layer *layers, int num_layers, cr_out_dtype out_dtype,
+                          cudaStream_t stream, bool pdl)
 {
     using namespace cr;
     using C = gv::Prod;
@@ -174,17 +177,45 @@ cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *x
         }
         attr_set = true;
     }
-    CUtensorMap tc, ts, tx;
-    const uint64_t uK = (uint64_t)K, uN = (uint64_t)N, uM = (uint64_t)M;
-    if (!make_tmap_3d(&tc, qdata, CU_TENSOR_MAP_DATA_TYPE_UINT32, {16, uN, uK / gv::kSlice}, {uK / 2, 64},
-                      {16, (uint32_t)gv::kRows, (uint32_t)(gv::kChunk / gv::kSlice)}, false) ||
-        !make_tmap_3d(&ts, srel, CU_TENSOR_MAP_DATA_TYPE_UINT8, {16, uN, uK / 256}, {uK / 16, 16},
-                      {16, (uint32_t)gv::kRows, (uint32_t)(gv::kChunk / 256)}, false) ||
-        !make_tmap_3d(&tx, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, {(uint64_t)gv::kSlice, uM, uK / gv::kSlice},
+    gv::GemvArgs args;
+    memset(&args, 0, sizeof(args));
+    const uint64_t uK = (uint64_t)K, uM = (uint64_t)M;
+    int64_t tiles = 0;
+    for (int l = 0; l < num_layers; ++l) {
+        const cr_w4a8_layer &ly = layers[l];
+        args.layer[l].tile0 = (int)tiles;
+        if (ly.N == 0)
+            continue; // no tiles; its pointers may be null
+        const uint64_t uN = (uint64_t)ly.N;
+        if (!make_tmap_3d(&args.tm_codes[l], ly.qdata, CU_TENSOR_MAP_DATA_TYPE_UINT32, {16, uN, uK / gv::kSlice},
+                          {uK / 2, 64}, {16, (uint32_t)gv::kRows, (uint32_t)(gv::kChunk / gv::kSlice)}, false) ||
+            !make_tmap_3d(&args.tm_srel[l], ly.srel, CU_TENSOR_MAP_DATA_TYPE_UINT8, {16, uN, uK / 256}, {uK / 16, 16},
+                          {16, (uint32_t)gv::kRows, (uint32_t)(gv::kChunk / 256)}, false))
+            return CR_ERR_CUDA;
+        args.layer[l].ws = ly.s_channel;
+        args.layer[l].bias = ly.bias;
+        args.layer[l].out = ly.out;
+        args.layer[l].acc_out = ly.acc_out;
+        args.layer[l].N = (int)ly.N;
+        tiles += (ly.N + gv::kRows - 1) / gv::kRows;
+    }
+    if (tiles == 0)
+        return CR_OK;
+    if (tiles > INT_MAX)
+        return CR_ERR_UNSUPPORTED;
+    if (!make_tmap_3d(&args.tm_x, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, {(uint64_t)gv::kSlice, uM, uK / gv::kSlice},
                       {uK, (uint64_t)gv::kSlice},
                       {(uint32_t)gv::kSlice, (uint32_t)gv::kTokens, (uint32_t)(gv::kChunk / gv::kSlice)}, true))
         return CR_ERR_CUDA;
-    const int64_t tiles = (N + gv::kRows - 1) / gv::kRows;
+    args.xs = xs;
+    args.codebook = codebook;
+    args.M = (int)M;
+    args.K = (int)K;
+    args.num_layers = num_layers;
+    args.num_tiles = (int)tiles;
+    args.out_f32 = out_dtype == CR_OUT_F32 ? 1 : 0;
+    args.lut_step = (uint32_t)(C::kCopies * sizeof(uint4));
+    args.ahead = gv::kPrefetchAhead;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -198,9 +229,24 @@ cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *x
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return launched(cudaLaunchKernelEx(&cfg, gv::gemv_kernel<C>, tc, ts, tx, xs, codebook, s_channel, bias, (int)M,
-                                       (int)N, (int)K, out_dtype == CR_OUT_F32 ? 1 : 0, out, acc_out,
-                                       (uint32_t)(C::kCopies * sizeof(uint4)), gv::kPrefetchAhead));
+    return launched(cudaLaunchKernelEx(&cfg, gv::gemv_kernel<C>, args));
+}
+
+// One layer.
+cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const uint8_t *qdata,
+                   const uint8_t *srel, const float *codebook, const float *s_channel, const float *bias, int64_t M,
+                   int64_t N, int64_t K, cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream,
+                   bool pdl)
+{
+    cr_w4a8_layer ly;
+    ly.qdata = qdata;
+    ly.srel = srel;
+    ly.s_channel = s_channel;
+    ly.bias = bias;
+    ly.N = N;
+    ly.out = out;
+    ly.acc_out = acc_out;
+    return run_gemv_layers(num_sms, attr_set, xq, xs, codebook, M, K, &ly, 1, out_dtype, stream, pdl);
 }
 
 // Shared validation of the contraction entry points.
@@ -225,6 +271,39 @@ cr_status check_contraction(const int8_t *xq, const float *xs, const uint8_t *qd
         !aligned16(s_channel) || !aligned16(out) || (bias && !aligned16(bias)) || (acc_out && !aligned16(acc_out)))
         return CR_ERR_ALIGNMENT;
     return CR_OK;
+}
+
+// Validation of a layer list: the count, each layer as in check_contraction
+// with the shared xq/xs/codebook, and acc_out only where `allow_acc`.
+// Output channels of all layers together.
+int64_t total_rows(const cr_w4a8_layer *layers, int num_layers)
+{
+    int64_t n = 0;
+    for (int l = 0; l < num_layers; ++l)
+        n += layers[l].N;
+    return n;
+}
+
+static_assert(cr::gv::kMaxLayers == CR_MAX_LAYERS, "layer count of the decode GEMV");
+
+cr_status check_layers(const int8_t *xq, const float *xs, const float *codebook, int64_t M, int64_t K,
+                       const cr_w4a8_layer *layers, int num_layers, cr_out_dtype out_dtype, bool allow_acc)
+{
+    if (!layers || num_layers < 1 || num_layers > CR_MAX_LAYERS)
+        return CR_ERR_INVALID_ARG;
+    cr_status worst = CR_OK;
+    for (int l = 0; l < num_layers; ++l) {
+        const cr_w4a8_layer &ly = layers[l];
+        if (!allow_acc && ly.acc_out)
+            return CR_ERR_INVALID_ARG;
+        const cr_status st = check_contraction(xq, xs, ly.qdata, ly.srel, codebook, ly.s_channel, ly.bias, M, ly.N,
+                                               K, out_dtype, ly.out, ly.acc_out);
+        if (st == CR_ERR_INVALID_ARG || st == CR_ERR_ALIGNMENT)
+            return st;
+        if (st != CR_OK)
+            worst = st;
+    }
+    return worst;
 }
 
 // The side stream and fork/join events of a device, created on first use.
@@ -519,6 +598,71 @@ cr_status cr_w4a8_linear(const uint16_t *x, const uint8_t *qdata, const uint8_t 
         return st;
     return run_gemv(d->num_sms, d->gemv_attr_set, xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K,
                     out_dtype, out, nullptr, stream, /*pdl=*/true);
+}
+
+cr_status cr_w4a8_gemv_grouped(const int8_t *xq, const float *xs, const float *codebook, int64_t M, int64_t K,
+                               const cr_w4a8_layer *layers, int num_layers, cr_out_dtype out_dtype,
+                               cr_stream_t stream)
+{
+    if (M > CR_GEMV_MAX_M)
+        return CR_ERR_UNSUPPORTED;
+    cr_status st = check_layers(xq, xs, codebook, M, K, layers, num_layers, out_dtype, /*allow_acc=*/true);
+    if (st != CR_OK || M == 0 || total_rows(layers, num_layers) == 0)
+        return st;
+    DeviceState *d = nullptr;
+    st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    return run_gemv_layers(d->num_sms, d->gemv_attr_set, xq, xs, codebook, M, K, layers, num_layers, out_dtype,
+                           stream, /*pdl=*/true);
+}
+
+cr_status cr_w4a8_linear_grouped(const uint16_t *x, const float *codebook, int64_t M, int64_t K,
+                                 const cr_w4a8_layer *layers, int num_layers, int act_qmax,
+                                 cr_out_dtype out_dtype, int8_t *xq_work, float *xs_work, cr_stream_t stream)
+{
+    if (M < 0 || K < 0 || act_qmax < 1 || act_qmax > 127)
+        return CR_ERR_INVALID_ARG;
+    int64_t MP = M;
+    if (M >= 1 && M <= CR_GEMV_MAX_M) {
+        MP = 1;
+        while (MP < M)
+            MP <<= 1;
+    }
+    cr_status st = check_layers(xq_work, xs_work, codebook, M, K, layers, num_layers, out_dtype,
+                                /*allow_acc=*/false);
+    if (st != CR_OK || M == 0 || total_rows(layers, num_layers) == 0)
+        return st;
+    if (!x)
+        return CR_ERR_INVALID_ARG;
+    if (!aligned16(x))
+        return CR_ERR_ALIGNMENT;
+    DeviceState *d = nullptr;
+    st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    auto activations = [&]() { return launched(cr::rq::launch(x, M, K, MP, act_qmax, xq_work, xs_work, stream)); };
+    if (M <= CR_GEMV_MAX_M) {
+        st = activations();
+        if (st != CR_OK)
+            return st;
+        return run_gemv_layers(d->num_sms, d->gemv_attr_set, xq_work, xs_work, codebook, M, K, layers, num_layers,
+                               out_dtype, stream, /*pdl=*/true);
+    }
+    // the first layer's weight decode overlaps the activation kernel
+    const std::function<cr_status()> act = activations;
+    bool first = true;
+    for (int l = 0; l < num_layers; ++l) {
+        const cr_w4a8_layer &ly = layers[l];
+        if (ly.N == 0)
+            continue;
+        st = run_gemm(*d, xq_work, xs_work, ly.qdata, ly.srel, codebook, ly.s_channel, ly.bias, M, ly.N, K, out_dtype,
+                      ly.out, nullptr, stream, first ? &act : nullptr);
+        if (st != CR_OK)
+            return st;
+        first = false;
+    }
+    return CR_OK;
 }
 
 // ---------------------------------------------------------------- decode forward without allocation

@@ -147,24 +147,58 @@ __device__ __forceinline__ void slice_mma(const Ops &o, int32_t (&c)[4], int32_t
     mma_s8(d, e0, e1, e2, e3, o.X1.z, o.X1.w);
 }
 
-// tm_codes: the packed codes as 32-bit words, dims {16, N, K / 128}, strides
-//           {K / 2, 64} bytes, box {16, 16, 8}.
-// tm_srel:  the scale bytes, dims {16, N, K / 256}, strides {K / 16, 16}, box {16, 16, 4}.
-// tm_x:     xq, dims {128, M, K / 128}, strides {K, 128}, box {128, 8, 8}, 128-byte swizzle.
-// lut_step: bytes between the table entries of consecutive scale bytes in one
-//           copy (kCopies * 16).  ahead: L2 prefetch distance in stages.
+// The layers one launch covers: every layer is contracted with the same
+// activations (xq, xs) and was quantised with the same codebook; their row
+// tiles are numbered one after the other (layer l owns the tiles
+// [tile0, tile0 + ceil(N / 16))).
+constexpr int kMaxLayers = 4;
+
+struct GemvLayer {
+    const float *ws;    // [N] per-channel scales
+    const float *bias;  // [N] or null
+    void *out;          // [M, N] bf16 or fp32
+    int32_t *acc_out;   // [M, N] or null
+    int N;
+    int tile0;
+};
+
+// tm_codes[l]: layer l's packed codes as 32-bit words, dims {16, N, K / 128},
+//              strides {K / 2, 64} bytes, box {16, 16, 8}.
+// tm_srel[l]:  its scale bytes, dims {16, N, K / 256}, strides {K / 16, 16}, box {16, 16, 4}.
+// tm_x:        xq, dims {128, M, K / 128}, strides {K, 128}, box {128, 8, 8}, 128-byte swizzle.
+// lut_step:    bytes between the table entries of consecutive scale bytes in one
+//              copy (kCopies * 16).  ahead: L2 prefetch distance in stages.
+struct GemvArgs {
+    CUtensorMap tm_codes[kMaxLayers];
+    CUtensorMap tm_srel[kMaxLayers];
+    CUtensorMap tm_x;
+    GemvLayer layer[kMaxLayers];
+    const float *xs;
+    const float *codebook;
+    int M, K, num_layers, num_tiles, out_f32;
+    uint32_t lut_step;
+    int ahead;
+};
+
+// The layer that owns global row tile `tile`.
+__device__ __forceinline__ int layer_of(const GemvArgs &a, int tile)
+{
+    int l = 0;
+#pragma unroll
+    for (int i = 1; i < kMaxLayers; ++i)
+        if (i < a.num_layers && tile >= a.layer[i].tile0)
+            l = i;
+    return l;
+}
+
 template <class C>
-__global__ void __launch_bounds__(kThreads, C::kMinBlocks)
-    gemv_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_srel,
-                const __grid_constant__ CUtensorMap tm_x, const float *__restrict__ xs,
-                const float *__restrict__ codebook, const float *__restrict__ ws, const float *__restrict__ bias,
-                int M, int N, int K, int out_f32, void *__restrict__ out, int32_t *__restrict__ acc_out,
-                uint32_t lut_step, int ahead)
+__global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __grid_constant__ GemvArgs a)
 {
     constexpr int STAGES = C::kStages;
     using Smem = typename C::Smem;
     extern __shared__ uint8_t smem_raw[];
     Smem &sh = smem_aligned_1024<Smem>(smem_raw);
+    const int M = a.M, K = a.K;
 
     // The next kernel on the stream may launch now: a GEMV of the next layer
     // starts its weight stream in the SM slots this grid frees, and whatever
@@ -173,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
     asm volatile("griddepcontrol.launch_dependents;" :::);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int ntiles = (N + kRows - 1) / kRows;
+    const int ntiles = a.num_tiles;
     const int nchunks = (K + kChunk - 1) / kChunk;
     // Persistent grid: this CTA takes row tiles blockIdx.x, + gridDim.x, ...,
     // each as nchunks stages; `total` stages in all.
@@ -194,20 +228,25 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     if (tid < 16)
-        sh.cb[tid] = codebook[tid];
+        sh.cb[tid] = a.codebook[tid];
     __syncthreads();
     volatile int *abort = &sh.abort;
 
     if (warp == kProducerWarp) {
         // ------------------------------------------------ producer
         if (lane == 0) {
-            prefetch_tmap(&tm_codes);
-            prefetch_tmap(&tm_srel);
-            prefetch_tmap(&tm_x);
+            for (int l = 0; l < a.num_layers; ++l) {
+                if (a.layer[l].N == 0)
+                    continue; // its maps are left empty
+                prefetch_tmap(&a.tm_codes[l]);
+                prefetch_tmap(&a.tm_srel[l]);
+            }
+            prefetch_tmap(&a.tm_x);
             auto weights = [&](int q, int s) {
                 const int i = q / nchunks, tile = (int)blockIdx.x + i * (int)gridDim.x, c = q - i * nchunks;
-                tma_load_3d(sh.codes[s], &tm_codes, 0, tile * kRows, c * (kChunk / kSlice), &sh.full[s]);
-                tma_load_3d(sh.srel[s], &tm_srel, 0, tile * kRows, c * (kChunk / 256), &sh.full[s]);
+                const int l = layer_of(a, tile), row = (tile - a.layer[l].tile0) * kRows;
+                tma_load_3d(sh.codes[s], &a.tm_codes[l], 0, row, c * (kChunk / kSlice), &sh.full[s]);
+                tma_load_3d(sh.srel[s], &a.tm_srel[l], 0, row, c * (kChunk / 256), &sh.full[s]);
             };
             // L2 prefetch of the weights of stage q: `ahead` stages of HBM reads
             // in flight beyond the shared-memory ring, so that a refill of the
@@ -215,12 +254,13 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
             auto prefetch = [&](int q) {
                 if (q < total) {
                     const int i = q / nchunks, tile = (int)blockIdx.x + i * (int)gridDim.x, c = q - i * nchunks;
-                    tma_prefetch_3d(&tm_codes, 0, tile * kRows, c * (kChunk / kSlice));
-                    tma_prefetch_3d(&tm_srel, 0, tile * kRows, c * (kChunk / 256));
+                    const int l = layer_of(a, tile), row = (tile - a.layer[l].tile0) * kRows;
+                    tma_prefetch_3d(&a.tm_codes[l], 0, row, c * (kChunk / kSlice));
+                    tma_prefetch_3d(&a.tm_srel[l], 0, row, c * (kChunk / 256));
                 }
             };
             auto acts = [&](int q, int s) {
-                tma_load_3d(sh.x[s], &tm_x, 0, 0, (q % nchunks) * (kChunk / kSlice), &sh.full[s]);
+                tma_load_3d(sh.x[s], &a.tm_x, 0, 0, (q % nchunks) * (kChunk / kSlice), &sh.full[s]);
             };
             // The first stages' weights go out before the activation kernel has
             // finished; their activation copies follow the dependency wait.
@@ -229,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
                 mbar_arrive_expect_tx(&sh.full[q], kStageTx);
                 weights(q, q);
             }
-            for (int q = pre; q < pre + ahead; ++q)
+            for (int q = pre; q < pre + a.ahead; ++q)
                 prefetch(q);
             asm volatile("griddepcontrol.wait;" ::: "memory");
             for (int q = 0; q < pre; ++q)
@@ -247,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
                 mbar_arrive_expect_tx(&sh.full[s], kStageTx);
                 weights(q, s);
                 acts(q, s);
-                prefetch(q + ahead);
+                prefetch(q + a.ahead);
             }
             if (!ok) {
                 // let the copies in flight land before the CTA exits
@@ -309,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
                     if (ok && ch < nvalid) {
                         Ops o;
                         fetch_ops(o, sh.x[s] + off_x0, sh.x[s] + off_x1, sh.codes[s] + off_code,
-                                  sh.srel[s] + off_srel, lutb, lut_step);
+                                  sh.srel[s] + off_srel, lutb, a.lut_step);
                         slice_mma(o, c, d);
                     }
                     __syncwarp();
@@ -330,14 +370,18 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
         asm volatile("griddepcontrol.wait;" ::: "memory");
         for (int seg = 0; seg < my_tiles; ++seg) {
             const int tile = (int)blockIdx.x + seg * (int)gridDim.x;
+            const GemvLayer &ly = a.layer[layer_of(a, tile)];
+            const int N = ly.N, row0 = (tile - ly.tile0) * kRows;
+            const float *__restrict__ ws = ly.ws;
+            const float *__restrict__ bias = ly.bias;
             // this lane's outputs: e = lane + 32 u -> row e / 8, token e % 8
             float exs[4], ews[4], eb[4];
             bool live[4];
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-                const int e = lane + 32 * u, r = e >> 3, m = e & 7, n = tile * kRows + r;
+                const int e = lane + 32 * u, r = e >> 3, m = e & 7, n = row0 + r;
                 live[u] = m < M && n < N;
-                exs[u] = live[u] ? xs[m] : 0.0f;
+                exs[u] = live[u] ? a.xs[m] : 0.0f;
                 ews[u] = live[u] ? ws[n] : 0.0f;
                 eb[u] = (live[u] && bias != nullptr) ? bias[n] : 0.0f;
             }
@@ -361,17 +405,17 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks)
                 for (int u = 0; u < 4; ++u) {
                     if (!live[u])
                         continue;
-                    const int e = lane + 32 * u, n = tile * kRows + (e >> 3), m = e & 7;
+                    const int e = lane + 32 * u, n = row0 + (e >> 3), m = e & 7;
                     float y = __fmul_rn(__int2float_rn(acc[u]), __fmul_rn(exs[u], ews[u]));
                     if (bias != nullptr)
                         y = __fadd_rn(y, eb[u]);
                     const int64_t o = (int64_t)m * N + n;
-                    if (out_f32)
-                        reinterpret_cast<float *>(out)[o] = y;
+                    if (a.out_f32)
+                        reinterpret_cast<float *>(ly.out)[o] = y;
                     else
-                        reinterpret_cast<uint16_t *>(out)[o] = to_bf16_bits(y);
-                    if (acc_out != nullptr)
-                        acc_out[o] = acc[u];
+                        reinterpret_cast<uint16_t *>(ly.out)[o] = to_bf16_bits(y);
+                    if (ly.acc_out != nullptr)
+                        ly.acc_out[o] = acc[u];
                 }
             }
         }
