@@ -55,6 +55,7 @@ def parse():
     p.add_argument("--workload", default="c2_decode_m8_4k")
     p.add_argument("--prefill-workload", default="c3_prefill_2k_4k")
     p.add_argument("--no-prefill", action="store_true")
+    p.add_argument("--no-grouped", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     return p.parse_args()
@@ -429,6 +430,10 @@ def run_ours(args):
     if not args.no_prefill:
         prefill = run_prefill(args, world, rank, local, pk)
 
+    grouped = None
+    if not args.no_grouped:
+        grouped = run_grouped(args, world, rank, local, case)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(case, args.cpu_seconds)
@@ -443,7 +448,7 @@ def run_ours(args):
                    "timing": "one CUDA-graph replay of K steps (graph uploaded beforehand), CUDA events on the capture stream",
                    "parallelism": f"replica x{world}"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps,
-        "clocks": clocks, "prefill": prefill,
+        "clocks": clocks, "prefill": prefill, "grouped": grouped,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -522,6 +527,51 @@ def run_prefill(args, world, rank, local, pk):
                          "kernel": "cr_w4a8_gemm call (weight decode to an int8 transient + tcgen05 GEMM)",
                          "peak_source": f"{pk['source']} bf16_tflops x {INT8_OVER_BF16} (nominal int8/bf16 ratio)",
                          "us_per_call": round(tg * 1e6, 2)}}
+
+
+GROUPED_NS = (4096, 1024, 1024)  # q, k, v of an attention block with 8-way grouped k/v heads
+
+
+def run_grouped(args, world, rank, local, case):
+    """Three layers fed the same decode batch (q/k/v): cr_w4a8_linear_grouped
+    (one rotate+quant, one grouped GEMV launch) against three
+    cr_w4a8_linear calls, in weight GB/s of the three layers together."""
+    import torch
+
+    import w4a8_codebook_quantized_b200 as cr
+    from w4a8_codebook_quantized_b200 import inputs
+    M, K = case.M, case.K
+    wb = sum(weight_bytes(n, K) for n in GROUPED_NS)
+    R = max(2, int(math.ceil(1.25 * L2_BYTES / wb)))
+    cb = torch.from_numpy(inputs.codebook()).cuda()
+    base = []
+    for i, n in enumerate(GROUPED_NS):
+        ly = inputs.layer(n, K, rank_seed(case.seed + 10 + i, rank))
+        base.append(tuple(torch.from_numpy(a).cuda() for a in (ly.qdata, ly.srel, ly.s_channel)))
+    sets = [[tuple(t.clone() for t in ly) for ly in base] for _ in range(R)]
+    x = inputs.activations(M, K, rank_seed(case.seed, rank), case.dist)
+    xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    rows = cr.gemv_rows(M)
+    xq = torch.empty(rows, K, dtype=torch.int8, device="cuda")
+    xs = torch.empty(rows, dtype=torch.float32, device="cuda")
+    outs = [torch.empty(M, n, dtype=torch.bfloat16, device="cuda") for n in GROUPED_NS]
+
+    def grouped_step(i):
+        cr.cr_w4a8_linear_grouped(xd, cb, sets[i % R], outs=outs, xq_work=xq, xs_work=xs)
+
+    def separate_step(i):
+        for (q, s, ws), o in zip(sets[i % R], outs):
+            cr.cr_w4a8_linear(xd, q, s, cb, ws, out=o, xq_work=xq, xs_work=xs)
+
+    tg, _ = graph_time(grouped_step, args.steps, args.warmup, world, local)
+    ts, _ = graph_time(separate_step, args.steps, args.warmup, world, local)
+    tg, ts = max_over_ranks(tg, world), max_over_ranks(ts, world)
+    return {"workload": f"q/k/v of the decode batch: M={M}, K={K}, N={'+'.join(map(str, GROUPED_NS))}",
+            "value": round(aggregate_value(wb, args.steps, world, tg), 2), "unit": "GB/s",
+            "us_per_step": round(tg / args.steps * 1e6, 3),
+            "separate_calls": {"value": round(aggregate_value(wb, args.steps, world, ts), 2),
+                               "us_per_step": round(ts / args.steps * 1e6, 3)},
+            "gpu_launches_per_step": 2, "l2": f"rotating {R} copies of the three layers"}
 
 
 # ---------------------------------------------------------------- reference arm

@@ -32,6 +32,7 @@ struct DeviceState {
     bool gemm_attr_set = false;
     bool gemm_pair_attr_set = false;
     bool gemv_attr_set = false;
+    bool gemv_grouped_attr_set = false;
     // side stream and events on which cr_w4a8_linear's prefill path decodes
     // the weight while the activations are rotated and quantised
     cudaStream_t side = nullptr;
@@ -163,21 +164,22 @@ bool make_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype,
 // tiles of all layers are numbered one after the other and run on a
 // persistent grid of as many CTAs as fit on the SMs, optionally as a
 // programmatic dependent of the previous kernel on the stream.
-cr_status run_gemv_layers(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const float *codebook,
-                          int64_t M, int64_t K, const cr_w4a8_layer *layers, int num_layers, cr_out_dtype out_dtype,
-                          cudaStream_t stream, bool pdl)
+template <int L>
+cr_status launch_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const float *codebook,
+                      int64_t M, int64_t K, const cr_w4a8_layer *layers, int num_layers, cr_out_dtype out_dtype,
+                      cudaStream_t stream, bool pdl)
 {
     using namespace cr;
     using C = gv::Prod;
     if (!attr_set) {
-        if (cudaFuncSetAttribute(gv::gemv_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gv::gemv_kernel<C, L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)C::kSmemBytes) != cudaSuccess) {
             cudaGetLastError();
             return CR_ERR_CUDA;
         }
         attr_set = true;
     }
-    gv::GemvArgs args;
+    gv::GemvArgs<L> args;
     memset(&args, 0, sizeof(args));
     const uint64_t uK = (uint64_t)K, uM = (uint64_t)M;
     int64_t tiles = 0;
@@ -229,7 +231,19 @@ cr_status run_gemv_layers(int num_sms, bool &attr_set, const int8_t *xq, const f
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return launched(cudaLaunchKernelEx(&cfg, gv::gemv_kernel<C>, args));
+    return launched(cudaLaunchKernelEx(&cfg, gv::gemv_kernel<C, L>, args));
+}
+
+
+cr_status run_gemv_layers(DeviceState &d, const int8_t *xq, const float *xs, const float *codebook, int64_t M,
+                          int64_t K, const cr_w4a8_layer *layers, int num_layers, cr_out_dtype out_dtype,
+                          cudaStream_t stream, bool pdl)
+{
+    if (num_layers == 1)
+        return launch_gemv<1>(d.num_sms, d.gemv_attr_set, xq, xs, codebook, M, K, layers, 1, out_dtype, stream,
+                              pdl);
+    return launch_gemv<cr::gv::kMaxLayers>(d.num_sms, d.gemv_grouped_attr_set, xq, xs, codebook, M, K, layers,
+                                           num_layers, out_dtype, stream, pdl);
 }
 
 // One layer.
@@ -246,7 +260,7 @@ cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *x
     ly.N = N;
     ly.out = out;
     ly.acc_out = acc_out;
-    return run_gemv_layers(num_sms, attr_set, xq, xs, codebook, M, K, &ly, 1, out_dtype, stream, pdl);
+    return launch_gemv<1>(num_sms, attr_set, xq, xs, codebook, M, K, &ly, 1, out_dtype, stream, pdl);
 }
 
 // Shared validation of the contraction entry points.
@@ -613,7 +627,7 @@ cr_status cr_w4a8_gemv_grouped(const int8_t *xq, const float *xs, const float *c
     st = current_device(&d);
     if (st != CR_OK)
         return st;
-    return run_gemv_layers(d->num_sms, d->gemv_attr_set, xq, xs, codebook, M, K, layers, num_layers, out_dtype,
+    return run_gemv_layers(*d, xq, xs, codebook, M, K, layers, num_layers, out_dtype,
                            stream, /*pdl=*/true);
 }
 
@@ -646,7 +660,7 @@ cr_status cr_w4a8_linear_grouped(const uint16_t *x, const float *codebook, int64
         st = activations();
         if (st != CR_OK)
             return st;
-        return run_gemv_layers(d->num_sms, d->gemv_attr_set, xq_work, xs_work, codebook, M, K, layers, num_layers,
+        return run_gemv_layers(*d, xq_work, xs_work, codebook, M, K, layers, num_layers,
                                out_dtype, stream, /*pdl=*/true);
     }
     // the first layer's weight decode overlaps the activation kernel

@@ -168,11 +168,14 @@ struct GemvLayer {
 // tm_x:        xq, dims {128, M, K / 128}, strides {K, 128}, box {128, 8, 8}, 128-byte swizzle.
 // lut_step:    bytes between the table entries of consecutive scale bytes in one
 //              copy (kCopies * 16).  ahead: L2 prefetch distance in stages.
+// L: the layer slots of the launch (1, or kMaxLayers for a grouped call), so
+// a single layer keeps a small parameter block and a constant layer index.
+template <int L>
 struct GemvArgs {
-    CUtensorMap tm_codes[kMaxLayers];
-    CUtensorMap tm_srel[kMaxLayers];
+    CUtensorMap tm_codes[L];
+    CUtensorMap tm_srel[L];
     CUtensorMap tm_x;
-    GemvLayer layer[kMaxLayers];
+    GemvLayer layer[L];
     const float *xs;
     const float *codebook;
     int M, K, num_layers, num_tiles, out_f32;
@@ -181,18 +184,32 @@ struct GemvArgs {
 };
 
 // The layer that owns global row tile `tile`.
-__device__ __forceinline__ int layer_of(const GemvArgs &a, int tile)
+template <int L>
+__device__ __forceinline__ int layer_of(const GemvArgs<L> &a, int tile)
 {
     int l = 0;
 #pragma unroll
-    for (int i = 1; i < kMaxLayers; ++i)
+    for (int i = 1; i < L; ++i)
         if (i < a.num_layers && tile >= a.layer[i].tile0)
             l = i;
     return l;
 }
 
-template <class C>
-__global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __grid_constant__ GemvArgs a)
+// Layer and first row of global row tile `tile` (compile-time for one layer).
+template <int L>
+__device__ __forceinline__ void locate(const GemvArgs<L> &a, int tile, int &l, int &row)
+{
+    if constexpr (L == 1) {
+        l = 0;
+        row = tile * kRows;
+    } else {
+        l = layer_of(a, tile);
+        row = (tile - a.layer[l].tile0) * kRows;
+    }
+}
+
+template <class C, int L>
+__global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __grid_constant__ GemvArgs<L> a)
 {
     constexpr int STAGES = C::kStages;
     using Smem = typename C::Smem;
@@ -235,16 +252,22 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
     if (warp == kProducerWarp) {
         // ------------------------------------------------ producer
         if (lane == 0) {
-            for (int l = 0; l < a.num_layers; ++l) {
-                if (a.layer[l].N == 0)
-                    continue; // its maps are left empty
-                prefetch_tmap(&a.tm_codes[l]);
-                prefetch_tmap(&a.tm_srel[l]);
+            if constexpr (L == 1) {
+                prefetch_tmap(&a.tm_codes[0]);
+                prefetch_tmap(&a.tm_srel[0]);
+            } else {
+                for (int l = 0; l < a.num_layers; ++l) {
+                    if (a.layer[l].N == 0)
+                        continue; // its maps are left empty
+                    prefetch_tmap(&a.tm_codes[l]);
+                    prefetch_tmap(&a.tm_srel[l]);
+                }
             }
             prefetch_tmap(&a.tm_x);
             auto weights = [&](int q, int s) {
                 const int i = q / nchunks, tile = (int)blockIdx.x + i * (int)gridDim.x, c = q - i * nchunks;
-                const int l = layer_of(a, tile), row = (tile - a.layer[l].tile0) * kRows;
+                int l, row;
+                locate(a, tile, l, row);
                 tma_load_3d(sh.codes[s], &a.tm_codes[l], 0, row, c * (kChunk / kSlice), &sh.full[s]);
                 tma_load_3d(sh.srel[s], &a.tm_srel[l], 0, row, c * (kChunk / 256), &sh.full[s]);
             };
@@ -254,7 +277,8 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
             auto prefetch = [&](int q) {
                 if (q < total) {
                     const int i = q / nchunks, tile = (int)blockIdx.x + i * (int)gridDim.x, c = q - i * nchunks;
-                    const int l = layer_of(a, tile), row = (tile - a.layer[l].tile0) * kRows;
+                    int l, row;
+                    locate(a, tile, l, row);
                     tma_prefetch_3d(&a.tm_codes[l], 0, row, c * (kChunk / kSlice));
                     tma_prefetch_3d(&a.tm_srel[l], 0, row, c * (kChunk / 256));
                 }
@@ -370,10 +394,16 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
         asm volatile("griddepcontrol.wait;" ::: "memory");
         for (int seg = 0; seg < my_tiles; ++seg) {
             const int tile = (int)blockIdx.x + seg * (int)gridDim.x;
-            const GemvLayer &ly = a.layer[layer_of(a, tile)];
-            const int N = ly.N, row0 = (tile - ly.tile0) * kRows;
+            int l, row0;
+            locate(a, tile, l, row0);
+            const GemvLayer &ly = a.layer[l];
+            const int N = ly.N;
             const float *__restrict__ ws = ly.ws;
             const float *__restrict__ bias = ly.bias;
+            const float *__restrict__ xs = a.xs;
+            void *__restrict__ out = ly.out;
+            int32_t *__restrict__ acc_out = ly.acc_out;
+            const bool out_f32 = a.out_f32 != 0;
             // this lane's outputs: e = lane + 32 u -> row e / 8, token e % 8
             float exs[4], ews[4], eb[4];
             bool live[4];
@@ -381,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
             for (int u = 0; u < 4; ++u) {
                 const int e = lane + 32 * u, r = e >> 3, m = e & 7, n = row0 + r;
                 live[u] = m < M && n < N;
-                exs[u] = live[u] ? a.xs[m] : 0.0f;
+                exs[u] = live[u] ? xs[m] : 0.0f;
                 ews[u] = live[u] ? ws[n] : 0.0f;
                 eb[u] = (live[u] && bias != nullptr) ? bias[n] : 0.0f;
             }
@@ -410,12 +440,12 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
                     if (bias != nullptr)
                         y = __fadd_rn(y, eb[u]);
                     const int64_t o = (int64_t)m * N + n;
-                    if (a.out_f32)
-                        reinterpret_cast<float *>(ly.out)[o] = y;
+                    if (out_f32)
+                        reinterpret_cast<float *>(out)[o] = y;
                     else
-                        reinterpret_cast<uint16_t *>(ly.out)[o] = to_bf16_bits(y);
-                    if (ly.acc_out != nullptr)
-                        ly.acc_out[o] = acc[u];
+                        reinterpret_cast<uint16_t *>(out)[o] = to_bf16_bits(y);
+                    if (acc_out != nullptr)
+                        acc_out[o] = acc[u];
                 }
             }
         }
