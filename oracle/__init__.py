@@ -55,6 +55,10 @@ def lib() -> ctypes.CDLL:
             L.or_gemm_s32_rows.restype = ctypes.c_int
             L.or_epilogue.argtypes = [P, P, P, P, i64, i64, ctypes.c_int, P]
             L.or_epilogue.restype = None
+            L.or_f64_to_bf16_rne.argtypes = [ctypes.c_double]
+            L.or_f64_to_bf16_rne.restype = ctypes.c_uint16
+            L.or_epilogue_swiglu.argtypes = [P, P, P, P, i64, i64, ctypes.c_int, P]
+            L.or_epilogue_swiglu.restype = None
             _lib = L
     return _lib
 
@@ -198,6 +202,58 @@ def epilogue(acc, xs, ws, bias=None, out: str = "bf16") -> np.ndarray:
         raise ValueError(out)
     lib().or_epilogue(_p(acc), _p(xs), _p(ws), _p(b), m, n, flag, _p(res))
     return res
+
+
+def f64_to_bf16(value: float) -> int:
+    """One double -> bf16 bits, rounded once (nearest, ties to even)."""
+    return int(lib().or_f64_to_bf16_rne(float(value)))
+
+
+def interleave_rows(a) -> np.ndarray:
+    """h3-rs src/weights.rs, interleave_rows: the two halves of the row
+    dimension [a0 .. aF-1, b0 .. bF-1] become [a0, b0, a1, b1, ...] (rows
+    carry their trailing dimensions with them)."""
+    a = np.ascontiguousarray(a)
+    n = a.shape[0]
+    if n % 2:
+        raise ValueError("an even number of rows is needed")
+    halves = a.reshape((2, n // 2) + a.shape[1:])
+    return np.ascontiguousarray(np.swapaxes(halves, 0, 1)).reshape(a.shape)
+
+
+def epilogue_swiglu(acc, xs, ws, bias=None, out: str = "bf16") -> np.ndarray:
+    """int32 [M, 2F] on interleaved gate/up rows -> silu(g) * u as bf16 bits
+    (uint16) or fp32 [M, F]."""
+    acc = _c(acc, np.int32)
+    m, n = acc.shape
+    if n % 2:
+        raise ValueError("interleaved gate/up needs an even number of columns")
+    f = n // 2
+    xs = _c(xs, np.float32)[:m]
+    ws = _c(ws, np.float32)
+    b = None if bias is None else _c(bias, np.float32)
+    if out == "bf16":
+        res = np.empty((m, f), dtype=np.uint16)
+        flag = 1
+    elif out == "f32":
+        res = np.empty((m, f), dtype=np.float32)
+        flag = 0
+    else:
+        raise ValueError(out)
+    lib().or_epilogue_swiglu(_p(acc), _p(xs), _p(ws), _p(b), m, f, flag, _p(res))
+    return res
+
+
+def linear_swiglu(x_bf16, qdata, srel, codebook, s_channel, bias=None, qmax: int = 127,
+                  out: str = "bf16", threads: int = 1) -> dict:
+    """The forward of a gate/up layer stored with interleaved rows, SwiGLU
+    fused into the epilogue: rotate + quantise x, decode W, contract, then
+    silu(gate) * up.  Returns xq, xs, w8, acc and y [M, N/2]."""
+    xq, xs = rotate_quant_act(x_bf16, None, qmax)
+    w8 = decode_w8(qdata, srel, codebook)
+    acc = gemm_s32(xq, w8, threads)
+    y = epilogue_swiglu(acc, xs, s_channel, bias, out)
+    return {"xq": xq, "xs": xs, "w8": w8, "acc": acc, "y": y}
 
 
 def linear(x_bf16, qdata, srel, codebook, s_channel, bias=None, qmax: int = 127,

@@ -19,7 +19,8 @@
  *         multiply-accumulate and epilogue), w4a8_act_quant_kernel, _gemv_mp,
  *         _w4a8_linear_ste_op (unpack -> act quant -> _int_mm -> epilogue),
  *         dequantize_w4a8.
- *   [H3]  h3-rs src/weights.rs -- hadamard(), rotate_activation().
+ *   [H3]  h3-rs src/weights.rs -- hadamard(), rotate_activation(),
+ *         interleave_rows / QLinear::interleave_swiglu, swiglu_interleaved.
  *
  * Every function restates one definition.  Where the pages leave a detail
  * open (the fp32 summation order of the rotation, NaN handling, the
@@ -78,6 +79,30 @@ uint16_t or_f32_to_bf16_rne(float f)
     uint32_t keep_lsb = (u >> 16) & 1u;
     u += 0x7FFFu + keep_lsb;
     return (uint16_t)(u >> 16);
+}
+
+/* double -> bf16 bits, one rounding to nearest, ties to even (used where the
+ * oracle computes a value in double and the output is bf16, so that it is not
+ * rounded twice through fp32).  Magnitudes below the smallest normal bf16 go
+ * through fp32; NaN stays a quiet NaN; overflow gives an infinity. */
+uint16_t or_f64_to_bf16_rne(double d)
+{
+    if (isnan(d))
+        return (uint16_t)(signbit(d) ? 0xFFC0u : 0x7FC0u);
+    if (fabs(d) < 1.1754943508222875e-38) /* 2^-126 */
+        return or_f32_to_bf16_rne((float)d);
+    uint64_t u;
+    memcpy(&u, &d, 8);
+    /* keep 7 of the 52 fraction bits: drop 45 with round-half-even */
+    uint64_t keep_lsb = (u >> 45) & 1u;
+    u += ((uint64_t)1 << 44) - 1 + keep_lsb;
+    u &= ~(((uint64_t)1 << 45) - 1);
+    double r;
+    memcpy(&r, &u, 8);
+    float f = (float)r; /* exact: 8 significant bits, in the fp32 exponent range, or an infinity */
+    uint32_t b;
+    memcpy(&b, &f, 4);
+    return (uint16_t)(b >> 16);
 }
 
 /* ------------------------------------------------------------------------
@@ -335,5 +360,39 @@ void or_epilogue(const int32_t *acc, const float *xs, const float *ws, const flo
                 ((uint16_t *)out)[m * N + n] = or_f32_to_bf16_rne(y);
             else
                 ((float *)out)[m * N + n] = y;
+        }
+}
+
+/* ------------------------------------------------------------------------
+ * SwiGLU on row-interleaved gate/up outputs.  [H3] QLinear::interleave_swiglu
+ * (a gate/up layer's output rows reordered to pairs g0, u0, g1, u1, ...) and
+ * swiglu_interleaved (silu(gate) * up of each pair).
+ * acc [M, 2F] int32.  g = the epilogue value of column 2f and u = that of
+ * column 2f + 1, each in fp32 exactly as or_epilogue computes it (the pages'
+ * fp32 rescale); then silu(g) * u = g * u / (1 + exp(-g)), which the pages
+ * do not pin to a precision: here in double, rounded once to the output
+ * type.  out [M, F].
+ * ------------------------------------------------------------------------ */
+void or_epilogue_swiglu(const int32_t *acc, const float *xs, const float *ws, const float *bias,
+                        int64_t M, int64_t F, int out_bf16, void *out)
+{
+    const int64_t N = 2 * F;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t f = 0; f < F; ++f) {
+            float v[2];
+            for (int h = 0; h < 2; ++h) {
+                const int64_t n = 2 * f + h;
+                float t = (float)acc[m * N + n];
+                float sc = xs[m] * ws[n];
+                v[h] = t * sc;
+                if (bias)
+                    v[h] = v[h] + bias[n];
+            }
+            const double g = v[0], up = v[1];
+            const double y = g / (1.0 + exp(-g)) * up;
+            if (out_bf16)
+                ((uint16_t *)out)[m * F + f] = or_f64_to_bf16_rne(y);
+            else
+                ((float *)out)[m * F + f] = (float)y;
         }
 }

@@ -368,3 +368,84 @@ def test_linear_random_within_quantisation_bound():
     assert (np.abs(res["y"] - ref) <= bound).all()
     # and a plausible slip (a dropped outlier channel) would break it
     assert np.abs(res["y"] - ref).max() < 0.05 * np.abs(ref).max()
+
+
+# ---------------------------------------------------------------- SwiGLU on interleaved gate/up rows
+
+def test_f64_to_bf16_rounds_once():
+    """One rounding from double: 1 + 2^-8 is a tie (goes to the even 1.0),
+    but 1 + 2^-8 + 2^-40 lies above it and rounds up, where a detour through
+    fp32 would lose the 2^-40 and round down."""
+    f = oracle.f64_to_bf16
+    assert f(1.0 + 2.0 ** -8) == 0x3F80
+    assert f(1.0 + 2.0 ** -8 + 2.0 ** -40) == 0x3F81
+    assert f(-(1.0 + 2.0 ** -8 + 2.0 ** -40)) == 0xBF81
+    assert f(1.0 + 3 * 2.0 ** -8) == 0x3F82          # tie between 0x3F81 and 0x3F82 -> even
+    assert f(3.4e38) == 0x7F80                        # above the bf16 maximum's halfway point
+    assert f(0.0) == 0x0000 and f(-0.0) == 0x8000
+    assert f(float("nan")) & 0x7FC0 == 0x7FC0
+    # on values exactly representable in fp32, the same as torch's fp32 -> bf16 cast
+    rng = np.random.default_rng(5)
+    v = (rng.standard_normal(2000) * np.exp(rng.uniform(-20, 20, 2000))).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert all(f(float(x)) == int(r) for x, r in zip(v, ref))
+
+
+def test_interleave_rows_hand_example():
+    """h3-rs interleave_rows: [a0 .. aF-1, b0 .. bF-1] -> [a0, b0, a1, b1, ...]."""
+    a = np.array([[0, 1], [2, 3], [4, 5], [10, 11], [12, 13], [14, 15]])
+    assert oracle.interleave_rows(a).tolist() == [[0, 1], [10, 11], [2, 3], [12, 13], [4, 5], [14, 15]]
+    assert oracle.interleave_rows(np.array([7, 8, 9, 1, 2, 3])).tolist() == [7, 1, 8, 2, 9, 3]
+    with pytest.raises(ValueError):
+        oracle.interleave_rows(np.zeros((3, 2)))
+
+
+def test_swiglu_closed_forms():
+    """silu(g) = g * sigmoid(g): sigmoid(ln 3) = 3/4 and sigmoid(-ln 3) = 1/4
+    exactly, silu(0) = 0, silu(g) -> g for large g and -> 0 for very negative
+    g; the up value multiplies."""
+    ln3 = np.float32(math.log(3.0))
+    gs = np.array([ln3, -ln3, 0.0, 30.0, -30.0, -100.0], dtype=np.float32)
+    us = np.array([1.0, 1.0, 5.0, 1.0, 1.0, 1.0], dtype=np.float32)
+    # acc holds the values themselves (integers would round them): use xs = ws = 1 and put g, u
+    # into the bias with zero accumulators
+    F = gs.size
+    acc = np.zeros((1, 2 * F), dtype=np.int32)
+    bias = np.empty(2 * F, dtype=np.float32)
+    bias[0::2], bias[1::2] = gs, us
+    y = oracle.epilogue_swiglu(acc, np.ones(1, np.float32), np.ones(2 * F, np.float32), bias, "f32")[0]
+    g = gs.astype(np.float64)
+    assert abs(y[0] - 0.75 * g[0]) <= 1e-7 * abs(g[0])
+    assert abs(y[1] - (-0.25 * g[0])) <= 1e-7 * abs(g[0])
+    assert y[2] == 0.0
+    assert y[3] == np.float32(30.0)                       # 30 * (1 - 9.4e-14) rounds to 30
+    assert -1e-11 < y[4] < 0 and abs(y[4] - (-30.0 * math.exp(-30.0))) <= 1e-6 * 30.0 * math.exp(-30.0)
+    assert y[5] <= 0 and abs(y[5]) < 1e-40
+    # the bf16 output is the same value rounded once
+    yb = oracle.epilogue_swiglu(acc, np.ones(1, np.float32), np.ones(2 * F, np.float32), bias, "bf16")[0]
+    assert int(yb[0]) == oracle.f64_to_bf16(float(g[0]) / (1.0 + math.exp(-float(g[0]))))
+
+
+def test_swiglu_pairs_gate_with_up():
+    """An interleaved gate/up layer's fused SwiGLU equals silu(gate(x)) * up(x)
+    computed from the two separate layers with the plain epilogue: a swapped
+    pair or a wrong row mapping fails."""
+    M, F, K = 5, 24, 512
+    gate, up = inputs.layer(F, K, 71, with_bias=True), inputs.layer(F, K, 72, with_bias=True)
+    x = inputs.activations(M, K, 73)
+    both = {}
+    for name, ly in (("g", gate), ("u", up)):
+        both[name] = oracle.linear(x, ly.qdata, ly.srel, ly.codebook, ly.s_channel, ly.bias, out="f32")["y"]
+    cat = lambda a, b: np.concatenate([a, b], axis=0)
+    q = oracle.interleave_rows(cat(gate.qdata, up.qdata))
+    s = oracle.interleave_rows(cat(gate.srel, up.srel))
+    ws = oracle.interleave_rows(cat(gate.s_channel, up.s_channel))
+    b = oracle.interleave_rows(cat(gate.bias, up.bias))
+    y = oracle.linear_swiglu(x, q, s, gate.codebook, ws, b, out="f32")["y"]
+    g, u = both["g"].astype(np.float64), both["u"].astype(np.float64)
+    ref = g / (1.0 + np.exp(-g)) * u
+    assert y.shape == (M, F)
+    np.testing.assert_array_max_ulp(y, ref.astype(np.float32), maxulp=1)
+    # and silu is not applied to the up half
+    wrong = u / (1.0 + np.exp(-u)) * g
+    assert np.abs(y - wrong).max() > 1e-3 * np.abs(ref).max()
