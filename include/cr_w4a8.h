@@ -277,6 +277,57 @@ cr_status cr_w4a8_linear_grouped(const uint16_t *x, const float *codebook, int64
                                  cr_out_dtype out_dtype, int8_t *xq_work, float *xs_work, cr_stream_t stream);
 
 /*
+ * (9) SwiGLU fused into the epilogue, for a gate/up layer whose output rows
+ * are interleaved.
+ *
+ * Defined by: h3-rs src/weights.rs, QLinear::interleave_swiglu (the gate and
+ * up projections' output rows reordered to pairs g0, u0, g1, u1, ... so the
+ * activation fuses into the int8 GEMM), swiglu_interleaved and run_swiglu
+ * (silu(gate) * up over each pair).
+ *
+ * The layer holds N = 2F rows in that order (cr_interleave_rows builds it
+ * from the two halves [gate; up]).  With g and u the fp32 epilogue values of
+ * rows 2f and 2f + 1, computed exactly as in (3),
+ *   out[m, f] = out_dtype( (g / (1 + exp(-g))) * u )
+ * in fp32 (CUDA expf, IEEE division, each op rounded on its own), rounded
+ * once to out_dtype.  out is [M, F]; N odd gives CR_ERR_INVALID_ARG.  There
+ * is no acc_out: the int32 accumulators are those of (3) and (4) on the same
+ * layer.  The decode GEMV and the GEMM give the same bits.
+ *
+ * (9a) on quantised activations, any M (the prefill GEMM of (3));
+ * (9b) on quantised activations, 1 <= M <= 8 (the decode GEMV of (4));
+ * (9c) the whole forward as (6).
+ */
+cr_status cr_w4a8_gemm_swiglu(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                              const float *codebook, const float *s_channel, const float *bias,
+                              int64_t M, int64_t N, int64_t K, cr_out_dtype out_dtype, void *out,
+                              cr_stream_t stream);
+cr_status cr_w4a8_gemv_swiglu(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                              const float *codebook, const float *s_channel, const float *bias,
+                              int64_t M, int64_t N, int64_t K, cr_out_dtype out_dtype, void *out,
+                              cr_stream_t stream);
+cr_status cr_w4a8_linear_swiglu(const uint16_t *x, const uint8_t *qdata, const uint8_t *srel,
+                                const float *codebook, const float *s_channel, const float *bias,
+                                int64_t M, int64_t N, int64_t K, int act_qmax, cr_out_dtype out_dtype,
+                                void *out, int8_t *xq_work, float *xs_work, cr_stream_t stream);
+
+/*
+ * (10) Row interleave of a gate/up layer's arrays.
+ *
+ * Defined by: h3-rs src/weights.rs, interleave_rows: rows [0, F) and
+ * [F, 2F) of src become pairs, dst row 2f = src row f and dst row 2f + 1 =
+ * src row F + f, each row `row_bytes` bytes.  Apply it to qdata (K/2 bytes a
+ * row), srel (K/16), s_channel (4) and bias (4) of the stacked [gate; up]
+ * layer to get the layout (9) reads.  A one-time preparation, not part of the
+ * forward.
+ *
+ * src, dst: device buffers of rows * row_bytes bytes that must not overlap
+ * (CR_ERR_INVALID_ARG otherwise); no alignment is required.  rows must be even
+ * (CR_ERR_INVALID_ARG otherwise); rows == 0 or row_bytes == 0 does nothing.
+ */
+cr_status cr_interleave_rows(const void *src, void *dst, int64_t rows, int64_t row_bytes, cr_stream_t stream);
+
+/*
  * Waits for `stream`, then reads and clears the library's device error word,
  * which a kernel sets when one of its bounded pipeline waits runs out (the
  * kernel then abandons its tile and exits; its outputs are unspecified).

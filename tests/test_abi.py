@@ -29,7 +29,8 @@ def test_header_declares_the_boundary():
     names = _declared()
     for n in ("cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv", "cr_epilogue",
               "cr_w4a8_linear", "cr_status_string", "cr_check_device_error", "cr_version",
-              "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped"):
+              "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped", "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu",
+              "cr_w4a8_linear_swiglu", "cr_interleave_rows"):
         assert n in names
 
 
@@ -156,6 +157,41 @@ def test_grouped_validation(L):
     assert f(MIS, A16, 2, 256, two, 2, 127, 0, A16, A16, None) == cr.CR_ERR_ALIGNMENT
     assert f(A16, A16, 2, 256, two, 2, 127, 0, MIS, A16, None) == cr.CR_ERR_ALIGNMENT
     assert f(None, A16, 2, 256, empty, 1, 127, 0, None, None, None) == cr.CR_OK
+
+
+@pytest.mark.parametrize("name", ["cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu"])
+def test_swiglu_contraction_validation(L, name):
+    f = getattr(L, name)
+    ok = [A16] * 7
+
+    def call(M=4, N=8, K=256, dtype=0, ptrs=None, out=A16):
+        return f(*(ptrs or ok), M, N, K, dtype, out, None)
+
+    assert call(N=7) == cr.CR_ERR_INVALID_ARG         # gate/up pairs need an even N
+    assert call(M=-1) == cr.CR_ERR_INVALID_ARG
+    assert call(dtype=2) == cr.CR_ERR_INVALID_ARG
+    assert call(K=320) == cr.CR_ERR_UNSUPPORTED
+    assert call(out=None) == cr.CR_ERR_INVALID_ARG
+    assert call(out=MIS) == cr.CR_ERR_ALIGNMENT
+    assert call(M=0) == cr.CR_OK and call(N=0) == cr.CR_OK
+    if name == "cr_w4a8_gemv_swiglu":
+        assert call(M=9) == cr.CR_ERR_UNSUPPORTED
+    g = L.cr_w4a8_linear_swiglu
+    assert g(A16, A16, A16, A16, A16, None, 2, 7, 256, 127, 0, A16, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert g(A16, A16, A16, A16, A16, None, 2, 8, 256, 0, 0, A16, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert g(MIS, A16, A16, A16, A16, None, 2, 8, 256, 127, 0, A16, A16, A16, None) == cr.CR_ERR_ALIGNMENT
+    assert g(None, None, None, None, None, None, 0, 8, 256, 127, 0, None, None, None, None) == cr.CR_OK
+
+
+def test_interleave_rows_validation(L):
+    f = L.cr_interleave_rows
+    assert f(A16, 0x20000, 3, 16, None) == cr.CR_ERR_INVALID_ARG      # odd row count
+    assert f(A16, 0x20000, -2, 16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, 0x20000, 2, -1, None) == cr.CR_ERR_INVALID_ARG
+    assert f(None, 0x20000, 2, 16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, A16 + 16, 2, 16, None) == cr.CR_ERR_INVALID_ARG     # overlapping buffers
+    assert f(None, None, 0, 16, None) == cr.CR_OK and f(None, None, 2, 0, None) == cr.CR_OK
+    assert f(A16, 0x20000, 2 ** 40, 2 ** 40, None) == cr.CR_ERR_INVALID_ARG  # size overflows
 
 
 def test_valid_call_without_a_gpu_fails_loudly(L):

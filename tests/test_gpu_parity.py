@@ -12,7 +12,7 @@ import oracle
 import w4a8_codebook_quantized_b200 as cr
 from w4a8_codebook_quantized_b200 import inputs
 
-from gpu_util import Guarded, assert_output_close, bf16_dev, dev, host
+from gpu_util import Guarded, assert_output_close, assert_swiglu_close, bf16_dev, dev, host
 
 pytestmark = pytest.mark.gpu
 
@@ -321,3 +321,89 @@ def test_linear_grouped_end_to_end(M):
     for ly, y in zip(layers, outs32):
         ref = oracle.linear(x, ly.qdata, ly.srel, ly.codebook, ly.s_channel, ly.bias, out="f32", threads=THREADS)
         assert_output_close(host(y), ref["y"], "f32")
+
+
+# ---------------------------------------------------------------- SwiGLU on interleaved gate/up rows
+
+def test_interleave_rows_matches_oracle():
+    """Bit-exact row interleave for 16-byte, 4-byte and 1-byte row units."""
+    rng = np.random.default_rng(9)
+    for shape, dtype in (((64, 512), np.uint8), ((2, 16), np.uint8), ((1000,), np.float32), ((6, 3), np.uint8),
+                         ((4, 2, 5), np.int16)):
+        a = rng.integers(0, 255, size=shape).astype(dtype) if dtype != np.float32 else \
+            rng.standard_normal(shape).astype(dtype)
+        got = cr.cr_interleave_rows(dev(a))
+        assert np.array_equal(host(got), oracle.interleave_rows(a)), (shape, dtype)
+
+
+def _swiglu_layer(F, K, seed, with_bias=False):
+    """An interleaved gate/up layer (numpy) built by the oracle's interleave."""
+    g = inputs.layer(F, K, seed, with_bias=with_bias)
+    u = inputs.layer(F, K, seed + 1, with_bias=with_bias)
+    il = lambda a, b: oracle.interleave_rows(np.concatenate([a, b], axis=0))
+    return (il(g.qdata, u.qdata), il(g.srel, u.srel), g.codebook, il(g.s_channel, u.s_channel),
+            None if g.bias is None else il(g.bias, u.bias))
+
+
+def _swiglu_case(fn, M, N, K, seed, kind="bf16", with_bias=False):
+    qd, sr, cbk, wsc, bs = _swiglu_layer(N // 2, K, seed, with_bias)
+    x = inputs.activations(M, K, seed)
+    xq_r, xs_r = oracle.rotate_quant_act(x, None, 127)
+    acc_r = oracle.gemm_s32(xq_r, oracle.decode_w8(qd, sr, cbk), THREADS)
+    y_r = oracle.epilogue_swiglu(acc_r, xs_r, wsc, bs, kind)
+    dt = torch.bfloat16 if kind == "bf16" else torch.float32
+    out = Guarded((M, N // 2), dt)
+    fn(dev(xq_r), dev(xs_r), dev(qd), dev(sr), dev(cbk), dev(wsc), None if bs is None else dev(bs), out=out.tensor)
+    torch.cuda.synchronize()
+    assert out.intact()
+    assert_swiglu_close(host(out.tensor), y_r, kind)
+    return host(out.tensor)
+
+
+@pytest.mark.parametrize("M,N,K,kind,bias", [(1, 32, 256, "bf16", False), (8, 4096, 1024, "bf16", False),
+                                             (3, 26, 512, "bf16", True), (5, 1000, 2048, "f32", True),
+                                             (7, 2048, 16384, "bf16", False)])
+def test_gemv_swiglu(M, N, K, kind, bias):
+    _swiglu_case(cr.cr_w4a8_gemv_swiglu, M, N, K, M + N + K, kind, bias)
+
+
+@pytest.mark.parametrize("M,N,K,kind,bias", [(100, 512, 512, "bf16", False),     # one-CTA kernel, TMA stores
+                                             (129, 26, 256, "bf16", True),       # F = 13: per-thread stores
+                                             (300, 1000, 1024, "f32", True),     # F = 500: fp32 TMA stores
+                                             (300, 1000, 1024, "bf16", False),   # F = 500: per-thread stores
+                                             (2048, 4096, 512, "bf16", True),    # CTA pairs
+                                             (2000, 4000, 256, "f32", False)])   # CTA pairs, ragged, fp32
+def test_gemm_swiglu(M, N, K, kind, bias):
+    _swiglu_case(cr.cr_w4a8_gemm_swiglu, M, N, K, M + N + K, kind, bias)
+
+
+@pytest.mark.parametrize("M", [1, 2, 5, 8])
+def test_gemv_swiglu_equals_gemm_swiglu_bitwise(M):
+    N, K = 768, 2048
+    qd, sr, cbk, wsc, bs = (None if a is None else dev(a) for a in _swiglu_layer(N // 2, K, 60 + M, True))
+    x = bf16_dev(inputs.activations(M, K, 60 + M))
+    xq, xs = cr.cr_rotate_quant_act(x, cr.gemv_rows(M), 127)
+    for dt in (torch.bfloat16, torch.float32):
+        o1 = cr.cr_w4a8_gemv_swiglu(xq, xs, qd, sr, cbk, wsc, bs, m=M, out_dtype=dt)
+        o2 = cr.cr_w4a8_gemm_swiglu(xq, xs, qd, sr, cbk, wsc, bs, m=M, out_dtype=dt)
+        assert torch.equal(o1.view(torch.int16) if dt == torch.bfloat16 else o1.view(torch.int32),
+                           o2.view(torch.int16) if dt == torch.bfloat16 else o2.view(torch.int32))
+
+
+@pytest.mark.parametrize("M", [4, 300])
+def test_linear_swiglu_from_separate_gate_and_up(M):
+    """interleave_gate_up on the device from separate gate and up layers,
+    then the fused forward: equal to the oracle's SwiGLU forward."""
+    F, K = 512, 1024
+    g = inputs.layer(F, K, 80, with_bias=True)
+    u = inputs.layer(F, K, 81, with_bias=True)
+    layer = cr.interleave_gate_up((dev(g.qdata), dev(g.srel), dev(g.s_channel), dev(g.bias)),
+                                  (dev(u.qdata), dev(u.srel), dev(u.s_channel), dev(u.bias)))
+    x = inputs.activations(M, K, 82)
+    cb = dev(g.codebook)
+    y = cr.cr_w4a8_linear_swiglu(bf16_dev(x), layer[0], layer[1], cb, layer[2], layer[3])
+    il = lambda a, b: oracle.interleave_rows(np.concatenate([a, b], axis=0))
+    ref = oracle.linear_swiglu(x, il(g.qdata, u.qdata), il(g.srel, u.srel), g.codebook,
+                               il(g.s_channel, u.s_channel), il(g.bias, u.bias), threads=THREADS)
+    assert y.shape == (M, F)
+    assert_swiglu_close(host(y), ref["y"], "bf16")

@@ -27,6 +27,8 @@ __all__ = [
     "cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv",
     "cr_epilogue", "cr_w4a8_linear", "cr_w4a8_linear_decode_noalloc", "cr_check_device_error",
     "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped", "CrLayer",
+    "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu", "cr_w4a8_linear_swiglu", "cr_interleave_rows",
+    "interleave_gate_up",
     "cr_status_string", "cr_version",
     "gemv_rows",
 ]
@@ -83,6 +85,10 @@ def lib() -> ctypes.CDLL:
             L.cr_w4a8_linear.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P, P, P]
             L.cr_check_device_error.argtypes = [P]
             L.cr_w4a8_linear_decode_noalloc.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P]
+            L.cr_w4a8_gemm_swiglu.argtypes = contraction[:-2] + [P]
+            L.cr_w4a8_gemv_swiglu.argtypes = contraction[:-2] + [P]
+            L.cr_w4a8_linear_swiglu.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P, P, P]
+            L.cr_interleave_rows.argtypes = [P, P, i64, i64, P]
             LP = ctypes.POINTER(CrLayer)
             L.cr_w4a8_gemv_grouped.argtypes = [P, P, P, i64, i64, LP, i32, i32, P]
             L.cr_w4a8_linear_grouped.argtypes = [P, P, i64, i64, LP, i32, i32, i32, P, P, P]
@@ -443,6 +449,111 @@ def cr_w4a8_linear_grouped(x, codebook, layers, act_qmax: int = 127, out_dtype=N
                                         _out_code(out_dtype), _ptr(xq_work), _ptr(xs_work), _stream(stream)),
            "cr_w4a8_linear_grouped")
     return res
+
+
+def _swiglu_contraction(fn_name, xq, xs, qdata, srel, codebook, s_channel, bias, m, out_dtype, out, stream):
+    torch = _torch()
+    N, K = _layer(qdata, srel, codebook, s_channel, bias)
+    if N % 2:
+        raise ValueError(f"an interleaved gate/up layer has an even number of rows, got {N}")
+    _need(xq, "xq", (torch.int8,), 2)
+    _need(xs, "xs", (torch.float32,), 1)
+    M = xq.shape[0] if m is None else int(m)
+    if xq.shape[1] != K or xq.shape[0] < M or xs.shape[0] < M:
+        raise ValueError(f"xq {tuple(xq.shape)} / xs {tuple(xs.shape)} do not match M={M}, K={K}")
+    if out is None:
+        out = torch.empty(M, N // 2, dtype=out_dtype, device=xq.device)
+    _need(out, "out", (torch.bfloat16, torch.float32), shape=(M, N // 2))
+    fn = getattr(lib(), fn_name)
+    _check(fn(_ptr(xq), _ptr(xs), _ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), _ptr(bias),
+              M, N, K, _out_code(out.dtype), _ptr(out), _stream(stream)), fn_name)
+    return out
+
+
+def cr_w4a8_gemm_swiglu(xq, xs, qdata, srel, codebook, s_channel, bias=None, m: Optional[int] = None,
+                        out_dtype=None, out=None, stream=None):
+    """Prefill GEMM of an interleaved gate/up layer [2F, K] with SwiGLU fused
+    into the epilogue: out [M, F] = silu(gate) * up."""
+    torch = _torch()
+    return _swiglu_contraction("cr_w4a8_gemm_swiglu", xq, xs, qdata, srel, codebook, s_channel, bias, m,
+                               out_dtype or torch.bfloat16, out, stream)
+
+
+def cr_w4a8_gemv_swiglu(xq, xs, qdata, srel, codebook, s_channel, bias=None, m: Optional[int] = None,
+                        out_dtype=None, out=None, stream=None):
+    """Decode GEMV (M <= 8) of an interleaved gate/up layer with SwiGLU fused;
+    bitwise equal to cr_w4a8_gemm_swiglu."""
+    torch = _torch()
+    return _swiglu_contraction("cr_w4a8_gemv_swiglu", xq, xs, qdata, srel, codebook, s_channel, bias, m,
+                               out_dtype or torch.bfloat16, out, stream)
+
+
+def cr_w4a8_linear_swiglu(x, qdata, srel, codebook, s_channel, bias=None, act_qmax: int = 127, out_dtype=None,
+                          out=None, xq_work=None, xs_work=None, stream=None):
+    """The forward of an interleaved gate/up layer with SwiGLU fused:
+    rotate + quantise x, then the decode GEMV (M <= 8) or the prefill GEMM."""
+    torch = _torch()
+    _need(x, "x", (torch.bfloat16,), 2)
+    M, K = x.shape
+    N, Kw = _layer(qdata, srel, codebook, s_channel, bias)
+    if Kw != K:
+        raise ValueError(f"x has K={K}, the layer K={Kw}")
+    if N % 2:
+        raise ValueError(f"an interleaved gate/up layer has an even number of rows, got {N}")
+    rows = gemv_rows(M) if 1 <= M <= CR_GEMV_MAX_M else M
+    if xq_work is None:
+        xq_work = torch.empty(rows, K, dtype=torch.int8, device=x.device)
+    if xs_work is None:
+        xs_work = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _need(xq_work, "xq_work", (torch.int8,), 2)
+    _need(xs_work, "xs_work", (torch.float32,), 1)
+    if xq_work.shape[0] < rows or xq_work.shape[1] != K or xs_work.shape[0] < rows:
+        raise ValueError(f"work buffers need {rows} rows of K={K}")
+    if out is None:
+        out = torch.empty(M, N // 2, dtype=out_dtype or torch.bfloat16, device=x.device)
+    _need(out, "out", (torch.bfloat16, torch.float32), shape=(M, N // 2))
+    _check(lib().cr_w4a8_linear_swiglu(_ptr(x), _ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel),
+                                       _ptr(bias), M, N, K, int(act_qmax), _out_code(out.dtype), _ptr(out),
+                                       _ptr(xq_work), _ptr(xs_work), _stream(stream)), "cr_w4a8_linear_swiglu")
+    return out
+
+
+def cr_interleave_rows(src, dst=None, stream=None):
+    """Rows [0, F) and [F, 2F) of src become pairs: dst[2f] = src[f],
+    dst[2f + 1] = src[F + f] (any dtype, rows along dim 0)."""
+    torch = _torch()
+    if not isinstance(src, torch.Tensor) or not src.is_cuda or not src.is_contiguous() or src.dim() < 1:
+        raise ValueError("src must be a contiguous CUDA tensor with at least one dimension")
+    rows = src.shape[0]
+    if rows % 2:
+        raise ValueError(f"an even number of rows is needed, got {rows}")
+    if dst is None:
+        dst = torch.empty_like(src)
+    if not dst.is_cuda or not dst.is_contiguous() or dst.shape != src.shape or dst.dtype != src.dtype:
+        raise ValueError("dst must be a contiguous CUDA tensor of src's shape and dtype")
+    row_bytes = src.numel() * src.element_size() // rows if rows else 0
+    _check(lib().cr_interleave_rows(_ptr(src), _ptr(dst), rows, row_bytes, _stream(stream)), "cr_interleave_rows")
+    return dst
+
+
+def interleave_gate_up(gate, up, stream=None):
+    """A gate/up pair of layers, each (qdata, srel, s_channel[, bias]) with
+    the same K, as one layer with interleaved rows for the SwiGLU entry points
+    (h3-rs weights.rs, QLinear::interleave_swiglu).  Returns (qdata, srel,
+    s_channel, bias or None)."""
+    torch = _torch()
+    gate, up = list(gate), list(up)
+    if len(gate) != len(up) or len(gate) not in (3, 4):
+        raise ValueError("gate and up are (qdata, srel, s_channel[, bias]) of the same form")
+    res = []
+    for i, (g, u) in enumerate(zip(gate, up)):
+        if g is None and u is None:
+            res.append(None)
+            continue
+        if g is None or u is None or g.shape != u.shape or g.dtype != u.dtype:
+            raise ValueError(f"gate and up differ in field {i}")
+        res.append(cr_interleave_rows(torch.cat([g, u], dim=0).contiguous(), stream=stream))
+    return tuple(res) + ((None,) if len(res) == 3 else ())
 
 
 def cr_check_device_error(stream=None) -> None:

@@ -119,6 +119,15 @@ __device__ __forceinline__ float epilogue_value(int32_t acc, float xs, float ws,
     return y;
 }
 
+// SwiGLU of one gate/up pair of epilogue values (h3-rs weights.rs,
+// swiglu_interleaved): silu(g) * u = g / (1 + e^-g) * u, in fp32 with CUDA's
+// expf and IEEE division.  e^-g overflows to +inf for g < -88.7, which gives
+// a zero of g's sign.
+__device__ __forceinline__ float swiglu_value(float g, float u)
+{
+    return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+}
+
 __device__ __forceinline__ uint16_t to_bf16_bits(float y)
 {
     return __bfloat16_as_ushort(__float2bfloat16_rn(y));

@@ -167,7 +167,7 @@ bool make_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype,
 template <int L>
 cr_status launch_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const float *codebook,
                       int64_t M, int64_t K, const cr_w4a8_layer *layers, int num_layers, cr_out_dtype out_dtype,
-                      cudaStream_t stream, bool pdl)
+                      cudaStream_t stream, bool pdl, int swiglu = 0)
 {
     using namespace cr;
     using C = gv::Prod;
@@ -199,6 +199,7 @@ cr_status launch_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float
         args.layer[l].out = ly.out;
         args.layer[l].acc_out = ly.acc_out;
         args.layer[l].N = (int)ly.N;
+        args.layer[l].swiglu = swiglu;
         tiles += (ly.N + gv::kRows - 1) / gv::kRows;
     }
     if (tiles == 0)
@@ -250,7 +251,7 @@ cr_status run_gemv_layers(DeviceState &d, const int8_t *xq, const float *xs, con
 cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const uint8_t *qdata,
                    const uint8_t *srel, const float *codebook, const float *s_channel, const float *bias, int64_t M,
                    int64_t N, int64_t K, cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream,
-                   bool pdl)
+                   bool pdl, int swiglu = 0)
 {
     cr_w4a8_layer ly;
     ly.qdata = qdata;
@@ -260,7 +261,7 @@ cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *x
     ly.N = N;
     ly.out = out;
     ly.acc_out = acc_out;
-    return launch_gemv<1>(num_sms, attr_set, xq, xs, codebook, M, K, &ly, 1, out_dtype, stream, pdl);
+    return launch_gemv<1>(num_sms, attr_set, xq, xs, codebook, M, K, &ly, 1, out_dtype, stream, pdl, swiglu);
 }
 
 // Shared validation of the contraction entry points.
@@ -350,7 +351,7 @@ cr_status side_stream(DeviceState &d)
 cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
                    const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K,
                    cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream,
-                   const std::function<cr_status()> *activations = nullptr)
+                   const std::function<cr_status()> *activations = nullptr, int swiglu = 0)
 {
     using namespace cr;
     if (!d.gemm_attr_set) {
@@ -393,7 +394,8 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
     }
     CUtensorMap ta, tb, to;
     const int out_f32 = out_dtype == CR_OUT_F32;
-    const int vec_ok = out_f32 ? (N % 4 == 0) : (N % 8 == 0);
+    const int64_t OC = swiglu ? N / 2 : N;  // output columns
+    const int vec_ok = out_f32 ? (OC % 4 == 0) : (OC % 8 == 0);
     // Output through TMA bulk stores when rows are 16-byte multiples and the
     // int32 accumulators are not requested: 32-row x 128-byte boxes, 128B swizzle.
     const int tma_out = vec_ok && acc_out == nullptr;
@@ -403,8 +405,8 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
     if (st == CR_OK) {
         to = ta;  // placeholder when the output does not go through TMA
         if (tma_out) {
-            const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)M};
-            const cuuint64_t strides[1] = {(cuuint64_t)N * (out_f32 ? 4u : 2u)};
+            const cuuint64_t dims[2] = {(cuuint64_t)OC, (cuuint64_t)M};
+            const cuuint64_t strides[1] = {(cuuint64_t)OC * (out_f32 ? 4u : 2u)};
             const cuuint32_t box[2] = {out_f32 ? 32u : 64u, 32u};
             const cuuint32_t estr[2] = {1u, 1u};
             if (g_encode_tiled(&to, out_f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out,
@@ -445,13 +447,13 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
             cfg.attrs = attr;
             cfg.numAttrs = 1;
             st = launched(cudaLaunchKernelEx(&cfg, gm::gemm_pair_kernel, ta, tb_half, to, xs, s_channel, bias, (int)M,
-                                             (int)N, (int)K, out_f32, vec_ok, tma_out, out, acc_out));
+                                             (int)N, (int)K, out_f32, swiglu, tma_out, out, acc_out));
         }
     } else if (st == CR_OK) {
         const int64_t tiles = ((M + gm::BM - 1) / gm::BM) * ((N + gm::BN - 1) / gm::BN);
         const int grid = (int)(tiles < d.num_sms ? tiles : d.num_sms);
         gm::gemm_kernel<<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(ta, tb, to, xs, s_channel, bias, (int)M,
-                                                                         (int)N, (int)K, out_f32, vec_ok, tma_out, out,
+                                                                         (int)N, (int)K, out_f32, swiglu, tma_out, out,
                                                                          acc_out);
         st = launched(cudaGetLastError());
     }
@@ -577,11 +579,20 @@ cr_status cr_epilogue(const int32_t *acc, const float *xs, const float *s_channe
                                             stream));
 }
 
-cr_status cr_w4a8_linear(const uint16_t *x, const uint8_t *qdata, const uint8_t *srel, const float *codebook,
-                         const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K, int act_qmax,
-                         cr_out_dtype out_dtype, void *out, int8_t *xq_work, float *xs_work, cr_stream_t stream)
+}  // extern "C"
+
+namespace {
+
+// cr_w4a8_linear and cr_w4a8_linear_swiglu: rotate + quantise, then the GEMV
+// (M <= 8) or the GEMM with the weight decode overlapping the activations.
+cr_status linear_impl(const uint16_t *x, const uint8_t *qdata, const uint8_t *srel, const float *codebook,
+                      const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K, int act_qmax,
+                      cr_out_dtype out_dtype, void *out, int8_t *xq_work, float *xs_work, cudaStream_t stream,
+                      int swiglu)
 {
     if (M < 0 || N < 0 || K < 0 || act_qmax < 1 || act_qmax > 127)
+        return CR_ERR_INVALID_ARG;
+    if (swiglu && N % 2 != 0)
         return CR_ERR_INVALID_ARG;
     int64_t MP = M;
     if (M >= 1 && M <= CR_GEMV_MAX_M) {
@@ -605,13 +616,89 @@ cr_status cr_w4a8_linear(const uint16_t *x, const uint8_t *qdata, const uint8_t 
     if (M > CR_GEMV_MAX_M) {
         const std::function<cr_status()> act = activations;
         return run_gemm(*d, xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, nullptr,
-                        stream, &act);
+                        stream, &act, swiglu);
     }
     st = activations();
     if (st != CR_OK)
         return st;
     return run_gemv(d->num_sms, d->gemv_attr_set, xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K,
-                    out_dtype, out, nullptr, stream, /*pdl=*/true);
+                    out_dtype, out, nullptr, stream, /*pdl=*/true, swiglu);
+}
+
+// cr_w4a8_gemm_swiglu and cr_w4a8_gemv_swiglu.
+cr_status contraction_swiglu(bool gemv, const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                             const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N,
+                             int64_t K, cr_out_dtype out_dtype, void *out, cudaStream_t stream)
+{
+    if (gemv && M > CR_GEMV_MAX_M)
+        return CR_ERR_UNSUPPORTED;
+    if (N % 2 != 0)
+        return CR_ERR_INVALID_ARG;
+    cr_status st = check_contraction(xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, nullptr);
+    if (st != CR_OK || M == 0 || N == 0)
+        return st;
+    DeviceState *d = nullptr;
+    st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    if (gemv)
+        return run_gemv(d->num_sms, d->gemv_attr_set, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K,
+                        out_dtype, out, nullptr, stream, /*pdl=*/true, /*swiglu=*/1);
+    return run_gemm(*d, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, nullptr, stream,
+                    nullptr, /*swiglu=*/1);
+}
+
+}  // namespace
+
+extern "C" {
+
+cr_status cr_w4a8_linear(const uint16_t *x, const uint8_t *qdata, const uint8_t *srel, const float *codebook,
+                         const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K, int act_qmax,
+                         cr_out_dtype out_dtype, void *out, int8_t *xq_work, float *xs_work, cr_stream_t stream)
+{
+    return linear_impl(x, qdata, srel, codebook, s_channel, bias, M, N, K, act_qmax, out_dtype, out, xq_work, xs_work,
+                       stream, 0);
+}
+
+cr_status cr_w4a8_linear_swiglu(const uint16_t *x, const uint8_t *qdata, const uint8_t *srel, const float *codebook,
+                                const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K,
+                                int act_qmax, cr_out_dtype out_dtype, void *out, int8_t *xq_work, float *xs_work,
+                                cr_stream_t stream)
+{
+    return linear_impl(x, qdata, srel, codebook, s_channel, bias, M, N, K, act_qmax, out_dtype, out, xq_work, xs_work,
+                       stream, 1);
+}
+
+cr_status cr_w4a8_gemm_swiglu(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                              const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N,
+                              int64_t K, cr_out_dtype out_dtype, void *out, cr_stream_t stream)
+{
+    return contraction_swiglu(false, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, stream);
+}
+
+cr_status cr_w4a8_gemv_swiglu(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                              const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N,
+                              int64_t K, cr_out_dtype out_dtype, void *out, cr_stream_t stream)
+{
+    return contraction_swiglu(true, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, stream);
+}
+
+cr_status cr_interleave_rows(const void *src, void *dst, int64_t rows, int64_t row_bytes, cr_stream_t stream)
+{
+    if (rows < 0 || row_bytes < 0 || rows % 2 != 0)
+        return CR_ERR_INVALID_ARG;
+    if (rows == 0 || row_bytes == 0)
+        return CR_OK;
+    if (!src || !dst || rows > INT64_MAX / row_bytes)
+        return CR_ERR_INVALID_ARG;
+    const uintptr_t s0 = (uintptr_t)src, d0 = (uintptr_t)dst, n = (uintptr_t)(rows * row_bytes);
+    if (s0 < d0 + n && d0 < s0 + n)
+        return CR_ERR_INVALID_ARG;  // the copy is not in place
+    DeviceState *d = nullptr;
+    const cr_status st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    return launched(cr::ew::launch_interleave_rows(src, dst, rows, row_bytes, d->num_sms, stream));
 }
 
 cr_status cr_w4a8_gemv_grouped(const int8_t *xq, const float *xs, const float *codebook, int64_t M, int64_t K,

@@ -145,5 +145,50 @@ inline cudaError_t launch_epilogue(const int32_t *acc, const float *xs, const fl
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- row interleave
+//
+// h3-rs weights.rs, interleave_rows: the two halves of the row dimension,
+// rows [0, F) and [F, 2F), become pairs: dst row 2f = src row f and dst row
+// 2f + 1 = src row F + f.  Applied to a gate/up layer's qdata, srel,
+// s_channel and bias it gives the row order the SwiGLU epilogues read.  A
+// grid-stride copy in units of V bytes (16, 4 or 1, the largest that divides
+// the row and both addresses).
+template <class V>
+__global__ void __launch_bounds__(kThreads) interleave_rows_kernel(const V *__restrict__ src, V *__restrict__ dst,
+                                                                   int64_t rows, int64_t units_per_row)
+{
+    const int64_t half = rows >> 1, total = rows * units_per_row;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t drow = i / units_per_row, c = i - drow * units_per_row;
+        const int64_t srow = (drow & 1) ? half + (drow >> 1) : (drow >> 1);
+        dst[i] = src[srow * units_per_row + c];
+    }
+}
+
+inline cudaError_t launch_interleave_rows(const void *src, void *dst, int64_t rows, int64_t row_bytes, int num_sms,
+                                          cudaStream_t stream)
+{
+    const uintptr_t align = (uintptr_t)src | (uintptr_t)dst | (uintptr_t)row_bytes;
+    const int vec = (align & 15) == 0 ? 16 : (align & 3) == 0 ? 4 : 1;
+    const int64_t units = row_bytes / vec, total = rows * units;
+    int64_t blocks = (total + kThreads - 1) / kThreads;
+    const int64_t cap = (int64_t)num_sms * 8;
+    if (blocks > cap)
+        blocks = cap;
+    if (blocks < 1)
+        blocks = 1;
+    if (vec == 16)
+        interleave_rows_kernel<uint4><<<(unsigned)blocks, kThreads, 0, stream>>>(
+            static_cast<const uint4 *>(src), static_cast<uint4 *>(dst), rows, units);
+    else if (vec == 4)
+        interleave_rows_kernel<uint32_t><<<(unsigned)blocks, kThreads, 0, stream>>>(
+            static_cast<const uint32_t *>(src), static_cast<uint32_t *>(dst), rows, units);
+    else
+        interleave_rows_kernel<uint8_t><<<(unsigned)blocks, kThreads, 0, stream>>>(
+            static_cast<const uint8_t *>(src), static_cast<uint8_t *>(dst), rows, units);
+    return cudaGetLastError();
+}
+
 }  // namespace ew
 }  // namespace cr

@@ -24,6 +24,8 @@
 
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "cr_device.cuh"
 
 namespace cr {
@@ -73,7 +75,8 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_n, int &tm, int 
 template <class Release>
 __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row0, int col_base, int lane, float xm, bool row_ok,
                                               const float *wsv, const float *bsv, bool has_bias, int M, int N,
-                                              int out_f32, int tma_out, const CUtensorMap *tmOut, uint8_t *stage_buf,
+                                              int out_f32, int swiglu, int tma_out, const CUtensorMap *tmOut,
+                                              uint8_t *stage_buf,
                                               uint32_t &units_issued, void *__restrict__ out,
                                               int32_t *__restrict__ acc_out, const float *__restrict__ ws,
                                               const float *__restrict__ bias, Release release)
@@ -125,6 +128,83 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row0, int col_
         ++units_issued;
     };
     uint32_t cur[32], nxt[32], packed[32];
+    if (swiglu) {
+        // Interleaved gate/up rows: accumulator columns 2f and 2f + 1 are one
+        // pair and give output column f of [M, N / 2].  Each 32-column TMEM
+        // load yields 16 outputs; a 128-byte unit (64 bf16 or 32 fp32 outputs)
+        // takes 4 or 2 loads.
+        const int F = N >> 1, ocol_base = col_base >> 1;
+        auto pairs16 = [&](int c0, float (&y)[16]) {
+#pragma unroll
+            for (int p = 0; p < 16; ++p) {
+                float g = __fmul_rn(__int2float_rn((int32_t)cur[2 * p]), __fmul_rn(xm, wsv[c0 + 2 * p]));
+                float u = __fmul_rn(__int2float_rn((int32_t)cur[2 * p + 1]), __fmul_rn(xm, wsv[c0 + 2 * p + 1]));
+                if (has_bias) {
+                    g = __fadd_rn(g, bsv[c0 + 2 * p]);
+                    u = __fadd_rn(u, bsv[c0 + 2 * p + 1]);
+                }
+                y[p] = swiglu_value(g, u);
+            }
+        };
+        // uo: output columns per 128-byte unit (compile-time, so that `packed`
+        // stays in registers)
+        auto units = [&](auto uo_c) {
+            constexpr int uo = decltype(uo_c)::value;
+            for (int un = 0; un < BN / (2 * uo); ++un) {
+#pragma unroll
+                for (int k = 0; k < uo / 16; ++k) {
+                    const int c0 = 2 * uo * un + 32 * k;
+                    __syncwarp();
+                    tmem_ld_32cols(tbase + (uint32_t)c0, cur);
+                    tmem_ld_wait();
+                    if (c0 + 32 == BN)
+                        release();
+                    float y[16];
+                    pairs16(c0, y);
+                    if constexpr (uo == 32) {
+#pragma unroll
+                        for (int p = 0; p < 16; ++p)
+                            packed[16 * k + p] = __float_as_uint(y[p]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            packed[8 * k + i] = to_bf16x2_bits(y[2 * i], y[2 * i + 1]);
+                    }
+                }
+                store_unit(packed, ocol_base + uo * un);
+            }
+        };
+        if (tma_out && out_f32) {
+            units(std::integral_constant<int, 32>{});
+        } else if (tma_out) {
+            units(std::integral_constant<int, 64>{});
+        } else {
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                const int c0 = 32 * ch;
+                __syncwarp();
+                tmem_ld_32cols(tbase + (uint32_t)c0, cur);
+                tmem_ld_wait();
+                if (ch + 1 == BN / 32)
+                    release();
+                float y[16];
+                pairs16(c0, y);
+                const int f0 = ocol_base + 16 * ch;
+                if (row_ok && f0 < F) {
+                    const int64_t base = (int64_t)row * F + f0;
+#pragma unroll
+                    for (int p = 0; p < 16; ++p) {
+                        if (f0 + p >= F)
+                            break;
+                        if (out_f32)
+                            reinterpret_cast<float *>(out)[base + p] = y[p];
+                        else
+                            reinterpret_cast<uint16_t *>(out)[base + p] = to_bf16_bits(y[p]);
+                    }
+                }
+            }
+        }
+        return;
+    }
     __syncwarp();
     tmem_ld_32cols(tbase, cur);
     tmem_ld_wait();
@@ -175,8 +255,11 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row0, int col_
             const int col0 = col_base + 32 * ch;
             if (row_ok && col0 < N) {
                 const int64_t base = (int64_t)row * N + col0;
-                for (int j = 0; j < 32 && col0 + j < N; ++j) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
                     const int n = col0 + j;
+                    if (n >= N)
+                        break;
                     const float y = epilogue_value((int32_t)cur[j], xm, ws[n], bias, n);
                     if (out_f32)
                         reinterpret_cast<float *>(out)[base + j] = y;
@@ -200,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmOut, const float *__restrict__ xs,
                 const float *__restrict__ ws, const float *__restrict__ bias, int M, int N, int K, int out_f32,
-                int vec_ok, int tma_out, void *__restrict__ out, int32_t *__restrict__ acc_out)
+                int swiglu, int tma_out, void *__restrict__ out, int32_t *__restrict__ acc_out)
 {
     extern __shared__ uint8_t smem_raw[];
     Smem &sh = smem_aligned_1024<Smem>(smem_raw);
@@ -351,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float xm = row_ok ? xs[row] : 0.0f;
             const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN);
             epilogue_tile(tbase, tm * BM + 32 * q, tn * BN, lane, xm, row_ok, sh.wsb[buf], sh.biasb[buf],
-                          bias != nullptr, M, N, out_f32, tma_out, &tmOut, sh.epi[q], units_issued, out, acc_out, ws,
+                          bias != nullptr, M, N, out_f32, swiglu, tma_out, &tmOut, sh.epi[q], units_issued, out, acc_out, ws,
                           bias, [&]() {
                               tc_fence_before();
                               __syncwarp();
@@ -409,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmOut, const float *__restrict__ xs,
                      const float *__restrict__ ws, const float *__restrict__ bias, int M, int N, int K, int out_f32,
-                     int vec_ok, int tma_out, void *__restrict__ out, int32_t *__restrict__ acc_out)
+                     int swiglu, int tma_out, void *__restrict__ out, int32_t *__restrict__ acc_out)
 {
     extern __shared__ uint8_t smem_raw[];
     pair::Smem &sh = smem_aligned_1024<pair::Smem>(smem_raw);
@@ -567,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN);
             const uint32_t release_addr = mapa_shared(smem_u32(&sh.tmem_empty[buf]), 0);
             epilogue_tile(tbase, row0, tn * BN, lane, xm, row_ok, sh.wsb[buf], sh.biasb[buf], bias != nullptr, M,
-                          N, out_f32, tma_out, &tmOut, sh.epi[q], units_issued, out, acc_out, ws, bias, [&]() {
+                          N, out_f32, swiglu, tma_out, &tmOut, sh.epi[q], units_issued, out, acc_out, ws, bias, [&]() {
                               tc_fence_before();
                               __syncwarp();
                               if (lane == 0)

@@ -160,6 +160,7 @@ struct GemvLayer {
     int32_t *acc_out;   // [M, N] or null
     int N;
     int tile0;
+    int swiglu;         // rows interleaved as gate/up pairs; out is [M, N / 2] of silu(gate) * up
 };
 
 // tm_codes[l]: layer l's packed codes as 32-bit words, dims {16, N, K / 128},
@@ -430,7 +431,29 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
             __syncwarp();
             if (ok && lane == 0)
                 mbar_arrive(&sh.red_empty[rb]);
-            if (ok && !*abort) {
+            // warp-uniform, as the SwiGLU path shuffles across lanes
+            const bool go = __shfl_sync(0xffffffffu, (int)(ok && !*abort), 0) != 0;
+            if (go && ly.swiglu) {
+                // rows 2f (gate) and 2f + 1 (up) of a pair are lanes l and l + 8
+                // of the same u (row0 is a multiple of 16)
+                const int F = N >> 1;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = lane + 32 * u, n = row0 + (e >> 3), m = e & 7;
+                    float y = __fmul_rn(__int2float_rn(acc[u]), __fmul_rn(exs[u], ews[u]));
+                    if (bias != nullptr)
+                        y = __fadd_rn(y, eb[u]);
+                    const float up = __shfl_down_sync(0xffffffffu, y, 8);
+                    if (live[u] && ((lane >> 3) & 1) == 0) {
+                        const float v = swiglu_value(y, up);
+                        const int64_t o = (int64_t)m * F + (n >> 1);
+                        if (out_f32)
+                            reinterpret_cast<float *>(out)[o] = v;
+                        else
+                            reinterpret_cast<uint16_t *>(out)[o] = to_bf16_bits(v);
+                    }
+                }
+            } else if (go) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     if (!live[u])
