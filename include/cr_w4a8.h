@@ -289,8 +289,8 @@ cr_status cr_w4a8_linear_grouped(const uint16_t *x, const float *codebook, int64
  * from the two halves [gate; up]).  With g and u the fp32 epilogue values of
  * rows 2f and 2f + 1, computed exactly as in (3),
  *   out[m, f] = out_dtype( (g / (1 + exp(-g))) * u )
- * in fp32 (CUDA expf, IEEE division, each op rounded on its own), rounded
- * once to out_dtype.  out is [M, F]; N odd gives CR_ERR_INVALID_ARG.  There
+ * in fp32 (CUDA expf, the fast division __fdividef with at most 2 ulp of
+ * error, each op rounded on its own), rounded once to out_dtype.  out is [M, F]; N odd gives CR_ERR_INVALID_ARG.  There
  * is no acc_out: the int32 accumulators are those of (3) and (4) on the same
  * layer.  The decode GEMV and the GEMM give the same bits.
  *

@@ -121,11 +121,13 @@ __device__ __forceinline__ float epilogue_value(int32_t acc, float xs, float ws,
 
 // SwiGLU of one gate/up pair of epilogue values (h3-rs weights.rs,
 // swiglu_interleaved): silu(g) * u = g / (1 + e^-g) * u, in fp32 with CUDA's
-// expf and IEEE division.  e^-g overflows to +inf for g < -88.7, which gives
-// a zero of g's sign.
+// expf and its fast division __fdividef (at most 2 ulp; the IEEE division's
+// slow-path branch would keep the compiler from overlapping the independent
+// pairs of a thread).  For g < -88.7, e^-g is +inf and the quotient is a zero
+// of g's sign.
 __device__ __forceinline__ float swiglu_value(float g, float u)
 {
-    return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+    return __fmul_rn(__fdividef(g, __fadd_rn(1.0f, expf(-g))), u);
 }
 
 __device__ __forceinline__ uint16_t to_bf16_bits(float y)
