@@ -56,6 +56,8 @@ def parse():
     p.add_argument("--prefill-workload", default="c3_prefill_2k_4k")
     p.add_argument("--no-prefill", action="store_true")
     p.add_argument("--no-grouped", action="store_true")
+    p.add_argument("--no-swiglu", action="store_true")
+    p.add_argument("--swiglu-workload", default="c4_mlp_up")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
     return p.parse_args()
@@ -434,6 +436,10 @@ def run_ours(args):
     if not args.no_grouped:
         grouped = run_grouped(args, world, rank, local, case)
 
+    swiglu = None
+    if not args.no_swiglu:
+        swiglu = run_swiglu(args, world, rank, pk)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(case, args.cpu_seconds)
@@ -448,7 +454,7 @@ def run_ours(args):
                    "timing": "one CUDA-graph replay of K steps (graph uploaded beforehand), CUDA events on the capture stream",
                    "parallelism": f"replica x{world}"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps,
-        "clocks": clocks, "prefill": prefill, "grouped": grouped,
+        "clocks": clocks, "prefill": prefill, "grouped": grouped, "swiglu": swiglu,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -527,6 +533,71 @@ def run_prefill(args, world, rank, local, pk):
                          "kernel": "cr_w4a8_gemm call (weight decode to an int8 transient + tcgen05 GEMM)",
                          "peak_source": f"{pk['source']} bf16_tflops x {INT8_OVER_BF16} (nominal int8/bf16 ratio)",
                          "us_per_call": round(tg * 1e6, 2)}}
+
+
+def flushed_medians(fns, steps):
+    """Each fn() captured once as a CUDA graph (uploaded first) and replayed
+    `steps` times, a 256 MiB L2 flush before every replay outside the CUDA
+    events on the replay stream; the median seconds of each."""
+    import torch
+    stream = torch.cuda.Stream()
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    graphs = []
+    for fn in fns:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        upload_graph(g, stream)
+        graphs.append(g)
+    res = []
+    with torch.cuda.stream(stream):
+        for g in graphs:
+            t = []
+            for i in range(steps):
+                flush.fill_(i & 0xFF)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                t.append(e0.elapsed_time(e1) / 1000.0)
+            res.append(statistics.median(t))
+    del graphs
+    return res
+
+
+def run_swiglu(args, world, rank, pk):
+    """A gate/up projection stored with interleaved rows (N = 2F), SwiGLU fused
+    into the GEMM epilogue (cr_w4a8_linear_swiglu, out [M, F]) against the
+    plain forward of the same layer (cr_w4a8_linear, out [M, N])."""
+    import torch
+
+    import w4a8_codebook_quantized_b200 as cr
+    from w4a8_codebook_quantized_b200 import inputs
+    case = inputs.CASES[args.swiglu_workload]
+    M, N, K = case.M, case.N, case.K
+    layer = inputs.layer(N, K, rank_seed(case.seed, rank))
+    x = inputs.activations(M, K, rank_seed(case.seed, rank), case.dist)
+    q, s, cb, ws = (torch.from_numpy(a).cuda() for a in (layer.qdata, layer.srel, layer.codebook, layer.s_channel))
+    xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+    xs = torch.empty(M, dtype=torch.float32, device="cuda")
+    out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    out_sw = torch.empty(M, N // 2, dtype=torch.bfloat16, device="cuda")
+    fused = lambda: cr.cr_w4a8_linear_swiglu(xd, q, s, cb, ws, out=out_sw, xq_work=xq, xs_work=xs)
+    plain = lambda: cr.cr_w4a8_linear(xd, q, s, cb, ws, out=out, xq_work=xq, xs_work=xs)
+    for _ in range(max(3, args.warmup)):
+        fused()
+        plain()
+    steps = max(3, min(args.steps, 20))
+    tf, tp = flushed_medians([fused, plain], steps)
+    tf, tp = max_over_ranks(tf, world), max_over_ranks(tp, world)
+    ops = 2.0 * M * N * K
+    return {"workload": f"{case.name} as interleaved gate/up: M={M}, N=2F={N}, K={K}, out [M, {N // 2}]",
+            "value": round(world * ops / tf / 1e12, 2), "unit": "TOPS", "ms_per_step": round(tf * 1e3, 4),
+            "plain_forward": {"value": round(world * ops / tp / 1e12, 2), "ms_per_step": round(tp * 1e3, 4)},
+            "steps": steps, "l2": "256 MiB write between steps, outside the timed events"}
 
 
 GROUPED_NS = (4096, 1024, 1024)  # q, k, v of an attention block with 8-way grouped k/v heads
