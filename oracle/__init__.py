@@ -59,6 +59,20 @@ def lib() -> ctypes.CDLL:
             L.or_f64_to_bf16_rne.restype = ctypes.c_uint16
             L.or_epilogue_swiglu.argtypes = [P, P, P, P, i64, i64, ctypes.c_int, P]
             L.or_epilogue_swiglu.restype = None
+            L.or_f32_to_fp8_e4m3fn.argtypes = [ctypes.c_float]
+            L.or_f32_to_fp8_e4m3fn.restype = ctypes.c_uint8
+            L.or_nearest_level.argtypes = [P, ctypes.c_int, ctypes.c_float]
+            L.or_nearest_level.restype = ctypes.c_int
+            L.or_stochastic_level.argtypes = [P, ctypes.c_int, ctypes.c_float, ctypes.c_float]
+            L.or_stochastic_level.restype = ctypes.c_int
+            L.or_grid_levels.argtypes = [P, ctypes.c_uint8, P]
+            L.or_grid_levels.restype = None
+            L.or_group_scale_als.argtypes = [P, P, P]
+            L.or_group_scale_als.restype = ctypes.c_float
+            L.or_quantize_rotated.argtypes = [P, i64, i64, P, P, P, P]
+            L.or_quantize_rotated.restype = ctypes.c_int
+            L.or_assign_codes.argtypes = [P, P, P, P, P, i64, i64, P]
+            L.or_assign_codes.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -254,6 +268,66 @@ def linear_swiglu(x_bf16, qdata, srel, codebook, s_channel, bias=None, qmax: int
     acc = gemm_s32(xq, w8, threads)
     y = epilogue_swiglu(acc, xs, s_channel, bias, out)
     return {"xq": xq, "xs": xs, "w8": w8, "acc": acc, "y": y}
+
+
+# ---------------------------------------------------------------- offline quantiser
+
+def f32_to_fp8(value: float) -> int:
+    """One fp32 -> fp8 e4m3fn byte with torch's cast semantics (NaN on overflow)."""
+    return int(lib().or_f32_to_fp8_e4m3fn(float(np.float32(value))))
+
+
+def nearest_level(levels, x: float) -> int:
+    """Index of the nearest of the sorted levels to fp32 x (ties to the lower)."""
+    lv = _c(levels, np.float32)
+    return int(lib().or_nearest_level(_p(lv), lv.size, float(np.float32(x))))
+
+
+def stochastic_level(levels, x: float, u: float) -> int:
+    lv = _c(levels, np.float32)
+    return int(lib().or_stochastic_level(_p(lv), lv.size, float(np.float32(x)), float(np.float32(u))))
+
+
+def grid_levels(codebook, srel_byte: int) -> np.ndarray:
+    """The 16 int8 grid values of one fp8 group scale, as fp32."""
+    cb = _c(codebook, np.float32)
+    out = np.empty(16, dtype=np.float32)
+    lib().or_grid_levels(_p(cb), int(srel_byte), _p(out))
+    return out
+
+
+def group_scale_als(gw, codebook):
+    """(gs, codes) of one 16-weight group after the ALS passes."""
+    g = _c(gw, np.float32)
+    cb = _c(codebook, np.float32)
+    q = np.empty(16, dtype=np.int32)
+    gs = lib().or_group_scale_als(_p(g), _p(cb), _p(q))
+    return float(np.float32(gs)), q
+
+
+def quantize_rotated(w_rot, codebook):
+    """w_rot fp32 [N, K] -> (qdata uint8 [N, K/2], srel uint8 [N, K/16], s_channel fp32 [N])."""
+    w = _c(w_rot, np.float32)
+    n, k = w.shape
+    cb = _c(codebook, np.float32)
+    q = np.empty((n, k // 2), dtype=np.uint8)
+    s = np.empty((n, k // 16), dtype=np.uint8)
+    ch = np.empty(n, dtype=np.float32)
+    if lib().or_quantize_rotated(_p(w), n, k, _p(cb), _p(q), _p(s), _p(ch)) != 0:
+        raise ValueError("K must be a multiple of 16")
+    return q, s, ch
+
+
+def assign_codes(w_rot, srel, s_channel, codebook, rand=None) -> np.ndarray:
+    """New packed codes on stored scales; rand [N, K] fp32 draws for the stochastic choice."""
+    w = _c(w_rot, np.float32)
+    n, k = w.shape
+    s, ch, cb = _c(srel, np.uint8), _c(s_channel, np.float32), _c(codebook, np.float32)
+    r = None if rand is None else _c(rand, np.float32)
+    q = np.empty((n, k // 2), dtype=np.uint8)
+    if lib().or_assign_codes(_p(w), _p(s), _p(ch), _p(cb), _p(r), n, k, _p(q)) != 0:
+        raise ValueError("K must be a multiple of 16")
+    return q
 
 
 def linear(x_bf16, qdata, srel, codebook, s_channel, bias=None, qmax: int = 127,

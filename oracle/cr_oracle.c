@@ -396,3 +396,232 @@ void or_epilogue_swiglu(const int32_t *acc, const float *xs, const float *ws, co
                 ((float *)out)[m * F + f] = (float)y;
         }
 }
+
+/* ========================================================================
+ * Offline quantiser.  [CR] quantize_w4a8_rotated / _quantize_rotated_rows,
+ * _assign_codes, _assign_grid, grid_levels, _ALS_ITERS = 2.
+ * ======================================================================== */
+
+/* fp32 -> fp8 e4m3fn byte, as torch's .to(torch.float8_e4m3fn) does (the
+ * quantiser's s_rel cast): the value rounded to the nearest e4m3 number,
+ * ties to even, where the pattern S.1111.111 (which would be 480) is NaN, so
+ * a magnitude that rounds above 448 becomes NaN; no saturation.  Subnormals
+ * (steps of 2^-9 below 2^-6) are kept; NaN and infinities give NaN. */
+uint8_t or_f32_to_fp8_e4m3fn(float f)
+{
+    const uint8_t sign = signbit(f) ? 0x80 : 0x00;
+    if (isnan(f) || isinf(f))
+        return (uint8_t)(sign | 0x7F);
+    double a = fabs((double)f);
+    /* the grid step at a's binade: 2^(e-3) for normals, 2^-9 below 2^-6 */
+    int e;
+    frexp(a, &e); /* a = m * 2^e, m in [0.5, 1): the binade is [2^(e-1), 2^e) */
+    int exp2 = e - 1;
+    if (exp2 < -6)
+        exp2 = -6;
+    const double step = ldexp(1.0, exp2 - 3);
+    double units = a / step; /* exact: a power-of-two division */
+    double r = nearbyint(units); /* the default rounding mode: to nearest, ties to even */
+    const double v = r * step;
+    if (v >= 480.0)
+        return (uint8_t)(sign | 0x7F);
+    /* encode v (a multiple of step) */
+    uint8_t code;
+    if (v < ldexp(1.0, -6)) {
+        code = (uint8_t)(v / ldexp(1.0, -9)); /* 0..8; 8 is 2^-6, the smallest normal */
+    } else {
+        int ev;
+        const double m = frexp(v, &ev); /* v = m 2^ev, m in [0.5, 1) */
+        const int ebias = ev - 1 + 7;
+        const int mant = (int)((m * 2.0 - 1.0) * 8.0);
+        code = (uint8_t)((ebias << 3) | mant);
+    }
+    return (uint8_t)(sign | code);
+}
+
+/* Count of the n non-decreasing levels strictly below x, i.e.
+ * torch.searchsorted(levels, x) (left side) on a sorted row. */
+static int or_searchsorted_left(const float *levels, int n, float x)
+{
+    int pos = 0;
+    while (pos < n && levels[pos] < x)
+        ++pos;
+    return pos;
+}
+
+/* [CR] _assign_codes / deterministic _assign_grid: the bracketing pair of the
+ * search position, each distance |x - level| in fp32, the upper level only
+ * when strictly nearer (ties go to the lower index). */
+int or_nearest_level(const float *levels, int n, float x)
+{
+    const int last = n - 1;
+    const int pos = or_searchsorted_left(levels, n, x);
+    const int lo = pos - 1 < 0 ? 0 : (pos - 1 > last ? last : pos - 1);
+    const int hi = pos > last ? last : pos;
+    const float dlo = fabsf(x - levels[lo]);
+    const float dhi = fabsf(x - levels[hi]);
+    return dhi < dlo ? hi : lo;
+}
+
+/* [CR] stochastic _assign_grid: lo = clamp(pos - 1, 0, n - 2), the threshold
+ * u * (levels[lo + 1] - levels[lo]) + levels[lo] (a multiply, then an add,
+ * each rounded to fp32), and the upper level when x is strictly above it.
+ * u is the uniform [0, 1) draw for this weight (an input). */
+int or_stochastic_level(const float *levels, int n, float x, float u)
+{
+    const int last = n - 1;
+    const int pos = or_searchsorted_left(levels, n, x);
+    int lo = pos - 1;
+    if (lo < 0)
+        lo = 0;
+    if (lo > last - 1)
+        lo = last - 1;
+    const float level_lo = levels[lo];
+    const float width = levels[lo + 1] - level_lo;
+    const float uw = u * width;
+    const float thr = uw + level_lo;
+    int code = lo + (x > thr ? 1 : 0);
+    return code > last ? last : code;
+}
+
+/* [CR] grid_levels: the int8 value each of the 16 codebook levels decodes to
+ * for one fp8 group scale, round(codebook[i] * s_rel) (one fp32 multiply,
+ * round half to even) clamped to [-127, 127]. */
+void or_grid_levels(const float *codebook, uint8_t srel_byte, float *levels /* [16] */)
+{
+    const float s = or_fp8_e4m3fn_to_f32(srel_byte);
+    for (int i = 0; i < 16; ++i) {
+        float v = nearbyintf(codebook[i] * s);
+        if (v < -127.0f)
+            v = -127.0f;
+        if (v > 127.0f)
+            v = 127.0f;
+        levels[i] = v;
+    }
+}
+
+/* Sum of 16 fp32 values in a fixed pairwise order: ((v0+v1)+(v2+v3)) + ...,
+ * then pairs of those, down to one.  The pages sum a group's 16 products with
+ * torch's .sum(-1), whose order they do not fix; this order is the reading
+ * taken (the GPU follows it exactly). */
+static float or_sum16_pairwise(const float *v)
+{
+    float a[8], b[4], c[2];
+    for (int i = 0; i < 8; ++i)
+        a[i] = v[2 * i] + v[2 * i + 1];
+    for (int i = 0; i < 4; ++i)
+        b[i] = a[2 * i] + a[2 * i + 1];
+    for (int i = 0; i < 2; ++i)
+        c[i] = b[2 * i] + b[2 * i + 1];
+    return c[0] + c[1];
+}
+
+static float or_clamp_min(float v, float lo)
+{
+    return v < lo ? lo : v; /* torch clamp(min=lo): NaN stays NaN */
+}
+
+/* Per group of 16 rotated weights gw: the group scale after the ALS passes
+ * ([CR] _quantize_rotated_rows): gs = clamp(max|gw|, 1e-8); codes = nearest
+ * codebook index of gw / gs; then _ALS_ITERS = 2 times: lv = codebook[codes],
+ * gs = clamp(sum(gw * lv) / clamp(sum(lv * lv), 1e-8), 1e-8), codes = nearest
+ * index of gw / gs.  Writes the final codes of this stage to q. */
+float or_group_scale_als(const float *gw, const float *codebook, int *q /* [16] */)
+{
+    const float eps = 1e-8f;
+    float amax = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        const float a = fabsf(gw[i]);
+        if (a > amax)
+            amax = a;
+    }
+    float gs = or_clamp_min(amax, eps);
+    for (int i = 0; i < 16; ++i)
+        q[i] = or_nearest_level(codebook, 16, gw[i] / gs);
+    for (int it = 0; it < 2; ++it) {
+        float p[16], l2[16];
+        for (int i = 0; i < 16; ++i) {
+            const float lv = codebook[q[i]];
+            p[i] = gw[i] * lv;
+            l2[i] = lv * lv;
+        }
+        const float num = or_sum16_pairwise(p);
+        const float den = or_clamp_min(or_sum16_pairwise(l2), eps);
+        gs = or_clamp_min(num / den, eps);
+        for (int i = 0; i < 16; ++i)
+            q[i] = or_nearest_level(codebook, 16, gw[i] / gs);
+    }
+    return gs;
+}
+
+/* [CR] quantize_w4a8_rotated (row chunking does not change the result: rows
+ * are independent).  w_rot [N, K] fp32 (already rotated), K a multiple of 16.
+ * Per row: the group scales gs and codes of or_group_scale_als; s_channel =
+ * clamp(max |codebook[code] * gs| / 127, 1e-8); s_rel = fp8(gs / s_channel);
+ * final codes = nearest level of w_rot / s_channel on grid_levels(s_rel);
+ * packed with column 2j in the low nibble of byte j.
+ * Outputs: qdata [N, K/2], srel [N, K/16] fp8 bytes, s_channel [N]. */
+int or_quantize_rotated(const float *w_rot, int64_t N, int64_t K, const float *codebook, uint8_t *qdata,
+                        uint8_t *srel, float *s_channel)
+{
+    if (K % 16 != 0 || N < 0 || K < 0)
+        return -1;
+    const int64_t G = K / 16;
+    float *gs = (float *)malloc((size_t)(G > 0 ? G : 1) * sizeof(float));
+    if (!gs)
+        return -1;
+    for (int64_t n = 0; n < N; ++n) {
+        const float *row = w_rot + n * K;
+        float rowmax = 0.0f;
+        for (int64_t g = 0; g < G; ++g) {
+            int q[16];
+            gs[g] = or_group_scale_als(row + 16 * g, codebook, q);
+            for (int i = 0; i < 16; ++i) {
+                const float a = fabsf(codebook[q[i]] * gs[g]);
+                if (a > rowmax)
+                    rowmax = a;
+            }
+        }
+        const float sch = or_clamp_min(rowmax / 127.0f, 1e-8f);
+        s_channel[n] = sch;
+        for (int64_t g = 0; g < G; ++g) {
+            const uint8_t b = or_f32_to_fp8_e4m3fn(gs[g] / sch);
+            srel[n * G + g] = b;
+            float levels[16];
+            or_grid_levels(codebook, b, levels);
+            for (int i = 0; i < 16; i += 2) {
+                const int c0 = or_nearest_level(levels, 16, row[16 * g + i] / sch);
+                const int c1 = or_nearest_level(levels, 16, row[16 * g + i + 1] / sch);
+                qdata[n * (K / 2) + 8 * g + i / 2] = (uint8_t)(c0 | (c1 << 4));
+            }
+        }
+    }
+    free(gs);
+    return 0;
+}
+
+/* [CR] requantize_codes_ without its rotation: new codes for rotated weights
+ * on STORED scales.  target = w_rot / s_channel; levels = grid_levels(s_rel);
+ * deterministic nearest level, or (rand != NULL) the stochastic choice with
+ * rand[n, k] as the uniform draw of weight (n, k).  Output packed qdata. */
+int or_assign_codes(const float *w_rot, const uint8_t *srel, const float *s_channel, const float *codebook,
+                    const float *rand, int64_t N, int64_t K, uint8_t *qdata)
+{
+    if (K % 16 != 0 || N < 0 || K < 0)
+        return -1;
+    const int64_t G = K / 16;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < G; ++g) {
+            float levels[16];
+            or_grid_levels(codebook, srel[n * G + g], levels);
+            int c[16];
+            for (int i = 0; i < 16; ++i) {
+                const int64_t k = 16 * g + i;
+                const float t = w_rot[n * K + k] / s_channel[n];
+                c[i] = rand ? or_stochastic_level(levels, 16, t, rand[n * K + k]) : or_nearest_level(levels, 16, t);
+            }
+            for (int i = 0; i < 16; i += 2)
+                qdata[n * (K / 2) + 8 * g + i / 2] = (uint8_t)(c[i] | (c[i + 1] << 4));
+        }
+    return 0;
+}

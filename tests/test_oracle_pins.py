@@ -449,3 +449,164 @@ def test_swiglu_pairs_gate_with_up():
     # and silu is not applied to the up half
     wrong = u / (1.0 + np.exp(-u)) * g
     assert np.abs(y - wrong).max() > 1e-3 * np.abs(ref).max()
+
+
+# ---------------------------------------------------------------- offline quantiser
+
+def _fp8_candidates():
+    """fp32 values around every positive e4m3 number: the values, the midpoints
+    to the next one, one fp32 ulp either side of each, and the range ends."""
+    vals = sorted({float(oracle.fp8_e4m3fn_to_f32(b)) for b in range(0x00, 0x7F)})
+    out = []
+    for a, b in zip(vals, vals[1:] + [480.0]):
+        mid = np.float32((a + b) / 2)
+        for v in (np.float32(a), mid):
+            out += [v, np.nextafter(v, np.float32(np.inf)), np.nextafter(v, np.float32(-np.inf))]
+    out += [np.float32(v) for v in (448.0, 463.99, 464.0, 464.01, 479.0, 480.0, 500.0, 1e6, 3e38, 1e-12, 0.0)]
+    out = np.array(out, dtype=np.float32)
+    return np.concatenate([out, -out])
+
+
+def test_fp8_cast_matches_torch():
+    """The quantiser's s_rel cast, pinned to torch's float8_e4m3fn conversion
+    (the library routine the page calls) on every e4m3 value, every midpoint
+    and their fp32 neighbours, subnormals, overflow and infinities."""
+    v = _fp8_candidates()
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.f32_to_fp8(x) for x in v], dtype=np.uint8)
+    nan = (ref & 0x7F) == 0x7F
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.all((got[nan] & 0x7F) == 0x7F)
+    for special in (np.inf, -np.inf, np.nan):
+        assert oracle.f32_to_fp8(special) & 0x7F == 0x7F
+
+
+def test_grid_levels_rounding_and_clamp():
+    """grid_levels: one fp32 product, round half to even, clamp to +-127 (not -128)."""
+    cb = np.array([-3.5, -2.5, -1.5, -0.5, 0.5, 1.5, 2.5, 3.5] * 2, dtype=np.float32)
+    one = 0x38  # fp8 1.0
+    assert oracle.grid_levels(cb, one)[:8].tolist() == [-4, -2, -2, -0, 0, 2, 2, 4]
+    big = oracle.grid_levels(inputs.codebook(), 0x7E)  # 448: every level saturates or is large
+    assert big.min() == -127 and big.max() == 127
+    # against torch's round on every finite scale byte
+    cbf = torch.from_numpy(inputs.codebook())
+    for b in range(256):
+        if (b & 0x7F) == 0x7F:
+            continue
+        s = torch.tensor([b], dtype=torch.uint8).view(torch.float8_e4m3fn).float()
+        ref = torch.round(cbf * s).clamp(-127, 127).numpy()
+        assert np.array_equal(oracle.grid_levels(inputs.codebook(), b), ref), hex(b)
+
+
+def _nearest_by_scan(levels, x):
+    """The page's rule restated by a scan: the level value nearest to x in fp32
+    distance, the one below x on a tie; its last index if it lies below x,
+    else its first index."""
+    lv = [np.float32(v) for v in levels]
+    x = np.float32(x)
+    best = None
+    for v in lv:
+        d = np.float32(abs(np.float32(x - v)))
+        key = (d, 0 if v < x else 1)
+        if best is None or key < best[0]:
+            best = (key, v)
+    v = best[1]
+    idx = [i for i, w in enumerate(lv) if w == v]
+    return idx[-1] if v < x else idx[0]
+
+
+def test_nearest_level_by_scan():
+    """Search + neighbour compare equals the scan on the codebook and on int8
+    grids with repeated levels, at the levels themselves, at exact midpoints
+    and at random points (ties go to the lower level)."""
+    rng = np.random.default_rng(11)
+    cb = inputs.codebook()
+    pts = list(cb) + [np.float32((a + b) / 2) for a, b in zip(cb, cb[1:])] + list(rng.uniform(-1.2, 1.2, 300))
+    for x in pts:
+        assert oracle.nearest_level(cb, x) == _nearest_by_scan(cb, x)
+    for b in (0x08, 0x20, 0x30, 0x40, 0x58, 0x6C, 0x70):
+        lv = oracle.grid_levels(cb, b)
+        xs = list(lv) + [np.float32(v + 0.5) for v in lv] + list(rng.uniform(lv.min() - 3, lv.max() + 3, 200))
+        for x in xs:
+            assert oracle.nearest_level(lv, x) == _nearest_by_scan(lv, x), (hex(b), x)
+
+
+def test_stochastic_level_properties():
+    """u = 0 takes the upper level for any x strictly inside a bracket, u just
+    below 1 the lower; outside the grid the end levels; and the choice is
+    unbiased: over u = (j + 0.5) / 4096 the mean level equals x."""
+    lv = oracle.grid_levels(inputs.codebook(), 0x6C)   # 96: levels about -94 .. 94
+    for x in (-50.3, -1.2, 0.7, 33.3, 80.9):
+        j = int(np.searchsorted(lv, np.float32(x))) - 1
+        assert oracle.stochastic_level(lv, x, 0.0) == j + 1
+        assert oracle.stochastic_level(lv, x, np.float32(0.99999994)) == j
+        us = (np.arange(4096) + 0.5) / 4096
+        mean = np.mean([lv[oracle.stochastic_level(lv, x, u)] for u in us])
+        assert abs(mean - x) <= (lv[j + 1] - lv[j]) / 2048
+    assert oracle.stochastic_level(lv, lv[0] - 5, 0.3) == 0
+    assert oracle.stochastic_level(lv, lv[-1] + 5, 0.3) == 15
+
+
+def test_group_scale_closed_form():
+    """A group that is exactly c * codebook[q] (its largest magnitude present)
+    keeps the codes q through both ALS passes, and the ALS scale is c."""
+    cb = inputs.codebook()
+    rng = np.random.default_rng(12)
+    for c in (0.01, 0.37, 3.0):
+        q = rng.integers(0, 16, size=16)
+        q[3] = 15
+        gw = (np.float32(c) * cb[q]).astype(np.float32)
+        gs, codes = oracle.group_scale_als(gw, cb)
+        assert codes.tolist() == q.tolist()
+        assert abs(gs - c) <= 4e-7 * c
+
+
+def test_quantize_hand_example():
+    """One row of 16 weights w = 0.01 * codebook, worked by hand: the codes are
+    0..15 in order (packed low nibble first: 0x10, 0x32, ..., 0xFE), the ALS
+    scale is 0.01, s_channel = 0.980671 * 0.01 / 127 and s_rel = 127 / 0.980671
+    = 129.5, which rounds to the e4m3 value 128 (byte 0x70)."""
+    cb = inputs.codebook()
+    w = (np.float32(0.01) * cb).reshape(1, 16).astype(np.float32)
+    q, s, ch = oracle.quantize_rotated(w, cb)
+    assert q[0].tolist() == [0x10, 0x32, 0x54, 0x76, 0x98, 0xBA, 0xDC, 0xFE]
+    assert s[0].tolist() == [0x70]
+    assert abs(ch[0] - 0.980671 * 0.01 / 127) <= 1e-6 * ch[0]
+
+
+def test_quantize_properties():
+    """On the synthetic rotated weights: scaling w by a power of two leaves the
+    codes and s_rel unchanged and scales s_channel exactly; the largest grid
+    level of each row is within fp8 rounding of 127; the stored layer decodes
+    (through the forward's decode) to w within the 4-bit codebook's error; and
+    re-assigning codes on the stored scales reproduces the stored codes."""
+    cb = inputs.codebook()
+    w = inputs.rotated_weights(24, 512, 5)
+    q, s, ch = oracle.quantize_rotated(w, cb)
+    for e in (-3, 5):
+        q2, s2, ch2 = oracle.quantize_rotated((w * np.float32(2.0 ** e)).astype(np.float32), cb)
+        assert np.array_equal(q2, q) and np.array_equal(s2, s)
+        assert np.array_equal(ch2, (ch * np.float32(2.0 ** e)).astype(np.float32))
+    w8 = oracle.decode_w8(q, s, cb).astype(np.float64)
+    top = np.abs(w8).max(axis=1)
+    assert np.all(top >= 110) and np.all(top <= 128)
+    deq = w8 * ch[:, None]
+    rel = np.sqrt(((deq - w) ** 2).sum(axis=1) / (w.astype(np.float64) ** 2).sum(axis=1))
+    assert np.all(rel < 0.15), rel.max()
+    assert np.array_equal(oracle.assign_codes(w, s, ch, cb), q)
+
+
+def test_stochastic_assignment_is_unbiased():
+    """Averaged over many draws, the stochastically assigned layer decodes to
+    the weight itself (deterministic assignment does not)."""
+    cb = inputs.codebook()
+    w = inputs.rotated_weights(4, 256, 6)
+    q, s, ch = oracle.quantize_rotated(w, cb)
+    acc = np.zeros(w.shape)
+    draws = 200
+    for d in range(draws):
+        qs = oracle.assign_codes(w, s, ch, cb, inputs.uniforms(4, 256, 100 + d))
+        acc += oracle.decode_w8(qs, s, cb) * ch[:, None].astype(np.float64)
+    mean = acc / draws
+    det = oracle.decode_w8(q, s, cb) * ch[:, None].astype(np.float64)
+    assert np.abs(mean - w).mean() < 0.25 * np.abs(det - w).mean()

@@ -20,6 +20,12 @@ or trained checkpoint is involved):
   the fp8 byte.
 * per-channel scales s_channel [N]: fp32 U[1e-4, 5e-4].
 * codebook[16]: the page's FIXED_CODEBOOK rounded to fp32.
+* rotated fp weights w_rot [N, K] fp32 (input of the offline quantiser):
+  the page motivates the codebook by ConvRot making rotated groups
+  Gaussian, so w = sigma_n * a_g * z with z ~ N(0, 1), a row scale sigma_n
+  log-uniform on [0.005, 0.05] and a per-16-group factor a_g = exp(N(0,
+  0.25^2)) so that group scales differ; drawn in fp64, rounded to fp32.
+* uniform draws u [N, K] fp32 in [0, 1) for the stochastic code assignment.
 
 Every tensor has its own counter-derived stream (seed, tag), so the weights
 of a layer do not depend on M and vice versa.
@@ -41,6 +47,7 @@ FIXED_CODEBOOK = (
 )
 
 _TAG_X, _TAG_OUTLIER, _TAG_Q, _TAG_S, _TAG_C, _TAG_BIAS = 1, 2, 3, 4, 5, 6
+_TAG_W, _TAG_WROW, _TAG_WGROUP, _TAG_U = 7, 8, 9, 10
 
 
 def _rng(seed: int, tag: int, extra: int = 0) -> np.random.Generator:
@@ -91,6 +98,21 @@ def layer(N: int, K: int, seed: int, with_bias: bool = False) -> Layer:
     if with_bias:
         b = _rng(seed, _TAG_BIAS).normal(0.0, 0.1, size=(N,)).astype(np.float32)
     return Layer(q, s, c, codebook(), b)
+
+
+def rotated_weights(N: int, K: int, seed: int) -> np.ndarray:
+    """fp32 [N, K] rotated weights for the offline quantiser (see the recipe)."""
+    if K % 16:
+        raise ValueError("K must be a multiple of 16")
+    sigma = np.exp(_rng(seed, _TAG_WROW).uniform(math.log(0.005), math.log(0.05), size=(N, 1, 1)))
+    a = np.exp(_rng(seed, _TAG_WGROUP).normal(0.0, 0.25, size=(N, K // 16, 1)))
+    z = _rng(seed, _TAG_W).standard_normal(size=(N, K // 16, 16))
+    return (sigma * a * z).reshape(N, K).astype(np.float32)
+
+
+def uniforms(N: int, K: int, seed: int) -> np.ndarray:
+    """fp32 [N, K] uniform draws in [0, 1)."""
+    return _rng(seed, _TAG_U).random(size=(N, K), dtype=np.float32)
 
 
 def outlier_channels(K: int, seed: int) -> np.ndarray:
