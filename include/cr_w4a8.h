@@ -328,6 +328,54 @@ cr_status cr_w4a8_linear_swiglu(const uint16_t *x, const uint8_t *qdata, const u
 cr_status cr_interleave_rows(const void *src, void *dst, int64_t rows, int64_t row_bytes, cr_stream_t stream);
 
 /*
+ * (11) Offline quantiser: rotated fp32 weights -> the layer's storage.
+ *
+ * Defined by: ai-toolkit convrot_w4a8_quant.py, quantize_w4a8_rotated and
+ * _quantize_rotated_rows, with _assign_codes, grid_levels and _assign_grid
+ * (deterministic) and _ALS_ITERS = 2.  Per row n and group g of 16 columns,
+ * with "nearest" the pages' rule (search the sorted table, compare the fp32
+ * distances to the two neighbours, the upper one only when strictly nearer):
+ *   gs     = clamp(max |w|, 1e-8); codes = nearest codebook index of w / gs
+ *   twice: lv = codebook[codes];
+ *          gs = clamp(sum(w * lv) / clamp(sum(lv * lv), 1e-8), 1e-8);
+ *          codes = nearest codebook index of w / gs
+ *   s_channel[n] = clamp(max over the row of |codebook[code] * gs| / 127, 1e-8)
+ *   srel[n, g]   = fp8_e4m3fn(gs / s_channel[n])  (nearest, ties to even;
+ *                  a magnitude rounding above 448 gives NaN, as torch's cast)
+ *   final code   = nearest level of w / s_channel[n] among
+ *                  clamp(rint(codebook[i] * fp8(srel[n, g])), -127, 127)
+ * Every operation is one IEEE fp32 operation; each sum of 16 products is
+ * taken pairwise, ((p0 + p1) + (p2 + p3)) + ... (the pages leave that order
+ * open).
+ *
+ * w_rot [N, K] fp32 (the weight already rotated block-wise), codebook [16]
+ * sorted ascending; qdata [N, K/2], srel [N, K/16] (fp8 bytes) and
+ * s_channel [N] are written.  K must be a positive multiple of 16, at most
+ * CR_MAX_K (CR_ERR_UNSUPPORTED otherwise); N == 0 does nothing.  The weights
+ * must be finite.
+ */
+cr_status cr_w4a8_quantize_rotated(const float *w_rot, const float *codebook, int64_t N, int64_t K,
+                                   uint8_t *qdata, uint8_t *srel, float *s_channel, cr_stream_t stream);
+
+/*
+ * (12) New codes on stored scales.
+ *
+ * Defined by: ai-toolkit convrot_w4a8_quant.py, requantize_codes_ (after its
+ * rotation) and _assign_grid.  target = w_rot[n, k] / s_channel[n] on the
+ * levels clamp(rint(codebook[i] * fp8(srel[n, k / 16])), -127, 127):
+ *   rand == NULL: the nearest level, as in (11);
+ *   otherwise the stochastic choice: with lo the lower level of the bracket
+ *     around target (lo = clamp(pos - 1, 0, 14)), the upper level when
+ *     target > rand[n, k] * (level[lo + 1] - level[lo]) + level[lo]
+ *     (a multiply, then an add), so that the expected level is the target.
+ * rand [N, K] fp32 uniform draws in [0, 1) are an input (the caller owns the
+ * random numbers).  qdata [N, K/2] is written; shapes and K as in (11).
+ */
+cr_status cr_w4a8_assign_codes(const float *w_rot, const uint8_t *srel, const float *s_channel,
+                               const float *codebook, const float *rand, int64_t N, int64_t K,
+                               uint8_t *qdata, cr_stream_t stream);
+
+/*
  * Waits for `stream`, then reads and clears the library's device error word,
  * which a kernel sets when one of its bounded pipeline waits runs out (the
  * kernel then abandons its tile and exits; its outputs are unspecified).

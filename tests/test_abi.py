@@ -30,7 +30,7 @@ def test_header_declares_the_boundary():
     for n in ("cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv", "cr_epilogue",
               "cr_w4a8_linear", "cr_status_string", "cr_check_device_error", "cr_version",
               "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped", "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu",
-              "cr_w4a8_linear_swiglu", "cr_interleave_rows"):
+              "cr_w4a8_linear_swiglu", "cr_interleave_rows", "cr_w4a8_quantize_rotated", "cr_w4a8_assign_codes"):
         assert n in names
 
 
@@ -192,6 +192,21 @@ def test_interleave_rows_validation(L):
     assert f(A16, A16 + 16, 2, 16, None) == cr.CR_ERR_INVALID_ARG     # overlapping buffers
     assert f(None, None, 0, 16, None) == cr.CR_OK and f(None, None, 2, 0, None) == cr.CR_OK
     assert f(A16, 0x20000, 2 ** 40, 2 ** 40, None) == cr.CR_ERR_INVALID_ARG  # size overflows
+
+
+def test_quantiser_validation(L):
+    f, g = L.cr_w4a8_quantize_rotated, L.cr_w4a8_assign_codes
+    assert f(A16, A16, -1, 16, A16, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, A16, 4, 24, A16, A16, A16, None) == cr.CR_ERR_UNSUPPORTED      # K % 16
+    assert f(A16, A16, 4, 0, A16, A16, A16, None) == cr.CR_ERR_UNSUPPORTED
+    assert f(A16, A16, 4, 131072 + 16, A16, A16, A16, None) == cr.CR_ERR_UNSUPPORTED
+    assert f(None, A16, 4, 16, A16, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, A16, 4, 16, A16, MIS, A16, None) == cr.CR_ERR_ALIGNMENT
+    assert f(None, None, 0, 16, None, None, None, None) == cr.CR_OK
+    assert g(A16, A16, A16, A16, None, 4, 24, A16, None) == cr.CR_ERR_UNSUPPORTED
+    assert g(A16, A16, A16, A16, MIS, 4, 16, A16, None) == cr.CR_ERR_ALIGNMENT   # rand
+    assert g(A16, None, A16, A16, None, 4, 16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert g(None, None, None, None, None, 0, 16, None, None) == cr.CR_OK
 
 
 def test_valid_call_without_a_gpu_fails_loudly(L):

@@ -407,3 +407,88 @@ def test_linear_swiglu_from_separate_gate_and_up(M):
                                il(g.s_channel, u.s_channel), il(g.bias, u.bias), threads=THREADS)
     assert y.shape == (M, F)
     assert_swiglu_close(host(y), ref["y"], "bf16")
+
+
+# ---------------------------------------------------------------- offline quantiser
+
+def _edge_rows(K):
+    """Rows that reach the quantiser's corner cases: an all-zero row (every
+    clamp at 1e-8), zero and tiny groups next to normal ones (fp8 zero and
+    subnormal s_rel), exact codebook multiples, one-hot groups, a negative
+    row and a row of equal values."""
+    cb = inputs.codebook()
+    rng = np.random.default_rng(21)
+    rows = [np.zeros(K)]
+    r = rng.standard_normal(K) * 0.02
+    r[:16] = 0.0
+    r[16:32] *= 1e-4
+    r[32:48] *= 1e-7
+    rows.append(r)
+    rows.append(np.tile(cb, K // 16) * 0.03)
+    oh = np.zeros(K)
+    oh[::16] = 0.5
+    oh[5::16] = -0.01
+    rows.append(oh)
+    rows.append(-np.abs(rng.standard_normal(K)))
+    rows.append(np.full(K, 0.125))
+    return np.array(rows, dtype=np.float32)
+
+
+@pytest.mark.parametrize("N,K", [(1, 16), (3, 48), (37, 512), (300, 4096), (64, 16384), (6, 1024)])
+def test_quantize_rotated_bit_exact(N, K):
+    w = inputs.rotated_weights(N, K, N + K) if (N, K) != (6, 1024) else _edge_rows(K)
+    cb = inputs.codebook()
+    q_r, s_r, ch_r = oracle.quantize_rotated(w, cb)
+    q, s, ch, _ = cr.cr_w4a8_quantize_rotated(dev(w), dev(cb))
+    torch.cuda.synchronize()
+    assert np.array_equal(host(s), s_r)
+    assert np.array_equal(host(ch).view(np.uint32), ch_r.view(np.uint32))
+    assert np.array_equal(host(q), q_r)
+
+
+def test_quantize_rotated_sampled_rows_full_size():
+    """16384 x 16384 on the GPU; rows are independent, so a sample of rows is
+    checked against the oracle run on those rows alone."""
+    N = K = 16384
+    cb = inputs.codebook()
+    w = torch.empty(N, K, dtype=torch.float32, device="cuda")
+    chunk = 2048
+    for r0 in range(0, N, chunk):
+        w[r0:r0 + chunk] = dev(inputs.rotated_weights(chunk, K, 1000 + r0))
+    q, s, ch, _ = cr.cr_w4a8_quantize_rotated(w, dev(cb))
+    torch.cuda.synchronize()
+    for r in (0, 1, 2047, 2048, 9000, N - 1):
+        wr = host(w[r:r + 1])
+        q_r, s_r, ch_r = oracle.quantize_rotated(wr, cb)
+        assert np.array_equal(host(q[r:r + 1]), q_r) and np.array_equal(host(s[r:r + 1]), s_r)
+        assert np.array_equal(host(ch[r:r + 1]).view(np.uint32), ch_r.view(np.uint32))
+
+
+@pytest.mark.parametrize("stochastic", [False, True])
+def test_assign_codes_bit_exact(stochastic):
+    """Codes for updated weights on the stored scales (requantize_codes_),
+    deterministic and with uniform draws passed in."""
+    N, K = 200, 2048
+    cb = inputs.codebook()
+    w = inputs.rotated_weights(N, K, 31)
+    _, s, ch = oracle.quantize_rotated(w, cb)
+    w2 = (w + 0.1 * inputs.rotated_weights(N, K, 32)).astype(np.float32)
+    u = inputs.uniforms(N, K, 33) if stochastic else None
+    q_r = oracle.assign_codes(w2, s, ch, cb, u)
+    q = cr.cr_w4a8_assign_codes(dev(w2), dev(s), dev(ch), dev(cb), None if u is None else dev(u))
+    torch.cuda.synchronize()
+    assert np.array_equal(host(q), q_r)
+
+
+def test_quantised_layer_runs_through_the_forward():
+    """A layer quantised on the GPU feeds the forward directly, and its output
+    equals the oracle forward of the oracle-quantised layer bit for bit."""
+    N, K, M = 512, 1024, 4
+    cb = inputs.codebook()
+    w = inputs.rotated_weights(N, K, 41)
+    q, s, ch, cbd = cr.cr_w4a8_quantize_rotated(dev(w), dev(cb))
+    x = inputs.activations(M, K, 42)
+    y = cr.cr_w4a8_linear(bf16_dev(x), q, s, cbd, ch)
+    q_r, s_r, ch_r = oracle.quantize_rotated(w, cb)
+    ref = oracle.linear(x, q_r, s_r, cb, ch_r, threads=THREADS)
+    assert_output_close(host(y), ref["y"], "bf16")

@@ -28,7 +28,7 @@ __all__ = [
     "cr_epilogue", "cr_w4a8_linear", "cr_w4a8_linear_decode_noalloc", "cr_check_device_error",
     "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped", "CrLayer",
     "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu", "cr_w4a8_linear_swiglu", "cr_interleave_rows",
-    "interleave_gate_up",
+    "interleave_gate_up", "cr_w4a8_quantize_rotated", "cr_w4a8_assign_codes",
     "cr_status_string", "cr_version",
     "gemv_rows",
 ]
@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
             L.cr_w4a8_gemv_swiglu.argtypes = contraction[:-2] + [P]
             L.cr_w4a8_linear_swiglu.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P, P, P]
             L.cr_interleave_rows.argtypes = [P, P, i64, i64, P]
+            L.cr_w4a8_quantize_rotated.argtypes = [P, P, i64, i64, P, P, P, P]
+            L.cr_w4a8_assign_codes.argtypes = [P, P, P, P, P, i64, i64, P, P]
             LP = ctypes.POINTER(CrLayer)
             L.cr_w4a8_gemv_grouped.argtypes = [P, P, P, i64, i64, LP, i32, i32, P]
             L.cr_w4a8_linear_grouped.argtypes = [P, P, i64, i64, LP, i32, i32, i32, P, P, P]
@@ -554,6 +556,54 @@ def interleave_gate_up(gate, up, stream=None):
             raise ValueError(f"gate and up differ in field {i}")
         res.append(cr_interleave_rows(torch.cat([g, u], dim=0).contiguous(), stream=stream))
     return tuple(res) + ((None,) if len(res) == 3 else ())
+
+
+def _fixed_codebook(device):
+    from .inputs import FIXED_CODEBOOK
+    return _torch().tensor(FIXED_CODEBOOK, dtype=_torch().float32, device=device)
+
+
+def cr_w4a8_quantize_rotated(w_rot, codebook=None, qdata=None, srel=None, s_channel=None, stream=None):
+    """Offline quantiser: rotated fp32 weights [N, K] (K a multiple of 16) ->
+    (qdata uint8 [N, K/2], srel uint8 [N, K/16] fp8 bytes, s_channel fp32 [N],
+    codebook fp32 [16]).  codebook=None uses the pages' fixed codebook."""
+    torch = _torch()
+    _need(w_rot, "w_rot", (torch.float32,), 2)
+    N, K = w_rot.shape
+    if codebook is None:
+        codebook = _fixed_codebook(w_rot.device)
+    _need(codebook, "codebook", (torch.float32,), shape=(16,))
+    if qdata is None:
+        qdata = torch.empty(N, K // 2, dtype=torch.uint8, device=w_rot.device)
+    if srel is None:
+        srel = torch.empty(N, K // 16, dtype=torch.uint8, device=w_rot.device)
+    if s_channel is None:
+        s_channel = torch.empty(N, dtype=torch.float32, device=w_rot.device)
+    _need(qdata, "qdata", (torch.uint8, torch.int8), shape=(N, K // 2))
+    _need(srel, "srel", (torch.uint8, torch.float8_e4m3fn), shape=(N, K // 16))
+    _need(s_channel, "s_channel", (torch.float32,), shape=(N,))
+    _check(lib().cr_w4a8_quantize_rotated(_ptr(w_rot), _ptr(codebook), N, K, _ptr(qdata), _ptr(srel),
+                                          _ptr(s_channel), _stream(stream)), "cr_w4a8_quantize_rotated")
+    return qdata, srel, s_channel, codebook
+
+
+def cr_w4a8_assign_codes(w_rot, srel, s_channel, codebook, rand=None, qdata=None, stream=None):
+    """New packed codes for rotated weights on stored scales: the nearest grid
+    level, or with rand [N, K] fp32 uniform draws the unbiased stochastic one."""
+    torch = _torch()
+    _need(w_rot, "w_rot", (torch.float32,), 2)
+    N, K = w_rot.shape
+    _need(srel, "srel", (torch.uint8, torch.float8_e4m3fn), shape=(N, K // 16))
+    _need(s_channel, "s_channel", (torch.float32,), shape=(N,))
+    _need(codebook, "codebook", (torch.float32,), shape=(16,))
+    if rand is not None:
+        _need(rand, "rand", (torch.float32,), shape=(N, K))
+    if qdata is None:
+        qdata = torch.empty(N, K // 2, dtype=torch.uint8, device=w_rot.device)
+    _need(qdata, "qdata", (torch.uint8, torch.int8), shape=(N, K // 2))
+    _check(lib().cr_w4a8_assign_codes(_ptr(w_rot), _ptr(srel), _ptr(s_channel), _ptr(codebook), _ptr(rand), N, K,
+                                      _ptr(qdata), _stream(stream)), "cr_w4a8_assign_codes")
+    return qdata
 
 
 def cr_check_device_error(stream=None) -> None:

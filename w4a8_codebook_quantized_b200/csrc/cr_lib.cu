@@ -18,6 +18,7 @@
 #include "k_elementwise.cuh"
 #include "k_gemm.cuh"
 #include "k_gemv.cuh"
+#include "k_quant.cuh"
 #include "k_rotquant.cuh"
 
 namespace {
@@ -681,6 +682,55 @@ cr_status cr_w4a8_gemv_swiglu(const int8_t *xq, const float *xs, const uint8_t *
                               int64_t K, cr_out_dtype out_dtype, void *out, cr_stream_t stream)
 {
     return contraction_swiglu(true, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, stream);
+}
+
+namespace {
+// Validation shared by the quantiser entry points: N >= 0, K a positive
+// multiple of 16 up to CR_MAX_K, 16-byte aligned non-null buffers.
+cr_status check_quant(const float *w_rot, const float *codebook, int64_t N, int64_t K, const void *a, const void *b,
+                      const void *c)
+{
+    if (N < 0 || K < 0)
+        return CR_ERR_INVALID_ARG;
+    if (K == 0 || K % 16 != 0 || K > CR_MAX_K)
+        return CR_ERR_UNSUPPORTED;
+    if (N == 0)
+        return CR_OK;
+    if (!w_rot || !codebook || !a || !b || !c)
+        return CR_ERR_INVALID_ARG;
+    if (!aligned16(w_rot) || !aligned16(codebook) || !aligned16(a) || !aligned16(b) || !aligned16(c))
+        return CR_ERR_ALIGNMENT;
+    return CR_OK;
+}
+}  // namespace
+
+cr_status cr_w4a8_quantize_rotated(const float *w_rot, const float *codebook, int64_t N, int64_t K, uint8_t *qdata,
+                                   uint8_t *srel, float *s_channel, cr_stream_t stream)
+{
+    cr_status st = check_quant(w_rot, codebook, N, K, qdata, srel, s_channel);
+    if (st != CR_OK || N == 0)
+        return st;
+    DeviceState *d = nullptr;
+    st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    return launched(cr::qz::launch_quantize(w_rot, codebook, N, (int)K, qdata, srel, s_channel, d->num_sms, stream));
+}
+
+cr_status cr_w4a8_assign_codes(const float *w_rot, const uint8_t *srel, const float *s_channel, const float *codebook,
+                               const float *rand, int64_t N, int64_t K, uint8_t *qdata, cr_stream_t stream)
+{
+    cr_status st = check_quant(w_rot, codebook, N, K, srel, s_channel, qdata);
+    if (st != CR_OK || N == 0)
+        return st;
+    if (rand && !aligned16(rand))
+        return CR_ERR_ALIGNMENT;
+    DeviceState *d = nullptr;
+    st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    return launched(
+        cr::qz::launch_assign(w_rot, srel, s_channel, codebook, rand, N, (int)K, qdata, d->num_sms, stream));
 }
 
 cr_status cr_interleave_rows(const void *src, void *dst, int64_t rows, int64_t row_bytes, cr_stream_t stream)
