@@ -73,6 +73,10 @@ def lib() -> ctypes.CDLL:
             L.or_quantize_rotated.restype = ctypes.c_int
             L.or_assign_codes.argtypes = [P, P, P, P, P, i64, i64, P]
             L.or_assign_codes.restype = ctypes.c_int
+            L.or_dequant_bf16.argtypes = [P, P, P, P, i64, i64, P]
+            L.or_dequant_bf16.restype = None
+            L.or_ste_backward.argtypes = [P, P, P, P, P, i64, i64, i64, P]
+            L.or_ste_backward.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -328,6 +332,31 @@ def assign_codes(w_rot, srel, s_channel, codebook, rand=None) -> np.ndarray:
     if lib().or_assign_codes(_p(w), _p(s), _p(ch), _p(cb), _p(r), n, k, _p(q)) != 0:
         raise ValueError("K must be a multiple of 16")
     return q
+
+
+# ---------------------------------------------------------------- straight-through backward
+
+def dequant_bf16(qdata, srel, codebook, s_channel) -> np.ndarray:
+    """bf16 bits [N, K] of w8 * bf16(s_channel), as the backward builds it."""
+    q = _c(qdata, np.uint8)
+    n, kh = q.shape
+    out = np.empty((n, 2 * kh), dtype=np.uint16)
+    lib().or_dequant_bf16(_p(q), _p(_c(srel, np.uint8)), _p(_c(codebook, np.float32)),
+                          _p(_c(s_channel, np.float32)), n, 2 * kh, _p(out))
+    return out
+
+
+def ste_backward(grad_bf16, qdata, srel, codebook, s_channel) -> np.ndarray:
+    """dx bf16 bits [M, K] = grad [M, N] @ dequant_bf16 [N, K] (double sums, one rounding)."""
+    g = _c(grad_bf16, np.uint16)
+    m, n = g.shape
+    q = _c(qdata, np.uint8)
+    k = 2 * q.shape[1]
+    out = np.empty((m, k), dtype=np.uint16)
+    if lib().or_ste_backward(_p(g), _p(q), _p(_c(srel, np.uint8)), _p(_c(codebook, np.float32)),
+                             _p(_c(s_channel, np.float32)), m, n, k, _p(out)) != 0:
+        raise MemoryError("oracle backward")
+    return out
 
 
 def linear(x_bf16, qdata, srel, codebook, s_channel, bias=None, qmax: int = 127,

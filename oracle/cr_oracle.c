@@ -625,3 +625,60 @@ int or_assign_codes(const float *w_rot, const uint8_t *srel, const float *s_chan
         }
     return 0;
 }
+
+/* ========================================================================
+ * Straight-through backward.  [CR] _w4a8_linear_ste_backward: the codes are
+ * decoded again, w = w8.to(grad.dtype) * s_channel.to(grad.dtype), and the
+ * input gradient is grad @ w.
+ * ======================================================================== */
+
+/* The dequantised weight in bf16, as the backward builds it for bf16
+ * gradients: w8 (exact in bf16) times bf16(s_channel[n]), the product of two
+ * bf16 values (exact in fp32) rounded once to bf16.  w [N, K] bf16 bits. */
+void or_dequant_bf16(const uint8_t *qdata, const uint8_t *srel, const float *codebook, const float *s_channel,
+                     int64_t N, int64_t K, uint16_t *w)
+{
+    int8_t *w8 = (int8_t *)malloc((size_t)(N * K > 0 ? N * K : 1));
+    if (!w8)
+        return;
+    or_decode_w8(qdata, srel, codebook, N, K, w8);
+    for (int64_t n = 0; n < N; ++n) {
+        const float s = or_bf16_to_f32(or_f32_to_bf16_rne(s_channel[n]));
+        for (int64_t k = 0; k < K; ++k)
+            w[n * K + k] = or_f32_to_bf16_rne((float)w8[n * K + k] * s);
+    }
+    free(w8);
+}
+
+/* dx [M, K] bf16 = grad [M, N] bf16 @ w [N, K] bf16 (or_dequant_bf16).  The
+ * pages leave the accumulation to the matmul; here every product and sum is
+ * in double and the result is rounded once to bf16. */
+int or_ste_backward(const uint16_t *grad, const uint8_t *qdata, const uint8_t *srel, const float *codebook,
+                    const float *s_channel, int64_t M, int64_t N, int64_t K, uint16_t *dx)
+{
+    uint16_t *w = (uint16_t *)malloc((size_t)(N * K > 0 ? N * K : 1) * sizeof(uint16_t));
+    double *row = (double *)malloc((size_t)(K > 0 ? K : 1) * sizeof(double));
+    if (!w || !row) {
+        free(w);
+        free(row);
+        return -1;
+    }
+    or_dequant_bf16(qdata, srel, codebook, s_channel, N, K, w);
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t k = 0; k < K; ++k)
+            row[k] = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            const double g = or_bf16_to_f32(grad[m * N + n]);
+            if (g == 0.0)
+                continue;
+            const uint16_t *wr = w + n * K;
+            for (int64_t k = 0; k < K; ++k)
+                row[k] += g * (double)or_bf16_to_f32(wr[k]);
+        }
+        for (int64_t k = 0; k < K; ++k)
+            dx[m * K + k] = or_f64_to_bf16_rne(row[k]);
+    }
+    free(w);
+    free(row);
+    return 0;
+}

@@ -610,3 +610,38 @@ def test_stochastic_assignment_is_unbiased():
     mean = acc / draws
     det = oracle.decode_w8(q, s, cb) * ch[:, None].astype(np.float64)
     assert np.abs(mean - w).mean() < 0.25 * np.abs(det - w).mean()
+
+
+# ---------------------------------------------------------------- straight-through backward
+
+def test_dequant_bf16_matches_torch():
+    """The backward's weight, w8.to(bf16) * s_channel.to(bf16), evaluated with
+    torch's own bf16 ops on the oracle's decoded grid."""
+    layer = inputs.layer(64, 512, 51)
+    w8 = torch.from_numpy(oracle.decode_w8(layer.qdata, layer.srel, layer.codebook))
+    ref = (w8.to(torch.bfloat16) * torch.from_numpy(layer.s_channel).to(torch.bfloat16).unsqueeze(1))
+    got = oracle.dequant_bf16(layer.qdata, layer.srel, layer.codebook, layer.s_channel)
+    assert np.array_equal(got, ref.view(torch.int16).numpy().view(np.uint16))
+
+
+def test_ste_backward_one_hot_and_fp64():
+    """A one-hot gradient row returns that weight row exactly; a random
+    gradient matches a float64 matmul of the same bf16 operands, rounded to
+    bf16, within one ulp (and equal almost everywhere); the operands are not
+    transposed (M, N, K all different)."""
+    M, N, K = 5, 48, 256
+    layer = inputs.layer(N, K, 52)
+    w = oracle.dequant_bf16(layer.qdata, layer.srel, layer.codebook, layer.s_channel)
+    g = np.zeros((M, N), dtype=np.uint16)
+    g[2, 17] = 0x3F80  # 1.0
+    g[4, 40] = 0xC000  # -2.0
+    dx = oracle.ste_backward(g, layer.qdata, layer.srel, layer.codebook, layer.s_channel)
+    assert np.array_equal(dx[2], w[17])
+    assert np.array_equal(dx[4], _bf16(-2.0 * _bf16_to_f64(w[40])))
+    assert not dx[0].any()
+    rng = np.random.default_rng(53)
+    g = _bf16(rng.standard_normal((M, N)))
+    dx = oracle.ste_backward(g, layer.qdata, layer.srel, layer.codebook, layer.s_channel)
+    ref = _bf16(_bf16_to_f64(g) @ _bf16_to_f64(w))
+    diff = np.abs(dx.astype(np.int32) - ref.astype(np.int32))
+    assert diff.max() <= 1 and (diff == 0).mean() > 0.99
