@@ -376,6 +376,33 @@ cr_status cr_w4a8_assign_codes(const float *w_rot, const uint8_t *srel, const fl
                                uint8_t *qdata, cr_stream_t stream);
 
 /*
+ * (13) Straight-through backward: the gradient of the layer's input.
+ *
+ * Defined by: ai-toolkit convrot_w4a8_quant.py, _w4a8_linear_ste_backward
+ * (the training path keeps only the packed codes and decodes them again in
+ * the backward):
+ *   w[n, k]  = bf16( w8[n, k] * bf16(s_channel[n]) )   (w8 as in (2); the
+ *              product is exact in fp32 and rounded once to bf16)
+ *   dx[m, k] = bf16( sum_n grad[m, n] * w[n, k] )       (fp32 accumulation)
+ * dx is the gradient with respect to the layer's (rotated) input, as the
+ * pages' operator returns it; the rotation's own backward is the caller's.
+ *
+ * grad [M, N] bf16 bits, dx [M, K] bf16 bits (written); the layer as in (3).
+ * K as for the forward; N must be a multiple of 8 (CR_ERR_UNSUPPORTED
+ * otherwise).  N == 0 writes dx = 0.  Internally the transposed weight (13a)
+ * is built in a transient of 2 N K bytes and contracted on the tensor cores
+ * (bf16 x bf16 -> fp32).
+ *
+ * (13a) The transposed backward weight alone: wt [K, N] bf16 bits,
+ * wt[k, n] = w[n, k].
+ */
+cr_status cr_w4a8_ste_backward(const uint16_t *grad, const uint8_t *qdata, const uint8_t *srel,
+                               const float *codebook, const float *s_channel, int64_t M, int64_t N, int64_t K,
+                               uint16_t *dx, cr_stream_t stream);
+cr_status cr_w4a8_dequant_t_bf16(const uint8_t *qdata, const uint8_t *srel, const float *codebook,
+                                 const float *s_channel, int64_t N, int64_t K, uint16_t *wt, cr_stream_t stream);
+
+/*
  * Waits for `stream`, then reads and clears the library's device error word,
  * which a kernel sets when one of its bounded pipeline waits runs out (the
  * kernel then abandons its tile and exits; its outputs are unspecified).

@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
     for n in ("cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv", "cr_epilogue",
               "cr_w4a8_linear", "cr_status_string", "cr_check_device_error", "cr_version",
               "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped", "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu",
-              "cr_w4a8_linear_swiglu", "cr_interleave_rows", "cr_w4a8_quantize_rotated", "cr_w4a8_assign_codes"):
+              "cr_w4a8_linear_swiglu", "cr_interleave_rows", "cr_w4a8_quantize_rotated", "cr_w4a8_assign_codes",
+              "cr_w4a8_ste_backward", "cr_w4a8_dequant_t_bf16"):
         assert n in names
 
 
@@ -207,6 +208,19 @@ def test_quantiser_validation(L):
     assert g(A16, A16, A16, A16, MIS, 4, 16, A16, None) == cr.CR_ERR_ALIGNMENT   # rand
     assert g(A16, None, A16, A16, None, 4, 16, A16, None) == cr.CR_ERR_INVALID_ARG
     assert g(None, None, None, None, None, 0, 16, None, None) == cr.CR_OK
+
+
+def test_backward_validation(L):
+    f, g = L.cr_w4a8_ste_backward, L.cr_w4a8_dequant_t_bf16
+    assert f(A16, A16, A16, A16, A16, -1, 8, 256, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, A16, A16, A16, A16, 4, 12, 256, A16, None) == cr.CR_ERR_UNSUPPORTED   # N % 8
+    assert f(A16, A16, A16, A16, A16, 4, 8, 320, A16, None) == cr.CR_ERR_UNSUPPORTED    # K % 256
+    assert f(None, A16, A16, A16, A16, 4, 8, 256, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, A16, A16, A16, A16, 4, 8, 256, MIS, None) == cr.CR_ERR_ALIGNMENT
+    assert f(None, None, None, None, None, 0, 8, 256, None, None) == cr.CR_OK
+    assert g(A16, A16, A16, A16, 12, 256, A16, None) == cr.CR_ERR_UNSUPPORTED
+    assert g(A16, A16, MIS, A16, 8, 256, A16, None) == cr.CR_ERR_ALIGNMENT
+    assert g(None, None, None, None, 0, 256, None, None) == cr.CR_OK
 
 
 def test_valid_call_without_a_gpu_fails_loudly(L):

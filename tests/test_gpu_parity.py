@@ -492,3 +492,58 @@ def test_quantised_layer_runs_through_the_forward():
     q_r, s_r, ch_r = oracle.quantize_rotated(w, cb)
     ref = oracle.linear(x, q_r, s_r, cb, ch_r, threads=THREADS)
     assert_output_close(host(y), ref["y"], "bf16")
+
+
+# ---------------------------------------------------------------- straight-through backward
+
+@pytest.mark.parametrize("N,K", [(8, 256), (520, 1024), (4096, 4096), (200, 2048)])
+def test_dequant_t_bf16_bit_exact(N, K):
+    layer = inputs.layer(N, K, N + K)
+    q, s, cb, ws, _ = _layer_dev(layer)
+    wt = cr.cr_w4a8_dequant_t_bf16(q, s, cb, ws)
+    torch.cuda.synchronize()
+    ref = oracle.dequant_bf16(layer.qdata, layer.srel, layer.codebook, layer.s_channel)
+    assert np.array_equal(host(wt), np.ascontiguousarray(ref.T))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 256), (64, 512, 1024), (300, 1000, 768), (129, 72, 2048),
+                                   (1024, 2048, 1024)])
+def test_ste_backward(M, N, K):
+    """dx against the oracle (double sums, one rounding) and against torch's
+    fp32 matmul of the same bf16 operands, elementwise within the bound the
+    arithmetic gives: half a bf16 ulp for each side's final rounding plus the
+    fp32 accumulation error of a sum of N products, N * 2^-24 * sum|g * w|
+    (the pages leave the accumulation order to the matmul); ragged M, N not a
+    multiple of 64, K tails of the 256-column tiles."""
+    layer = inputs.layer(N, K, 3 * N + K)
+    rng = np.random.default_rng(M + N + K)
+    g = torch.from_numpy(rng.standard_normal((M, N)).astype(np.float32)).to(torch.bfloat16)
+    g_bits = g.view(torch.int16).numpy().view(np.uint16)
+    q, s, cb, ws, _ = _layer_dev(layer)
+    dx = Guarded((M, K), torch.bfloat16)
+    cr.cr_w4a8_ste_backward(g.cuda(), q, s, cb, ws, dx=dx.tensor)
+    torch.cuda.synchronize()
+    assert dx.intact()
+    got = host(dx.tensor)
+    ref = oracle.ste_backward(g_bits, layer.qdata, layer.srel, layer.codebook, layer.s_channel)
+    from gpu_util import bf16_bits_to_f64
+    w = torch.from_numpy(oracle.dequant_bf16(layer.qdata, layer.srel, layer.codebook, layer.s_channel)
+                         .view(np.int16)).view(torch.bfloat16).float()
+    absum = np.abs(g.float().numpy().astype(np.float64)) @ np.abs(w.numpy().astype(np.float64))
+    acc = N * 2.0 ** -24 * absum
+    gf, rf = bf16_bits_to_f64(got), bf16_bits_to_f64(ref)
+    bound = 2.0 ** -8 * (np.abs(gf) + np.abs(rf)) + acc + 1e-30
+    assert np.all(np.abs(gf - rf) <= bound), np.max(np.abs(gf - rf) / bound)
+    t32 = (g.float() @ w).numpy().astype(np.float64)
+    assert np.all(np.abs(gf - t32) <= 2.0 ** -8 * np.abs(gf) + 2 * acc + 1e-30)
+    # and most elements agree with the oracle exactly
+    assert (got == ref).mean() > 0.9
+
+
+def test_ste_backward_empty_layer_gives_zero():
+    layer = inputs.layer(8, 256, 1)
+    q, s, cb, ws, _ = _layer_dev(layer)
+    dx = torch.full((4, 256), 7.0, dtype=torch.bfloat16, device="cuda")
+    cr.cr_w4a8_ste_backward(torch.empty(4, 0, dtype=torch.bfloat16, device="cuda"), q[:0], s[:0], cb, ws[:0], dx=dx)
+    torch.cuda.synchronize()
+    assert not dx.float().abs().sum().item()

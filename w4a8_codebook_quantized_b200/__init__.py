@@ -29,6 +29,7 @@ __all__ = [
     "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped", "CrLayer",
     "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu", "cr_w4a8_linear_swiglu", "cr_interleave_rows",
     "interleave_gate_up", "cr_w4a8_quantize_rotated", "cr_w4a8_assign_codes",
+    "cr_w4a8_ste_backward", "cr_w4a8_dequant_t_bf16",
     "cr_status_string", "cr_version",
     "gemv_rows",
 ]
@@ -91,6 +92,8 @@ def lib() -> ctypes.CDLL:
             L.cr_interleave_rows.argtypes = [P, P, i64, i64, P]
             L.cr_w4a8_quantize_rotated.argtypes = [P, P, i64, i64, P, P, P, P]
             L.cr_w4a8_assign_codes.argtypes = [P, P, P, P, P, i64, i64, P, P]
+            L.cr_w4a8_ste_backward.argtypes = [P, P, P, P, P, i64, i64, i64, P, P]
+            L.cr_w4a8_dequant_t_bf16.argtypes = [P, P, P, P, i64, i64, P, P]
             LP = ctypes.POINTER(CrLayer)
             L.cr_w4a8_gemv_grouped.argtypes = [P, P, P, i64, i64, LP, i32, i32, P]
             L.cr_w4a8_linear_grouped.argtypes = [P, P, i64, i64, LP, i32, i32, i32, P, P, P]
@@ -604,6 +607,35 @@ def cr_w4a8_assign_codes(w_rot, srel, s_channel, codebook, rand=None, qdata=None
     _check(lib().cr_w4a8_assign_codes(_ptr(w_rot), _ptr(srel), _ptr(s_channel), _ptr(codebook), _ptr(rand), N, K,
                                       _ptr(qdata), _stream(stream)), "cr_w4a8_assign_codes")
     return qdata
+
+
+def cr_w4a8_ste_backward(grad, qdata, srel, codebook, s_channel, dx=None, stream=None):
+    """Straight-through input gradient: dx [M, K] bf16 = grad [M, N] bf16 @
+    (w8 * s_channel in bf16), the layer's codes decoded again (N % 8 == 0)."""
+    torch = _torch()
+    N, K = _layer(qdata, srel, codebook, s_channel, None)
+    _need(grad, "grad", (torch.bfloat16,), 2)
+    M = grad.shape[0]
+    if grad.shape[1] != N:
+        raise ValueError(f"grad has {grad.shape[1]} columns, the layer N={N}")
+    if dx is None:
+        dx = torch.empty(M, K, dtype=torch.bfloat16, device=grad.device)
+    _need(dx, "dx", (torch.bfloat16,), shape=(M, K))
+    _check(lib().cr_w4a8_ste_backward(_ptr(grad), _ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), M, N,
+                                      K, _ptr(dx), _stream(stream)), "cr_w4a8_ste_backward")
+    return dx
+
+
+def cr_w4a8_dequant_t_bf16(qdata, srel, codebook, s_channel, wt=None, stream=None):
+    """The backward's weight, transposed: wt [K, N] bf16, wt[k, n] = bf16(w8[n, k] * bf16(s_channel[n]))."""
+    torch = _torch()
+    N, K = _layer(qdata, srel, codebook, s_channel, None)
+    if wt is None:
+        wt = torch.empty(K, N, dtype=torch.bfloat16, device=qdata.device)
+    _need(wt, "wt", (torch.bfloat16,), shape=(K, N))
+    _check(lib().cr_w4a8_dequant_t_bf16(_ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), N, K, _ptr(wt),
+                                        _stream(stream)), "cr_w4a8_dequant_t_bf16")
+    return wt
 
 
 def cr_check_device_error(stream=None) -> None:

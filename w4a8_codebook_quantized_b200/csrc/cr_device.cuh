@@ -384,6 +384,19 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t
         : "memory");
 }
 
+// D[tmem] (+)= A[smem] x B[smem]^T, bf16 x bf16 -> fp32 (kind::f16; A and B
+// of the same type).
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // 32 consecutive 32-bit TMEM columns of this warp's 32 lanes -> 32 registers.
 __device__ __forceinline__ void tmem_ld_32cols(uint32_t taddr, uint32_t (&r)[32])
 {
@@ -506,6 +519,18 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N)
     return (2u << 4)                        // D format: s32
            | (1u << 7)                      // A: signed 8-bit
            | (1u << 10)                     // B: signed 8-bit
+           | ((uint32_t)(N >> 3) << 17)     // N / 8
+           | ((uint32_t)(M >> 4) << 24);    // M / 16
+}
+
+// Instruction descriptor for kind::f16 with bf16 A and B and an fp32
+// accumulator, both operands K-major: D format 1 (f32) in bits 4-5, A and B
+// format 1 (bf16) in bits 7-9 and 10-12, N / 8 in bits 17-22, M / 16 in 24-28.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N)
+{
+    return (1u << 4)                        // D format: f32
+           | (1u << 7)                      // A: bf16
+           | (1u << 10)                     // B: bf16
            | ((uint32_t)(N >> 3) << 17)     // N / 8
            | ((uint32_t)(M >> 4) << 24);    // M / 16
 }

@@ -34,6 +34,7 @@ struct DeviceState {
     bool gemm_pair_attr_set = false;
     bool gemv_attr_set = false;
     bool gemv_grouped_attr_set = false;
+    bool gemm_bf16_attr_set = false;
     // side stream and events on which cr_w4a8_linear's prefill path decodes
     // the weight while the activations are rotated and quantised
     cudaStream_t side = nullptr;
@@ -135,6 +136,21 @@ bool make_tmap_i8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t r
     const cuuint32_t estr[2] = {1u, 1u};
     const CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
                                       box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// 2-D bf16 tensor map for the tcgen05 GEMM: rows of `inner` elements, boxes
+// of 64 elements (128 bytes, 128-byte swizzle) x box_rows rows.
+bool make_tmap_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+                    uint32_t box_rows)
+{
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+                                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -356,7 +372,7 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
 {
     using namespace cr;
     if (!d.gemm_attr_set) {
-        if (cudaFuncSetAttribute(gm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(gm::gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gm::kSmemBytes) != cudaSuccess) {
             cudaGetLastError();
             return CR_ERR_CUDA;
@@ -453,7 +469,7 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
     } else if (st == CR_OK) {
         const int64_t tiles = ((M + gm::BM - 1) / gm::BM) * ((N + gm::BN - 1) / gm::BN);
         const int grid = (int)(tiles < d.num_sms ? tiles : d.num_sms);
-        gm::gemm_kernel<<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(ta, tb, to, xs, s_channel, bias, (int)M,
+        gm::gemm_kernel<false><<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(ta, tb, to, xs, s_channel, bias, (int)M,
                                                                          (int)N, (int)K, out_f32, swiglu, tma_out, out,
                                                                          acc_out);
         st = launched(cudaGetLastError());
@@ -682,6 +698,102 @@ cr_status cr_w4a8_gemv_swiglu(const int8_t *xq, const float *xs, const uint8_t *
                               int64_t K, cr_out_dtype out_dtype, void *out, cr_stream_t stream)
 {
     return contraction_swiglu(true, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, stream);
+}
+
+namespace {
+// Validation shared by the backward entry points: K as for the forward, N a
+// multiple of 8 (16-byte rows of the bf16 operands), 16-byte aligned buffers.
+cr_status check_backward(const uint8_t *qdata, const uint8_t *srel, const float *codebook, const float *s_channel,
+                         int64_t N, int64_t K, const void *a, const void *b, bool empty = false)
+{
+    if (N < 0 || K < 0)
+        return CR_ERR_INVALID_ARG;
+    const cr_status k = check_k(K);
+    if (k != CR_OK)
+        return k;
+    if (N % 8 != 0 || N > INT_MAX)
+        return CR_ERR_UNSUPPORTED;
+    if (N == 0 || empty)
+        return CR_OK;
+    if (!qdata || !srel || !codebook || !s_channel || !a || !b)
+        return CR_ERR_INVALID_ARG;
+    if (!aligned16(qdata) || !aligned16(srel) || !aligned16(codebook) || !aligned16(s_channel) || !aligned16(a) ||
+        !aligned16(b))
+        return CR_ERR_ALIGNMENT;
+    return CR_OK;
+}
+}  // namespace
+
+cr_status cr_w4a8_dequant_t_bf16(const uint8_t *qdata, const uint8_t *srel, const float *codebook,
+                                 const float *s_channel, int64_t N, int64_t K, uint16_t *wt, cr_stream_t stream)
+{
+    cr_status st = check_backward(qdata, srel, codebook, s_channel, N, K, wt, wt);
+    if (st != CR_OK || N == 0)
+        return st;
+    DeviceState *d = nullptr;
+    st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    return launched(cr::ew::launch_dequant_t_bf16(qdata, srel, codebook, s_channel, (int)N, (int)K, wt, d->num_sms,
+                                                  stream));
+}
+
+cr_status cr_w4a8_ste_backward(const uint16_t *grad, const uint8_t *qdata, const uint8_t *srel,
+                               const float *codebook, const float *s_channel, int64_t M, int64_t N, int64_t K,
+                               uint16_t *dx, cr_stream_t stream)
+{
+    if (M < 0)
+        return CR_ERR_INVALID_ARG;
+    if (M > INT_MAX)
+        return CR_ERR_UNSUPPORTED;
+    cr_status st = check_backward(qdata, srel, codebook, s_channel, N, K, grad, dx, /*empty=*/M == 0);
+    if (st != CR_OK || M == 0)
+        return st;
+    if (N == 0) {  // an empty sum: dx = 0
+        if (!dx)
+            return CR_ERR_INVALID_ARG;
+        return cudaMemsetAsync(dx, 0, (size_t)(M * K) * 2, stream) == cudaSuccess ? CR_OK : CR_ERR_CUDA;
+    }
+    DeviceState *d = nullptr;
+    st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    using namespace cr;
+    if (!d->gemm_bf16_attr_set) {
+        if (cudaFuncSetAttribute(gm::gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)gm::kSmemBytes) != cudaSuccess) {
+            cudaGetLastError();
+            return CR_ERR_CUDA;
+        }
+        d->gemm_bf16_attr_set = true;
+    }
+    // the transposed bf16 weight, from the stream-ordered pool
+    uint16_t *wt = nullptr;
+    if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&wt), (size_t)(N * K) * 2, d->pool, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return CR_ERR_CUDA;
+    }
+    st = launched(ew::launch_dequant_t_bf16(qdata, srel, codebook, s_channel, (int)N, (int)K, wt, d->num_sms, stream));
+    // dx [M, K] = grad [M, N] x wt [K, N]^T: the GEMM's rows are M, its columns K, its reduction N
+    CUtensorMap ta, tb, to;
+    if (st == CR_OK && (!make_tmap_bf16(&ta, grad, (uint64_t)N, (uint64_t)M, 64u, (uint32_t)gm::BM) ||
+                        !make_tmap_bf16(&tb, wt, (uint64_t)N, (uint64_t)K, 64u, (uint32_t)gm::BN) ||
+                        !make_tmap_bf16(&to, dx, (uint64_t)K, (uint64_t)M, 64u, 32u)))
+        st = CR_ERR_CUDA;
+    if (st == CR_OK) {
+        const int64_t tiles = ((M + gm::BM - 1) / gm::BM) * ((K + gm::BN - 1) / gm::BN);
+        const int grid = (int)(tiles < d->num_sms ? tiles : d->num_sms);
+        gm::gemm_kernel<true><<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(
+            ta, tb, to, nullptr, nullptr, nullptr, (int)M, (int)K, (int)N, /*out_f32=*/0, /*swiglu=*/0,
+            /*tma_out=*/1, dx, nullptr);
+        st = launched(cudaGetLastError());
+    }
+    if (cudaFreeAsync(wt, stream) != cudaSuccess) {
+        cudaGetLastError();
+        if (st == CR_OK)
+            st = CR_ERR_CUDA;
+    }
+    return st;
 }
 
 namespace {

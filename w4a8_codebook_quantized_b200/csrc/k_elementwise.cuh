@@ -190,5 +190,71 @@ inline cudaError_t launch_interleave_rows(const void *src, void *dst, int64_t ro
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- backward weight
+//
+// ai-toolkit convrot_w4a8_quant.py, _w4a8_linear_ste_backward: the weight of
+// the input gradient, w = w8.to(bf16) * s_channel.to(bf16), here written
+// transposed, wt[k, n] = bf16(w8[n, k] * bf16(s_channel[n])) [K, N], the
+// K-major B operand of dx = grad @ w.  w8 is the forward's decode; the
+// product of an int8 and a bf16 is exact in fp32 and is rounded once.
+// A CTA per 64 (n) x 128 (k) tile: thread (c = tid / 64, r = tid % 64)
+// decodes the 32 weights of row n0 + r, columns k0 + 32c .. + 32 (one 16-byte
+// load of codes) into a shared tile [128 k][72] (lanes on consecutive n: no
+// bank conflicts), then the tile leaves as 128 rows of 64 bf16 (16-byte
+// stores).  N must be a multiple of 8 and K of 128.
+constexpr int kTN = 64, kTK = 128, kTPad = 72;
+
+__global__ void __launch_bounds__(kThreads) dequant_t_bf16_kernel(const uint8_t *__restrict__ qdata,
+                                                                  const uint8_t *__restrict__ srel,
+                                                                  const float *__restrict__ codebook,
+                                                                  const float *__restrict__ s_channel, int N, int K,
+                                                                  uint16_t *__restrict__ wt)
+{
+    __shared__ __align__(16) uint16_t tile[kTK][kTPad];
+    __shared__ float cb[16];
+    if (threadIdx.x < 16)
+        cb[threadIdx.x] = codebook[threadIdx.x];
+    __syncthreads();
+    const int tiles_k = K / kTK, tiles_n = (N + kTN - 1) / kTN;
+    const int r = threadIdx.x & (kTN - 1), c = threadIdx.x >> 6;
+    for (int t = blockIdx.x; t < tiles_k * tiles_n; t += gridDim.x) {
+        const int tn = t / tiles_k, tk = t - tn * tiles_k;
+        const int n0 = tn * kTN, k0 = tk * kTK, n = n0 + r;
+        if (n < N) {
+            const int kc = k0 + 32 * c;
+            const uint4 codes = *reinterpret_cast<const uint4 *>(qdata + (int64_t)n * (K / 2) + kc / 2);
+            const uint8_t *sr = srel + (int64_t)n * (K / 16) + kc / 16;
+            const float sv0 = fp8e4m3fn_to_float(sr[0]), sv1 = fp8e4m3fn_to_float(sr[1]);
+            const float sch = __bfloat162float(__float2bfloat16_rn(s_channel[n]));
+            const uint32_t words[4] = {codes.x, codes.y, codes.z, codes.w};
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const uint32_t code = (words[j >> 3] >> (4 * (j & 7))) & 0xFu;
+                const int32_t w8 = sat_s8_rne(__fmul_rn(cb[code], j < 16 ? sv0 : sv1));
+                tile[32 * c + j][r] = to_bf16_bits(__fmul_rn((float)w8, sch));
+            }
+        }
+        __syncthreads();
+        for (int i = threadIdx.x; i < kTK * (kTN / 8); i += kThreads) {
+            const int kr = i >> 3, ch = i & 7, nn = n0 + 8 * ch;
+            if (nn < N)  // N % 8 == 0: a 16-byte chunk is wholly inside or outside
+                *reinterpret_cast<uint4 *>(wt + (int64_t)(k0 + kr) * N + nn) =
+                    *reinterpret_cast<const uint4 *>(&tile[kr][8 * ch]);
+        }
+        __syncthreads();
+    }
+}
+
+inline cudaError_t launch_dequant_t_bf16(const uint8_t *qdata, const uint8_t *srel, const float *codebook,
+                                         const float *s_channel, int N, int K, uint16_t *wt, int num_sms,
+                                         cudaStream_t stream)
+{
+    const int64_t tiles = (int64_t)(K / kTK) * ((N + kTN - 1) / kTN);
+    const int64_t cap = (int64_t)num_sms * 8;
+    const int grid = (int)(tiles < cap ? tiles : cap);
+    dequant_t_bf16_kernel<<<grid < 1 ? 1 : grid, kThreads, 0, stream>>>(qdata, srel, codebook, s_channel, N, K, wt);
+    return cudaGetLastError();
+}
+
 }  // namespace ew
 }  // namespace cr

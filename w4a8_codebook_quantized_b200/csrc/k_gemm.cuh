@@ -72,7 +72,9 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_n, int &tm, int 
 // TMEM load is in flight while the current chunk is converted.  Otherwise each
 // thread stores its own row.  release() hands the accumulator back once every
 // column is in registers.
-template <class Release>
+// RAW: the accumulator holds fp32 values that are the outputs themselves
+// (bf16 GEMM); no scales, bias or SwiGLU.
+template <bool RAW, class Release>
 __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row0, int col_base, int lane, float xm, bool row_ok,
                                               const float *wsv, const float *bsv, bool has_bias, int M, int N,
                                               int out_f32, int swiglu, int tma_out, const CUtensorMap *tmOut,
@@ -86,16 +88,22 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row0, int col_
     auto convert32 = [&](const uint32_t (&v)[32], int c0, uint32_t *dst) {
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
-            const float4 w4 = *reinterpret_cast<const float4 *>(wsv + c0 + j);
-            const float4 b4 = *reinterpret_cast<const float4 *>(bsv + c0 + j);
-            const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
-            const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
             float y[4];
+            if constexpr (RAW) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                y[e] = __fmul_rn(__int2float_rn((int32_t)v[j + e]), __fmul_rn(xm, wv[e]));
-                if (has_bias)
-                    y[e] = __fadd_rn(y[e], bv[e]);
+                for (int e = 0; e < 4; ++e)
+                    y[e] = __uint_as_float(v[j + e]);
+            } else {
+                const float4 w4 = *reinterpret_cast<const float4 *>(wsv + c0 + j);
+                const float4 b4 = *reinterpret_cast<const float4 *>(bsv + c0 + j);
+                const float wv[4] = {w4.x, w4.y, w4.z, w4.w};
+                const float bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    y[e] = __fmul_rn(__int2float_rn((int32_t)v[j + e]), __fmul_rn(xm, wv[e]));
+                    if (has_bias)
+                        y[e] = __fadd_rn(y[e], bv[e]);
+                }
             }
             if (out_f32) {
 #pragma unroll
@@ -128,7 +136,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row0, int col_
         ++units_issued;
     };
     uint32_t cur[32], nxt[32], packed[32];
-    if (swiglu) {
+    if (!RAW && swiglu) {
         // Interleaved gate/up rows: accumulator columns 2f and 2f + 1 are one
         // pair and give output column f of [M, N / 2].  Each 32-column TMEM
         // load yields 16 outputs; a 128-byte unit (64 bf16 or 32 fp32 outputs)
@@ -260,7 +268,7 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row0, int col_
                     const int n = col0 + j;
                     if (n >= N)
                         break;
-                    const float y = epilogue_value((int32_t)cur[j], xm, ws[n], bias, n);
+                    const float y = RAW ? __uint_as_float(cur[j]) : epilogue_value((int32_t)cur[j], xm, ws[n], bias, n);
                     if (out_f32)
                         reinterpret_cast<float *>(out)[base + j] = y;
                     else
@@ -279,6 +287,10 @@ __device__ __forceinline__ void epilogue_tile(uint32_t tbase, int row0, int col_
     }
 }
 
+// BF16: A and B are bf16 (K counted in bf16 elements, 64 per 128-byte
+// stage row), tcgen05.mma kind::f16 into fp32, and the epilogue writes the
+// accumulators as they are (xs, ws, bias, swiglu and acc_out unused).
+template <bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmOut, const float *__restrict__ xs,
@@ -291,7 +303,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tiles_m = (M + BM - 1) / BM, tiles_n = (N + BN - 1) / BN;
     const int num_tiles = tiles_m * tiles_n;
-    const int kblocks = K / BK;
+    constexpr int BKE = BF16 ? BK / 2 : BK;  // K elements per stage
+    const int kblocks = (K + BKE - 1) / BKE;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -337,8 +350,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     mbar_arrive_expect_tx(&sh.full[stage], kStageBytes);
-                    tma_load_2d(sh.stage[stage], &tmA, kb * BK, tm * BM, &sh.full[stage]);
-                    tma_load_2d(sh.stage[stage] + kABytes, &tmB, kb * BK, tn * BN, &sh.full[stage]);
+                    tma_load_2d(sh.stage[stage], &tmA, kb * BKE, tm * BM, &sh.full[stage]);
+                    tma_load_2d(sh.stage[stage] + kABytes, &tmB, kb * BKE, tn * BN, &sh.full[stage]);
                     issued[stage] = 1;
                     issued_phase[stage] = phase;
                     if (++stage == kStages) {
@@ -384,7 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < BK / 32; ++kk) {
                         const uint64_t ad = sw128_kmajor_desc(a_addr + 32u * kk);
                         const uint64_t bd = sw128_kmajor_desc(b_addr + 32u * kk);
-                        mma_i8(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                        if constexpr (BF16)
+                            mma_bf16(d, ad, bd, idesc_bf16(BM, BN), (kb | kk) != 0 ? 1u : 0u);
+                        else
+                            mma_i8(d, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     tc_commit(&sh.empty[stage]);
                     if (++stage == kStages) {
@@ -419,10 +435,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tile_coords(tile, tiles_n, tm, tn);
             const int buf = local & 1;
             const uint32_t use = (uint32_t)(local >> 1) & 1u;
-            for (int j = et; j < BN; j += 128) {
-                const int n = tn * BN + j;
-                sh.wsb[buf][j] = n < N ? ws[n] : 0.0f;
-                sh.biasb[buf][j] = (bias != nullptr && n < N) ? bias[n] : 0.0f;
+            if constexpr (!BF16) {
+                for (int j = et; j < BN; j += 128) {
+                    const int n = tn * BN + j;
+                    sh.wsb[buf][j] = n < N ? ws[n] : 0.0f;
+                    sh.biasb[buf][j] = (bias != nullptr && n < N) ? bias[n] : 0.0f;
+                }
             }
             asm volatile("bar.sync 2, 128;" ::: "memory");
             const bool ok = mbar_wait_bounded_warp(&sh.tmem_full[buf], use, abort);
@@ -431,9 +449,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int row = tm * BM + 32 * q + lane;
             const bool row_ok = row < M;
-            const float xm = row_ok ? xs[row] : 0.0f;
+            const float xm = (!BF16 && row_ok) ? xs[row] : 0.0f;
             const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN);
-            epilogue_tile(tbase, tm * BM + 32 * q, tn * BN, lane, xm, row_ok, sh.wsb[buf], sh.biasb[buf],
+            epilogue_tile<BF16>(tbase, tm * BM + 32 * q, tn * BN, lane, xm, row_ok, sh.wsb[buf], sh.biasb[buf],
                           bias != nullptr, M, N, out_f32, swiglu, tma_out, &tmOut, sh.epi[q], units_issued, out, acc_out, ws,
                           bias, [&]() {
                               tc_fence_before();
@@ -649,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float xm = row_ok ? xs[row0 + lane] : 0.0f;
             const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN);
             const uint32_t release_addr = mapa_shared(smem_u32(&sh.tmem_empty[buf]), 0);
-            epilogue_tile(tbase, row0, tn * BN, lane, xm, row_ok, sh.wsb[buf], sh.biasb[buf], bias != nullptr, M,
+            epilogue_tile<false>(tbase, row0, tn * BN, lane, xm, row_ok, sh.wsb[buf], sh.biasb[buf], bias != nullptr, M,
                           N, out_f32, swiglu, tma_out, &tmOut, sh.epi[q], units_issued, out, acc_out, ws, bias, [&]() {
                               tc_fence_before();
                               __syncwarp();
