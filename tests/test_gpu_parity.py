@@ -507,7 +507,8 @@ def test_dequant_t_bf16_bit_exact(N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 8, 256), (64, 512, 1024), (300, 1000, 768), (129, 72, 2048),
-                                   (1024, 2048, 1024)])
+                                   (1024, 2048, 1024),
+                                   (1100, 256, 8192), (2000, 72, 4096)])  # the last two on CTA pairs
 def test_ste_backward(M, N, K):
     """dx against the oracle (double sums, one rounding) and against torch's
     fp32 matmul of the same bf16 operands, elementwise within the bound the

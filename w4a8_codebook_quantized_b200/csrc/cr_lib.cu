@@ -35,6 +35,7 @@ struct DeviceState {
     bool gemv_attr_set = false;
     bool gemv_grouped_attr_set = false;
     bool gemm_bf16_attr_set = false;
+    bool gemm_pair_bf16_attr_set = false;
     // side stream and events on which cr_w4a8_linear's prefill path decodes
     // the weight while the activations are rotated and quantised
     cudaStream_t side = nullptr;
@@ -439,7 +440,7 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
     if (st == CR_OK && use_pair) {
         CUtensorMap tb_half;
         if (!d.gemm_pair_attr_set) {
-            if (cudaFuncSetAttribute(gm::gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            if (cudaFuncSetAttribute(gm::gemm_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)gm::pair::kSmemBytes) != cudaSuccess) {
                 cudaGetLastError();
                 st = CR_ERR_CUDA;
@@ -463,7 +464,7 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
             attr[0].val.clusterDim.z = 1;
             cfg.attrs = attr;
             cfg.numAttrs = 1;
-            st = launched(cudaLaunchKernelEx(&cfg, gm::gemm_pair_kernel, ta, tb_half, to, xs, s_channel, bias, (int)M,
+            st = launched(cudaLaunchKernelEx(&cfg, gm::gemm_pair_kernel<false>, ta, tb_half, to, xs, s_channel, bias, (int)M,
                                              (int)N, (int)K, out_f32, swiglu, tma_out, out, acc_out));
         }
     } else if (st == CR_OK) {
@@ -780,7 +781,40 @@ cr_status cr_w4a8_ste_backward(const uint16_t *grad, const uint8_t *qdata, const
                         !make_tmap_bf16(&tb, wt, (uint64_t)N, (uint64_t)K, 64u, (uint32_t)gm::BN) ||
                         !make_tmap_bf16(&to, dx, (uint64_t)K, (uint64_t)M, 64u, 32u)))
         st = CR_ERR_CUDA;
-    if (st == CR_OK) {
+    // 256 x 256 tiles on CTA pairs when there is at least one per SM pair
+    const int64_t pair_tiles = ((M + 255) / 256) * ((K + gm::BN - 1) / gm::BN);
+    if (st == CR_OK && pair_tiles >= d->num_sms / 2) {
+        CUtensorMap tb_half;
+        if (!d->gemm_pair_bf16_attr_set) {
+            if (cudaFuncSetAttribute(gm::gemm_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)gm::pair::kSmemBytes) != cudaSuccess) {
+                cudaGetLastError();
+                st = CR_ERR_CUDA;
+            } else {
+                d->gemm_pair_bf16_attr_set = true;
+            }
+        }
+        if (st == CR_OK && !make_tmap_bf16(&tb_half, wt, (uint64_t)N, (uint64_t)K, 64u, 128u))
+            st = CR_ERR_CUDA;
+        if (st == CR_OK) {
+            const int64_t pairs = pair_tiles < d->num_sms / 2 ? pair_tiles : d->num_sms / 2;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)(2 * pairs));
+            cfg.blockDim = dim3(gm::kThreads);
+            cfg.dynamicSmemBytes = gm::pair::kSmemBytes;
+            cfg.stream = stream;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            st = launched(cudaLaunchKernelEx(&cfg, gm::gemm_pair_kernel<true>, ta, tb_half, to, (const float *)nullptr,
+                                             (const float *)nullptr, (const float *)nullptr, (int)M, (int)K, (int)N,
+                                             0, 0, 1, (void *)dx, (int32_t *)nullptr));
+        }
+    } else if (st == CR_OK) {
         const int64_t tiles = ((M + gm::BM - 1) / gm::BM) * ((K + gm::BN - 1) / gm::BN);
         const int grid = (int)(tiles < d->num_sms ? tiles : d->num_sms);
         gm::gemm_kernel<true><<<grid, gm::kThreads, gm::kSmemBytes, stream>>>(

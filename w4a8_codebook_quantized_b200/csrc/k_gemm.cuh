@@ -506,6 +506,8 @@ struct __align__(1024) Smem {
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 }  // namespace pair
 
+// BF16 as for gemm_kernel.
+template <bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmOut, const float *__restrict__ xs,
@@ -521,7 +523,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int npairs = gridDim.x >> 1, pair_id = blockIdx.x >> 1;
     const int tiles_m = (M + 255) / 256, tiles_n = (N + BN - 1) / BN;
     const int num_tiles = tiles_m * tiles_n;
-    const int kblocks = K / BK;
+    constexpr int BKE = BF16 ? BK / 2 : BK;  // K elements per stage
+    const int kblocks = (K + BKE - 1) / BKE;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < pair::kStages; ++s) {
@@ -569,8 +572,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t full_leader = mapa_shared(smem_u32(&sh.full[stage]), 0);
                     if (leader)
                         mbar_arrive_expect_tx(&sh.full[stage], 2 * pair::kStageBytes);
-                    tma_load_2d_pair(sh.stage[stage], &tmA, kb * BK, tm * 256 + (int)rank * 128, full_leader);
-                    tma_load_2d_pair(sh.stage[stage] + pair::kHalfBytes, &tmB, kb * BK, tn * BN + (int)rank * 128,
+                    tma_load_2d_pair(sh.stage[stage], &tmA, kb * BKE, tm * 256 + (int)rank * 128, full_leader);
+                    tma_load_2d_pair(sh.stage[stage] + pair::kHalfBytes, &tmB, kb * BKE, tn * BN + (int)rank * 128,
                                      full_leader);
                     issued[stage] = 1;
                     issued_phase[stage] = phase;
@@ -624,8 +627,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t b_addr = a_addr + pair::kHalfBytes;
 #pragma unroll
                     for (int kk = 0; kk < BK / 32; ++kk)
-                        mma_i8_pair(d, sw128_kmajor_desc(a_addr + 32u * kk), sw128_kmajor_desc(b_addr + 32u * kk),
-                                    pair::kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                        if constexpr (BF16)
+                            mma_bf16_pair(d, sw128_kmajor_desc(a_addr + 32u * kk),
+                                          sw128_kmajor_desc(b_addr + 32u * kk), idesc_bf16(256, BN),
+                                          (kb | kk) != 0 ? 1u : 0u);
+                        else
+                            mma_i8_pair(d, sw128_kmajor_desc(a_addr + 32u * kk),
+                                        sw128_kmajor_desc(b_addr + 32u * kk), pair::kIdesc,
+                                        (kb | kk) != 0 ? 1u : 0u);
                     const uint32_t e = smem_u32(&sh.empty[stage]);
                     tc_commit_pair(mapa_shared(e, 0));
                     tc_commit_pair(mapa_shared(e, peer));
@@ -652,10 +661,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tile_coords(tile, tiles_n, tm, tn);
             const int buf = local & 1;
             const uint32_t use = (uint32_t)(local >> 1) & 1u;
-            for (int j = et; j < BN; j += 128) {
-                const int n = tn * BN + j;
-                sh.wsb[buf][j] = n < N ? ws[n] : 0.0f;
-                sh.biasb[buf][j] = (bias != nullptr && n < N) ? bias[n] : 0.0f;
+            if constexpr (!BF16) {
+                for (int j = et; j < BN; j += 128) {
+                    const int n = tn * BN + j;
+                    sh.wsb[buf][j] = n < N ? ws[n] : 0.0f;
+                    sh.biasb[buf][j] = (bias != nullptr && n < N) ? bias[n] : 0.0f;
+                }
             }
             asm volatile("bar.sync 2, 128;" ::: "memory");
             const bool ok = mbar_wait_bounded_warp(&sh.tmem_full[buf], use, abort);
@@ -664,10 +675,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const int row0 = tm * 256 + (int)rank * 128 + 32 * q;
             const bool row_ok = row0 + lane < M;
-            const float xm = row_ok ? xs[row0 + lane] : 0.0f;
+            const float xm = (!BF16 && row_ok) ? xs[row0 + lane] : 0.0f;
             const uint32_t tbase = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * BN);
             const uint32_t release_addr = mapa_shared(smem_u32(&sh.tmem_empty[buf]), 0);
-            epilogue_tile<false>(tbase, row0, tn * BN, lane, xm, row_ok, sh.wsb[buf], sh.biasb[buf], bias != nullptr, M,
+            epilogue_tile<BF16>(tbase, row0, tn * BN, lane, xm, row_ok, sh.wsb[buf], sh.biasb[buf], bias != nullptr, M,
                           N, out_f32, swiglu, tma_out, &tmOut, sh.epi[q], units_issued, out, acc_out, ws, bias, [&]() {
                               tc_fence_before();
                               __syncwarp();
