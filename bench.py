@@ -57,6 +57,7 @@ def parse():
     p.add_argument("--no-prefill", action="store_true")
     p.add_argument("--no-grouped", action="store_true")
     p.add_argument("--no-swiglu", action="store_true")
+    p.add_argument("--no-backward", action="store_true")
     p.add_argument("--swiglu-workload", default="c4_mlp_up")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -440,6 +441,10 @@ def run_ours(args):
     if not args.no_swiglu:
         swiglu = run_swiglu(args, world, rank, pk)
 
+    backward = None
+    if not args.no_backward:
+        backward = run_backward(args, world, rank, pk)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(case, args.cpu_seconds)
@@ -454,7 +459,7 @@ def run_ours(args):
                    "timing": "one CUDA-graph replay of K steps (graph uploaded beforehand), CUDA events on the capture stream",
                    "parallelism": f"replica x{world}"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps,
-        "clocks": clocks, "prefill": prefill, "grouped": grouped, "swiglu": swiglu,
+        "clocks": clocks, "prefill": prefill, "grouped": grouped, "swiglu": swiglu, "ste_backward": backward,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -598,6 +603,38 @@ def run_swiglu(args, world, rank, pk):
             "value": round(world * ops / tf / 1e12, 2), "unit": "TOPS", "ms_per_step": round(tf * 1e3, 4),
             "plain_forward": {"value": round(world * ops / tp / 1e12, 2), "ms_per_step": round(tp * 1e3, 4)},
             "steps": steps, "l2": "256 MiB write between steps, outside the timed events"}
+
+
+def run_backward(args, world, rank, pk):
+    """The straight-through input gradient on the prefill shape: dx [M, K] =
+    grad [M, N] @ (w8 * s_channel in bf16), cr_w4a8_ste_backward (the codes
+    decoded again into a bf16 transient, then the tcgen05 bf16 GEMM)."""
+    import torch
+
+    import w4a8_codebook_quantized_b200 as cr
+    from w4a8_codebook_quantized_b200 import inputs
+    case = inputs.CASES[args.prefill_workload]
+    M, N, K = case.M, case.N, case.K
+    layer = inputs.layer(N, K, rank_seed(case.seed, rank))
+    q, s, cb, ws = (torch.from_numpy(a).cuda() for a in (layer.qdata, layer.srel, layer.codebook, layer.s_channel))
+    g = torch.from_numpy(np.random.default_rng(rank_seed(case.seed, rank)).standard_normal((M, N))
+                         .astype(np.float32)).to(torch.bfloat16).cuda()
+    dx = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    call = lambda: cr.cr_w4a8_ste_backward(g, q, s, cb, ws, dx=dx)
+    for _ in range(max(3, args.warmup)):
+        call()
+    steps = max(3, min(args.steps, 20))
+    (t,) = flushed_medians([call], steps)
+    t = max_over_ranks(t, world)
+    flops = 2.0 * M * N * K
+    peak = pk["bf16_tflops"]
+    return {"workload": f"{case.name} backward: grad [{M}, {N}] @ w [{N}, {K}]",
+            "value": round(world * flops / t / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(t * 1e3, 4),
+            "steps": steps, "l2": "256 MiB write between steps, outside the timed events",
+            "roofline": {"bound": "tensor", "achieved": round(flops / t / 1e12, 1), "peak": round(peak, 1),
+                         "unit": "TFLOP/s", "frac": round(flops / t / 1e12 / peak, 4),
+                         "peak_source": f"{pk['source']} bf16_tflops",
+                         "kernel": "cr_w4a8_ste_backward call (bf16 weight transient + tcgen05 bf16 GEMM)"}}
 
 
 GROUPED_NS = (4096, 1024, 1024)  # q, k, v of an attention block with 8-way grouped k/v heads
