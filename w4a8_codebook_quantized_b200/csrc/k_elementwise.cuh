@@ -13,14 +13,16 @@ constexpr int kThreads = 256;
 // ai-toolkit convrot_w4a8_quant.py, unpack_w4a8_eager / w4a8_unpack_kernel:
 // w8[n, k] = sat_s8(rne(codebook[code] * fp8(srel[n, k/16]))).
 //
-// Grid-stride over 16-byte chunks of packed codes (32 weights, two groups).
-// Each thread issues the loads of kDecodeUnroll chunks (64 bytes of codes and their
-// scale bytes) before it decodes any, so that enough bytes are in flight to
-// keep HBM busy; per chunk two lookups in the CTA's level table (4 copies, the
-// copy chosen by lane, to spread a quarter-warp's lookups over bank groups),
-// four byte-permute decodes and two 16-byte stores.  HBM traffic per weight:
-// 0.5 + 1/16 bytes in, 1 byte out.
-constexpr int kDecodeUnroll = 4;
+// Grid-stride over groups: a thread takes one group of 16 weights (8 bytes
+// of codes, one scale byte) and writes its 16 output bytes, so a warp's store
+// is one contiguous 512-byte run of whole sectors (two 16-byte stores per
+// 32-byte chunk, one per half-sector, were written back to DRAM about 2.6
+// times over).  Each thread issues the loads of kDecodeUnroll groups before it
+// decodes any, to keep enough bytes in flight; per group one lookup in the
+// CTA's level table (4 copies, the copy chosen by lane, to spread a
+// quarter-warp's lookups over bank groups) and two byte-permute decodes.
+// HBM traffic per weight: 0.5 + 1/16 bytes in, 1 byte out.
+constexpr int kDecodeUnroll = 8;
 constexpr int kDecodeLutCopies = 4;
 
 __global__ void __launch_bounds__(kThreads) decode_int8_kernel(const uint8_t *__restrict__ qdata,
@@ -42,36 +44,30 @@ __global__ void __launch_bounds__(kThreads) decode_int8_kernel(const uint8_t *__
     __syncthreads();
 
     const uint4 *lutc = lut + (threadIdx.x & (kDecodeLutCopies - 1));
-    const int64_t chunks_per_row = K / 32;
-    const int64_t total = N * chunks_per_row;
+    // groups are contiguous across rows: group i has its codes at 8 i, its
+    // scale byte at i and its output at 16 i
+    const int64_t total = N * (K / 16);
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     for (int64_t i0 = (int64_t)blockIdx.x * kThreads + threadIdx.x; i0 < total; i0 += kDecodeUnroll * stride) {
-        uint4 c[kDecodeUnroll];
+        uint2 c[kDecodeUnroll];
         uint32_t sb[kDecodeUnroll];
 #pragma unroll
         for (int u = 0; u < kDecodeUnroll; ++u) {
             const int64_t i = i0 + u * stride;
             if (i < total) {
-                const int64_t n = i / chunks_per_row;
-                const int64_t j = i - n * chunks_per_row;
-                c[u] = ldg_stream16(qdata + n * (K / 2) + 16 * j);
-                sb[u] = __ldg(reinterpret_cast<const uint16_t *>(srel + n * (K / 16) + 2 * j));
+                c[u] = ldg_stream8(qdata + 8 * i);
+                sb[u] = __ldg(srel + i);
             }
         }
 #pragma unroll
         for (int u = 0; u < kDecodeUnroll; ++u) {
             const int64_t i = i0 + u * stride;
             if (i < total) {
-                const uint4 T0 = lutc[kDecodeLutCopies * (sb[u] & 0xFFu)];
-                const uint4 T1 = lutc[kDecodeLutCopies * (sb[u] >> 8)];
-                uint4 o0, o1;
-                decode8(c[u].x, T0, o0.x, o0.y);
-                decode8(c[u].y, T0, o0.z, o0.w);
-                decode8(c[u].z, T1, o1.x, o1.y);
-                decode8(c[u].w, T1, o1.z, o1.w);
-                uint4 *dst = reinterpret_cast<uint4 *>(w8 + 32 * i);  // rows are K bytes: chunk i starts at 32 i
-                dst[0] = o0;
-                dst[1] = o1;
+                const uint4 T = lutc[kDecodeLutCopies * sb[u]];
+                uint4 o;
+                decode8(c[u].x, T, o.x, o.y);
+                decode8(c[u].y, T, o.z, o.w);
+                *reinterpret_cast<uint4 *>(w8 + 16 * i) = o;
             }
         }
     }
@@ -80,7 +76,7 @@ __global__ void __launch_bounds__(kThreads) decode_int8_kernel(const uint8_t *__
 inline cudaError_t launch_decode(const uint8_t *qdata, const uint8_t *srel, const float *codebook, int64_t N,
                                  int64_t K, int8_t *w8, int num_sms, cudaStream_t stream)
 {
-    const int64_t total = N * (K / 32);
+    const int64_t total = N * (K / 16);
     int64_t blocks = (total + (int64_t)kThreads * kDecodeUnroll - 1) / ((int64_t)kThreads * kDecodeUnroll);
     const int64_t cap = (int64_t)num_sms * 8;
     if (blocks > cap)
