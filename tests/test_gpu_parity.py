@@ -146,8 +146,9 @@ def _contraction_case(fn, M, N, K, seed, kind="bf16", with_bias=False, dist="out
                                    (8, 4096, 4096), (5, 2048, 2048), (8, 256, 12288), (6, 33, 8192),
                                    (7, 3000, 16384), (2, 520, 20480)])
 def test_gemv(M, N, K):
-    """Up to K = 12288 the activations stay resident in shared memory; at
-    K = 16384 and 20480 they stream through the ring with the weights."""
+    """Ragged N, every M, K from one stage (1024 columns) up to twenty: the
+    activations stream through the ring with the weights, one 1024-column
+    chunk per stage."""
     _contraction_case(cr.cr_w4a8_gemv, M, N, K, seed=M + N + K)
 
 
