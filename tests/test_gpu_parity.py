@@ -160,10 +160,11 @@ def test_gemm(M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(2048, 4096, 512), (2000, 4000, 768), (4096, 2560, 256), (1100, 9000, 256),
-                                   (4352, 2304, 512)])
+                                   (4352, 2304, 512), (512, 18944, 256), (2048, 4096, 2048)])
 def test_gemm_cta_pairs(M, N, K):
     """Shapes with at least one 256 x 256 tile per SM pair take the CTA-pair
-    tcgen05 kernel (M = 256 per pair); ragged M and N included."""
+    tcgen05 kernel (M = 256 per pair); ragged M and N included, partial last
+    waves, and 512 x 18944 = 148 tiles, two whole waves on 74 pairs."""
     _contraction_case(cr.cr_w4a8_gemm, M, N, K, seed=M + N + K, with_bias=(K == 768))
 
 
