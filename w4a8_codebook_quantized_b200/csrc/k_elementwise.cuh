@@ -191,14 +191,16 @@ inline cudaError_t launch_interleave_rows(const void *src, void *dst, int64_t ro
 // ai-toolkit convrot_w4a8_quant.py, _w4a8_linear_ste_backward: the weight of
 // the input gradient, w = w8.to(bf16) * s_channel.to(bf16), here written
 // transposed, wt[k, n] = bf16(w8[n, k] * bf16(s_channel[n])) [K, N], the
-// K-major B operand of dx = grad @ w.  w8 is the forward's decode; the
+// K-major B operand of dx = grad @ w.  w8 is the forward's decode (the same
+// per-CTA table of 16 int8 levels per scale byte and byte permutes); the
 // product of an int8 and a bf16 is exact in fp32 and is rounded once.
-// A CTA per 64 (n) x 128 (k) tile: thread (c = tid / 64, r = tid % 64)
-// decodes the 32 weights of row n0 + r, columns k0 + 32c .. + 32 (one 16-byte
-// load of codes) into a shared tile [128 k][72] (lanes on consecutive n: no
-// bank conflicts), then the tile leaves as 128 rows of 64 bf16 (16-byte
-// stores).  N must be a multiple of 8 and K of 128.
-constexpr int kTN = 64, kTK = 128, kTPad = 72;
+// A CTA per 64 (n) x 128 (k) tile: thread (g = tid / 32, p = tid % 32)
+// decodes group g (16 columns) of rows n0 + 2p and n0 + 2p + 1 and stores
+// the 16 bf16 pairs (row 2p, row 2p + 1) of those columns into a shared tile
+// of 4-byte pairs [128 k][36] (lanes on consecutive pairs: no bank
+// conflicts); the tile then leaves as 128 rows of 64 bf16 (16-byte stores, 8
+// lanes per 128-byte row).  N must be a multiple of 8 and K of 128.
+constexpr int kTN = 64, kTK = 128, kTPairs = 36;  // 32 row pairs + 4 of padding (16-byte aligned rows)
 
 __global__ void __launch_bounds__(kThreads) dequant_t_bf16_kernel(const uint8_t *__restrict__ qdata,
                                                                   const uint8_t *__restrict__ srel,
@@ -206,28 +208,48 @@ __global__ void __launch_bounds__(kThreads) dequant_t_bf16_kernel(const uint8_t 
                                                                   const float *__restrict__ s_channel, int N, int K,
                                                                   uint16_t *__restrict__ wt)
 {
-    __shared__ __align__(16) uint16_t tile[kTK][kTPad];
+    __shared__ __align__(16) uint32_t tile[kTK][kTPairs];
+    __shared__ uint4 lut[256];
     __shared__ float cb[16];
     if (threadIdx.x < 16)
         cb[threadIdx.x] = codebook[threadIdx.x];
     __syncthreads();
+    lut[threadIdx.x] = lut_entry(threadIdx.x, cb);  // kThreads == 256 scale bytes
+    __syncthreads();
     const int tiles_k = K / kTK, tiles_n = (N + kTN - 1) / kTN;
-    const int r = threadIdx.x & (kTN - 1), c = threadIdx.x >> 6;
+    const int p = threadIdx.x & 31, g = threadIdx.x >> 5;
+    // n fastest: CTAs running together write neighbouring 128-byte strips of
+    // the same 128 rows of wt (whole rows between them), not one strip each
+    // of rows 8 KB apart
     for (int t = blockIdx.x; t < tiles_k * tiles_n; t += gridDim.x) {
-        const int tn = t / tiles_k, tk = t - tn * tiles_k;
-        const int n0 = tn * kTN, k0 = tk * kTK, n = n0 + r;
-        if (n < N) {
-            const int kc = k0 + 32 * c;
-            const uint4 codes = *reinterpret_cast<const uint4 *>(qdata + (int64_t)n * (K / 2) + kc / 2);
-            const uint8_t *sr = srel + (int64_t)n * (K / 16) + kc / 16;
-            const float sv0 = fp8e4m3fn_to_float(sr[0]), sv1 = fp8e4m3fn_to_float(sr[1]);
-            const float sch = __bfloat162float(__float2bfloat16_rn(s_channel[n]));
-            const uint32_t words[4] = {codes.x, codes.y, codes.z, codes.w};
+        const int tk = t / tiles_n, tn = t - tk * tiles_n;
+        const int n0 = tn * kTN, k0 = tk * kTK, n = n0 + 2 * p;
+        if (n < N) {  // N % 8 == 0: both rows of the pair exist
+            const int kg = k0 / 16 + g;  // this thread's group
+            uint32_t lo[4], hi[4];
+            float sch[2];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const uint32_t code = (words[j >> 3] >> (4 * (j & 7))) & 0xFu;
-                const int32_t w8 = sat_s8_rne(__fmul_rn(cb[code], j < 16 ? sv0 : sv1));
-                tile[32 * c + j][r] = to_bf16_bits(__fmul_rn((float)w8, sch));
+            for (int r = 0; r < 2; ++r) {
+                const uint2 c = *reinterpret_cast<const uint2 *>(qdata + (int64_t)(n + r) * (K / 2) + 8 * kg);
+                const uint4 T = lut[srel[(int64_t)(n + r) * (K / 16) + kg]];
+                uint32_t *w = r ? hi : lo;
+                decode8(c.x, T, w[0], w[1]);
+                decode8(c.y, T, w[2], w[3]);
+                sch[r] = __bfloat162float(__float2bfloat16_rn(s_channel[n + r]));
+            }
+            // int8 -> fp32 without the conversion unit: with the sign bit
+            // flipped, byte j is w + 128 in 0..255; placed as the low mantissa
+            // byte of 2^23 (bits 0x4B000000) it reads as 2^23 + w + 128, and
+            // subtracting 2^23 + 128 leaves w exactly
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const uint32_t sel = 0x7650u | (uint32_t)(j & 3);
+                const uint32_t ab = prmt(lo[j >> 2] ^ 0x80808080u, 0x4B000000u, sel);
+                const uint32_t bb = prmt(hi[j >> 2] ^ 0x80808080u, 0x4B000000u, sel);
+                const float a = __fsub_rn(__uint_as_float(ab), 8388736.0f);
+                const float b = __fsub_rn(__uint_as_float(bb), 8388736.0f);
+                const __nv_bfloat162 v = __floats2bfloat162_rn(__fmul_rn(a, sch[0]), __fmul_rn(b, sch[1]));
+                tile[16 * g + j][p] = *reinterpret_cast<const uint32_t *>(&v);
             }
         }
         __syncthreads();
@@ -235,7 +257,7 @@ __global__ void __launch_bounds__(kThreads) dequant_t_bf16_kernel(const uint8_t 
             const int kr = i >> 3, ch = i & 7, nn = n0 + 8 * ch;
             if (nn < N)  // N % 8 == 0: a 16-byte chunk is wholly inside or outside
                 *reinterpret_cast<uint4 *>(wt + (int64_t)(k0 + kr) * N + nn) =
-                    *reinterpret_cast<const uint4 *>(&tile[kr][8 * ch]);
+                    *reinterpret_cast<const uint4 *>(&tile[kr][4 * ch]);
         }
         __syncthreads();
     }
