@@ -285,12 +285,12 @@ class Sets:
         cr.cr_w4a8_gemv(self.xq[r], self.xs[r], self.q[r], self.s[r], self.cb, self.ws[r], m=M, out=self.out[r])
 
     def e2e_step(self, i):
-        """Through the public API (a W4A8Linear layer, buffers checked once) with
-        host buffers: H2D of x, forward, D2H of y."""
+        """Through the public API with host buffers: a prepared W4A8Linear
+        layer's forward_host (the C-ABI call cr_w4a8_plan_forward_host), which
+        queues the H2D copy of x from pinned memory, the forward and the D2H
+        copy of y."""
         r = i % self.R
-        self.x[r].copy_(self.x_host, non_blocking=True)
-        self.lin[r](self.x[r], out=self.out[r], xq_work=self.xq[r], xs_work=self.xs[r])
-        self.out_host.copy_(self.out[r], non_blocking=True)
+        self.lin[r].forward_host(self.x_host, self.out_host, self.x[r], self.out[r], self.xq[r], self.xs[r])
 
 
 def upload_graph(g, stream):

@@ -403,6 +403,41 @@ cr_status cr_w4a8_dequant_t_bf16(const uint8_t *qdata, const uint8_t *srel, cons
                                  const float *s_channel, int64_t N, int64_t K, uint16_t *wt, cr_stream_t stream);
 
 /*
+ * (14) A prepared layer for repeated forwards (serving loops).
+ *
+ * The same computation as (6) for one layer, with its arguments checked and
+ * the decode GEMV's weight tensor maps encoded once, at plan creation; the
+ * activation map is re-encoded only when the work buffer or M changes.  The
+ * pages' ConvRotW4A8Quantizer likewise prepares a layer's buffers once
+ * (attach_) and reuses them on every forward.
+ *
+ * cr_w4a8_plan_create: the layer as in (3), act_qmax and out_dtype as in (6);
+ *   the buffers must stay valid and unchanged while the plan exists.  The plan
+ *   belongs to the device current at creation; *plan is written.
+ * cr_w4a8_plan_forward: (6) on that device with the plan's layer: x [M, K]
+ *   bf16, out [M, N], xq_work / xs_work as in (6).  Calls on one plan may come
+ *   from several host threads.
+ * cr_w4a8_plan_forward_host: the same with x and out in HOST memory (pinned
+ *   memory lets the copies run asynchronously): queues the copy of x_host
+ *   [M, K] into x_dev, the forward into out_dev [M, N], and the copy of out_dev
+ *   into out_host, all on `stream`; out_host is valid once the stream has
+ *   reached that point.  x_dev, out_dev, xq_work and xs_work are device
+ *   buffers of the caller.
+ * cr_w4a8_plan_destroy: frees the plan (NULL is allowed).
+ * Errors as in (6); a plan used on another device gives CR_ERR_INVALID_ARG.
+ */
+typedef struct cr_w4a8_plan_st *cr_w4a8_plan;
+cr_status cr_w4a8_plan_create(const uint8_t *qdata, const uint8_t *srel, const float *codebook,
+                              const float *s_channel, const float *bias, int64_t N, int64_t K, int act_qmax,
+                              cr_out_dtype out_dtype, cr_w4a8_plan *plan);
+cr_status cr_w4a8_plan_forward(cr_w4a8_plan plan, const uint16_t *x, int64_t M, void *out, int8_t *xq_work,
+                               float *xs_work, cr_stream_t stream);
+cr_status cr_w4a8_plan_forward_host(cr_w4a8_plan plan, const uint16_t *x_host, int64_t M, void *out_host,
+                                    uint16_t *x_dev, void *out_dev, int8_t *xq_work, float *xs_work,
+                                    cr_stream_t stream);
+cr_status cr_w4a8_plan_destroy(cr_w4a8_plan plan);
+
+/*
  * Waits for `stream`, then reads and clears the library's device error word,
  * which a kernel sets when one of its bounded pipeline waits runs out (the
  * kernel then abandons its tile and exits; its outputs are unspecified).

@@ -31,7 +31,8 @@ def test_header_declares_the_boundary():
               "cr_w4a8_linear", "cr_status_string", "cr_check_device_error", "cr_version",
               "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped", "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu",
               "cr_w4a8_linear_swiglu", "cr_interleave_rows", "cr_w4a8_quantize_rotated", "cr_w4a8_assign_codes",
-              "cr_w4a8_ste_backward", "cr_w4a8_dequant_t_bf16"):
+              "cr_w4a8_ste_backward", "cr_w4a8_dequant_t_bf16", "cr_w4a8_plan_create", "cr_w4a8_plan_forward",
+              "cr_w4a8_plan_forward_host", "cr_w4a8_plan_destroy"):
         assert n in names
 
 
@@ -221,6 +222,20 @@ def test_backward_validation(L):
     assert g(A16, A16, A16, A16, 12, 256, A16, None) == cr.CR_ERR_UNSUPPORTED
     assert g(A16, A16, MIS, A16, 8, 256, A16, None) == cr.CR_ERR_ALIGNMENT
     assert g(None, None, None, None, 0, 256, None, None) == cr.CR_OK
+
+
+def test_plan_validation(L):
+    plan = ctypes.c_void_p()
+    f = L.cr_w4a8_plan_create
+    assert f(A16, A16, A16, A16, None, 8, 256, 0, 0, ctypes.byref(plan)) == cr.CR_ERR_INVALID_ARG   # act_qmax
+    assert f(A16, A16, A16, A16, None, 8, 256, 127, 9, ctypes.byref(plan)) == cr.CR_ERR_INVALID_ARG  # out dtype
+    assert f(A16, A16, A16, A16, None, 8, 320, 127, 0, ctypes.byref(plan)) == cr.CR_ERR_UNSUPPORTED
+    assert f(None, A16, A16, A16, None, 8, 256, 127, 0, ctypes.byref(plan)) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, MIS, A16, A16, None, 8, 256, 127, 0, ctypes.byref(plan)) == cr.CR_ERR_ALIGNMENT
+    assert f(A16, A16, A16, A16, None, 8, 256, 127, 0, None) == cr.CR_ERR_INVALID_ARG
+    assert L.cr_w4a8_plan_forward(None, A16, 2, A16, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert L.cr_w4a8_plan_forward_host(None, A16, 2, A16, A16, A16, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert L.cr_w4a8_plan_destroy(None) == cr.CR_OK
 
 
 def test_valid_call_without_a_gpu_fails_loudly(L):

@@ -258,6 +258,40 @@ def test_w4a8_linear_layer_object(M):
         lin(bf16_dev(inputs.activations(M, 512, 1)))
     with pytest.raises(ValueError):
         lin(x, xq_work=torch.empty(cr.gemv_rows(M) if M <= 8 else M, K, dtype=torch.int8))  # host tensor
+    # through host buffers: copy in, forward, copy out on one stream, with
+    # new contents in the same host buffer on the last call
+    x_host = x.cpu().pin_memory()
+    out_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    x_dev, out_dev = torch.empty_like(x), torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    for rep in range(3):
+        if rep == 2:
+            x2 = bf16_dev(inputs.activations(M, K, 190 + M))
+            x_host.copy_(x2.cpu())
+            y2 = cr.cr_w4a8_linear(x2, q, s, cb, ws, b)
+        out_host.zero_()
+        lin.forward_host(x_host, out_host, x_dev, out_dev)
+        torch.cuda.synchronize()
+        assert torch.equal(out_host.view(torch.int16), y2.cpu().view(torch.int16)), rep
+
+
+def test_plan_reencodes_the_activation_map_when_buffers_change():
+    """A prepared layer re-encodes its cached activation map whenever the work
+    buffer or M changes: alternating two work buffers and several M on one
+    layer gives every call the output of a fresh cr_w4a8_linear."""
+    N, K = 1000, 2048
+    layer = inputs.layer(N, K, 95)
+    q, s, cb, ws, _ = _layer_dev(layer)
+    lin = cr.W4A8Linear(q, s, cb, ws)
+    works = [(torch.empty(8, K, dtype=torch.int8, device="cuda"), torch.empty(8, device="cuda")) for _ in range(2)]
+    for i, M in enumerate([1, 8, 8, 3, 5, 2, 8, 1, 7]):
+        x = bf16_dev(inputs.activations(M, K, 200 + i))
+        xq, xs = works[i % 2] if i < 6 else works[0]
+        y = lin(x, xq_work=xq, xs_work=xs)
+        ref = cr.cr_w4a8_linear(x, q, s, cb, ws)
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16)), (i, M)
+    f32 = cr.W4A8Linear(q, s, cb, ws, out_dtype=torch.float32)
+    x = bf16_dev(inputs.activations(4, K, 300))
+    assert torch.equal(f32(x), cr.cr_w4a8_linear(x, q, s, cb, ws, out_dtype=torch.float32))
 
 
 # ---------------------------------------------------------------- grouped decode (several layers, one input)

@@ -93,6 +93,10 @@ def lib() -> ctypes.CDLL:
             L.cr_w4a8_quantize_rotated.argtypes = [P, P, i64, i64, P, P, P, P]
             L.cr_w4a8_assign_codes.argtypes = [P, P, P, P, P, i64, i64, P, P]
             L.cr_w4a8_ste_backward.argtypes = [P, P, P, P, P, i64, i64, i64, P, P]
+            L.cr_w4a8_plan_create.argtypes = [P, P, P, P, P, i64, i64, i32, i32, ctypes.POINTER(P)]
+            L.cr_w4a8_plan_forward.argtypes = [P, P, i64, P, P, P, P]
+            L.cr_w4a8_plan_forward_host.argtypes = [P, P, i64, P, P, P, P, P, P]
+            L.cr_w4a8_plan_destroy.argtypes = [P]
             L.cr_w4a8_dequant_t_bf16.argtypes = [P, P, P, P, i64, i64, P, P]
             LP = ctypes.POINTER(CrLayer)
             L.cr_w4a8_gemv_grouped.argtypes = [P, P, P, i64, i64, LP, i32, i32, P]
@@ -309,21 +313,53 @@ def cr_w4a8_linear(x, qdata, srel, codebook, s_channel, bias=None, act_qmax: int
 
 
 class W4A8Linear:
-    """A layer whose buffers are checked once, for repeated forwards.
+    """A prepared layer for repeated forwards (cr_w4a8_plan_*).
 
     Holds qdata, srel, codebook, s_channel (and bias) as given (no copies) and
-    their device pointers; forward() checks only the activations, the output
-    and the work buffers, then makes the cr_w4a8_linear call.  The caller must
-    not resize or free the layer's tensors while the object is in use."""
+    a library plan over them: the layer is checked and the decode GEMV's
+    weight maps are encoded once, here.  forward() checks only the
+    activations, the output and the work buffers; forward_host() takes x and
+    the output in host memory and queues both copies with the forward.  The
+    caller must not resize or free the layer's tensors while the object is in
+    use."""
 
-    def __init__(self, qdata, srel, codebook, s_channel, bias=None, act_qmax: int = 127):
+    def __init__(self, qdata, srel, codebook, s_channel, bias=None, act_qmax: int = 127, out_dtype=None):
+        torch = _torch()
         self.N, self.K = _layer(qdata, srel, codebook, s_channel, bias)
         if not 1 <= int(act_qmax) <= 127:
             raise ValueError("act_qmax must be in 1..127")
         self.act_qmax = int(act_qmax)
+        self.out_dtype = out_dtype or torch.bfloat16
         self._tensors = (qdata, srel, codebook, s_channel, bias)  # keep them alive
-        self._ptrs = (_ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), _ptr(bias))
-        self._fn = lib().cr_w4a8_linear
+        self._L = lib()
+        handle = ctypes.c_void_p()
+        with torch.cuda.device(qdata.device):
+            _check(self._L.cr_w4a8_plan_create(_ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel),
+                                               _ptr(bias), self.N, self.K, self.act_qmax, _out_code(self.out_dtype),
+                                               ctypes.byref(handle)), "cr_w4a8_plan_create")
+        self._plan = handle
+        self._fwd = self._L.cr_w4a8_plan_forward
+        self._fwd_host = self._L.cr_w4a8_plan_forward_host
+
+    def __del__(self):
+        plan = getattr(self, "_plan", None)
+        if plan is not None and plan.value:
+            self._L.cr_w4a8_plan_destroy(plan)
+            self._plan = None
+
+    def _work(self, x, M, xq_work, xs_work):
+        torch = _torch()
+        rows = gemv_rows(M) if 1 <= M <= CR_GEMV_MAX_M else M
+        if xq_work is None:
+            xq_work = torch.empty(rows, self.K, dtype=torch.int8, device=x.device)
+        elif not xq_work.is_cuda or xq_work.dtype != torch.int8 or xq_work.dim() != 2 or xq_work.shape[0] < rows \
+                or xq_work.shape[1] != self.K or not xq_work.is_contiguous():
+            raise ValueError(f"xq_work must be a contiguous CUDA int8 [>= {rows}, {self.K}] tensor")
+        if xs_work is None:
+            xs_work = torch.empty(rows, dtype=torch.float32, device=x.device)
+        elif not xs_work.is_cuda or xs_work.dtype != torch.float32 or xs_work.dim() != 1 or xs_work.shape[0] < rows:
+            raise ValueError(f"xs_work must be a CUDA float32 [>= {rows}] tensor")
+        return xq_work, xs_work
 
     def forward(self, x, out=None, xq_work=None, xs_work=None, stream=None):
         torch = _torch()
@@ -331,25 +367,38 @@ class W4A8Linear:
         M, K = x.shape
         if K != self.K:
             raise ValueError(f"x has K={K}, the layer K={self.K}")
-        rows = gemv_rows(M) if 1 <= M <= CR_GEMV_MAX_M else M
-        if xq_work is None:
-            xq_work = torch.empty(rows, K, dtype=torch.int8, device=x.device)
-        elif not xq_work.is_cuda or xq_work.dtype != torch.int8 or xq_work.dim() != 2 or xq_work.shape[0] < rows \
-                or xq_work.shape[1] != K or not xq_work.is_contiguous():
-            raise ValueError(f"xq_work must be a contiguous CUDA int8 [>= {rows}, {K}] tensor")
-        if xs_work is None:
-            xs_work = torch.empty(rows, dtype=torch.float32, device=x.device)
-        elif not xs_work.is_cuda or xs_work.dtype != torch.float32 or xs_work.dim() != 1 or xs_work.shape[0] < rows:
-            raise ValueError(f"xs_work must be a CUDA float32 [>= {rows}] tensor")
+        xq_work, xs_work = self._work(x, M, xq_work, xs_work)
         if out is None:
-            out = torch.empty(M, self.N, dtype=torch.bfloat16, device=x.device)
-        _need(out, "out", (torch.bfloat16, torch.float32), shape=(M, self.N))
-        q, s, cb, ws, b = self._ptrs
-        _check(self._fn(x.data_ptr(), q, s, cb, ws, b, M, self.N, K, self.act_qmax, _out_code(out.dtype),
-                        out.data_ptr(), xq_work.data_ptr(), xs_work.data_ptr(), _stream(stream)), "cr_w4a8_linear")
+            out = torch.empty(M, self.N, dtype=self.out_dtype, device=x.device)
+        _need(out, "out", (self.out_dtype,), shape=(M, self.N))
+        _check(self._fwd(self._plan, x.data_ptr(), M, out.data_ptr(), xq_work.data_ptr(), xs_work.data_ptr(),
+                         _stream(stream)), "cr_w4a8_plan_forward")
         return out
 
     __call__ = forward
+
+    def forward_host(self, x_host, out_host, x_dev, out_dev, xq_work=None, xs_work=None, stream=None):
+        """x_host [M, K] bf16 and out_host [M, N] in host memory (pinned for
+        asynchronous copies), x_dev / out_dev their device buffers: queues the
+        copy in, the forward and the copy out on the stream; out_host is ready
+        once the stream has reached that point."""
+        torch = _torch()
+        if x_host.is_cuda or out_host.is_cuda:
+            raise ValueError("x_host and out_host must be host tensors")
+        if x_host.dtype != torch.bfloat16 or x_host.dim() != 2 or not x_host.is_contiguous():
+            raise ValueError("x_host must be a contiguous bf16 [M, K] tensor")
+        M, K = x_host.shape
+        if K != self.K:
+            raise ValueError(f"x has K={K}, the layer K={self.K}")
+        if out_host.dtype != self.out_dtype or tuple(out_host.shape) != (M, self.N) or not out_host.is_contiguous():
+            raise ValueError(f"out_host must be a contiguous {self.out_dtype} [{M}, {self.N}] tensor")
+        _need(x_dev, "x_dev", (torch.bfloat16,), shape=(M, K))
+        _need(out_dev, "out_dev", (self.out_dtype,), shape=(M, self.N))
+        xq_work, xs_work = self._work(x_dev, M, xq_work, xs_work)
+        _check(self._fwd_host(self._plan, x_host.data_ptr(), M, out_host.data_ptr(), x_dev.data_ptr(),
+                              out_dev.data_ptr(), xq_work.data_ptr(), xs_work.data_ptr(), _stream(stream)),
+               "cr_w4a8_plan_forward_host")
+        return out_host
 
 
 def cr_w4a8_linear_decode_noalloc(x, qdata, srel, codebook, s_channel, bias=None, act_qmax: int = 127,

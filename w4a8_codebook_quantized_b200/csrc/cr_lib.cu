@@ -11,6 +11,7 @@
 #include <functional>
 #include <cstdint>
 #include <cstring>
+#include <new>
 #include <mutex>
 
 #include "cr_w4a8.h"
@@ -182,25 +183,30 @@ bool make_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype,
 // tiles of all layers are numbered one after the other and run on a
 // persistent grid of as many CTAs as fit on the SMs, optionally as a
 // programmatic dependent of the previous kernel on the stream.
+// The activation map of the decode GEMV over xq [>= M, K] (a stage's box of
+// 8 rows x 1024 columns lands as [slice][token][128 B], 128-byte swizzle).
+bool encode_gemv_x_map(CUtensorMap *map, const int8_t *xq, int64_t M, int64_t K)
+{
+    const uint64_t uK = (uint64_t)K;
+    return make_tmap_3d(map, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, {(uint64_t)cr::gv::kSlice, (uint64_t)M,
+                                                                   uK / cr::gv::kSlice},
+                        {uK, (uint64_t)cr::gv::kSlice},
+                        {(uint32_t)cr::gv::kSlice, (uint32_t)cr::gv::kTokens,
+                         (uint32_t)(cr::gv::kChunk / cr::gv::kSlice)},
+                        true);
+}
+
+// Everything of a GEMV launch's arguments but the activations (tm_x, xs, M).
+// `tiles` returns the row tiles of all layers (0: nothing to launch).
 template <int L>
-cr_status launch_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const float *codebook,
-                      int64_t M, int64_t K, const cr_w4a8_layer *layers, int num_layers, cr_out_dtype out_dtype,
-                      cudaStream_t stream, bool pdl, int swiglu = 0)
+cr_status build_gemv_args(cr::gv::GemvArgs<L> &args, const float *codebook, int64_t K, const cr_w4a8_layer *layers,
+                          int num_layers, cr_out_dtype out_dtype, int swiglu, int64_t &tiles)
 {
     using namespace cr;
     using C = gv::Prod;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(gv::gemv_kernel<C, L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)C::kSmemBytes) != cudaSuccess) {
-            cudaGetLastError();
-            return CR_ERR_CUDA;
-        }
-        attr_set = true;
-    }
-    gv::GemvArgs<L> args;
     memset(&args, 0, sizeof(args));
-    const uint64_t uK = (uint64_t)K, uM = (uint64_t)M;
-    int64_t tiles = 0;
+    const uint64_t uK = (uint64_t)K;
+    tiles = 0;
     for (int l = 0; l < num_layers; ++l) {
         const cr_w4a8_layer &ly = layers[l];
         args.layer[l].tile0 = (int)tiles;
@@ -220,29 +226,41 @@ cr_status launch_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float
         args.layer[l].swiglu = swiglu;
         tiles += (ly.N + gv::kRows - 1) / gv::kRows;
     }
-    if (tiles == 0)
-        return CR_OK;
     if (tiles > INT_MAX)
         return CR_ERR_UNSUPPORTED;
-    if (!make_tmap_3d(&args.tm_x, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, {(uint64_t)gv::kSlice, uM, uK / gv::kSlice},
-                      {uK, (uint64_t)gv::kSlice},
-                      {(uint32_t)gv::kSlice, (uint32_t)gv::kTokens, (uint32_t)(gv::kChunk / gv::kSlice)}, true))
-        return CR_ERR_CUDA;
-    args.xs = xs;
     args.codebook = codebook;
-    args.M = (int)M;
     args.K = (int)K;
     args.num_layers = num_layers;
     args.num_tiles = (int)tiles;
     args.out_f32 = out_dtype == CR_OUT_F32 ? 1 : 0;
     args.lut_step = (uint32_t)(C::kCopies * sizeof(uint4));
     args.ahead = gv::kPrefetchAhead;
+    return CR_OK;
+}
+
+// Launch the decode GEMV with complete arguments: a persistent grid of as
+// many CTAs as fit on the SMs, optionally as a programmatic dependent of the
+// previous kernel on the stream.
+template <int L>
+cr_status launch_gemv_args(int num_sms, bool &attr_set, const cr::gv::GemvArgs<L> &args, cudaStream_t stream,
+                           bool pdl)
+{
+    using namespace cr;
+    using C = gv::Prod;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(gv::gemv_kernel<C, L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)C::kSmemBytes) != cudaSuccess) {
+            cudaGetLastError();
+            return CR_ERR_CUDA;
+        }
+        attr_set = true;
+    }
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     // persistent grid of several CTAs per SM, at most one wave
     const int64_t slots = (int64_t)C::kMinBlocks * num_sms;
-    const int64_t grid = tiles < slots ? tiles : slots;
+    const int64_t grid = args.num_tiles < slots ? args.num_tiles : slots;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(gv::kThreads);
@@ -251,6 +269,23 @@ cr_status launch_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
     return launched(cudaLaunchKernelEx(&cfg, gv::gemv_kernel<C, L>, args));
+}
+
+template <int L>
+cr_status launch_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const float *codebook,
+                      int64_t M, int64_t K, const cr_w4a8_layer *layers, int num_layers, cr_out_dtype out_dtype,
+                      cudaStream_t stream, bool pdl, int swiglu = 0)
+{
+    cr::gv::GemvArgs<L> args;
+    int64_t tiles = 0;
+    cr_status st = build_gemv_args<L>(args, codebook, K, layers, num_layers, out_dtype, swiglu, tiles);
+    if (st != CR_OK || tiles == 0)
+        return st;
+    if (!encode_gemv_x_map(&args.tm_x, xq, M, K))
+        return CR_ERR_CUDA;
+    args.xs = xs;
+    args.M = (int)M;
+    return launch_gemv_args<L>(num_sms, attr_set, args, stream, pdl);
 }
 
 
@@ -484,6 +519,24 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
 }
 
 }  // namespace
+
+// A prepared layer (cr_w4a8_plan_*): the validated layer, its device, and
+// the decode GEMV's arguments with the weight maps encoded; tm_x holds the
+// activation map of (xmap_base, xmap_M) once a forward has set it.
+struct cr_w4a8_plan_st {
+    int device = -1;
+    DeviceState *d = nullptr;
+    const uint8_t *qdata = nullptr, *srel = nullptr;
+    const float *codebook = nullptr, *s_channel = nullptr, *bias = nullptr;
+    int64_t N = 0, K = 0;
+    int act_qmax = 127;
+    cr_out_dtype out_dtype = CR_OUT_BF16;
+    cr::gv::GemvArgs<1> gemv;
+    int64_t tiles = 0;
+    const int8_t *xmap_base = nullptr;
+    int64_t xmap_M = -1;
+    std::mutex mu;
+};
 
 extern "C" {
 
@@ -877,6 +930,147 @@ cr_status cr_w4a8_assign_codes(const float *w_rot, const uint8_t *srel, const fl
         return st;
     return launched(
         cr::qz::launch_assign(w_rot, srel, s_channel, codebook, rand, N, (int)K, qdata, d->num_sms, stream));
+}
+
+cr_status cr_w4a8_plan_create(const uint8_t *qdata, const uint8_t *srel, const float *codebook,
+                              const float *s_channel, const float *bias, int64_t N, int64_t K, int act_qmax,
+                              cr_out_dtype out_dtype, cr_w4a8_plan *plan)
+{
+    if (!plan)
+        return CR_ERR_INVALID_ARG;
+    *plan = nullptr;
+    if (N < 0 || K < 0 || act_qmax < 1 || act_qmax > 127)
+        return CR_ERR_INVALID_ARG;
+    if (out_dtype != CR_OUT_BF16 && out_dtype != CR_OUT_F32)
+        return CR_ERR_INVALID_ARG;
+    cr_status st = check_k(K);
+    if (st != CR_OK)
+        return st;
+    if (N > INT_MAX)
+        return CR_ERR_UNSUPPORTED;
+    if (N > 0) {
+        if (!qdata || !srel || !codebook || !s_channel)
+            return CR_ERR_INVALID_ARG;
+        if (!aligned16(qdata) || !aligned16(srel) || !aligned16(codebook) || !aligned16(s_channel) ||
+            (bias && !aligned16(bias)))
+            return CR_ERR_ALIGNMENT;
+    }
+    DeviceState *d = nullptr;
+    st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    cr_w4a8_plan_st *p = new (std::nothrow) cr_w4a8_plan_st;
+    if (!p)
+        return CR_ERR_CUDA;
+    cudaGetDevice(&p->device);
+    p->d = d;
+    p->qdata = qdata;
+    p->srel = srel;
+    p->codebook = codebook;
+    p->s_channel = s_channel;
+    p->bias = bias;
+    p->N = N;
+    p->K = K;
+    p->act_qmax = act_qmax;
+    p->out_dtype = out_dtype;
+    if (N > 0) {
+        cr_w4a8_layer ly{qdata, srel, s_channel, bias, N, nullptr, nullptr};
+        st = build_gemv_args<1>(p->gemv, codebook, K, &ly, 1, out_dtype, 0, p->tiles);
+        if (st != CR_OK) {
+            delete p;
+            return st;
+        }
+    }
+    *plan = p;
+    return CR_OK;
+}
+
+cr_status cr_w4a8_plan_destroy(cr_w4a8_plan plan)
+{
+    delete plan;
+    return CR_OK;
+}
+
+cr_status cr_w4a8_plan_forward(cr_w4a8_plan plan, const uint16_t *x, int64_t M, void *out, int8_t *xq_work,
+                               float *xs_work, cr_stream_t stream)
+{
+    if (!plan || M < 0)
+        return CR_ERR_INVALID_ARG;
+    if (M > INT_MAX)
+        return CR_ERR_UNSUPPORTED;
+    if (M == 0 || plan->N == 0)
+        return CR_OK;
+    if (!x || !out || !xq_work || !xs_work)
+        return CR_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(out) || !aligned16(xq_work) || !aligned16(xs_work))
+        return CR_ERR_ALIGNMENT;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != plan->device) {
+        cudaGetLastError();
+        return CR_ERR_INVALID_ARG;
+    }
+    if (M > CR_GEMV_MAX_M)
+        return linear_impl(x, plan->qdata, plan->srel, plan->codebook, plan->s_channel, plan->bias, M, plan->N,
+                           plan->K, plan->act_qmax, plan->out_dtype, out, xq_work, xs_work, stream, 0);
+    int64_t MP = 1;
+    while (MP < M)
+        MP <<= 1;
+    cr_status st = launched(cr::rq::launch(x, M, plan->K, MP, plan->act_qmax, xq_work, xs_work, stream));
+    if (st != CR_OK)
+        return st;
+    cr::gv::GemvArgs<1> args;
+    {
+        std::lock_guard<std::mutex> lock(plan->mu);
+        if (plan->xmap_base != xq_work || plan->xmap_M != M) {
+            if (!encode_gemv_x_map(&plan->gemv.tm_x, xq_work, M, plan->K))
+                return CR_ERR_CUDA;
+            plan->xmap_base = xq_work;
+            plan->xmap_M = M;
+        }
+        args = plan->gemv;
+    }
+    args.xs = xs_work;
+    args.M = (int)M;
+    args.layer[0].out = out;
+    return launch_gemv_args<1>(plan->d->num_sms, plan->d->gemv_attr_set, args, stream, /*pdl=*/true);
+}
+
+cr_status cr_w4a8_plan_forward_host(cr_w4a8_plan plan, const uint16_t *x_host, int64_t M, void *out_host,
+                                    uint16_t *x_dev, void *out_dev, int8_t *xq_work, float *xs_work,
+                                    cr_stream_t stream)
+{
+    if (!plan || M < 0)
+        return CR_ERR_INVALID_ARG;
+    if (M == 0 || plan->N == 0)
+        return CR_OK;
+    if (!x_host || !out_host)
+        return CR_ERR_INVALID_ARG;
+    const size_t xb = (size_t)(M * plan->K) * 2;
+    const size_t ob = (size_t)(M * plan->N) * (plan->out_dtype == CR_OUT_F32 ? 4 : 2);
+    // everything the forward checks, checked before the first copy is queued
+    if (!x_dev || !out_dev || !xq_work || !xs_work)
+        return CR_ERR_INVALID_ARG;
+    if (!aligned16(x_dev) || !aligned16(out_dev) || !aligned16(xq_work) || !aligned16(xs_work))
+        return CR_ERR_ALIGNMENT;
+    if (M > INT_MAX)
+        return CR_ERR_UNSUPPORTED;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != plan->device) {
+        cudaGetLastError();
+        return CR_ERR_INVALID_ARG;
+    }
+    if (cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return CR_ERR_CUDA;
+    }
+    const cr_status st = cr_w4a8_plan_forward(plan, x_dev, M, out_dev, xq_work, xs_work, stream);
+    if (st != CR_OK)
+        return st;
+    if (cudaMemcpyAsync(out_host, out_dev, ob, cudaMemcpyDeviceToHost, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return CR_ERR_CUDA;
+    }
+    return CR_OK;
 }
 
 cr_status cr_interleave_rows(const void *src, void *dst, int64_t rows, int64_t row_bytes, cr_stream_t stream)
