@@ -438,6 +438,17 @@ cr_status cr_w4a8_plan_forward_host(cr_w4a8_plan plan, const uint16_t *x_host, i
 cr_status cr_w4a8_plan_destroy(cr_w4a8_plan plan);
 
 /*
+ * (15) Self-test of the failure path: launches one CTA whose thread waits,
+ * with the library's bounded wait, on an mbarrier that nothing completes.
+ * After limit_ns (1 ms .. 1 s, CR_ERR_INVALID_ARG otherwise) the wait gives
+ * up, sets the device error word exactly as a stalled pipeline would, and
+ * the kernel returns; cr_check_device_error then reports CR_ERR_TIMEOUT and
+ * clears the word.  No fault, trap or hang is involved and the context stays
+ * usable.
+ */
+cr_status cr_selftest_wait_timeout(uint64_t limit_ns, cr_stream_t stream);
+
+/*
  * Waits for `stream`, then reads and clears the library's device error word,
  * which a kernel sets when one of its bounded pipeline waits runs out (the
  * kernel then abandons its tile and exits; its outputs are unspecified).

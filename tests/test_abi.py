@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
               "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped", "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu",
               "cr_w4a8_linear_swiglu", "cr_interleave_rows", "cr_w4a8_quantize_rotated", "cr_w4a8_assign_codes",
               "cr_w4a8_ste_backward", "cr_w4a8_dequant_t_bf16", "cr_w4a8_plan_create", "cr_w4a8_plan_forward",
-              "cr_w4a8_plan_forward_host", "cr_w4a8_plan_destroy"):
+              "cr_w4a8_plan_forward_host", "cr_w4a8_plan_destroy", "cr_selftest_wait_timeout"):
         assert n in names
 
 
@@ -236,6 +236,11 @@ def test_plan_validation(L):
     assert L.cr_w4a8_plan_forward(None, A16, 2, A16, A16, A16, None) == cr.CR_ERR_INVALID_ARG
     assert L.cr_w4a8_plan_forward_host(None, A16, 2, A16, A16, A16, A16, A16, None) == cr.CR_ERR_INVALID_ARG
     assert L.cr_w4a8_plan_destroy(None) == cr.CR_OK
+
+
+def test_selftest_validation(L):
+    assert L.cr_selftest_wait_timeout(10, None) == cr.CR_ERR_INVALID_ARG        # below 1 ms
+    assert L.cr_selftest_wait_timeout(2 * 10 ** 9, None) == cr.CR_ERR_INVALID_ARG  # above 1 s
 
 
 def test_valid_call_without_a_gpu_fails_loudly(L):

@@ -584,3 +584,24 @@ def test_ste_backward_empty_layer_gives_zero():
     cr.cr_w4a8_ste_backward(torch.empty(4, 0, dtype=torch.bfloat16, device="cuda"), q[:0], s[:0], cb, ws[:0], dx=dx)
     torch.cuda.synchronize()
     assert not dx.float().abs().sum().item()
+
+
+# ---------------------------------------------------------------- failure detection
+
+def test_bounded_wait_runs_out_and_is_reported():
+    """A wait that nothing completes gives up after its limit, the host reads
+    CR_ERR_TIMEOUT once (the word is cleared), and the context keeps working."""
+    cr.cr_check_device_error()
+    cr.cr_selftest_wait_timeout(0.005)
+    with pytest.raises(cr.CrError) as err:
+        cr.cr_check_device_error()
+    assert err.value.status == cr.CR_ERR_TIMEOUT
+    cr.cr_check_device_error()  # cleared
+    layer = inputs.layer(256, 1024, 7)
+    q, s, cb, ws, _ = _layer_dev(layer)
+    x = bf16_dev(inputs.activations(4, 1024, 7))
+    xq, xs = cr.cr_rotate_quant_act(x, 4)
+    o1, a1 = cr.cr_w4a8_gemv(xq, xs, q, s, cb, ws, m=4, acc_out=True)
+    o2, a2 = cr.cr_w4a8_gemm(xq, xs, q, s, cb, ws, m=4, acc_out=True)
+    cr.cr_check_device_error()
+    assert torch.equal(a1, a2)

@@ -29,7 +29,7 @@ __all__ = [
     "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped", "CrLayer",
     "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu", "cr_w4a8_linear_swiglu", "cr_interleave_rows",
     "interleave_gate_up", "cr_w4a8_quantize_rotated", "cr_w4a8_assign_codes",
-    "cr_w4a8_ste_backward", "cr_w4a8_dequant_t_bf16",
+    "cr_w4a8_ste_backward", "cr_w4a8_dequant_t_bf16", "cr_selftest_wait_timeout",
     "cr_status_string", "cr_version",
     "gemv_rows",
 ]
@@ -97,6 +97,7 @@ def lib() -> ctypes.CDLL:
             L.cr_w4a8_plan_forward.argtypes = [P, P, i64, P, P, P, P]
             L.cr_w4a8_plan_forward_host.argtypes = [P, P, i64, P, P, P, P, P, P]
             L.cr_w4a8_plan_destroy.argtypes = [P]
+            L.cr_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
             L.cr_w4a8_dequant_t_bf16.argtypes = [P, P, P, P, i64, i64, P, P]
             LP = ctypes.POINTER(CrLayer)
             L.cr_w4a8_gemv_grouped.argtypes = [P, P, P, i64, i64, LP, i32, i32, P]
@@ -685,6 +686,12 @@ def cr_w4a8_dequant_t_bf16(qdata, srel, codebook, s_channel, wt=None, stream=Non
     _check(lib().cr_w4a8_dequant_t_bf16(_ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), N, K, _ptr(wt),
                                         _stream(stream)), "cr_w4a8_dequant_t_bf16")
     return wt
+
+
+def cr_selftest_wait_timeout(seconds: float = 0.005, stream=None) -> None:
+    """Queue a bounded wait that nothing completes; after `seconds` it sets the
+    device error word, which cr_check_device_error then reports."""
+    _check(lib().cr_selftest_wait_timeout(int(seconds * 1e9), _stream(stream)), "cr_selftest_wait_timeout")
 
 
 def cr_check_device_error(stream=None) -> None:

@@ -1255,6 +1255,18 @@ cr_status cr_w4a8_linear_decode_noalloc(const uint16_t *x, const uint8_t *qdata,
                     out_dtype, out, nullptr, stream, /*pdl=*/true);
 }
 
+cr_status cr_selftest_wait_timeout(uint64_t limit_ns, cr_stream_t stream)
+{
+    if (limit_ns < 1000000ull || limit_ns > 1000000000ull)
+        return CR_ERR_INVALID_ARG;
+    DeviceState *d = nullptr;
+    const cr_status st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    cr::ew::selftest_timeout_kernel<<<1, 32, 0, stream>>>(limit_ns);
+    return launched(cudaGetLastError());
+}
+
 cr_status cr_check_device_error(cr_stream_t stream)
 {
     DeviceState *d = nullptr;

@@ -274,5 +274,25 @@ inline cudaError_t launch_dequant_t_bf16(const uint8_t *qdata, const uint8_t *sr
     return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------- failure-path self-test
+//
+// A wait that nothing completes: one thread initialises an mbarrier expecting
+// one arrival that never comes and waits for its first phase with the
+// library's bounded wait.  The wait runs out after limit_ns, sets the device
+// error word (as any of the pipelines' waits would) and the kernel returns:
+// the error path is exercised without a fault, a trap or a hang.
+__global__ void selftest_timeout_kernel(uint64_t limit_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        volatile int *ab = &abort_flag;
+        mbar_wait_bounded(&bar, 0u, ab, limit_ns);
+    }
+}
+
 }  // namespace ew
 }  // namespace cr
