@@ -152,6 +152,14 @@ def test_gemv(M, N, K):
     _contraction_case(cr.cr_w4a8_gemv, M, N, K, seed=M + N + K)
 
 
+@pytest.mark.parametrize("M,N,K", [(8, 8192, 8192), (3, 6000, 2048), (1, 5000, 256), (8, 12288, 4096),
+                                   (5, 4752, 7936)])
+def test_gemv_several_tiles_per_cta(M, N, K):
+    """More row tiles than CTA slots: CTAs walk several tiles, their rings
+    running across tile boundaries (chunk counts 1 to 8)."""
+    _contraction_case(cr.cr_w4a8_gemv, M, N, K, seed=M + N + K)
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 256, 256), (8, 256, 512), (100, 300, 1024), (128, 256, 256),
                                    (129, 257, 256), (300, 1000, 1024), (256, 4096, 2048), (2048, 512, 4096),
                                    (17, 17, 768), (640, 1536, 1280)])
