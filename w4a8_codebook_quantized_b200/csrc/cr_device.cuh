@@ -145,20 +145,11 @@ __device__ __forceinline__ uint32_t to_bf16x2_bits(float lo, float hi)
 
 // ---------------------------------------------------------------- loads
 
-// 16-byte streaming load that bypasses L1 (weights are read once).
+// 8-byte streaming load that bypasses L1 (weights are read once).
 __device__ __forceinline__ uint2 ldg_stream8(const void *p)
 {
     uint2 v;
     asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-    return v;
-}
-
-__device__ __forceinline__ uint4 ldg_stream16(const void *p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
     return v;
 }
 
