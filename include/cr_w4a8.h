@@ -438,6 +438,20 @@ cr_status cr_w4a8_plan_forward_host(cr_w4a8_plan plan, const uint16_t *x_host, i
 cr_status cr_w4a8_plan_destroy(cr_w4a8_plan plan);
 
 /*
+ * (16) The prefill contraction on an int8 weight already on the grid.
+ *
+ * Defined by: ai-toolkit convrot_w4a8_quant.py, _w4a8_linear_ste_op after
+ * its unpack: torch._int_mm(aq, w8.t()) and the epilogue, i.e. (3) without
+ * the decode.  w8 [N, K] int8 (from (2), or a weight a caller keeps decoded
+ * across calls, trading 8 bits per weight of memory for the decode); the
+ * other arguments as in (3), and the results equal those of (3) on the same
+ * layer bit for bit.
+ */
+cr_status cr_gemm_s8(const int8_t *xq, const float *xs, const int8_t *w8, const float *s_channel,
+                     const float *bias, int64_t M, int64_t N, int64_t K, cr_out_dtype out_dtype, void *out,
+                     int32_t *acc_out, cr_stream_t stream);
+
+/*
  * (15) Self-test of the failure path: launches one CTA whose thread waits,
  * with the library's bounded wait, on an mbarrier that nothing completes.
  * After limit_ns (1 ms .. 1 s, CR_ERR_INVALID_ARG otherwise) the wait gives

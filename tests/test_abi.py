@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
               "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped", "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu",
               "cr_w4a8_linear_swiglu", "cr_interleave_rows", "cr_w4a8_quantize_rotated", "cr_w4a8_assign_codes",
               "cr_w4a8_ste_backward", "cr_w4a8_dequant_t_bf16", "cr_w4a8_plan_create", "cr_w4a8_plan_forward",
-              "cr_w4a8_plan_forward_host", "cr_w4a8_plan_destroy", "cr_selftest_wait_timeout"):
+              "cr_w4a8_plan_forward_host", "cr_w4a8_plan_destroy", "cr_selftest_wait_timeout", "cr_gemm_s8"):
         assert n in names
 
 
@@ -86,6 +86,16 @@ def test_decode_validation(L):
     assert f(None, A16, A16, 4, 256, A16, None) == cr.CR_ERR_INVALID_ARG
     assert f(A16, MIS, A16, 4, 256, A16, None) == cr.CR_ERR_ALIGNMENT
     assert f(None, None, None, 0, 256, None, None) == cr.CR_OK
+
+
+def test_gemm_s8_validation(L):
+    f = L.cr_gemm_s8
+    assert f(A16, A16, A16, A16, None, -1, 8, 256, 0, A16, None, None) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, A16, A16, A16, None, 4, 8, 320, 0, A16, None, None) == cr.CR_ERR_UNSUPPORTED
+    assert f(A16, A16, None, A16, None, 4, 8, 256, 0, A16, None, None) == cr.CR_ERR_INVALID_ARG
+    assert f(A16, A16, MIS, A16, None, 4, 8, 256, 0, A16, None, None) == cr.CR_ERR_ALIGNMENT
+    assert f(A16, A16, A16, A16, None, 4, 8, 256, 3, A16, None, None) == cr.CR_ERR_INVALID_ARG
+    assert f(None, None, None, None, None, 0, 8, 256, 0, None, None, None) == cr.CR_OK
 
 
 @pytest.mark.parametrize("name", ["cr_w4a8_gemm", "cr_w4a8_gemv"])

@@ -176,6 +176,22 @@ def test_gemm_cta_pairs(M, N, K):
     _contraction_case(cr.cr_w4a8_gemm, M, N, K, seed=M + N + K, with_bias=(K == 768))
 
 
+@pytest.mark.parametrize("M,N,K", [(100, 300, 1024), (2048, 4096, 512), (129, 257, 256)])
+def test_gemm_s8_on_a_decoded_weight(M, N, K):
+    """The contraction on an int8 weight decoded beforehand equals
+    cr_w4a8_gemm on the packed layer bit for bit (1-CTA and CTA-pair tiles)."""
+    layer = inputs.layer(N, K, M + 3 * N, with_bias=True)
+    q, s, cb, ws, b = _layer_dev(layer)
+    x = bf16_dev(inputs.activations(M, K, M + 1))
+    xq, xs = cr.cr_rotate_quant_act(x)
+    w8 = cr.cr_w4a8_decode_int8(q, s, cb)
+    o1, a1 = cr.cr_gemm_s8(xq, xs, w8, ws, b, acc_out=True)
+    o2, a2 = cr.cr_w4a8_gemm(xq, xs, q, s, cb, ws, b, acc_out=True)
+    assert torch.equal(a1, a2) and torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    o3 = cr.cr_gemm_s8(xq, xs, w8, ws, b)  # the TMA-store epilogue path
+    assert torch.equal(o3.view(torch.int16), o2.view(torch.int16))
+
+
 @pytest.mark.parametrize("kind,with_bias", [("f32", False), ("f32", True), ("bf16", True)])
 def test_output_kinds_and_bias(kind, with_bias):
     _contraction_case(cr.cr_w4a8_gemv, 3, 520, 1024, 11, kind, with_bias)

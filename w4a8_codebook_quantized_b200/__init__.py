@@ -29,7 +29,7 @@ __all__ = [
     "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped", "CrLayer",
     "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu", "cr_w4a8_linear_swiglu", "cr_interleave_rows",
     "interleave_gate_up", "cr_w4a8_quantize_rotated", "cr_w4a8_assign_codes",
-    "cr_w4a8_ste_backward", "cr_w4a8_dequant_t_bf16", "cr_selftest_wait_timeout",
+    "cr_w4a8_ste_backward", "cr_w4a8_dequant_t_bf16", "cr_selftest_wait_timeout", "cr_gemm_s8",
     "cr_status_string", "cr_version",
     "gemv_rows",
 ]
@@ -98,6 +98,7 @@ def lib() -> ctypes.CDLL:
             L.cr_w4a8_plan_forward_host.argtypes = [P, P, i64, P, P, P, P, P, P]
             L.cr_w4a8_plan_destroy.argtypes = [P]
             L.cr_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
+            L.cr_gemm_s8.argtypes = [P, P, P, P, P, i64, i64, i64, i32, P, P, P]
             L.cr_w4a8_dequant_t_bf16.argtypes = [P, P, P, P, i64, i64, P, P]
             LP = ctypes.POINTER(CrLayer)
             L.cr_w4a8_gemv_grouped.argtypes = [P, P, P, i64, i64, LP, i32, i32, P]
@@ -263,6 +264,36 @@ def cr_w4a8_gemv(xq, xs, qdata, srel, codebook, s_channel, bias=None, m: Optiona
     torch = _torch()
     return _contraction("cr_w4a8_gemv", xq, xs, qdata, srel, codebook, s_channel, bias, m,
                         out_dtype or torch.bfloat16, out, acc_out, stream)
+
+
+def cr_gemm_s8(xq, xs, w8, s_channel, bias=None, m: Optional[int] = None, out_dtype=None, out=None, acc_out=None,
+               stream=None):
+    """The prefill contraction + epilogue on an int8 weight w8 [N, K] already
+    on the grid (cr_w4a8_gemm without its decode); acc_out=True also returns
+    the int32 accumulators."""
+    torch = _torch()
+    _need(w8, "w8", (torch.int8,), 2)
+    N, K = w8.shape
+    _need(s_channel, "s_channel", (torch.float32,), shape=(N,))
+    if bias is not None:
+        _need(bias, "bias", (torch.float32,), shape=(N,))
+    _need(xq, "xq", (torch.int8,), 2)
+    _need(xs, "xs", (torch.float32,), 1)
+    M = xq.shape[0] if m is None else int(m)
+    if xq.shape[1] != K or xq.shape[0] < M or xs.shape[0] < M:
+        raise ValueError(f"xq {tuple(xq.shape)} / xs {tuple(xs.shape)} do not match M={M}, K={K}")
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype or torch.bfloat16, device=xq.device)
+    _need(out, "out", (torch.bfloat16, torch.float32), shape=(M, N))
+    if acc_out is True:
+        acc_out = torch.empty(M, N, dtype=torch.int32, device=xq.device)
+    if acc_out is not None and acc_out is not False:
+        _need(acc_out, "acc_out", (torch.int32,), shape=(M, N))
+    else:
+        acc_out = None
+    _check(lib().cr_gemm_s8(_ptr(xq), _ptr(xs), _ptr(w8), _ptr(s_channel), _ptr(bias), M, N, K,
+                            _out_code(out.dtype), _ptr(out), _ptr(acc_out), _stream(stream)), "cr_gemm_s8")
+    return (out, acc_out) if acc_out is not None else out
 
 
 def cr_epilogue(acc, xs, s_channel, bias=None, out_dtype=None, out=None, stream=None):

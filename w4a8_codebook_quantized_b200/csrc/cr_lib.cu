@@ -398,15 +398,15 @@ cr_status side_stream(DeviceState &d)
     return CR_OK;
 }
 
-// The prefill contraction.  When `activations` is given (cr_w4a8_linear), it
-// launches the activation kernel on `stream` while the weight decode runs on
-// the device's side stream (the two are independent); the GEMM waits for both.
-cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
-                   const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K,
-                   cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream,
-                   const std::function<cr_status()> *activations = nullptr, int swiglu = 0)
+// The int8 contraction with the fused epilogue on an int8 weight w8 [N, K]
+// (already decoded): tcgen05 GEMM on CTA pairs (256 x 256 tiles) when there
+// is at least one tile per SM pair, otherwise one CTA per 128 x 256 tile.
+cr_status gemm_on_w8(DeviceState &d, const int8_t *xq, const float *xs, const int8_t *w8, const float *s_channel,
+                     const float *bias, int64_t M, int64_t N, int64_t K, cr_out_dtype out_dtype, void *out,
+                     int32_t *acc_out, cudaStream_t stream, int swiglu)
 {
     using namespace cr;
+    cr_status st = CR_OK;
     if (!d.gemm_attr_set) {
         if (cudaFuncSetAttribute(gm::gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)gm::kSmemBytes) != cudaSuccess) {
@@ -414,36 +414,6 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
             return CR_ERR_CUDA;
         }
         d.gemm_attr_set = true;
-    }
-    // The int8 grid of the weight, decoded once per call into a transient
-    // from the library's stream-ordered pool.
-    int8_t *w8 = nullptr;
-    if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&w8), (size_t)(N * K), d.pool, stream) != cudaSuccess) {
-        cudaGetLastError();
-        return CR_ERR_CUDA;
-    }
-    cr_status st = CR_OK;
-    if (activations != nullptr) {
-        st = side_stream(d);
-        if (st == CR_OK && (cudaEventRecord(d.fork, stream) != cudaSuccess ||
-                            cudaStreamWaitEvent(d.side, d.fork, 0) != cudaSuccess)) {
-            cudaGetLastError();
-            st = CR_ERR_CUDA;
-        }
-        if (st == CR_OK)
-            st = launched(ew::launch_decode(qdata, srel, codebook, N, K, w8, d.num_sms, d.side));
-        if (st == CR_OK && cudaEventRecord(d.join, d.side) != cudaSuccess) {
-            cudaGetLastError();
-            st = CR_ERR_CUDA;
-        }
-        if (st == CR_OK)
-            st = (*activations)();
-        if (st == CR_OK && cudaStreamWaitEvent(stream, d.join, 0) != cudaSuccess) {
-            cudaGetLastError();
-            st = CR_ERR_CUDA;
-        }
-    } else {
-        st = launched(ew::launch_decode(qdata, srel, codebook, N, K, w8, d.num_sms, stream));
     }
     CUtensorMap ta, tb, to;
     const int out_f32 = out_dtype == CR_OUT_F32;
@@ -468,8 +438,6 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
                 st = CR_ERR_CUDA;
         }
     }
-    // 256 x 256 tiles on CTA pairs when there is at least one per SM pair;
-    // otherwise 128 x 256 tiles on single CTAs.
     const int64_t pair_tiles = ((M + 255) / 256) * ((N + gm::BN - 1) / gm::BN);
     const bool use_pair = pair_tiles >= d.num_sms / 2;
     if (st == CR_OK && use_pair) {
@@ -510,6 +478,50 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
                                                                          acc_out);
         st = launched(cudaGetLastError());
     }
+    return st;
+}
+
+// The prefill contraction.  When `activations` is given (cr_w4a8_linear), it
+// launches the activation kernel on `stream` while the weight decode runs on
+// the device's side stream (the two are independent); the GEMM waits for both.
+cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                   const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K,
+                   cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream,
+                   const std::function<cr_status()> *activations = nullptr, int swiglu = 0)
+{
+    using namespace cr;
+    // The int8 grid of the weight, decoded once per call into a transient
+    // from the library's stream-ordered pool.
+    int8_t *w8 = nullptr;
+    if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&w8), (size_t)(N * K), d.pool, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return CR_ERR_CUDA;
+    }
+    cr_status st = CR_OK;
+    if (activations != nullptr) {
+        st = side_stream(d);
+        if (st == CR_OK && (cudaEventRecord(d.fork, stream) != cudaSuccess ||
+                            cudaStreamWaitEvent(d.side, d.fork, 0) != cudaSuccess)) {
+            cudaGetLastError();
+            st = CR_ERR_CUDA;
+        }
+        if (st == CR_OK)
+            st = launched(ew::launch_decode(qdata, srel, codebook, N, K, w8, d.num_sms, d.side));
+        if (st == CR_OK && cudaEventRecord(d.join, d.side) != cudaSuccess) {
+            cudaGetLastError();
+            st = CR_ERR_CUDA;
+        }
+        if (st == CR_OK)
+            st = (*activations)();
+        if (st == CR_OK && cudaStreamWaitEvent(stream, d.join, 0) != cudaSuccess) {
+            cudaGetLastError();
+            st = CR_ERR_CUDA;
+        }
+    } else {
+        st = launched(ew::launch_decode(qdata, srel, codebook, N, K, w8, d.num_sms, stream));
+    }
+    if (st == CR_OK)
+        st = gemm_on_w8(d, xq, xs, w8, s_channel, bias, M, N, K, out_dtype, out, acc_out, stream, swiglu);
     if (cudaFreeAsync(w8, stream) != cudaSuccess) {
         cudaGetLastError();
         if (st == CR_OK)
@@ -1253,6 +1265,33 @@ cr_status cr_w4a8_linear_decode_noalloc(const uint16_t *x, const uint8_t *qdata,
         return st;
     return run_gemv(ns->num_sms, ns->gemv_attr_set, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K,
                     out_dtype, out, nullptr, stream, /*pdl=*/true);
+}
+
+cr_status cr_gemm_s8(const int8_t *xq, const float *xs, const int8_t *w8, const float *s_channel, const float *bias,
+                     int64_t M, int64_t N, int64_t K, cr_out_dtype out_dtype, void *out, int32_t *acc_out,
+                     cr_stream_t stream)
+{
+    if (M < 0 || N < 0 || K < 0)
+        return CR_ERR_INVALID_ARG;
+    if (out_dtype != CR_OUT_BF16 && out_dtype != CR_OUT_F32)
+        return CR_ERR_INVALID_ARG;
+    cr_status st = check_k(K);
+    if (st != CR_OK)
+        return st;
+    if (M > INT_MAX || N > INT_MAX)
+        return CR_ERR_UNSUPPORTED;
+    if (M == 0 || N == 0)
+        return CR_OK;
+    if (!xq || !xs || !w8 || !s_channel || !out)
+        return CR_ERR_INVALID_ARG;
+    if (!aligned16(xq) || !aligned16(xs) || !aligned16(w8) || !aligned16(s_channel) || !aligned16(out) ||
+        (bias && !aligned16(bias)) || (acc_out && !aligned16(acc_out)))
+        return CR_ERR_ALIGNMENT;
+    DeviceState *d = nullptr;
+    st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    return gemm_on_w8(*d, xq, xs, w8, s_channel, bias, M, N, K, out_dtype, out, acc_out, stream, 0);
 }
 
 cr_status cr_selftest_wait_timeout(uint64_t limit_ns, cr_stream_t stream)
