@@ -183,16 +183,18 @@ bool make_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype,
 // tiles of all layers are numbered one after the other and run on a
 // persistent grid of as many CTAs as fit on the SMs, optionally as a
 // programmatic dependent of the previous kernel on the stream.
-// The activation map of the decode GEMV over xq [>= M, K] (a stage's box of
-// 8 rows x 1024 columns lands as [slice][token][128 B], 128-byte swizzle).
+// The activation map of the decode GEMV over xq [>= M, K], 1 <= M <= 8 (a
+// stage's box of M rows x 1024 columns lands as [slice][token][128 B],
+// 128-byte swizzle).
 bool encode_gemv_x_map(CUtensorMap *map, const int8_t *xq, int64_t M, int64_t K)
 {
+    if (M < 1 || M > cr::gv::kTokens)
+        return false;
     const uint64_t uK = (uint64_t)K;
     return make_tmap_3d(map, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, {(uint64_t)cr::gv::kSlice, (uint64_t)M,
                                                                    uK / cr::gv::kSlice},
                         {uK, (uint64_t)cr::gv::kSlice},
-                        {(uint32_t)cr::gv::kSlice, (uint32_t)cr::gv::kTokens,
-                         (uint32_t)(cr::gv::kChunk / cr::gv::kSlice)},
+                        {(uint32_t)cr::gv::kSlice, (uint32_t)M, (uint32_t)(cr::gv::kChunk / cr::gv::kSlice)},
                         true);
 }
 

@@ -10,7 +10,7 @@
 //  * Streaming: a persistent grid (two CTAs per SM).  In each CTA one
 //    producer warp moves, per stage, the packed codes (16 weight rows x 1024
 //    columns, 8 KB), their group scales (1 KB) and the matching 1024 columns
-//    of the (at most 8) activation rows (8 KB) into a ring of shared-memory
+//    of the M <= 8 activation rows (M KB) into a ring of shared-memory
 //    stages with 3-D TMA copies; eight consumer warps decode and contract each
 //    stage while the following ones are in flight; an epilogue warp reduces
 //    the consumers' partial sums and writes the outputs of a tile while the
@@ -20,8 +20,12 @@
 //  * Shared-memory layouts chosen for conflict-free reads: the tensor maps
 //    order the box so that a stage holds the codes as [slice][row][64 B], the
 //    scales as [256-column block][row][16 B] and the activations as
-//    [slice][token][128 B] with the 128-byte swizzle; every quarter-warp
-//    request then touches 8 distinct 16-byte bank groups.
+//    [slice][token < M][128 B] with the 128-byte swizzle; every quarter-warp
+//    request then touches 8 distinct 16-byte bank groups.  The activation box
+//    has exactly M rows: no rows are zero-filled by the copy engine (which
+//    measurably slows a stage), and the stage carries M KB of activations
+//    rather than 8.  Lanes of tokens m >= M read stale bytes of the stage;
+//    they only feed accumulator columns that are never written out.
 //  * Decode: a per-CTA table of the 16 int8 levels of every fp8 scale byte
 //    (exact: the decoded value depends only on the pair), replicated so that
 //    the lanes of a quarter-warp mostly read distinct bank groups; byte
@@ -60,8 +64,7 @@ constexpr int kChunk = kConsumerWarps * kSlice;      // columns per stage
 constexpr int kTokens = 8;                           // activation rows of a stage (the MMA's N)
 constexpr int kCodeBytes = kRows * kChunk / 2;
 constexpr int kSrelBytes = kRows * kChunk / 16;
-constexpr int kXBytes = kTokens * kChunk;
-constexpr int kStageTx = kCodeBytes + kSrelBytes + kXBytes;
+constexpr int kXBytes = kTokens * kChunk;  // room for M = 8; a stage carries M * kChunk
 constexpr int kPrefetchAhead = 3;  // L2 prefetch distance of the weight stream, in stages
 constexpr int kRedBufs = 1;  // partial-sum mailboxes between the consumers and the epilogue warp
 
@@ -74,7 +77,7 @@ struct Cfg {
     static constexpr int kMinBlocks = MINB;
     static constexpr int kCopies = COPIES;
     struct __align__(1024) Smem {
-        uint8_t x[STAGES][kXBytes];          // [slice][token][128 B], 128-byte swizzle (1024-aligned)
+        uint8_t x[STAGES][kXBytes];          // [slice][token < M][128 B], 128-byte swizzle (1024-aligned)
         uint8_t codes[STAGES][kCodeBytes];   // [slice][row][64 B]
         uint8_t srel[STAGES][kSrelBytes];    // [256-column block][row][16 B]
         uint4 lut[256 * COPIES];             // lut[s * COPIES + c]: copy c of the levels of scale byte s
@@ -166,7 +169,7 @@ struct GemvLayer {
 // tm_codes[l]: layer l's packed codes as 32-bit words, dims {16, N, K / 128},
 //              strides {K / 2, 64} bytes, box {16, 16, 8}.
 // tm_srel[l]:  its scale bytes, dims {16, N, K / 256}, strides {K / 16, 16}, box {16, 16, 4}.
-// tm_x:        xq, dims {128, M, K / 128}, strides {K, 128}, box {128, 8, 8}, 128-byte swizzle.
+// tm_x:        xq, dims {128, M, K / 128}, strides {K, 128}, box {128, M, 8}, 128-byte swizzle.
 // lut_step:    bytes between the table entries of consecutive scale bytes in one
 //              copy (kCopies * 16).  ahead: L2 prefetch distance in stages.
 // L: the layer slots of the launch (1, or kMaxLayers for a grouped call), so
@@ -217,6 +220,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
     extern __shared__ uint8_t smem_raw[];
     Smem &sh = smem_aligned_1024<Smem>(smem_raw);
     const int M = a.M, K = a.K;
+    const uint32_t stage_tx = (uint32_t)(kCodeBytes + kSrelBytes + M * kChunk);
 
     // The next kernel on the stream may launch now: a GEMV of the next layer
     // starts its weight stream in the SM slots this grid frees, and whatever
@@ -232,26 +236,28 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
     const int my_tiles = (int)blockIdx.x < ntiles ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
     const int total = my_tiles * nchunks;
 
-    if (tid == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&sh.full[s], 1);
-            mbar_init(&sh.empty[s], kConsumerWarps);
-        }
-        for (int b = 0; b < kRedBufs; ++b) {
-            mbar_init(&sh.red_full[b], kConsumerWarps);
-            mbar_init(&sh.red_empty[b], 1);
-        }
-        sh.abort = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    }
-    if (tid < 16)
-        sh.cb[tid] = a.codebook[tid];
-    __syncthreads();
+    // The producer initialises the barriers and starts the weight stream at
+    // once; the other warps pass named barrier 2 only after the
+    // initialisation, and the consumers' codebook load stays off the path to
+    // the first copy.
     volatile int *abort = &sh.abort;
-
     if (warp == kProducerWarp) {
         // ------------------------------------------------ producer
+        if (lane == 0) {
+            for (int s = 0; s < STAGES; ++s) {
+                mbar_init(&sh.full[s], 1);
+                mbar_init(&sh.empty[s], kConsumerWarps);
+            }
+            for (int b = 0; b < kRedBufs; ++b) {
+                mbar_init(&sh.red_full[b], kConsumerWarps);
+                mbar_init(&sh.red_empty[b], 1);
+            }
+            sh.abort = 0;
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        }
+        __syncwarp();
+        asm volatile("bar.arrive 2, %0;" ::"n"(kThreads) : "memory");
         if (lane == 0) {
             if constexpr (L == 1) {
                 prefetch_tmap(&a.tm_codes[0]);
@@ -291,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
             // finished; their activation copies follow the dependency wait.
             const int pre = total < STAGES ? total : STAGES;
             for (int q = 0; q < pre; ++q) {
-                mbar_arrive_expect_tx(&sh.full[q], kStageTx);
+                mbar_arrive_expect_tx(&sh.full[q], stage_tx);
                 weights(q, q);
             }
             for (int q = pre; q < pre + a.ahead; ++q)
@@ -309,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
                     issued_upto = q;
                     break;
                 }
-                mbar_arrive_expect_tx(&sh.full[s], kStageTx);
+                mbar_arrive_expect_tx(&sh.full[s], stage_tx);
                 weights(q, s);
                 acts(q, s);
                 prefetch(q + a.ahead);
@@ -324,6 +330,9 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
         }
     } else if (warp < kConsumerWarps) {
         // ------------------------------------------------ consumers
+        if (tid < 16)
+            sh.cb[tid] = a.codebook[tid];
+        asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
         {
             const uint4 e = lut_entry((uint32_t)tid, sh.cb);
 #pragma unroll
@@ -339,8 +348,11 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
         // this thread's offsets inside a stage
         const int off_code = sl * (kRows * 64) + g * 64 + 16 * t;                       // row g; g + 8 at +512
         const int off_srel = (sl >> 1) * (kRows * 16) + g * 16 + 8 * (sl & 1) + 2 * t;  // row g; g + 8 at +128
-        const int off_x0 = sl * (kTokens * 128) + g * 128 + 16 * ((2 * t) ^ g);
-        const int off_x1 = sl * (kTokens * 128) + g * 128 + 16 * ((2 * t + 1) ^ g);
+        // 128-byte line of (slice sl, token g); the swizzle permutes the
+        // 16-byte chunks of a line by its index mod 8
+        const int xl = sl * M + g;
+        const int off_x0 = xl * 128 + 16 * ((2 * t) ^ (xl & 7));
+        const int off_x1 = xl * 128 + 16 * ((2 * t + 1) ^ (xl & 7));
         // chunks in which this warp's slice lies inside K (K is a multiple of 256)
         const int nvalid = (K - kSlice * sl + kChunk - 1) / kChunk;
         // hand a tile's partial sums to the epilogue warp and go on
@@ -392,6 +404,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
         // ------------------------------------------------ epilogue warp
         // Per tile: sum the eight warps' partials and write the outputs, while
         // the consumers already decode the next tile.
+        asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
         asm volatile("griddepcontrol.wait;" ::: "memory");
         for (int seg = 0; seg < my_tiles; ++seg) {
             const int tile = (int)blockIdx.x + seg * (int)gridDim.x;
