@@ -421,8 +421,17 @@ cr_status cr_w4a8_dequant_t_bf16(const uint8_t *qdata, const uint8_t *srel, cons
  *   memory lets the copies run asynchronously): queues the copy of x_host
  *   [M, K] into x_dev, the forward into out_dev [M, N], and the copy of out_dev
  *   into out_host, all on `stream`; out_host is valid once the stream has
- *   reached that point.  x_dev, out_dev, xq_work and xs_work are device
- *   buffers of the caller.
+ *   reached that point, and x_host must stay unchanged until then.  x_dev,
+ *   out_dev, xq_work and xs_work are device buffers of the caller.  A copy of
+ *   at most 1 MiB whose host buffer is page-locked memory mapped for the
+ *   device (cudaHostAlloc, cudaMallocHost, or cudaHostRegister with mapping;
+ *   every such allocation under unified addressing), 16-byte aligned and a
+ *   multiple of 16 bytes long, is done by a kernel of the library on the SMs
+ *   (a decode step's few tens of KB cost far less that way than a copy-engine
+ *   transfer between two kernels); other copies use cudaMemcpyAsync.  The
+ *   kernel copying x_host reads it before the previous kernel on the stream
+ *   has finished: x_host must not be written by a kernel that immediately
+ *   precedes this call and allows early launch of its dependents.
  * cr_w4a8_plan_destroy: frees the plan (NULL is allowed).
  * Errors as in (6); a plan used on another device gives CR_ERR_INVALID_ARG.
  */

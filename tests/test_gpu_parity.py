@@ -298,6 +298,35 @@ def test_w4a8_linear_layer_object(M):
         assert torch.equal(out_host.view(torch.int16), y2.cpu().view(torch.int16)), rep
 
 
+@pytest.mark.parametrize("pinned,out_kind", [(True, "bf16"), (True, "f32"), (False, "bf16")])
+@pytest.mark.parametrize("M,N,K", [(8, 4096, 4096), (5, 776, 2048), (1, 16, 256), (64, 1032, 512)])
+def test_forward_host_copy_paths(pinned, out_kind, M, N, K):
+    """Host-buffer forwards over both copy paths: mapped page-locked buffers
+    of at most 1 MiB (16-byte multiples) are copied by the library's kernel,
+    pageable ones and ragged sizes by the copy engine; every call gives
+    cr_w4a8_linear's output bit for bit, over repeated calls with the host
+    input rewritten in between."""
+    odt = torch.float32 if out_kind == "f32" else torch.bfloat16
+    layer = inputs.layer(N, K, 7 * M + N, with_bias=True)
+    q, s, cb, ws, b = _layer_dev(layer)
+    lin = cr.W4A8Linear(q, s, cb, ws, b, out_dtype=odt)
+    x_host = torch.empty(M, K, dtype=torch.bfloat16)
+    out_host = torch.empty(M, N, dtype=odt)
+    if pinned:
+        x_host, out_host = x_host.pin_memory(), out_host.pin_memory()
+    x_dev = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    out_dev = torch.empty(M, N, dtype=odt, device="cuda")
+    for rep in range(3):
+        x = bf16_dev(inputs.activations(M, K, 500 + 11 * rep + M))
+        x_host.copy_(x.cpu())
+        ref = cr.cr_w4a8_linear(x, q, s, cb, ws, b, out_dtype=odt)
+        out_host.fill_(float("nan"))
+        lin.forward_host(x_host, out_host, x_dev, out_dev)
+        torch.cuda.synchronize()
+        view = torch.int32 if odt == torch.float32 else torch.int16
+        assert torch.equal(out_host.view(view), ref.cpu().view(view)), rep
+
+
 def test_plan_reencodes_the_activation_map_when_buffers_change():
     """A prepared layer re-encodes its cached activation map whenever the work
     buffer or M changes: alternating two work buffers and several M on one

@@ -372,6 +372,7 @@ class W4A8Linear:
         self._plan = handle
         self._fwd = self._L.cr_w4a8_plan_forward
         self._fwd_host = self._L.cr_w4a8_plan_forward_host
+        self._host_args = None  # (tensors, their storage and shapes, C arguments) of the last host forward
 
     def __del__(self):
         plan = getattr(self, "_plan", None)
@@ -414,6 +415,14 @@ class W4A8Linear:
         asynchronous copies), x_dev / out_dev their device buffers: queues the
         copy in, the forward and the copy out on the stream; out_host is ready
         once the stream has reached that point."""
+        key = (x_host, out_host, x_dev, out_dev, xq_work, xs_work)
+        hit = self._host_args
+        if hit is not None and all(a is b for a, b in zip(hit[0], key)):
+            # the same tensors as the last call, unchanged in storage and shape:
+            # skip re-validating them
+            if hit[1] == tuple(None if t is None else (t.data_ptr(), t.shape) for t in key):
+                _check(self._fwd_host(self._plan, *hit[2], _stream(stream)), "cr_w4a8_plan_forward_host")
+                return out_host
         torch = _torch()
         if x_host.is_cuda or out_host.is_cuda:
             raise ValueError("x_host and out_host must be host tensors")
@@ -426,10 +435,12 @@ class W4A8Linear:
             raise ValueError(f"out_host must be a contiguous {self.out_dtype} [{M}, {self.N}] tensor")
         _need(x_dev, "x_dev", (torch.bfloat16,), shape=(M, K))
         _need(out_dev, "out_dev", (self.out_dtype,), shape=(M, self.N))
-        xq_work, xs_work = self._work(x_dev, M, xq_work, xs_work)
-        _check(self._fwd_host(self._plan, x_host.data_ptr(), M, out_host.data_ptr(), x_dev.data_ptr(),
-                              out_dev.data_ptr(), xq_work.data_ptr(), xs_work.data_ptr(), _stream(stream)),
-               "cr_w4a8_plan_forward_host")
+        xq, xs = self._work(x_dev, M, xq_work, xs_work)
+        ptrs = (x_host.data_ptr(), M, out_host.data_ptr(), x_dev.data_ptr(), out_dev.data_ptr(), xq.data_ptr(),
+                xs.data_ptr())
+        _check(self._fwd_host(self._plan, *ptrs, _stream(stream)), "cr_w4a8_plan_forward_host")
+        if xq_work is not None and xs_work is not None:  # caller-owned work buffers: the call can be repeated as is
+            self._host_args = (key, tuple(None if t is None else (t.data_ptr(), t.shape) for t in key), ptrs)
         return out_host
 
 

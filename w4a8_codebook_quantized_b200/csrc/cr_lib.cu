@@ -733,6 +733,30 @@ cr_status contraction_swiglu(bool gemv, const int8_t *xq, const float *xs, const
                     nullptr, /*swiglu=*/1);
 }
 
+// The device address of host buffer [p, p + bytes) when it is at most
+// kHostCopyMax bytes, 16-byte aligned, a multiple of 16 bytes long, and both
+// its first and last byte lie in page-locked host memory mapped for the
+// device at addresses `bytes - 1` apart; otherwise null.
+constexpr size_t kHostCopyMax = 1u << 20;
+
+const void *small_mapped_host(const void *p, size_t bytes)
+{
+    if (bytes == 0 || bytes > kHostCopyMax || bytes % 16 != 0 || !aligned16(p))
+        return nullptr;
+    cudaPointerAttributes a0, a1;
+    const char *last = static_cast<const char *>(p) + bytes - 1;
+    if (cudaPointerGetAttributes(&a0, p) != cudaSuccess || cudaPointerGetAttributes(&a1, last) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    if (a0.type != cudaMemoryTypeHost || a1.type != cudaMemoryTypeHost || !a0.devicePointer || !a1.devicePointer)
+        return nullptr;
+    if (static_cast<const char *>(a1.devicePointer) - static_cast<const char *>(a0.devicePointer) !=
+        (ptrdiff_t)(bytes - 1))
+        return nullptr;
+    return a0.devicePointer;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1073,13 +1097,28 @@ cr_status cr_w4a8_plan_forward_host(cr_w4a8_plan plan, const uint16_t *x_host, i
         cudaGetLastError();
         return CR_ERR_INVALID_ARG;
     }
-    if (cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, stream) != cudaSuccess) {
+    DeviceState *d = nullptr;
+    cr_status st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    // Small transfers between mapped page-locked host memory and the device
+    // go through the SMs (ew::host_copy_kernel), anything else through the
+    // copy engine.
+    const void *x_map = small_mapped_host(x_host, xb);
+    void *out_map = const_cast<void *>(small_mapped_host(out_host, ob));
+    if (x_map) {
+        st = launched(cr::ew::launch_host_copy(x_dev, x_map, (int64_t)xb, true, d->num_sms, stream));
+        if (st != CR_OK)
+            return st;
+    } else if (cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, stream) != cudaSuccess) {
         cudaGetLastError();
         return CR_ERR_CUDA;
     }
-    const cr_status st = cr_w4a8_plan_forward(plan, x_dev, M, out_dev, xq_work, xs_work, stream);
+    st = cr_w4a8_plan_forward(plan, x_dev, M, out_dev, xq_work, xs_work, stream);
     if (st != CR_OK)
         return st;
+    if (out_map)
+        return launched(cr::ew::launch_host_copy(out_map, out_dev, (int64_t)ob, false, d->num_sms, stream));
     if (cudaMemcpyAsync(out_host, out_dev, ob, cudaMemcpyDeviceToHost, stream) != cudaSuccess) {
         cudaGetLastError();
         return CR_ERR_CUDA;

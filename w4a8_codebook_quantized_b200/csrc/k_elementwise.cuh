@@ -276,6 +276,67 @@ inline cudaError_t launch_dequant_t_bf16(const uint8_t *qdata, const uint8_t *sr
 
 // ---------------------------------------------------------------- failure-path self-test
 //
+// Copy between page-locked host memory that the device can address and
+// device memory, done by the SMs with 16-byte accesses: one vector per thread
+// per pass, the grid spread wide so that no SM holds many host-link requests
+// in flight.  For the tens of kilobytes of a decode step's activations and
+// outputs this takes a fraction of the time of a copy-engine transfer queued
+// between kernels on the same stream.  Host addresses are read with
+// ld.global.cv (fetched again, never a stale cached line) and written with
+// st.global.wt (write-through to system memory).
+//
+// Launched as a programmatic dependent of the previous kernel on the stream.
+// Host to device: the host loads are issued before waiting for that kernel
+// (the host wrote the source before queuing the call) and the device stores
+// after it.  Device to host: the loads wait for that kernel, which produced
+// the source.
+constexpr int kCopyThreads = 128;
+
+template <bool kToDevice>
+__global__ void __launch_bounds__(kCopyThreads) host_copy_kernel(uint4 *__restrict__ dst,
+                                                                 const uint4 *__restrict__ src, int64_t n16)
+{
+    asm volatile("griddepcontrol.launch_dependents;" :::);
+    const int64_t stride = (int64_t)gridDim.x * kCopyThreads;
+    const int64_t i0 = (int64_t)blockIdx.x * kCopyThreads + threadIdx.x;
+    if (kToDevice) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (i0 < n16)
+            v = __ldcv(src + i0);
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        if (i0 < n16)
+            dst[i0] = v;
+        for (int64_t i = i0 + stride; i < n16; i += stride)
+            dst[i] = __ldcv(src + i);
+    } else {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        for (int64_t i = i0; i < n16; i += stride)
+            __stwt(dst + i, src[i]);
+    }
+}
+
+inline cudaError_t launch_host_copy(void *dst, const void *src, int64_t bytes, bool to_device, int num_sms,
+                                    cudaStream_t stream)
+{
+    const int64_t n16 = bytes / 16;
+    const int64_t want = (n16 + kCopyThreads - 1) / kCopyThreads;
+    const int64_t cap = 4 * (int64_t)num_sms;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(want < cap ? want : cap));
+    cfg.blockDim = dim3(kCopyThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (to_device)
+        return cudaLaunchKernelEx(&cfg, host_copy_kernel<true>, reinterpret_cast<uint4 *>(dst),
+                                  reinterpret_cast<const uint4 *>(src), n16);
+    return cudaLaunchKernelEx(&cfg, host_copy_kernel<false>, reinterpret_cast<uint4 *>(dst),
+                              reinterpret_cast<const uint4 *>(src), n16);
+}
+
 // A wait that nothing completes: one thread initialises an mbarrier expecting
 // one arrival that never comes and waits for its first phase with the
 // library's bounded wait.  The wait runs out after limit_ns, sets the device
