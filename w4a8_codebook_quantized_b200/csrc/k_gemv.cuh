@@ -82,6 +82,7 @@ struct Cfg {
         uint8_t srel[STAGES][kSrelBytes];    // [256-column block][row][16 B]
         uint4 lut[256 * COPIES];             // lut[s * COPIES + c]: copy c of the levels of scale byte s
         int32_t red[kRedBufs][kConsumerWarps][kRows][8];  // per-warp partial sums
+        alignas(16) uint16_t ostage[kTokens][kRows];      // a tile's bf16 outputs, token-major
         float cb[16];
         uint64_t full[STAGES];
         uint64_t empty[STAGES];
@@ -466,6 +467,24 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
                             reinterpret_cast<uint16_t *>(out)[o] = to_bf16_bits(v);
                     }
                 }
+            } else if (go && !out_f32 && acc_out == nullptr && (N & 7) == 0 && row0 + kRows <= N) {
+                // a whole tile of bf16 outputs: staged token-major, then each
+                // token's 16 outputs leave as two 16-byte stores
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = lane + 32 * u;
+                    float y = __fmul_rn(__int2float_rn(acc[u]), __fmul_rn(exs[u], ews[u]));
+                    if (bias != nullptr)
+                        y = __fadd_rn(y, eb[u]);
+                    sh.ostage[e & 7][e >> 3] = to_bf16_bits(y);
+                }
+                __syncwarp();
+                if (lane < 2 * M) {
+                    const int m = lane >> 1, h = lane & 1;
+                    const uint4 v = *reinterpret_cast<const uint4 *>(&sh.ostage[m][8 * h]);
+                    *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(out) + (int64_t)m * N + row0 + 8 * h) = v;
+                }
+                __syncwarp();
             } else if (go) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
