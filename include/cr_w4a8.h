@@ -447,6 +447,29 @@ cr_status cr_w4a8_plan_forward_host(cr_w4a8_plan plan, const uint16_t *x_host, i
 cr_status cr_w4a8_plan_destroy(cr_w4a8_plan plan);
 
 /*
+ * (17) A host-buffer forward bound to its buffers (serving loops that call
+ * the same layer with the same buffers again and again).
+ *
+ * cr_w4a8_plan_bind_host: checks the arguments of cr_w4a8_plan_forward_host
+ *   once (with the same meaning), decides each copy's path (kernel or copy
+ *   engine, as there) and prepares the decode GEMV's complete arguments;
+ *   *call is written (NULL on error).  The plan and every buffer must stay
+ *   valid, and the host buffers page-locked, while the call exists.
+ * cr_w4a8_host_call_run: queues exactly what cr_w4a8_plan_forward_host with
+ *   those arguments queues (results bit for bit the same), without checking
+ *   or resolving anything again; only the current device is checked
+ *   (CR_ERR_INVALID_ARG if it is not the plan's).
+ * cr_w4a8_host_call_destroy: frees the call (NULL is allowed); the plan and
+ *   the buffers are not touched.
+ */
+typedef struct cr_w4a8_host_call_st *cr_w4a8_host_call;
+cr_status cr_w4a8_plan_bind_host(cr_w4a8_plan plan, const uint16_t *x_host, int64_t M, void *out_host,
+                                 uint16_t *x_dev, void *out_dev, int8_t *xq_work, float *xs_work,
+                                 cr_w4a8_host_call *call);
+cr_status cr_w4a8_host_call_run(cr_w4a8_host_call call, cr_stream_t stream);
+cr_status cr_w4a8_host_call_destroy(cr_w4a8_host_call call);
+
+/*
  * (16) The prefill contraction on an int8 weight already on the grid.
  *
  * Defined by: ai-toolkit convrot_w4a8_quant.py, _w4a8_linear_ste_op after

@@ -32,7 +32,8 @@ def test_header_declares_the_boundary():
               "cr_w4a8_gemv_grouped", "cr_w4a8_linear_grouped", "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu",
               "cr_w4a8_linear_swiglu", "cr_interleave_rows", "cr_w4a8_quantize_rotated", "cr_w4a8_assign_codes",
               "cr_w4a8_ste_backward", "cr_w4a8_dequant_t_bf16", "cr_w4a8_plan_create", "cr_w4a8_plan_forward",
-              "cr_w4a8_plan_forward_host", "cr_w4a8_plan_destroy", "cr_selftest_wait_timeout", "cr_gemm_s8"):
+              "cr_w4a8_plan_forward_host", "cr_w4a8_plan_destroy", "cr_selftest_wait_timeout", "cr_gemm_s8",
+              "cr_w4a8_plan_bind_host", "cr_w4a8_host_call_run", "cr_w4a8_host_call_destroy"):
         assert n in names
 
 
@@ -86,6 +87,15 @@ def test_decode_validation(L):
     assert f(None, A16, A16, 4, 256, A16, None) == cr.CR_ERR_INVALID_ARG
     assert f(A16, MIS, A16, 4, 256, A16, None) == cr.CR_ERR_ALIGNMENT
     assert f(None, None, None, 0, 256, None, None) == cr.CR_OK
+
+
+def test_bound_host_call_validation(L):
+    call = ctypes.c_void_p(1)
+    assert L.cr_w4a8_plan_bind_host(None, A16, 2, A16, A16, A16, A16, A16, ctypes.byref(call)) == cr.CR_ERR_INVALID_ARG
+    assert call.value is None  # written NULL on error
+    assert L.cr_w4a8_plan_bind_host(None, A16, 2, A16, A16, A16, A16, A16, None) == cr.CR_ERR_INVALID_ARG
+    assert L.cr_w4a8_host_call_run(None, None) == cr.CR_ERR_INVALID_ARG
+    assert L.cr_w4a8_host_call_destroy(None) == cr.CR_OK
 
 
 def test_gemm_s8_validation(L):

@@ -298,12 +298,15 @@ def test_w4a8_linear_layer_object(M):
         assert torch.equal(out_host.view(torch.int16), y2.cpu().view(torch.int16)), rep
 
 
+@pytest.mark.parametrize("bound", [False, True])
 @pytest.mark.parametrize("pinned,out_kind", [(True, "bf16"), (True, "f32"), (False, "bf16")])
-@pytest.mark.parametrize("M,N,K", [(8, 4096, 4096), (5, 776, 2048), (1, 16, 256), (64, 1032, 512)])
-def test_forward_host_copy_paths(pinned, out_kind, M, N, K):
+@pytest.mark.parametrize("M,N,K", [(8, 4096, 4096), (5, 776, 2048), (1, 16, 256), (64, 1032, 512), (3, 520, 1024)])
+def test_forward_host_copy_paths(bound, pinned, out_kind, M, N, K):
     """Host-buffer forwards over both copy paths: mapped page-locked buffers
     of at most 1 MiB (16-byte multiples) are copied by the library's kernel,
-    pageable ones and ragged sizes by the copy engine; every call gives
+    pageable ones and ragged sizes (3 x 520 bf16) by the copy engine; with
+    caller-owned work buffers the layer binds the call once
+    (cr_w4a8_plan_bind_host) and then only runs it.  Every call gives
     cr_w4a8_linear's output bit for bit, over repeated calls with the host
     input rewritten in between."""
     odt = torch.float32 if out_kind == "f32" else torch.bfloat16
@@ -316,12 +319,16 @@ def test_forward_host_copy_paths(pinned, out_kind, M, N, K):
         x_host, out_host = x_host.pin_memory(), out_host.pin_memory()
     x_dev = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
     out_dev = torch.empty(M, N, dtype=odt, device="cuda")
+    rows = cr.gemv_rows(M) if M <= 8 else M
+    work = (torch.empty(rows, K, dtype=torch.int8, device="cuda"), torch.empty(rows, device="cuda")) if bound \
+        else (None, None)
     for rep in range(3):
         x = bf16_dev(inputs.activations(M, K, 500 + 11 * rep + M))
         x_host.copy_(x.cpu())
         ref = cr.cr_w4a8_linear(x, q, s, cb, ws, b, out_dtype=odt)
         out_host.fill_(float("nan"))
-        lin.forward_host(x_host, out_host, x_dev, out_dev)
+        lin.forward_host(x_host, out_host, x_dev, out_dev, *work)
+        assert (lin._host_args is not None) == bound
         torch.cuda.synchronize()
         view = torch.int32 if odt == torch.float32 else torch.int16
         assert torch.equal(out_host.view(view), ref.cpu().view(view)), rep

@@ -552,6 +552,24 @@ struct cr_w4a8_plan_st {
     std::mutex mu;
 };
 
+// A host-buffer forward bound to its buffers (cr_w4a8_plan_bind_host): the
+// checks, the host mappings and the decode GEMV's complete arguments are
+// resolved once; a run only queues the launches.
+struct cr_w4a8_host_call_st {
+    cr_w4a8_plan plan = nullptr;
+    const uint16_t *x_host = nullptr;
+    void *out_host = nullptr;
+    const void *x_map = nullptr;  // device address of x_host (copied by a kernel), or null (copy engine)
+    void *out_map = nullptr;      // the same for out_host
+    uint16_t *x_dev = nullptr;
+    void *out_dev = nullptr;
+    int8_t *xq = nullptr;
+    float *xs = nullptr;
+    int64_t M = 0, MP = 0;
+    size_t xb = 0, ob = 0;
+    cr::gv::GemvArgs<1> gemv;  // M <= CR_GEMV_MAX_M: the GEMV launch's arguments, activation map included
+};
+
 extern "C" {
 
 const char *cr_status_string(cr_status s)
@@ -1123,6 +1141,110 @@ cr_status cr_w4a8_plan_forward_host(cr_w4a8_plan plan, const uint16_t *x_host, i
         cudaGetLastError();
         return CR_ERR_CUDA;
     }
+    return CR_OK;
+}
+
+cr_status cr_w4a8_plan_bind_host(cr_w4a8_plan plan, const uint16_t *x_host, int64_t M, void *out_host,
+                                 uint16_t *x_dev, void *out_dev, int8_t *xq_work, float *xs_work,
+                                 cr_w4a8_host_call *call)
+{
+    if (!call)
+        return CR_ERR_INVALID_ARG;
+    *call = nullptr;
+    if (!plan || M < 0)
+        return CR_ERR_INVALID_ARG;
+    if (M > INT_MAX)
+        return CR_ERR_UNSUPPORTED;
+    cr_w4a8_host_call_st *c = new (std::nothrow) cr_w4a8_host_call_st();
+    if (!c)
+        return CR_ERR_CUDA;
+    c->plan = plan;
+    c->M = M;
+    if (M > 0 && plan->N > 0) {
+        cr_status st = CR_OK;
+        int dev = -1;
+        if (!x_host || !out_host || !x_dev || !out_dev || !xq_work || !xs_work)
+            st = CR_ERR_INVALID_ARG;
+        else if (!aligned16(x_dev) || !aligned16(out_dev) || !aligned16(xq_work) || !aligned16(xs_work))
+            st = CR_ERR_ALIGNMENT;
+        else if (cudaGetDevice(&dev) != cudaSuccess || dev != plan->device) {
+            cudaGetLastError();
+            st = CR_ERR_INVALID_ARG;
+        }
+        if (st == CR_OK && M <= CR_GEMV_MAX_M) {
+            std::lock_guard<std::mutex> lock(plan->mu);
+            c->gemv = plan->gemv;
+            if (!encode_gemv_x_map(&c->gemv.tm_x, xq_work, M, plan->K))
+                st = CR_ERR_CUDA;
+        }
+        if (st != CR_OK) {
+            delete c;
+            return st;
+        }
+        c->x_host = x_host;
+        c->out_host = out_host;
+        c->x_dev = x_dev;
+        c->out_dev = out_dev;
+        c->xq = xq_work;
+        c->xs = xs_work;
+        c->xb = (size_t)(M * plan->K) * 2;
+        c->ob = (size_t)(M * plan->N) * (plan->out_dtype == CR_OUT_F32 ? 4 : 2);
+        c->x_map = small_mapped_host(x_host, c->xb);
+        c->out_map = const_cast<void *>(small_mapped_host(out_host, c->ob));
+        c->MP = 1;
+        while (c->MP < M)
+            c->MP <<= 1;
+        c->gemv.xs = xs_work;
+        c->gemv.M = (int)M;
+        c->gemv.layer[0].out = out_dev;
+    }
+    *call = c;
+    return CR_OK;
+}
+
+cr_status cr_w4a8_host_call_run(cr_w4a8_host_call c, cr_stream_t stream)
+{
+    if (!c)
+        return CR_ERR_INVALID_ARG;
+    cr_w4a8_plan plan = c->plan;
+    if (c->M == 0 || plan->N == 0)
+        return CR_OK;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != plan->device) {
+        cudaGetLastError();
+        return CR_ERR_INVALID_ARG;
+    }
+    DeviceState *d = plan->d;
+    cr_status st = CR_OK;
+    if (c->x_map)
+        st = launched(cr::ew::launch_host_copy(c->x_dev, c->x_map, (int64_t)c->xb, true, d->num_sms, stream));
+    else if (cudaMemcpyAsync(c->x_dev, c->x_host, c->xb, cudaMemcpyHostToDevice, stream) != cudaSuccess) {
+        cudaGetLastError();
+        st = CR_ERR_CUDA;
+    }
+    if (st != CR_OK)
+        return st;
+    if (c->M > CR_GEMV_MAX_M) {
+        st = cr_w4a8_plan_forward(plan, c->x_dev, c->M, c->out_dev, c->xq, c->xs, stream);
+    } else {
+        st = launched(cr::rq::launch(c->x_dev, c->M, plan->K, c->MP, plan->act_qmax, c->xq, c->xs, stream));
+        if (st == CR_OK)
+            st = launch_gemv_args<1>(d->num_sms, d->gemv_attr_set, c->gemv, stream, /*pdl=*/true);
+    }
+    if (st != CR_OK)
+        return st;
+    if (c->out_map)
+        return launched(cr::ew::launch_host_copy(c->out_map, c->out_dev, (int64_t)c->ob, false, d->num_sms, stream));
+    if (cudaMemcpyAsync(c->out_host, c->out_dev, c->ob, cudaMemcpyDeviceToHost, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return CR_ERR_CUDA;
+    }
+    return CR_OK;
+}
+
+cr_status cr_w4a8_host_call_destroy(cr_w4a8_host_call call)
+{
+    delete call;
     return CR_OK;
 }
 
