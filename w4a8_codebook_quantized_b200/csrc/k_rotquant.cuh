@@ -177,8 +177,13 @@ __global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__re
     asm volatile("griddepcontrol.launch_dependents;" :::);
     // Launched as a programmatic dependent itself, this grid may be resident
     // before the previous kernel on the stream has finished: x may still be
-    // in the making and xq / xs still being read, so nothing is touched
-    // before that kernel completes.
+    // in the making and xq / xs still being read, so nothing is read or
+    // written before that kernel completes.  Only an L2 prefetch of this
+    // CTA's row of x goes out first: the L2 is where the device's writes
+    // become visible, so a prefetch cannot make a later load return an old
+    // value, and the row's loads after the wait then find it there.
+    if (threadIdx.x == 0 && (int64_t)blockIdx.x < M)
+        bulk_prefetch_l2(x + (int64_t)blockIdx.x * K, (uint32_t)(K * 2));
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
     const int tid = threadIdx.x;
