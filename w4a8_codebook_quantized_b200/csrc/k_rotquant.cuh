@@ -161,6 +161,21 @@ __device__ __forceinline__ void quantise_store(const float (&v)[16], float scale
     __syncwarp(hmask);
 }
 
+// max |v[i]| over 16 values as a tree of depth 4 (fmaxf drops NaN operands,
+// so the result is NaN-free and >= 0 for any inputs; max is exact in any
+// order).
+__device__ __forceinline__ float max_abs16(const float (&v)[16])
+{
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        m[i] = fmaxf(fabsf(v[i]), fabsf(v[i + 8]));
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        m[i] = fmaxf(m[i], m[i + 4]);
+    return fmaxf(fmaxf(m[0], m[2]), fmaxf(m[1], m[3]));
+}
+
 template <int J, bool kRecompute>
 __global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
                                                             int qmax, int8_t *__restrict__ xq,
@@ -213,24 +228,24 @@ __global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__re
             const int b = hw + kHalfWarps * j;
             if (b < NB) {
                 rotate_block(xrow + 256 * b, L, tr, hmask, v[j]);
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    amax = fmaxf(amax, fabsf(v[j][i]));
+                amax = fmaxf(amax, max_abs16(v[j]));
             }
         }
     } else {
         for (int b = hw; b < NB; b += kHalfWarps) {
             rotate_block(xrow + 256 * b, L, tr, hmask, v[0]);
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                amax = fmaxf(amax, fabsf(v[0][i]));
+            amax = fmaxf(amax, max_abs16(v[0]));
         }
     }
 
-    // row maximum (exact in any order)
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-        amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+    // row maximum (exact in any order).  amax is >= 0 and never NaN, and
+    // such floats order like their bit patterns as unsigned integers: one
+    // warp reduction instruction on the bits.
+    {
+        uint32_t bits = __float_as_uint(amax);
+        asm volatile("redux.sync.max.u32 %0, %0, 0xffffffff;" : "+r"(bits));
+        amax = __uint_as_float(bits);
+    }
     if (lane == 0)
         warp_max[warp] = amax;
     __syncthreads();
