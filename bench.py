@@ -452,7 +452,9 @@ def run_ours(args):
     esecs = max_over_ranks(esecs, world)
     e2e = {"value": round(aggregate_value(wb, args.steps, world, esecs), 2), "unit": "GB/s",
            "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N,
-           "ms_per_step": round(esecs / args.steps * 1e3, 5)}
+           "ms_per_step": round(esecs / args.steps * 1e3, 5),
+           "path": "W4A8Linear.forward_host (bound call, cr_w4a8_host_call_run), eager: x from pinned host memory "
+                   "by a copy kernel, rotate+quant, GEMV, y to pinned host memory by a copy kernel (4 launches)"}
 
     prefill = None
     if not args.no_prefill:
