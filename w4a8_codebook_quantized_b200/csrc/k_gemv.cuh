@@ -272,40 +272,59 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
                 }
             }
             prefetch_tmap(&a.tm_x);
-            auto weights = [&](int q, int s) {
-                const int i = q / nchunks, tile = (int)blockIdx.x + i * (int)gridDim.x, c = q - i * nchunks;
-                int l, row;
-                locate(a, tile, l, row);
-                tma_load_3d(sh.codes[s], &a.tm_codes[l], 0, row, c * (kChunk / kSlice), &sh.full[s]);
-                tma_load_3d(sh.srel[s], &a.tm_srel[l], 0, row, c * (kChunk / 256), &sh.full[s]);
+            // Stage q of this CTA's run is chunk q mod nchunks of its tile
+            // q / nchunks; the producer walks these positions with counters
+            // (no run-time division on its per-stage path).
+            struct Pos {
+                int c, tile;
             };
-            // L2 prefetch of the weights of stage q: `ahead` stages of HBM reads
-            // in flight beyond the shared-memory ring, so that a refill of the
-            // ring usually finds its data in L2
-            auto prefetch = [&](int q) {
-                if (q < total) {
-                    const int i = q / nchunks, tile = (int)blockIdx.x + i * (int)gridDim.x, c = q - i * nchunks;
-                    int l, row;
-                    locate(a, tile, l, row);
-                    tma_prefetch_3d(&a.tm_codes[l], 0, row, c * (kChunk / kSlice));
-                    tma_prefetch_3d(&a.tm_srel[l], 0, row, c * (kChunk / 256));
+            auto step = [&](Pos &p) {
+                if (++p.c == nchunks) {
+                    p.c = 0;
+                    p.tile += (int)gridDim.x;
                 }
             };
-            auto acts = [&](int q, int s) {
-                tma_load_3d(sh.x[s], &a.tm_x, 0, 0, (q % nchunks) * (kChunk / kSlice), &sh.full[s]);
+            auto weights = [&](const Pos &p, int s) {
+                int l, row;
+                locate(a, p.tile, l, row);
+                tma_load_3d(sh.codes[s], &a.tm_codes[l], 0, row, p.c * (kChunk / kSlice), &sh.full[s]);
+                tma_load_3d(sh.srel[s], &a.tm_srel[l], 0, row, p.c * (kChunk / 256), &sh.full[s]);
+            };
+            // L2 prefetch of the weights of a stage `ahead` stages beyond the
+            // shared-memory ring, so that a refill of the ring usually finds
+            // its data in L2
+            auto prefetch = [&](const Pos &p) {
+                int l, row;
+                locate(a, p.tile, l, row);
+                tma_prefetch_3d(&a.tm_codes[l], 0, row, p.c * (kChunk / kSlice));
+                tma_prefetch_3d(&a.tm_srel[l], 0, row, p.c * (kChunk / 256));
+            };
+            auto acts = [&](const Pos &p, int s) {
+                tma_load_3d(sh.x[s], &a.tm_x, 0, 0, p.c * (kChunk / kSlice), &sh.full[s]);
             };
             // The first stages' weights go out before the activation kernel has
             // finished; their activation copies follow the dependency wait.
             const int pre = total < STAGES ? total : STAGES;
+            Pos pw{0, (int)blockIdx.x};  // the next stage to issue
             for (int q = 0; q < pre; ++q) {
                 mbar_arrive_expect_tx(&sh.full[q], stage_tx);
-                weights(q, q);
+                weights(pw, q);
+                step(pw);
             }
-            for (int q = pre; q < pre + a.ahead; ++q)
-                prefetch(q);
+            Pos pp = pw;  // the next stage to prefetch
+            for (int q = pre; q < pre + a.ahead; ++q) {
+                if (q < total)
+                    prefetch(pp);
+                step(pp);
+            }
             asm volatile("griddepcontrol.wait;" ::: "memory");
-            for (int q = 0; q < pre; ++q)
-                acts(q, q);
+            {
+                Pos pa{0, (int)blockIdx.x};
+                for (int q = 0; q < pre; ++q) {
+                    acts(pa, q);
+                    step(pa);
+                }
+            }
             int issued_upto = pre;  // stages [0, issued_upto) of the run have been issued
             bool ok = true;
             for (int q = pre; q < total; ++q) {
@@ -317,9 +336,12 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
                     break;
                 }
                 mbar_arrive_expect_tx(&sh.full[s], stage_tx);
-                weights(q, s);
-                acts(q, s);
-                prefetch(q + a.ahead);
+                weights(pw, s);
+                acts(pw, s);
+                step(pw);
+                if (q + a.ahead < total)
+                    prefetch(pp);
+                step(pp);
             }
             if (!ok) {
                 // let the copies in flight land before the CTA exits
