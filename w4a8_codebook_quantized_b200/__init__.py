@@ -377,8 +377,9 @@ class W4A8Linear:
         self._fwd_host = self._L.cr_w4a8_plan_forward_host
         self._run_host = self._L.cr_w4a8_host_call_run
         # (tensors, their storage and shapes, bound call) of the last host forward
-        # with caller-owned work buffers (cr_w4a8_plan_bind_host)
+        # with caller-owned work buffers (cr_w4a8_plan_bind_host), and its lock
         self._host_args = None
+        self._host_lock = threading.Lock()
 
     def __del__(self):
         self._drop_host_call()
@@ -432,11 +433,14 @@ class W4A8Linear:
         and a repeat with the same tensors, unchanged in storage and shape,
         only queues the launches."""
         key = (x_host, out_host, x_dev, out_dev, xq_work, xs_work)
-        hit = self._host_args
-        if hit is not None and all(a is b for a, b in zip(hit[0], key)):
-            if hit[1] == tuple(None if t is None else (t.data_ptr(), t.shape) for t in key):
-                _check(self._run_host(hit[2], _stream(stream)), "cr_w4a8_host_call_run")
-                return out_host
+        # the bound call is used and replaced under the lock: the C call releases
+        # the GIL, and another thread must not free the call while it runs
+        with self._host_lock:
+            hit = self._host_args
+            if hit is not None and all(a is b for a, b in zip(hit[0], key)):
+                if hit[1] == tuple(None if t is None else (t.data_ptr(), t.shape) for t in key):
+                    _check(self._run_host(hit[2], _stream(stream)), "cr_w4a8_host_call_run")
+                    return out_host
         torch = _torch()
         if x_host.is_cuda or out_host.is_cuda:
             raise ValueError("x_host and out_host must be host tensors")
@@ -455,12 +459,13 @@ class W4A8Linear:
         if xq_work is None or xs_work is None:  # work buffers of this call only: nothing to bind
             _check(self._fwd_host(self._plan, *ptrs, _stream(stream)), "cr_w4a8_plan_forward_host")
             return out_host
-        self._drop_host_call()
-        call = ctypes.c_void_p()
-        _check(self._L.cr_w4a8_plan_bind_host(self._plan, *ptrs, ctypes.byref(call)), "cr_w4a8_plan_bind_host")
-        # the bound tensors are held with the call, so their memory outlives it
-        self._host_args = (key, tuple(None if t is None else (t.data_ptr(), t.shape) for t in key), call)
-        _check(self._run_host(call, _stream(stream)), "cr_w4a8_host_call_run")
+        with self._host_lock:
+            self._drop_host_call()
+            call = ctypes.c_void_p()
+            _check(self._L.cr_w4a8_plan_bind_host(self._plan, *ptrs, ctypes.byref(call)), "cr_w4a8_plan_bind_host")
+            # the bound tensors are held with the call, so their memory outlives it
+            self._host_args = (key, tuple(None if t is None else (t.data_ptr(), t.shape) for t in key), call)
+            _check(self._run_host(call, _stream(stream)), "cr_w4a8_host_call_run")
         return out_host
 
 
