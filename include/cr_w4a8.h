@@ -18,9 +18,28 @@
  *
  * Conventions for every entry point
  * ---------------------------------
- * - Pointers are DEVICE pointers unless stated otherwise; the caller owns all
- *   memory.  Every call is asynchronous on `stream` (NULL = the legacy default
- *   stream) and returns as soon as the work is queued.
+ * - Pointers are DEVICE pointers unless stated otherwise; the caller owns
+ *   every buffer it passes.  Every call is asynchronous on `stream` (NULL =
+ *   the legacy default stream) and returns as soon as the work is queued.
+ * - Device memory of the library.  The prefill paths need a weight
+ *   transient: cr_w4a8_gemm, cr_w4a8_gemm_swiglu, and cr_w4a8_linear,
+ *   cr_w4a8_linear_swiglu, cr_w4a8_linear_grouped and cr_w4a8_plan_forward
+ *   when M > 8, take N * K bytes (the int8 weight; grouped: the largest
+ *   layer's) and cr_w4a8_ste_backward 2 * N * K bytes (the transposed bf16
+ *   weight) from a stream-ordered pool of the library, allocated on `stream`
+ *   and freed on it at the end of the call.  The pool keeps nothing: its
+ *   memory goes back to the driver at the next stream, event or device
+ *   synchronisation after the free.  When that allocation fails the call
+ *   returns CR_ERR_CUDA and launches nothing.  The *_ws variants
+ *   (cr_w4a8_gemm_ws, cr_w4a8_linear_ws, cr_w4a8_ste_backward_ws) take the
+ *   transient from the caller instead and allocate nothing; every other entry
+ *   point allocates no device memory.
+ * - cr_w4a8_linear (and _swiglu, _ws, _grouped, cr_w4a8_plan_forward) with
+ *   M > 8 run the weight decode on a side stream of the library (one
+ *   non-blocking stream and two events per device, created on first use and
+ *   kept until exit), forked from and joined back into `stream` with events,
+ *   so the decode overlaps the activation kernel; `stream` orders the call
+ *   as usual.
  * - Arrays are dense and row-major, with exactly the shapes given.
  * - Every pointer must be 16-byte aligned (CR_ERR_ALIGNMENT otherwise).
  * - Sizes are int64_t.  M == 0 or N == 0 is an empty problem: CR_OK, nothing
@@ -156,6 +175,17 @@ cr_status cr_w4a8_gemm(const int8_t *xq, const float *xs, const uint8_t *qdata, 
                        int32_t *acc_out, cr_stream_t stream);
 
 /*
+ * (3w) (3) with the caller's weight transient: w8_work [N, K] int8 (16-byte
+ * aligned, required unless M == 0 or N == 0) receives the decoded weight (the
+ * int8 grid of (2)) and is then read by the contraction; on return it holds
+ * that grid.  Allocates nothing.  Results equal those of (3) bit for bit.
+ */
+cr_status cr_w4a8_gemm_ws(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                          const float *codebook, const float *s_channel, const float *bias,
+                          int64_t M, int64_t N, int64_t K, cr_out_dtype out_dtype, void *out,
+                          int32_t *acc_out, int8_t *w8_work, cr_stream_t stream);
+
+/*
  * (4) Decode forward for 1 <= M <= 8: a fused GEMV that streams the packed
  * codes, the fp8 group scales and the codebook (4.5 bits per weight) and
  * never materialises the int8 weight.
@@ -202,14 +232,25 @@ cr_status cr_w4a8_linear(const uint16_t *x, const uint8_t *qdata, const uint8_t 
                          void *out, int8_t *xq_work, float *xs_work, cr_stream_t stream);
 
 /*
+ * (6w) (6) with the caller's weight transient for the prefill path: when
+ * M > 8, w8_work [N, K] int8 (16-byte aligned; CR_ERR_INVALID_ARG if NULL)
+ * receives the decoded weight, as in (3w); when M <= 8 it is not used and may
+ * be NULL.  Allocates nothing.  Results equal those of (6) bit for bit.
+ */
+cr_status cr_w4a8_linear_ws(const uint16_t *x, const uint8_t *qdata, const uint8_t *srel,
+                            const float *codebook, const float *s_channel, const float *bias,
+                            int64_t M, int64_t N, int64_t K, int act_qmax, cr_out_dtype out_dtype,
+                            void *out, int8_t *xq_work, float *xs_work, int8_t *w8_work, cr_stream_t stream);
+
+/*
  * (7) The decode forward (1 <= M <= 8) without any allocation.
  *
  * The pages have no counterpart of this entry point; it exists for callers
  * that cannot allocate device memory at the time of the call and so cannot
- * supply the scratch buffers cr_w4a8_linear needs: code running while a CUDA
- * graph is being captured (cudaMalloc may not be called then), serving loops
- * whose device memory is owned by their own allocator, and real-time paths
- * that cannot afford the synchronisation an allocation can imply.
+ * supply the scratch buffers cr_w4a8_linear needs: serving loops whose device
+ * memory is all owned by their own allocator (nothing is left to carve
+ * scratch from), and real-time paths that cannot afford the synchronisation
+ * an allocation can imply.
  *
  * It computes exactly what cr_w4a8_linear computes for M <= 8 (rotate +
  * quantise, then the decode GEMV), with the quantised activations kept in a
@@ -288,9 +329,12 @@ cr_status cr_w4a8_linear_grouped(const uint16_t *x, const float *codebook, int64
  * The layer holds N = 2F rows in that order (cr_interleave_rows builds it
  * from the two halves [gate; up]).  With g and u the fp32 epilogue values of
  * rows 2f and 2f + 1, computed exactly as in (3),
- *   out[m, f] = out_dtype( (g / (1 + exp(-g))) * u )
- * in fp32 (CUDA expf, the fast division __fdividef with at most 2 ulp of
- * error, each op rounded on its own), rounded once to out_dtype.  out is [M, F]; N odd gives CR_ERR_INVALID_ARG.  There
+ *   out[m, f] = out_dtype( silu(g) * u ),  silu(g) = g / (1 + exp(-g))
+ * in fp32: with t = expf(-|g|), silu(g) = g / (1 + t) for g >= 0 and
+ * g * t / (1 + t) for g < 0 (the same value, and no overflow for very
+ * negative gates), the division by the fast __fdividef (at most 2 ulp for a
+ * divisor in [1, 2]), each op rounded on its own, then rounded once to
+ * out_dtype.  out is [M, F]; N odd gives CR_ERR_INVALID_ARG.  There
  * is no acc_out: the int32 accumulators are those of (3) and (4) on the same
  * layer.  The decode GEMV and the GEMM give the same bits.
  *
@@ -401,6 +445,12 @@ cr_status cr_w4a8_ste_backward(const uint16_t *grad, const uint8_t *qdata, const
                                uint16_t *dx, cr_stream_t stream);
 cr_status cr_w4a8_dequant_t_bf16(const uint8_t *qdata, const uint8_t *srel, const float *codebook,
                                  const float *s_channel, int64_t N, int64_t K, uint16_t *wt, cr_stream_t stream);
+/* (13w) (13) with the caller's transient: wt_work [K, N] bf16 (16-byte
+ * aligned; CR_ERR_INVALID_ARG if NULL when M > 0 and N > 0) receives the
+ * transposed weight of (13a).  Allocates nothing; dx equals that of (13). */
+cr_status cr_w4a8_ste_backward_ws(const uint16_t *grad, const uint8_t *qdata, const uint8_t *srel,
+                                  const float *codebook, const float *s_channel, int64_t M, int64_t N, int64_t K,
+                                  uint16_t *dx, uint16_t *wt_work, cr_stream_t stream);
 
 /*
  * (14) A prepared layer for repeated forwards (serving loops).

@@ -30,6 +30,7 @@ __all__ = [
     "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu", "cr_w4a8_linear_swiglu", "cr_interleave_rows",
     "interleave_gate_up", "cr_w4a8_quantize_rotated", "cr_w4a8_assign_codes",
     "cr_w4a8_ste_backward", "cr_w4a8_dequant_t_bf16", "cr_selftest_wait_timeout", "cr_gemm_s8",
+    "cr_w4a8_gemm_ws", "cr_w4a8_linear_ws", "cr_w4a8_ste_backward_ws",
     "cr_status_string", "cr_version",
     "gemv_rows",
 ]
@@ -103,12 +104,16 @@ def lib() -> ctypes.CDLL:
             L.cr_selftest_wait_timeout.argtypes = [ctypes.c_uint64, P]
             L.cr_gemm_s8.argtypes = [P, P, P, P, P, i64, i64, i64, i32, P, P, P]
             L.cr_w4a8_dequant_t_bf16.argtypes = [P, P, P, P, i64, i64, P, P]
+            L.cr_w4a8_gemm_ws.argtypes = contraction[:-1] + [P, P]
+            L.cr_w4a8_linear_ws.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P, P, P, P]
+            L.cr_w4a8_ste_backward_ws.argtypes = [P, P, P, P, P, i64, i64, i64, P, P, P]
             LP = ctypes.POINTER(CrLayer)
             L.cr_w4a8_gemv_grouped.argtypes = [P, P, P, i64, i64, LP, i32, i32, P]
             L.cr_w4a8_linear_grouped.argtypes = [P, P, i64, i64, LP, i32, i32, i32, P, P, P]
             for name in ("cr_rotate_quant_act", "cr_w4a8_decode_int8", "cr_w4a8_gemm", "cr_w4a8_gemv",
                          "cr_epilogue", "cr_w4a8_linear", "cr_check_device_error",
-                         "cr_w4a8_linear_decode_noalloc"):
+                         "cr_w4a8_linear_decode_noalloc", "cr_w4a8_gemm_ws", "cr_w4a8_linear_ws",
+                         "cr_w4a8_ste_backward_ws"):
                 getattr(L, name).restype = i32
             _lib = L
     return _lib
@@ -165,6 +170,51 @@ def _check(status: int, where: str) -> None:
         raise CrError(status, where)
 
 
+def _cuda_device_of(args, kwargs):
+    """The one device of the CUDA tensors among the arguments (searched one
+    level into lists and tuples), or None; ValueError when they differ."""
+    torch = _torch()
+    dev = None
+
+    def visit(v, depth):
+        nonlocal dev
+        if isinstance(v, torch.Tensor):
+            if v.is_cuda:
+                if dev is None:
+                    dev = v.device
+                elif v.device != dev:
+                    raise ValueError(f"CUDA tensors on different devices: {dev} and {v.device}")
+        elif depth < 2 and isinstance(v, (list, tuple)):
+            for e in v:
+                visit(e, depth + 1)
+
+    for a in args:
+        visit(a, 0)
+    for a in kwargs.values():
+        visit(a, 0)
+    return dev
+
+
+def _on_device(fn):
+    """Run an entry point with the device of its CUDA tensors current.
+
+    The C library launches on the current device and the binding passes the
+    current device's stream, so a call on tensors of another device must make
+    that device current first; all CUDA tensor arguments must share it."""
+    import functools
+
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        dev = _cuda_device_of(args, kwargs)
+        torch = _torch()
+        if dev is None or dev.index == torch.cuda.current_device():
+            return fn(*args, **kwargs)
+        with torch.cuda.device(dev):
+            return fn(*args, **kwargs)
+
+    return wrapper
+
+
 def _out_code(dtype) -> int:
     torch = _torch()
     if dtype == torch.bfloat16:
@@ -195,6 +245,7 @@ def _layer(qdata, srel, codebook, s_channel, bias):
 
 # ---------------------------------------------------------------- entry points
 
+@_on_device
 def cr_rotate_quant_act(x, mp: Optional[int] = None, act_qmax: int = 127, xq=None, xs=None,
                         stream=None) -> Tuple["torch.Tensor", "torch.Tensor"]:
     """x bf16 [M, K] -> (xq int8 [MP, K], xs fp32 [MP]); rows >= M are 0 / 1."""
@@ -213,6 +264,7 @@ def cr_rotate_quant_act(x, mp: Optional[int] = None, act_qmax: int = 127, xq=Non
     return xq, xs
 
 
+@_on_device
 def cr_w4a8_decode_int8(qdata, srel, codebook, w8=None, stream=None):
     """Packed codes -> the int8 grid w8 [N, K]."""
     torch = _torch()
@@ -228,7 +280,8 @@ def cr_w4a8_decode_int8(qdata, srel, codebook, w8=None, stream=None):
     return w8
 
 
-def _contraction(fn_name, xq, xs, qdata, srel, codebook, s_channel, bias, m, out_dtype, out, acc_out, stream):
+def _contraction(fn_name, xq, xs, qdata, srel, codebook, s_channel, bias, m, out_dtype, out, acc_out, stream,
+                 w8_work=None):
     torch = _torch()
     N, K = _layer(qdata, srel, codebook, s_channel, bias)
     _need(xq, "xq", (torch.int8,), 2)
@@ -246,21 +299,40 @@ def _contraction(fn_name, xq, xs, qdata, srel, codebook, s_channel, bias, m, out
         _need(acc_out, "acc_out", (torch.int32,), shape=(M, N))
     else:
         acc_out = None
+    args = [_ptr(xq), _ptr(xs), _ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), _ptr(bias),
+            M, N, K, code, _ptr(out), _ptr(acc_out)]
+    if w8_work is not None:
+        _need(w8_work, "w8_work", (torch.int8,), shape=(N, K))
+        fn_name = "cr_w4a8_gemm_ws"
+        args.append(_ptr(w8_work))
     fn = getattr(lib(), fn_name)
-    _check(fn(_ptr(xq), _ptr(xs), _ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), _ptr(bias),
-              M, N, K, code, _ptr(out), _ptr(acc_out), _stream(stream)), fn_name)
+    _check(fn(*args, _stream(stream)), fn_name)
     return (out, acc_out) if acc_out is not None else out
 
 
+@_on_device
 def cr_w4a8_gemm(xq, xs, qdata, srel, codebook, s_channel, bias=None, m: Optional[int] = None,
-                 out_dtype=None, out=None, acc_out=None, stream=None):
+                 out_dtype=None, out=None, acc_out=None, stream=None, w8_work=None):
     """Prefill forward on quantised activations.  acc_out=True also returns the
-    int32 accumulators (out, acc)."""
+    int32 accumulators (out, acc).  With w8_work (int8 [N, K]) the weight is
+    decoded there (cr_w4a8_gemm_ws) and the library allocates nothing."""
     torch = _torch()
     return _contraction("cr_w4a8_gemm", xq, xs, qdata, srel, codebook, s_channel, bias, m,
-                        out_dtype or torch.bfloat16, out, acc_out, stream)
+                        out_dtype or torch.bfloat16, out, acc_out, stream, w8_work)
 
 
+@_on_device
+def cr_w4a8_gemm_ws(xq, xs, qdata, srel, codebook, s_channel, w8_work, bias=None, m: Optional[int] = None,
+                    out_dtype=None, out=None, acc_out=None, stream=None):
+    """cr_w4a8_gemm with the caller's weight transient w8_work int8 [N, K]."""
+    torch = _torch()
+    if w8_work is None:
+        raise ValueError("w8_work is required")
+    return _contraction("cr_w4a8_gemm_ws", xq, xs, qdata, srel, codebook, s_channel, bias, m,
+                        out_dtype or torch.bfloat16, out, acc_out, stream, w8_work)
+
+
+@_on_device
 def cr_w4a8_gemv(xq, xs, qdata, srel, codebook, s_channel, bias=None, m: Optional[int] = None,
                  out_dtype=None, out=None, acc_out=None, stream=None):
     """Decode forward (M <= 8) on quantised activations; bitwise equal to cr_w4a8_gemm."""
@@ -269,6 +341,7 @@ def cr_w4a8_gemv(xq, xs, qdata, srel, codebook, s_channel, bias=None, m: Optiona
                         out_dtype or torch.bfloat16, out, acc_out, stream)
 
 
+@_on_device
 def cr_gemm_s8(xq, xs, w8, s_channel, bias=None, m: Optional[int] = None, out_dtype=None, out=None, acc_out=None,
                stream=None):
     """The prefill contraction + epilogue on an int8 weight w8 [N, K] already
@@ -299,6 +372,7 @@ def cr_gemm_s8(xq, xs, w8, s_channel, bias=None, m: Optional[int] = None, out_dt
     return (out, acc_out) if acc_out is not None else out
 
 
+@_on_device
 def cr_epilogue(acc, xs, s_channel, bias=None, out_dtype=None, out=None, stream=None):
     torch = _torch()
     _need(acc, "acc", (torch.int32,), 2)
@@ -318,10 +392,13 @@ def cr_epilogue(acc, xs, s_channel, bias=None, out_dtype=None, out=None, stream=
     return out
 
 
+@_on_device
 def cr_w4a8_linear(x, qdata, srel, codebook, s_channel, bias=None, act_qmax: int = 127, out_dtype=None,
-                   out=None, xq_work=None, xs_work=None, stream=None):
+                   out=None, xq_work=None, xs_work=None, stream=None, w8_work=None):
     """The whole layer forward: rotate + quantise x, then the decode GEMV when
-    M <= 8, else the prefill GEMM."""
+    M <= 8, else the prefill GEMM.  With w8_work (int8 [N, K]) the prefill
+    path decodes the weight there (cr_w4a8_linear_ws) instead of a transient
+    of the library."""
     torch = _torch()
     _need(x, "x", (torch.bfloat16,), 2)
     M, K = x.shape
@@ -341,9 +418,56 @@ def cr_w4a8_linear(x, qdata, srel, codebook, s_channel, bias=None, act_qmax: int
     if out is None:
         out = torch.empty(M, N, dtype=out_dtype, device=x.device)
     _need(out, "out", (torch.bfloat16, torch.float32), shape=(M, N))
-    _check(lib().cr_w4a8_linear(_ptr(x), _ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), _ptr(bias),
-                                M, N, K, int(act_qmax), _out_code(out.dtype), _ptr(out), _ptr(xq_work),
-                                _ptr(xs_work), _stream(stream)), "cr_w4a8_linear")
+    args = [_ptr(x), _ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), _ptr(bias), M, N, K, int(act_qmax),
+            _out_code(out.dtype), _ptr(out), _ptr(xq_work), _ptr(xs_work)]
+    if w8_work is not None:
+        _need(w8_work, "w8_work", (torch.int8,), shape=(N, K))
+        _check(lib().cr_w4a8_linear_ws(*args, _ptr(w8_work), _stream(stream)), "cr_w4a8_linear_ws")
+    else:
+        _check(lib().cr_w4a8_linear(*args, _stream(stream)), "cr_w4a8_linear")
+    return out
+
+
+@_on_device
+def cr_w4a8_linear_ws(x, qdata, srel, codebook, s_channel, w8_work, bias=None, act_qmax: int = 127,
+                      out_dtype=None, out=None, xq_work=None, xs_work=None, stream=None):
+    """cr_w4a8_linear with the caller's weight transient w8_work int8 [N, K]
+    (used when M > 8; may be None for M <= 8)."""
+    torch = _torch()
+    if w8_work is None:
+        M = x.shape[0]
+        if M > CR_GEMV_MAX_M:
+            raise ValueError("w8_work is required when M > 8")
+        return _linear_ws_decode(x, qdata, srel, codebook, s_channel, bias, act_qmax, out_dtype, out, xq_work,
+                                 xs_work, stream)
+    return cr_w4a8_linear(x, qdata, srel, codebook, s_channel, bias, act_qmax, out_dtype, out, xq_work, xs_work,
+                          stream, w8_work=w8_work)
+
+
+def _linear_ws_decode(x, qdata, srel, codebook, s_channel, bias, act_qmax, out_dtype, out, xq_work, xs_work,
+                      stream):
+    """cr_w4a8_linear_ws on the decode path (M <= 8), where no transient is used."""
+    torch = _torch()
+    _need(x, "x", (torch.bfloat16,), 2)
+    M, K = x.shape
+    N, Kw = _layer(qdata, srel, codebook, s_channel, bias)
+    if Kw != K:
+        raise ValueError(f"x has K={K}, the layer K={Kw}")
+    rows = gemv_rows(M) if M >= 1 else M
+    if xq_work is None:
+        xq_work = torch.empty(rows, K, dtype=torch.int8, device=x.device)
+    if xs_work is None:
+        xs_work = torch.empty(rows, dtype=torch.float32, device=x.device)
+    _need(xq_work, "xq_work", (torch.int8,), 2)
+    _need(xs_work, "xs_work", (torch.float32,), 1)
+    if xq_work.shape[0] < rows or xs_work.shape[0] < rows:
+        raise ValueError(f"work buffers need {rows} rows")
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype or torch.bfloat16, device=x.device)
+    _need(out, "out", (torch.bfloat16, torch.float32), shape=(M, N))
+    _check(lib().cr_w4a8_linear_ws(_ptr(x), _ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), _ptr(bias),
+                                   M, N, K, int(act_qmax), _out_code(out.dtype), _ptr(out), _ptr(xq_work),
+                                   _ptr(xs_work), None, _stream(stream)), "cr_w4a8_linear_ws")
     return out
 
 
@@ -366,9 +490,10 @@ class W4A8Linear:
         self.act_qmax = int(act_qmax)
         self.out_dtype = out_dtype or torch.bfloat16
         self._tensors = (qdata, srel, codebook, s_channel, bias)  # keep them alive
+        self.device = _cuda_device_of((qdata, srel, codebook, s_channel, bias), {})
         self._L = lib()
         handle = ctypes.c_void_p()
-        with torch.cuda.device(qdata.device):
+        with torch.cuda.device(self.device):
             _check(self._L.cr_w4a8_plan_create(_ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel),
                                                _ptr(bias), self.N, self.K, self.act_qmax, _out_code(self.out_dtype),
                                                ctypes.byref(handle)), "cr_w4a8_plan_create")
@@ -408,7 +533,25 @@ class W4A8Linear:
             raise ValueError(f"xs_work must be a CUDA float32 [>= {rows}] tensor")
         return xq_work, xs_work
 
+    def _device_ctx(self, *tensors):
+        """The plan's device made current (the plan runs only there); every
+        CUDA tensor given must be on it."""
+        import contextlib
+        torch = _torch()
+        for t in tensors:
+            if isinstance(t, torch.Tensor) and t.is_cuda and t.device != self.device:
+                raise ValueError(f"tensor on {t.device}, the layer is on {self.device}")
+        if torch.cuda.current_device() == self.device.index:
+            return contextlib.nullcontext()
+        return torch.cuda.device(self.device)
+
     def forward(self, x, out=None, xq_work=None, xs_work=None, stream=None):
+        with self._device_ctx(x, out, xq_work, xs_work):
+            return self._forward(x, out, xq_work, xs_work, stream)
+
+    __call__ = forward
+
+    def _forward(self, x, out, xq_work, xs_work, stream):
         torch = _torch()
         _need(x, "x", (torch.bfloat16,), 2)
         M, K = x.shape
@@ -422,8 +565,6 @@ class W4A8Linear:
                          _stream(stream)), "cr_w4a8_plan_forward")
         return out
 
-    __call__ = forward
-
     def forward_host(self, x_host, out_host, x_dev, out_dev, xq_work=None, xs_work=None, stream=None):
         """x_host [M, K] bf16 and out_host [M, N] in host memory (pinned for
         asynchronous copies), x_dev / out_dev their device buffers: queues the
@@ -432,6 +573,10 @@ class W4A8Linear:
         buffers the call is bound to its tensors (cr_w4a8_plan_bind_host),
         and a repeat with the same tensors, unchanged in storage and shape,
         only queues the launches."""
+        with self._device_ctx(x_dev, out_dev, xq_work, xs_work):
+            return self._forward_host(x_host, out_host, x_dev, out_dev, xq_work, xs_work, stream)
+
+    def _forward_host(self, x_host, out_host, x_dev, out_dev, xq_work, xs_work, stream):
         key = (x_host, out_host, x_dev, out_dev, xq_work, xs_work)
         # the bound call is used and replaced under the lock: the C call releases
         # the GIL, and another thread must not free the call while it runs
@@ -469,14 +614,17 @@ class W4A8Linear:
         return out_host
 
 
+@_on_device
 def cr_w4a8_linear_decode_noalloc(x, qdata, srel, codebook, s_channel, bias=None, act_qmax: int = 127,
                                   out_dtype=None, out=None, stream=None):
     """The decode forward (M <= 8) for callers that cannot allocate device
-    memory during the call (e.g. while a CUDA graph is being captured): the
-    quantised activations live in a small scratch array the library reserves
-    statically per device.  Pass `out` to allocate nothing at all.  Calls that
-    overlap on the GPU share that scratch and race; make the first call on a
-    device before any stream capture."""
+    memory during the call (a serving loop whose device memory all belongs to
+    its own allocator, or a real-time path that cannot take an allocation's
+    synchronisation): the quantised activations live in a small scratch array
+    the library reserves statically per device.  Pass `out` to allocate
+    nothing at all.  Calls that overlap on the GPU share that scratch and
+    race.  The first call on a device looks up the scratch array's address;
+    make it before any stream capture on that device."""
     torch = _torch()
     _need(x, "x", (torch.bfloat16,), 2)
     M, K = x.shape
@@ -525,6 +673,7 @@ def _grouped(layers, codebook, K, M, out_dtype, outs, acc_out, device):
     return arr, res, accs
 
 
+@_on_device
 def cr_w4a8_gemv_grouped(xq, xs, codebook, layers, m: Optional[int] = None, out_dtype=None, outs=None,
                          acc_out: bool = False, stream=None):
     """Decode GEMV of 1..4 layers on the same quantised activations in one
@@ -547,6 +696,7 @@ def cr_w4a8_gemv_grouped(xq, xs, codebook, layers, m: Optional[int] = None, out_
     return (res, accs) if acc_out else res
 
 
+@_on_device
 def cr_w4a8_linear_grouped(x, codebook, layers, act_qmax: int = 127, out_dtype=None, outs=None,
                            xq_work=None, xs_work=None, stream=None):
     """Forward of 1..4 layers fed the same x (q/k/v, gate/up): one rotate +
@@ -592,6 +742,7 @@ def _swiglu_contraction(fn_name, xq, xs, qdata, srel, codebook, s_channel, bias,
     return out
 
 
+@_on_device
 def cr_w4a8_gemm_swiglu(xq, xs, qdata, srel, codebook, s_channel, bias=None, m: Optional[int] = None,
                         out_dtype=None, out=None, stream=None):
     """Prefill GEMM of an interleaved gate/up layer [2F, K] with SwiGLU fused
@@ -601,6 +752,7 @@ def cr_w4a8_gemm_swiglu(xq, xs, qdata, srel, codebook, s_channel, bias=None, m: 
                                out_dtype or torch.bfloat16, out, stream)
 
 
+@_on_device
 def cr_w4a8_gemv_swiglu(xq, xs, qdata, srel, codebook, s_channel, bias=None, m: Optional[int] = None,
                         out_dtype=None, out=None, stream=None):
     """Decode GEMV (M <= 8) of an interleaved gate/up layer with SwiGLU fused;
@@ -610,6 +762,7 @@ def cr_w4a8_gemv_swiglu(xq, xs, qdata, srel, codebook, s_channel, bias=None, m: 
                                out_dtype or torch.bfloat16, out, stream)
 
 
+@_on_device
 def cr_w4a8_linear_swiglu(x, qdata, srel, codebook, s_channel, bias=None, act_qmax: int = 127, out_dtype=None,
                           out=None, xq_work=None, xs_work=None, stream=None):
     """The forward of an interleaved gate/up layer with SwiGLU fused:
@@ -640,6 +793,7 @@ def cr_w4a8_linear_swiglu(x, qdata, srel, codebook, s_channel, bias=None, act_qm
     return out
 
 
+@_on_device
 def cr_interleave_rows(src, dst=None, stream=None):
     """Rows [0, F) and [F, 2F) of src become pairs: dst[2f] = src[f],
     dst[2f + 1] = src[F + f] (any dtype, rows along dim 0)."""
@@ -658,6 +812,7 @@ def cr_interleave_rows(src, dst=None, stream=None):
     return dst
 
 
+@_on_device
 def interleave_gate_up(gate, up, stream=None):
     """A gate/up pair of layers, each (qdata, srel, s_channel[, bias]) with
     the same K, as one layer with interleaved rows for the SwiGLU entry points
@@ -683,6 +838,7 @@ def _fixed_codebook(device):
     return _torch().tensor(FIXED_CODEBOOK, dtype=_torch().float32, device=device)
 
 
+@_on_device
 def cr_w4a8_quantize_rotated(w_rot, codebook=None, qdata=None, srel=None, s_channel=None, stream=None):
     """Offline quantiser: rotated fp32 weights [N, K] (K a multiple of 16) ->
     (qdata uint8 [N, K/2], srel uint8 [N, K/16] fp8 bytes, s_channel fp32 [N],
@@ -707,6 +863,7 @@ def cr_w4a8_quantize_rotated(w_rot, codebook=None, qdata=None, srel=None, s_chan
     return qdata, srel, s_channel, codebook
 
 
+@_on_device
 def cr_w4a8_assign_codes(w_rot, srel, s_channel, codebook, rand=None, qdata=None, stream=None):
     """New packed codes for rotated weights on stored scales: the nearest grid
     level, or with rand [N, K] fp32 uniform draws the unbiased stochastic one."""
@@ -726,9 +883,12 @@ def cr_w4a8_assign_codes(w_rot, srel, s_channel, codebook, rand=None, qdata=None
     return qdata
 
 
-def cr_w4a8_ste_backward(grad, qdata, srel, codebook, s_channel, dx=None, stream=None):
+@_on_device
+def cr_w4a8_ste_backward(grad, qdata, srel, codebook, s_channel, dx=None, stream=None, wt_work=None):
     """Straight-through input gradient: dx [M, K] bf16 = grad [M, N] bf16 @
-    (w8 * s_channel in bf16), the layer's codes decoded again (N % 8 == 0)."""
+    (w8 * s_channel in bf16), the layer's codes decoded again (N % 8 == 0).
+    With wt_work (bf16 [K, N]) the transposed weight is built there
+    (cr_w4a8_ste_backward_ws) and the library allocates nothing."""
     torch = _torch()
     N, K = _layer(qdata, srel, codebook, s_channel, None)
     _need(grad, "grad", (torch.bfloat16,), 2)
@@ -738,11 +898,26 @@ def cr_w4a8_ste_backward(grad, qdata, srel, codebook, s_channel, dx=None, stream
     if dx is None:
         dx = torch.empty(M, K, dtype=torch.bfloat16, device=grad.device)
     _need(dx, "dx", (torch.bfloat16,), shape=(M, K))
+    if wt_work is not None:
+        _need(wt_work, "wt_work", (torch.bfloat16,), shape=(K, N))
+        _check(lib().cr_w4a8_ste_backward_ws(_ptr(grad), _ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel),
+                                             M, N, K, _ptr(dx), _ptr(wt_work), _stream(stream)),
+               "cr_w4a8_ste_backward_ws")
+        return dx
     _check(lib().cr_w4a8_ste_backward(_ptr(grad), _ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), M, N,
                                       K, _ptr(dx), _stream(stream)), "cr_w4a8_ste_backward")
     return dx
 
 
+@_on_device
+def cr_w4a8_ste_backward_ws(grad, qdata, srel, codebook, s_channel, wt_work, dx=None, stream=None):
+    """cr_w4a8_ste_backward with the caller's transient wt_work bf16 [K, N]."""
+    if wt_work is None:
+        raise ValueError("wt_work is required")
+    return cr_w4a8_ste_backward(grad, qdata, srel, codebook, s_channel, dx=dx, stream=stream, wt_work=wt_work)
+
+
+@_on_device
 def cr_w4a8_dequant_t_bf16(qdata, srel, codebook, s_channel, wt=None, stream=None):
     """The backward's weight, transposed: wt [K, N] bf16, wt[k, n] = bf16(w8[n, k] * bf16(s_channel[n]))."""
     torch = _torch()

@@ -120,14 +120,21 @@ __device__ __forceinline__ float epilogue_value(int32_t acc, float xs, float ws,
 }
 
 // SwiGLU of one gate/up pair of epilogue values (h3-rs weights.rs,
-// swiglu_interleaved): silu(g) * u = g / (1 + e^-g) * u, in fp32 with CUDA's
-// expf and its fast division __fdividef (at most 2 ulp; the IEEE division's
-// slow-path branch would keep the compiler from overlapping the independent
-// pairs of a thread).  For g < -88.7, e^-g is +inf and the quotient is a zero
-// of g's sign.
+// swiglu_interleaved): silu(g) * u = g * sigmoid(g) * u, in fp32.  With
+// t = e^-|g| (CUDA's expf; t lies in (0, 1], so it never overflows):
+//   silu(g) = g / (1 + t)        for g >= 0
+//           = g * t / (1 + t)    for g <  0   (the same value, e^g = t)
+// so the divisor always lies in [1, 2], where the fast division __fdividef
+// has at most 2 ulp of error (outside [2^-126, 2^126] it does not: a divisor
+// 1 + e^-g near 2^127 would return 0 for gates around -88, and e^-g overflows
+// below -88.7, where the true result is still a normal fp32 number).  The
+// IEEE division's slow-path branch would keep the compiler from overlapping
+// the independent pairs of a thread; this form has no branch.
 __device__ __forceinline__ float swiglu_value(float g, float u)
 {
-    return __fmul_rn(__fdividef(g, __fadd_rn(1.0f, expf(-g))), u);
+    const float t = expf(-fabsf(g));
+    const float num = g >= 0.0f ? g : __fmul_rn(g, t);
+    return __fmul_rn(__fdividef(num, __fadd_rn(1.0f, t)), u);
 }
 
 __device__ __forceinline__ uint16_t to_bf16_bits(float y)

@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <functional>
 #include <cstdint>
@@ -30,13 +31,15 @@ struct DeviceState {
     bool probed = false;
     bool usable = false;
     int num_sms = 0;
-    cudaMemPool_t pool = nullptr;  // stream-ordered pool for the prefill weight transient
-    bool gemm_attr_set = false;
-    bool gemm_pair_attr_set = false;
-    bool gemv_attr_set = false;
-    bool gemv_grouped_attr_set = false;
-    bool gemm_bf16_attr_set = false;
-    bool gemm_pair_bf16_attr_set = false;
+    cudaMemPool_t pool = nullptr;  // stream-ordered pool for the weight transients (release threshold 0)
+    // kernel attributes set once (cudaFuncSetAttribute is idempotent; atomic
+    // flags so that concurrent first calls do not race on the flag itself)
+    std::atomic<bool> gemm_attr_set{false};
+    std::atomic<bool> gemm_pair_attr_set{false};
+    std::atomic<bool> gemv_attr_set{false};
+    std::atomic<bool> gemv_grouped_attr_set{false};
+    std::atomic<bool> gemm_bf16_attr_set{false};
+    std::atomic<bool> gemm_pair_bf16_attr_set{false};
     // side stream and events on which cr_w4a8_linear's prefill path decodes
     // the weight while the activations are rotated and quantised
     cudaStream_t side = nullptr;
@@ -108,7 +111,10 @@ cr_status current_device(DeviceState **out)
                 cudaGetLastError();
                 d.usable = false;
             } else {
-                uint64_t keep = UINT64_MAX;
+                // hold nothing past a synchronisation: a transient's memory
+                // goes back to the driver at the next stream, event or device
+                // synchronisation after it was freed
+                uint64_t keep = 0;
                 cudaMemPoolSetAttribute(d.pool, cudaMemPoolAttrReleaseThreshold, &keep);
             }
         }
@@ -244,7 +250,7 @@ cr_status build_gemv_args(cr::gv::GemvArgs<L> &args, const float *codebook, int6
 // many CTAs as fit on the SMs, optionally as a programmatic dependent of the
 // previous kernel on the stream.
 template <int L>
-cr_status launch_gemv_args(int num_sms, bool &attr_set, const cr::gv::GemvArgs<L> &args, cudaStream_t stream,
+cr_status launch_gemv_args(int num_sms, std::atomic<bool> &attr_set, const cr::gv::GemvArgs<L> &args, cudaStream_t stream,
                            bool pdl)
 {
     using namespace cr;
@@ -274,7 +280,7 @@ cr_status launch_gemv_args(int num_sms, bool &attr_set, const cr::gv::GemvArgs<L
 }
 
 template <int L>
-cr_status launch_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const float *codebook,
+cr_status launch_gemv(int num_sms, std::atomic<bool> &attr_set, const int8_t *xq, const float *xs, const float *codebook,
                       int64_t M, int64_t K, const cr_w4a8_layer *layers, int num_layers, cr_out_dtype out_dtype,
                       cudaStream_t stream, bool pdl, int swiglu = 0)
 {
@@ -303,7 +309,7 @@ cr_status run_gemv_layers(DeviceState &d, const int8_t *xq, const float *xs, con
 }
 
 // One layer.
-cr_status run_gemv(int num_sms, bool &attr_set, const int8_t *xq, const float *xs, const uint8_t *qdata,
+cr_status run_gemv(int num_sms, std::atomic<bool> &attr_set, const int8_t *xq, const float *xs, const uint8_t *qdata,
                    const uint8_t *srel, const float *codebook, const float *s_channel, const float *bias, int64_t M,
                    int64_t N, int64_t K, cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream,
                    bool pdl, int swiglu = 0)
@@ -486,16 +492,20 @@ cr_status gemm_on_w8(DeviceState &d, const int8_t *xq, const float *xs, const in
 // The prefill contraction.  When `activations` is given (cr_w4a8_linear), it
 // launches the activation kernel on `stream` while the weight decode runs on
 // the device's side stream (the two are independent); the GEMM waits for both.
+// The weight is decoded into the caller's w8_work [N, K] when given, otherwise
+// into a transient from the device's stream-ordered pool, freed on `stream`
+// after the GEMM.
 cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
                    const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K,
                    cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream,
-                   const std::function<cr_status()> *activations = nullptr, int swiglu = 0)
+                   const std::function<cr_status()> *activations = nullptr, int swiglu = 0,
+                   int8_t *w8_work = nullptr)
 {
     using namespace cr;
-    // The int8 grid of the weight, decoded once per call into a transient
-    // from the library's stream-ordered pool.
-    int8_t *w8 = nullptr;
-    if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&w8), (size_t)(N * K), d.pool, stream) != cudaSuccess) {
+    // The int8 grid of the weight, decoded once per call.
+    int8_t *w8 = w8_work;
+    if (w8 == nullptr &&
+        cudaMallocFromPoolAsync(reinterpret_cast<void **>(&w8), (size_t)(N * K), d.pool, stream) != cudaSuccess) {
         cudaGetLastError();
         return CR_ERR_CUDA;
     }
@@ -524,7 +534,7 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
     }
     if (st == CR_OK)
         st = gemm_on_w8(d, xq, xs, w8, s_channel, bias, M, N, K, out_dtype, out, acc_out, stream, swiglu);
-    if (cudaFreeAsync(w8, stream) != cudaSuccess) {
+    if (w8_work == nullptr && cudaFreeAsync(w8, stream) != cudaSuccess) {
         cudaGetLastError();
         if (st == CR_OK)
             st = CR_ERR_CUDA;
@@ -646,6 +656,26 @@ cr_status cr_w4a8_gemm(const int8_t *xq, const float *xs, const uint8_t *qdata, 
     return run_gemm(*d, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, acc_out, stream);
 }
 
+cr_status cr_w4a8_gemm_ws(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
+                          const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N,
+                          int64_t K, cr_out_dtype out_dtype, void *out, int32_t *acc_out, int8_t *w8_work,
+                          cr_stream_t stream)
+{
+    cr_status st = check_contraction(xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, acc_out);
+    if (st != CR_OK || M == 0 || N == 0)
+        return st;
+    if (!w8_work)
+        return CR_ERR_INVALID_ARG;
+    if (!aligned16(w8_work))
+        return CR_ERR_ALIGNMENT;
+    DeviceState *d = nullptr;
+    st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    return run_gemm(*d, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, acc_out, stream,
+                    nullptr, 0, w8_work);
+}
+
 cr_status cr_w4a8_gemv(const int8_t *xq, const float *xs, const uint8_t *qdata, const uint8_t *srel,
                        const float *codebook, const float *s_channel, const float *bias, int64_t M, int64_t N,
                        int64_t K, cr_out_dtype out_dtype, void *out, int32_t *acc_out, cr_stream_t stream)
@@ -688,10 +718,13 @@ namespace {
 
 // cr_w4a8_linear and cr_w4a8_linear_swiglu: rotate + quantise, then the GEMV
 // (M <= 8) or the GEMM with the weight decode overlapping the activations.
+// With ws_given, the prefill path (M > 8) decodes the weight into the
+// caller's w8_work [N, K] (which must then be given) instead of a pool
+// transient.
 cr_status linear_impl(const uint16_t *x, const uint8_t *qdata, const uint8_t *srel, const float *codebook,
                       const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K, int act_qmax,
                       cr_out_dtype out_dtype, void *out, int8_t *xq_work, float *xs_work, cudaStream_t stream,
-                      int swiglu)
+                      int swiglu, bool ws_given = false, int8_t *w8_work = nullptr)
 {
     if (M < 0 || N < 0 || K < 0 || act_qmax < 1 || act_qmax > 127)
         return CR_ERR_INVALID_ARG;
@@ -711,6 +744,12 @@ cr_status linear_impl(const uint16_t *x, const uint8_t *qdata, const uint8_t *sr
         return CR_ERR_INVALID_ARG;
     if (!aligned16(x))
         return CR_ERR_ALIGNMENT;
+    if (ws_given && M > CR_GEMV_MAX_M) {
+        if (!w8_work)
+            return CR_ERR_INVALID_ARG;
+        if (!aligned16(w8_work))
+            return CR_ERR_ALIGNMENT;
+    }
     DeviceState *d = nullptr;
     st = current_device(&d);
     if (st != CR_OK)
@@ -719,7 +758,7 @@ cr_status linear_impl(const uint16_t *x, const uint8_t *qdata, const uint8_t *sr
     if (M > CR_GEMV_MAX_M) {
         const std::function<cr_status()> act = activations;
         return run_gemm(*d, xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, nullptr,
-                        stream, &act, swiglu);
+                        stream, &act, swiglu, ws_given ? w8_work : nullptr);
     }
     st = activations();
     if (st != CR_OK)
@@ -787,6 +826,15 @@ cr_status cr_w4a8_linear(const uint16_t *x, const uint8_t *qdata, const uint8_t 
                        stream, 0);
 }
 
+cr_status cr_w4a8_linear_ws(const uint16_t *x, const uint8_t *qdata, const uint8_t *srel, const float *codebook,
+                            const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K, int act_qmax,
+                            cr_out_dtype out_dtype, void *out, int8_t *xq_work, float *xs_work, int8_t *w8_work,
+                            cr_stream_t stream)
+{
+    return linear_impl(x, qdata, srel, codebook, s_channel, bias, M, N, K, act_qmax, out_dtype, out, xq_work, xs_work,
+                       stream, 0, /*ws_given=*/true, w8_work);
+}
+
 cr_status cr_w4a8_linear_swiglu(const uint16_t *x, const uint8_t *qdata, const uint8_t *srel, const float *codebook,
                                 const float *s_channel, const float *bias, int64_t M, int64_t N, int64_t K,
                                 int act_qmax, cr_out_dtype out_dtype, void *out, int8_t *xq_work, float *xs_work,
@@ -848,9 +896,12 @@ cr_status cr_w4a8_dequant_t_bf16(const uint8_t *qdata, const uint8_t *srel, cons
                                                   stream));
 }
 
-cr_status cr_w4a8_ste_backward(const uint16_t *grad, const uint8_t *qdata, const uint8_t *srel,
-                               const float *codebook, const float *s_channel, int64_t M, int64_t N, int64_t K,
-                               uint16_t *dx, cr_stream_t stream)
+namespace {
+// cr_w4a8_ste_backward(_ws): wt_work [K, N] bf16 is the caller's transient
+// when ws_given (it must then be given), otherwise one from the pool.
+cr_status ste_backward_impl(const uint16_t *grad, const uint8_t *qdata, const uint8_t *srel,
+                            const float *codebook, const float *s_channel, int64_t M, int64_t N, int64_t K,
+                            uint16_t *dx, cudaStream_t stream, bool ws_given, uint16_t *wt_work)
 {
     if (M < 0)
         return CR_ERR_INVALID_ARG;
@@ -863,6 +914,12 @@ cr_status cr_w4a8_ste_backward(const uint16_t *grad, const uint8_t *qdata, const
         if (!dx)
             return CR_ERR_INVALID_ARG;
         return cudaMemsetAsync(dx, 0, (size_t)(M * K) * 2, stream) == cudaSuccess ? CR_OK : CR_ERR_CUDA;
+    }
+    if (ws_given) {
+        if (!wt_work)
+            return CR_ERR_INVALID_ARG;
+        if (!aligned16(wt_work))
+            return CR_ERR_ALIGNMENT;
     }
     DeviceState *d = nullptr;
     st = current_device(&d);
@@ -877,9 +934,11 @@ cr_status cr_w4a8_ste_backward(const uint16_t *grad, const uint8_t *qdata, const
         }
         d->gemm_bf16_attr_set = true;
     }
-    // the transposed bf16 weight, from the stream-ordered pool
-    uint16_t *wt = nullptr;
-    if (cudaMallocFromPoolAsync(reinterpret_cast<void **>(&wt), (size_t)(N * K) * 2, d->pool, stream) != cudaSuccess) {
+    // the transposed bf16 weight: the caller's transient, or one from the
+    // stream-ordered pool
+    uint16_t *wt = wt_work;
+    if (!ws_given &&
+        cudaMallocFromPoolAsync(reinterpret_cast<void **>(&wt), (size_t)(N * K) * 2, d->pool, stream) != cudaSuccess) {
         cudaGetLastError();
         return CR_ERR_CUDA;
     }
@@ -931,12 +990,27 @@ cr_status cr_w4a8_ste_backward(const uint16_t *grad, const uint8_t *qdata, const
             /*tma_out=*/1, dx, nullptr);
         st = launched(cudaGetLastError());
     }
-    if (cudaFreeAsync(wt, stream) != cudaSuccess) {
+    if (!ws_given && cudaFreeAsync(wt, stream) != cudaSuccess) {
         cudaGetLastError();
         if (st == CR_OK)
             st = CR_ERR_CUDA;
     }
     return st;
+}
+}  // namespace
+
+cr_status cr_w4a8_ste_backward(const uint16_t *grad, const uint8_t *qdata, const uint8_t *srel,
+                               const float *codebook, const float *s_channel, int64_t M, int64_t N, int64_t K,
+                               uint16_t *dx, cr_stream_t stream)
+{
+    return ste_backward_impl(grad, qdata, srel, codebook, s_channel, M, N, K, dx, stream, false, nullptr);
+}
+
+cr_status cr_w4a8_ste_backward_ws(const uint16_t *grad, const uint8_t *qdata, const uint8_t *srel,
+                                  const float *codebook, const float *s_channel, int64_t M, int64_t N, int64_t K,
+                                  uint16_t *dx, uint16_t *wt_work, cr_stream_t stream)
+{
+    return ste_backward_impl(grad, qdata, srel, codebook, s_channel, M, N, K, dx, stream, true, wt_work);
 }
 
 namespace {
@@ -1346,13 +1420,14 @@ struct NoallocState {
     bool ready = false;
     uint8_t *scratch = nullptr;  // device address of g_noalloc_scratch on this device
     int num_sms = 0;
-    bool gemv_attr_set = false;
+    std::atomic<bool> gemv_attr_set{false};  // set in noalloc_scratch, under the lock
 };
 NoallocState g_noalloc[kMaxDevices];
 
 // Once per device, with that device current: check it is an sm_100 part,
 // look up the scratch array's device address, the SM count and the tensor-map
-// encoder.  Allocates nothing.
+// encoder, and set the decode GEMV's shared-memory attribute.  Allocates
+// nothing.
 cr_status noalloc_scratch(NoallocState **out)
 {
     int dev = -1;
@@ -1383,6 +1458,12 @@ cr_status noalloc_scratch(NoallocState **out)
             return CR_ERR_CUDA;
         }
         s.scratch = static_cast<uint8_t *>(p);
+        if (cudaFuncSetAttribute(cr::gv::gemv_kernel<cr::gv::Prod, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)cr::gv::Prod::kSmemBytes) != cudaSuccess) {
+            cudaGetLastError();
+            return CR_ERR_CUDA;
+        }
+        s.gemv_attr_set = true;
         s.ready = true;
     }
     *out = &s;
@@ -1403,6 +1484,8 @@ cr_status cr_w4a8_linear_decode_noalloc(const uint16_t *x, const uint8_t *qdata,
         return k;
     if (M > CR_GEMV_MAX_M)
         return CR_ERR_UNSUPPORTED;  // the padded activations would not fit the static scratch
+    if (N > INT_MAX)
+        return CR_ERR_UNSUPPORTED;
     if (M == 0 || N == 0)
         return CR_OK;
     int64_t MP = 1;
