@@ -52,8 +52,16 @@ def parse():
     p.add_argument("--steps", type=int, default=200)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    p.add_argument("--workload", default="c2_decode_m8_4k")
-    p.add_argument("--prefill-workload", default="c3_prefill_2k_4k")
+    p.add_argument("--workload", default="c5_m8_8k")
+    p.add_argument("--prefill-workload", default="c5_m16384_8k")
+    p.add_argument("--gemv-extra", default="c1_decode_m1_1k,c2_decode_m8_4k,c5_m1_8k,c5_m2_8k,c5_m4_8k",
+                   help="comma-separated decode workloads reported beside the headline (empty: none)")
+    p.add_argument("--prefill-extra", default="c3_prefill_2k_4k,c4_mlp_up,c4_mlp_down",
+                   help="comma-separated prefill workloads reported beside the prefill block (empty: none)")
+    p.add_argument("--backward-workload", default="c3_prefill_2k_4k")
+    p.add_argument("--only", default=None, choices=["headline", "decode-transient", "quantiser", "int8-peak"],
+                   help="run one piece alone (profiling runs): the headline step and GEMV, the prefill weight "
+                        "transient, the offline quantiser, or the INT8 rate kernel")
     p.add_argument("--no-prefill", action="store_true")
     p.add_argument("--no-grouped", action="store_true")
     p.add_argument("--no-swiglu", action="store_true")
@@ -412,6 +420,71 @@ def cpu_baseline(case, seconds):
             "cpu_model": model}
 
 
+def gemv_block(case, args, world, rank, local, pk, sets=None):
+    """One decode workload: the whole step (rotate+quant launch + GEMV
+    launch) as one CUDA-graph replay of K steps, and the GEMV kernel alone
+    the same way (its roofline).  Rotating copies of layer + activations
+    larger than L2 make every step stream its weights from HBM."""
+    if sets is None:
+        sets = Sets(case, rank)
+    M, N, K = case.M, case.N, case.K
+    secs, clocks = graph_time(sets.step, args.steps, args.warmup, world, local)
+    secs = max_over_ranks(secs, world)
+    wb = weight_bytes(N, K)
+    ksecs, _ = graph_time(sets.contraction_only, args.steps, args.warmup, world, local)
+    ksecs = max_over_ranks(ksecs, world)
+    per_launch = ksecs / args.steps
+    achieved = gemv_launch_bytes(M, N, K) / per_launch / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": prior_traffic(f"gemv_kernel_{case.name}"),
+                "kernel": "cr::gv::gemv_kernel", "peak_source": f"{pk['source']} (hbm_gbs)",
+                "algorithmic_bytes_per_launch": gemv_launch_bytes(M, N, K),
+                "us_per_launch": round(per_launch * 1e6, 3)}
+    return {"workload": f"{case.name}: decode batch M={M}, N={N}, K={K}, rot 256, group 16, seed {case.seed}",
+            "value": round(aggregate_value(wb, args.steps, world, secs), 2), "unit": "GB/s",
+            "us_per_step": round(secs / args.steps * 1e6, 3),
+            "l2": f"rotating {sets.R} copies of layer+activations ({sets.R * (wb + 2 * M * K) / 2**20:.0f} MiB)",
+            "roofline": roofline, "_secs": secs, "_clocks": clocks, "_sets": sets}
+
+
+def measure_int8_peak(world):
+    """The dense INT8 tensor-core rate of this GPU: the library's
+    measurement kernel (resident shared-memory operands, tcgen05 kind::i8 on
+    CTA pairs, the prefill GEMM's instruction shape), timed with CUDA events;
+    the best of several launches of about 2 ms."""
+    import torch
+
+    import w4a8_codebook_quantized_b200 as cr
+    stream = torch.cuda.Stream()
+    iters = 4096
+    with torch.cuda.stream(stream):
+        ops = cr.cr_mma_i8_peak(iters, stream=stream)
+        stream.synchronize()
+        # size the launch to about 2 ms
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        cr.cr_mma_i8_peak(iters, stream=stream)
+        e1.record(stream)
+        stream.synchronize()
+        t = e0.elapsed_time(e1) / 1000.0
+        iters = int(min(1 << 20, max(1024, iters * 2e-3 / max(t, 1e-6))))
+        best, times = None, []
+        for _ in range(5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            ops = cr.cr_mma_i8_peak(iters, stream=stream)
+            e1.record(stream)
+            stream.synchronize()
+            times.append(e0.elapsed_time(e1) / 1000.0)
+    cr.cr_check_device_error(stream)
+    t = min(times)
+    t = max_over_ranks(t, world)
+    return {"value": round(ops / t / 1e12, 1), "unit": "TOPS", "iters": iters, "ms_per_launch": round(t * 1e3, 4),
+            "kernel": "cr::pk::mma_i8_peak_kernel (tcgen05.mma.cta_group::2.kind::i8, M=N=256, K=32, operands "
+                      "resident in shared memory, one cluster of two CTAs per SM pair)",
+            "launches": len(times)}
+
+
 def run_ours(args):
     import torch
 
@@ -420,30 +493,19 @@ def run_ours(args):
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
     cr.lib()
+    if args.only in ("decode-transient", "quantiser", "int8-peak"):
+        return run_only(args, world, rank, local)
     pk = peaks()
     case = inputs.CASES[args.workload]
     if case.M > 8:
         raise SystemExit("the headline workload must be a decode batch (M <= 8)")
     M, N, K = case.M, case.N, case.K
-    sets = Sets(case, rank)
 
     # headline: the whole step (rotate+quant launch + GEMV launch), graph-replayed
-    secs, clocks = graph_time(sets.step, args.steps, args.warmup, world, local)
-    secs = max_over_ranks(secs, world)
+    head = gemv_block(case, args, world, rank, local, pk)
+    secs, clocks, sets = head.pop("_secs"), head.pop("_clocks"), head.pop("_sets")
     wb = weight_bytes(N, K)
     value = aggregate_value(wb, args.steps, world, secs)
-
-    # the dominant kernel alone (GEMV), for the roofline
-    ksecs, _ = graph_time(sets.contraction_only, args.steps, args.warmup, world, local)
-    ksecs = max_over_ranks(ksecs, world)
-    per_launch = ksecs / args.steps
-    achieved = gemv_launch_bytes(M, N, K) / per_launch / 1e9
-    traffic = prior_traffic("gemv_kernel_c2")
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
-                "kernel": "cr::gv::gemv_kernel", "peak_source": f"{pk['source']} (hbm_gbs)",
-                "algorithmic_bytes_per_launch": gemv_launch_bytes(M, N, K),
-                "us_per_launch": round(per_launch * 1e6, 3)}
 
     # end to end through the public API with host buffers
     # warm-up covers every rotating layer at least twice (first calls encode
@@ -455,21 +517,38 @@ def run_ours(args):
            "ms_per_step": round(esecs / args.steps * 1e3, 5),
            "path": "W4A8Linear.forward_host (bound call, cr_w4a8_host_call_run), eager: x from pinned host memory "
                    "by a copy kernel, rotate+quant, GEMV, y to pinned host memory by a copy kernel (4 launches)"}
+    del sets
 
-    prefill = None
-    if not args.no_prefill:
-        prefill = run_prefill(args, world, rank, local, pk)
+    gemv_extra = []
+    if args.only != "headline":
+        for name in [w for w in args.gemv_extra.split(",") if w and w != args.workload]:
+            blk = gemv_block(inputs.CASES[name], args, world, rank, local, pk)
+            for k in ("_secs", "_clocks", "_sets"):
+                blk.pop(k)
+            gemv_extra.append(blk)
+            torch.cuda.empty_cache()
+
+    int8_peak = None
+    prefill = prefill_extra = None
+    if not args.no_prefill and args.only != "headline":
+        int8_peak = measure_int8_peak(world)
+        prefill = run_prefill(args, world, rank, pk, int8_peak, args.prefill_workload)
+        torch.cuda.empty_cache()
+        prefill_extra = []
+        for name in [w for w in args.prefill_extra.split(",") if w and w != args.prefill_workload]:
+            prefill_extra.append(run_prefill(args, world, rank, pk, int8_peak, name))
+            torch.cuda.empty_cache()
 
     grouped = None
-    if not args.no_grouped:
-        grouped = run_grouped(args, world, rank, local, case)
+    if not args.no_grouped and args.only != "headline":
+        grouped = run_grouped(args, world, rank, local, inputs.CASES["c2_decode_m8_4k"])
 
     swiglu = None
-    if not args.no_swiglu:
+    if not args.no_swiglu and args.only != "headline":
         swiglu = run_swiglu(args, world, rank, pk)
 
     backward = None
-    if not args.no_backward:
+    if not args.no_backward and args.only != "headline":
         backward = run_backward(args, world, rank, pk)
 
     cpu = None
@@ -480,13 +559,14 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
-        "config": {"workload": f"{case.name}: decode batch M={M}, N={N}, K={K}, rot 256, group 16, seed {case.seed}",
+        "config": {"workload": head["workload"],
                    "path": "cr_w4a8_linear = rotate+quant kernel + fused decode GEMV kernel",
-                   "l2": f"rotating {sets.R} copies of layer+activations ({sets.R * (wb + 2 * M * K) / 2**20:.0f} MiB > 126 MiB L2)",
+                   "l2": head["l2"] + " > 126 MiB L2",
                    "timing": "one CUDA-graph replay of K steps (graph uploaded beforehand), CUDA events on the capture stream",
                    "parallelism": f"replica x{world}"},
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps,
-        "clocks": clocks, "prefill": prefill, "grouped": grouped, "swiglu": swiglu, "ste_backward": backward,
+        "roofline": head["roofline"], "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps,
+        "clocks": clocks, "gemv_extra": gemv_extra, "int8_peak": int8_peak, "prefill": prefill,
+        "prefill_extra": prefill_extra, "grouped": grouped, "swiglu": swiglu, "ste_backward": backward,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -495,16 +575,17 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_prefill(args, world, rank, local, pk):
-    """The prefill step through cr_w4a8_linear (rotate+quant overlapped with the
-    weight decode, then the tcgen05 GEMM); the GEMM kernel alone (cr_gemm_s8
-    on the decoded weight: the roofline) and the cr_w4a8_gemm call (decode +
-    GEMM) beside it."""
+def run_prefill(args, world, rank, pk, int8_peak, workload):
+    """One prefill workload: the step through cr_w4a8_linear (rotate+quant
+    overlapped with the weight decode, then the tcgen05 GEMM); the GEMM
+    kernel alone (cr_gemm_s8 on the decoded weight: the roofline, against the
+    INT8 rate measured in this run) and the cr_w4a8_gemm call (decode + GEMM)
+    beside it.  Each replay follows a 256 MiB L2 flush (outside the events)."""
     import torch
 
     import w4a8_codebook_quantized_b200 as cr
     from w4a8_codebook_quantized_b200 import inputs
-    case = inputs.CASES[args.prefill_workload]
+    case = inputs.CASES[workload]
     M, N, K = case.M, case.N, case.K
     layer = inputs.layer(N, K, rank_seed(case.seed, rank))
     x = inputs.activations(M, K, rank_seed(case.seed, rank), case.dist)
@@ -513,71 +594,94 @@ def run_prefill(args, world, rank, local, pk):
     cb = torch.from_numpy(layer.codebook).cuda()
     ws = torch.from_numpy(layer.s_channel).cuda()
     xd = torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    del x
     xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
     xs = torch.empty(M, dtype=torch.float32, device="cuda")
     out = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device="cuda")
     steps = max(3, min(args.steps, 50))
 
-    def step(i):
+    def step():
         cr.cr_w4a8_linear(xd, q, s, cb, ws, out=out, xq_work=xq, xs_work=xs)
 
     for i in range(max(3, args.warmup)):
-        step(i)
-    # The step (cr_w4a8_linear: rotate+quant, weight decode, GEMM) and the
-    # GEMM call alone are captured as CUDA graphs (uploaded before timing), so
-    # the events measure device time, not the host's argument checks and
-    # tensor-map encoding.  L2 flushed before every timed replay (outside the
-    # events).
-    stream = torch.cuda.Stream()
-    torch.cuda.synchronize()
-    # The GEMM kernel alone runs through cr_gemm_s8 on the weight decoded once
-    # beforehand (the same kernel cr_w4a8_gemm launches after its decode).
+        step()
+    # the GEMM kernel alone runs through cr_gemm_s8 on the weight decoded once
+    # beforehand (the same kernel and arguments cr_w4a8_gemm launches after
+    # its decode)
     w8 = cr.cr_w4a8_decode_int8(q, s, cb)
     cr.cr_gemm_s8(xq, xs, w8, ws, out=out)
     torch.cuda.synchronize()
-    g_step, g_mm, g_k = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step, stream=stream):
-        step(0)
-    with torch.cuda.graph(g_mm, stream=stream):
-        cr.cr_w4a8_gemm(xq, xs, q, s, cb, ws, out=out)
-    with torch.cuda.graph(g_k, stream=stream):
-        cr.cr_gemm_s8(xq, xs, w8, ws, out=out)
-    for g in (g_step, g_mm, g_k):
-        upload_graph(g, stream)
-
-    def timed(g):
-        res = []
-        with torch.cuda.stream(stream):
-            for i in range(steps):
-                flush.fill_(i & 0xFF)
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                g.replay()
-                e1.record(stream)
-                torch.cuda.synchronize()
-                res.append(e0.elapsed_time(e1) / 1000.0)
-        return res
-    times = timed(g_step)
-    ct = timed(g_mm)
-    kt = timed(g_k)
-    del g_step, g_mm, g_k, w8
-    t = max_over_ranks(statistics.median(times), world)
-    tc = max_over_ranks(statistics.median(ct), world)
-    tg = max_over_ranks(statistics.median(kt), world)
+    ts, tc, tg = flushed_medians([step, lambda: cr.cr_w4a8_gemm(xq, xs, q, s, cb, ws, out=out),
+                                  lambda: cr.cr_gemm_s8(xq, xs, w8, ws, out=out)], steps)
+    del w8
+    t, tc, tg = max_over_ranks(ts, world), max_over_ranks(tc, world), max_over_ranks(tg, world)
     ops = 2.0 * M * N * K
-    peak_tops = pk["bf16_tflops"] * INT8_OVER_BF16
     achieved = ops / tg / 1e12
+    if int8_peak is not None:
+        peak_tops, src = int8_peak["value"], "measured in this run (int8_peak: tcgen05 kind::i8 rate kernel)"
+    else:
+        peak_tops, src = pk["bf16_tflops"] * INT8_OVER_BF16, \
+            f"{pk['source']} bf16_tflops x {INT8_OVER_BF16} (nominal int8/bf16 ratio)"
     return {"workload": f"{case.name}: prefill M={M}, N={N}, K={K}", "value": round(world * ops / t / 1e12, 2),
             "unit": "TOPS", "ms_per_step": round(t * 1e3, 4), "steps": steps,
             "l2": "256 MiB write between steps, outside the timed events",
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak_tops, 1),
                          "unit": "TOPS", "frac": round(achieved / peak_tops, 4), "traffic": None,
                          "kernel": "tcgen05 int8 GEMM + epilogue (cr_gemm_s8 on the decoded int8 weight)",
-                         "peak_source": f"{pk['source']} bf16_tflops x {INT8_OVER_BF16} (nominal int8/bf16 ratio)",
-                         "us_per_call": round(tg * 1e6, 2)},
+                         "peak_source": src, "us_per_call": round(tg * 1e6, 2),
+                         "frac_of_bf16x2": round(achieved / (pk["bf16_tflops"] * INT8_OVER_BF16), 4)},
             "gemm_call": {"what": "cr_w4a8_gemm: weight decode to an int8 transient + the same GEMM",
-                          "us": round(tc * 1e6, 2), "tops": round(ops / tc / 1e12, 1)}}
+                          "us": round(tc * 1e6, 2), "tops": round(ops / tc / 1e12, 1),
+                          "frac": round(ops / tc / 1e12 / peak_tops, 4)}}
+
+
+def run_only(args, world, rank, local):
+    """Single pieces for profiling runs (one JSON line each)."""
+    import torch
+
+    import w4a8_codebook_quantized_b200 as cr
+    from w4a8_codebook_quantized_b200 import inputs
+    out = {"only": args.only}
+    if args.only == "int8-peak":
+        out.update(measure_int8_peak(world))
+    elif args.only == "decode-transient":
+        # the prefill's int8 weight transient on an [8192, 4096] layer: two
+        # warm launches, then 20 back to back timed with CUDA events
+        N, K = 8192, 4096
+        layer = inputs.layer(N, K, 1)
+        q, s, cb = (torch.from_numpy(a).cuda() for a in (layer.qdata, layer.srel, layer.codebook))
+        w8 = torch.empty(N, K, dtype=torch.int8, device="cuda")
+        for _ in range(2):
+            cr.cr_w4a8_decode_int8(q, s, cb, w8)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(20):
+            cr.cr_w4a8_decode_int8(q, s, cb, w8)
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) / 1000.0 / 20
+        out.update({"N": N, "K": K, "us": round(t * 1e6, 2),
+                    "gb_per_s": round(N * K * (0.5 + 1 / 16 + 1) / t / 1e9, 1)})
+    elif args.only == "quantiser":
+        # the offline quantiser and the stochastic re-assignment on an
+        # [8192, 4096] rotated weight
+        N, K = 8192, 4096
+        w = torch.from_numpy(inputs.rotated_weights(N, K, 1)).cuda()
+        cb = torch.tensor(inputs.FIXED_CODEBOOK, dtype=torch.float32, device="cuda")
+        u = torch.from_numpy(inputs.uniforms(N, K, 1)).cuda()
+        q, s, ch, _ = cr.cr_w4a8_quantize_rotated(w, cb)
+        cr.cr_w4a8_assign_codes(w, s, ch, cb, u, q)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        cr.cr_w4a8_quantize_rotated(w, cb, q, s, ch)
+        e1.record()
+        torch.cuda.synchronize()
+        out.update({"N": N, "K": K, "quantize_us": round(e0.elapsed_time(e1) * 1e3, 1)})
+    cr.cr_check_device_error()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
 
 
 def flushed_medians(fns, steps):
@@ -653,7 +757,7 @@ def run_backward(args, world, rank, pk):
 
     import w4a8_codebook_quantized_b200 as cr
     from w4a8_codebook_quantized_b200 import inputs
-    case = inputs.CASES[args.prefill_workload]
+    case = inputs.CASES[args.backward_workload]
     M, N, K = case.M, case.N, case.K
     layer = inputs.layer(N, K, rank_seed(case.seed, rank))
     q, s, cb, ws = (torch.from_numpy(a).cuda() for a in (layer.qdata, layer.srel, layer.codebook, layer.s_channel))
@@ -761,7 +865,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
-            "config": {"workload": f"{case.name}: decode batch M={M}, N={N}, K={K}, rot 256, group 16",
+            "config": {"workload": f"{case.name}: decode batch M={M}, N={N}, K={K}, rot 256, group 16, seed {case.seed}",
                        "parallelism": "host CPU, 1 thread"},
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": sample},

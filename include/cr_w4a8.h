@@ -545,6 +545,18 @@ cr_status cr_gemm_s8(const int8_t *xq, const float *xs, const int8_t *w8, const 
 cr_status cr_selftest_wait_timeout(uint64_t limit_ns, cr_stream_t stream);
 
 /*
+ * (18) Measurement of the dense INT8 tensor-core rate (the prefill GEMM's
+ * roofline denominator; not part of the layer).  Launches one cluster of two
+ * CTAs per SM pair; each pair issues `iters` (1 .. 2^20) groups of four
+ * tcgen05.mma.cta_group::2.kind::i8 (M = 256, N = 256, K = 32, the prefill
+ * GEMM's instruction) on int8 tiles resident in shared memory, accumulating
+ * in TMEM, with no global memory traffic.  *ops_per_launch (host) receives
+ * the int8 operations one launch performs (2 * 256 * 256 * 128 * iters per
+ * pair); the caller times the launch on `stream` (CUDA events) and divides.
+ */
+cr_status cr_mma_i8_peak(int64_t iters, double *ops_per_launch, cr_stream_t stream);
+
+/*
  * Waits for `stream`, then reads and clears the library's device error word,
  * which a kernel sets when one of its bounded pipeline waits runs out (the
  * kernel then abandons its tile and exits; its outputs are unspecified).

@@ -22,7 +22,7 @@ def test_reference_arm_json_line():
         assert key in d, key
     assert d["unit"] == "GB/s" and d["higher_is_better"] is True and d["steps"] == 1 and d["warmup"] == 1
     assert d["value"] > 0 and d["ms_per_step"] > 0
-    assert d["config"]["workload"].startswith("c2_decode_m8_4k")
+    assert d["config"]["workload"].startswith("c5_m8_8k")
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     e2e = d["e2e"]

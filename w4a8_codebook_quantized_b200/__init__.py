@@ -30,7 +30,7 @@ __all__ = [
     "cr_w4a8_gemm_swiglu", "cr_w4a8_gemv_swiglu", "cr_w4a8_linear_swiglu", "cr_interleave_rows",
     "interleave_gate_up", "cr_w4a8_quantize_rotated", "cr_w4a8_assign_codes",
     "cr_w4a8_ste_backward", "cr_w4a8_dequant_t_bf16", "cr_selftest_wait_timeout", "cr_gemm_s8",
-    "cr_w4a8_gemm_ws", "cr_w4a8_linear_ws", "cr_w4a8_ste_backward_ws",
+    "cr_w4a8_gemm_ws", "cr_w4a8_linear_ws", "cr_w4a8_ste_backward_ws", "cr_mma_i8_peak",
     "cr_status_string", "cr_version",
     "gemv_rows",
 ]
@@ -105,6 +105,7 @@ def lib() -> ctypes.CDLL:
             L.cr_gemm_s8.argtypes = [P, P, P, P, P, i64, i64, i64, i32, P, P, P]
             L.cr_w4a8_dequant_t_bf16.argtypes = [P, P, P, P, i64, i64, P, P]
             L.cr_w4a8_gemm_ws.argtypes = contraction[:-1] + [P, P]
+            L.cr_mma_i8_peak.argtypes = [i64, ctypes.POINTER(ctypes.c_double), P]
             L.cr_w4a8_linear_ws.argtypes = [P, P, P, P, P, P, i64, i64, i64, i32, i32, P, P, P, P, P]
             L.cr_w4a8_ste_backward_ws.argtypes = [P, P, P, P, P, i64, i64, i64, P, P, P]
             LP = ctypes.POINTER(CrLayer)
@@ -928,6 +929,15 @@ def cr_w4a8_dequant_t_bf16(qdata, srel, codebook, s_channel, wt=None, stream=Non
     _check(lib().cr_w4a8_dequant_t_bf16(_ptr(qdata), _ptr(srel), _ptr(codebook), _ptr(s_channel), N, K, _ptr(wt),
                                         _stream(stream)), "cr_w4a8_dequant_t_bf16")
     return wt
+
+
+def cr_mma_i8_peak(iters: int, stream=None) -> float:
+    """Queue the INT8 tensor-core rate measurement kernel on the current
+    device; returns the int8 operations of the launch (time it with CUDA
+    events on `stream`)."""
+    ops = ctypes.c_double()
+    _check(lib().cr_mma_i8_peak(int(iters), ctypes.byref(ops), _stream(stream)), "cr_mma_i8_peak")
+    return ops.value
 
 
 def cr_selftest_wait_timeout(seconds: float = 0.005, stream=None) -> None:

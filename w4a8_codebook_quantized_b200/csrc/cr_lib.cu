@@ -20,6 +20,7 @@
 #include "k_elementwise.cuh"
 #include "k_gemm.cuh"
 #include "k_gemv.cuh"
+#include "k_peak.cuh"
 #include "k_quant.cuh"
 #include "k_rotquant.cuh"
 
@@ -1538,6 +1539,40 @@ cr_status cr_gemm_s8(const int8_t *xq, const float *xs, const int8_t *w8, const 
     if (st != CR_OK)
         return st;
     return gemm_on_w8(*d, xq, xs, w8, s_channel, bias, M, N, K, out_dtype, out, acc_out, stream, 0);
+}
+
+cr_status cr_mma_i8_peak(int64_t iters, double *ops_per_launch, cr_stream_t stream)
+{
+    if (iters < 1 || iters > (1 << 20) || !ops_per_launch)
+        return CR_ERR_INVALID_ARG;
+    DeviceState *d = nullptr;
+    const cr_status st = current_device(&d);
+    if (st != CR_OK)
+        return st;
+    static std::atomic<bool> attr_set{false};
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(cr::pk::mma_i8_peak_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)cr::pk::kSmemBytes) != cudaSuccess) {
+            cudaGetLastError();
+            return CR_ERR_CUDA;
+        }
+        attr_set = true;
+    }
+    const int pairs = d->num_sms / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(cr::pk::kThreads);
+    cfg.dynamicSmemBytes = cr::pk::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    *ops_per_launch = 2.0 * 256.0 * 256.0 * 128.0 * (double)iters * (double)pairs;
+    return launched(cudaLaunchKernelEx(&cfg, cr::pk::mma_i8_peak_kernel, (int)iters));
 }
 
 cr_status cr_selftest_wait_timeout(uint64_t limit_ns, cr_stream_t stream)
