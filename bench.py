@@ -280,17 +280,16 @@ class Sets:
         self.out_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
 
     def step(self, i):
-        import w4a8_codebook_quantized_b200 as cr
+        """One decode step through a prepared layer (W4A8Linear.forward =
+        cr_w4a8_plan_forward): the rotate+quant kernel and the decode GEMV."""
         r = i % self.R
-        cr.cr_w4a8_linear(self.x[r], self.q[r], self.s[r], self.cb, self.ws[r], out=self.out[r],
-                          xq_work=self.xq[r], xs_work=self.xs[r])
+        self.lin[r].forward(self.x[r], out=self.out[r], xq_work=self.xq[r], xs_work=self.xs[r])
 
     def contraction_only(self, i):
-        """The dominant kernel alone: the GEMV (M <= 8) on prepared activations."""
-        import w4a8_codebook_quantized_b200 as cr
+        """The dominant kernel alone: the prepared layer's decode GEMV on the
+        quantised activations (W4A8Linear.gemv = cr_w4a8_plan_gemv)."""
         r = i % self.R
-        M = self.case.M
-        cr.cr_w4a8_gemv(self.xq[r], self.xs[r], self.q[r], self.s[r], self.cb, self.ws[r], m=M, out=self.out[r])
+        self.lin[r].gemv(self.xq[r], self.xs[r], m=self.case.M, out=self.out[r])
 
     def e2e_step(self, i):
         """Through the public API with host buffers: a prepared W4A8Linear
@@ -560,7 +559,8 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "s8", "data": "synthetic",
         "config": {"workload": head["workload"],
-                   "path": "cr_w4a8_linear = rotate+quant kernel + fused decode GEMV kernel",
+                   "path": "W4A8Linear.forward (cr_w4a8_plan_forward, a prepared layer) = rotate+quant kernel + fused "
+                           "decode GEMV kernel",
                    "l2": head["l2"] + " > 126 MiB L2",
                    "timing": "one CUDA-graph replay of K steps (graph uploaded beforehand), CUDA events on the capture stream",
                    "parallelism": f"replica x{world}"},

@@ -463,7 +463,13 @@ cr_status cr_w4a8_ste_backward_ws(const uint16_t *grad, const uint8_t *qdata, co
  *
  * cr_w4a8_plan_create: the layer as in (3), act_qmax and out_dtype as in (6);
  *   the buffers must stay valid and unchanged while the plan exists.  The plan
- *   belongs to the device current at creation; *plan is written.
+ *   belongs to the device current at creation; *plan is written.  Creation
+ *   reads the layer's scale bytes and the codebook once on the device (a check
+ *   kernel on the legacy default stream, waited for before the call returns):
+ *   when every scale byte's level table has the split form of the decode GEMV
+ *   (two tables whose byte-permute results add up to the level; it exists
+ *   unless a level of 127 pairs with a negative one), the plan's decode
+ *   forwards may use that faster decode.  Results are the same bit for bit.
  * cr_w4a8_plan_forward: (6) on that device with the plan's layer: x [M, K]
  *   bf16, out [M, N], xq_work / xs_work as in (6).  Calls on one plan may come
  *   from several host threads.
@@ -482,6 +488,10 @@ cr_status cr_w4a8_ste_backward_ws(const uint16_t *grad, const uint8_t *qdata, co
  *   kernel copying x_host reads it before the previous kernel on the stream
  *   has finished: x_host must not be written by a kernel that immediately
  *   precedes this call and allows early launch of its dependents.
+ * cr_w4a8_plan_gemv: the decode GEMV of (4) on the plan's layer and already
+ *   quantised activations (ai-toolkit convrot_w4a8_quant.py, gemv_prepared):
+ *   xq [>= M, K] int8, xs [M] fp32, 1 <= M <= 8 (CR_ERR_UNSUPPORTED above),
+ *   out [M, N]; the same results as cr_w4a8_gemv.
  * cr_w4a8_plan_destroy: frees the plan (NULL is allowed).
  * Errors as in (6); a plan used on another device gives CR_ERR_INVALID_ARG.
  */
@@ -494,6 +504,8 @@ cr_status cr_w4a8_plan_forward(cr_w4a8_plan plan, const uint16_t *x, int64_t M, 
 cr_status cr_w4a8_plan_forward_host(cr_w4a8_plan plan, const uint16_t *x_host, int64_t M, void *out_host,
                                     uint16_t *x_dev, void *out_dev, int8_t *xq_work, float *xs_work,
                                     cr_stream_t stream);
+cr_status cr_w4a8_plan_gemv(cr_w4a8_plan plan, const int8_t *xq, const float *xs, int64_t M, void *out,
+                            cr_stream_t stream);
 cr_status cr_w4a8_plan_destroy(cr_w4a8_plan plan);
 
 /*

@@ -242,3 +242,82 @@ def test_calls_on_a_device_that_is_not_current():
     torch.cuda.synchronize(0)
     torch.cuda.synchronize(1)
     assert torch.equal(y.cpu(), ref.cpu()) and torch.equal(y2.cpu(), ref.cpu())
+
+
+# ---------------------------------------------------------------- decode GEMV: both weight decodes
+
+def _codebook(kind):
+    if kind == "fixed":
+        return inputs.codebook()
+    if kind == "arange":
+        return np.arange(-8, 8, dtype=np.float32)
+    if kind == "wide":
+        return np.linspace(-300.0, 300.0, 16).astype(np.float32)
+    return np.array([3, -1, 0.5, 7, -6, 2, -0.25, 5, -3, 1, -7, 4, 0, -5, 6, -2], np.float32)  # unsorted
+
+
+@pytest.mark.parametrize("cb_kind", ["fixed", "arange", "wide", "unsorted"])
+@pytest.mark.parametrize("scales", ["all_bytes", "generator", "one_large"])
+def test_gemv_decodes_every_scale_byte(cb_kind, scales):
+    """The decode GEMV picks, per CTA, a split table decode (two byte
+    permutes whose int8 results add up to the level inside the MMA) when every
+    scale byte of its tiles allows it, and the general decode otherwise.  Both
+    must give the oracle's int32 sums and outputs bit for bit: every scale
+    byte (NaN and negative ones included), codebooks that saturate or are not
+    sorted, and a layer whose scales are ordinary except one large byte in
+    one row (so CTAs differ in the decode they take)."""
+    M, N, K, seed = 5, 4096 + 48, 2048, 77
+    layer = inputs.layer(N, K, seed)
+    cb = _codebook(cb_kind)
+    srel = layer.srel.copy()
+    rng = np.random.default_rng(seed)
+    if scales == "all_bytes":
+        srel = rng.integers(0, 256, size=srel.shape, dtype=np.uint8)
+        srel[:2, :] = np.arange(256, dtype=np.uint8).reshape(2, 128)  # every byte, in two rows
+    elif scales == "one_large":
+        srel[1000, 7] = 0x7E  # 448: saturates the top levels of the fixed codebook
+    x = inputs.activations(M, K, seed)
+    ref = oracle.linear(x, layer.qdata, srel, cb, layer.s_channel, threads=8)
+    xq, xs = oracle.rotate_quant_act(x, oracle.mp_for(M))
+    q, s, c, ws = dev(layer.qdata), dev(srel), dev(cb), dev(layer.s_channel)
+    out, acc = cr.cr_w4a8_gemv(dev(xq), dev(xs), q, s, c, ws, m=M, acc_out=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(acc), ref["acc"])
+    assert np.array_equal(host(out), ref["y"])
+    # the same through the prefill path (GEMV and GEMM agree bit for bit)
+    out2 = cr.cr_w4a8_gemm(dev(xq[:M]), dev(xs[:M]), q, s, c, ws)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(out2), host(out))
+
+
+@pytest.mark.parametrize("cb_kind", ["fixed", "arange", "unsorted"])
+@pytest.mark.parametrize("scales", ["all_bytes", "generator", "one_large"])
+@pytest.mark.parametrize("N", [4096 + 48, 12288])
+def test_prepared_layer_decode_matches_oracle(cb_kind, scales, N):
+    """A prepared layer (W4A8Linear) checks its scale bytes once and then
+    decodes with split tables when all of them have one (and each CTA has
+    at most two row tiles: N = 4144 here; N = 12288 has more).  Its forward
+    and its GEMV on quantised activations must equal the oracle and the
+    unprepared GEMV bit for bit, for layers whose bytes all allow the split
+    form, none do, or all but one."""
+    K, seed = 2048, 91
+    layer = inputs.layer(N, K, seed)
+    cb = _codebook(cb_kind)
+    srel = layer.srel.copy()
+    rng = np.random.default_rng(seed)
+    if scales == "all_bytes":
+        srel = rng.integers(0, 256, size=srel.shape, dtype=np.uint8)
+    elif scales == "one_large":
+        srel[N // 2, 3] = 0x7E
+    q, s, c, ws = dev(layer.qdata), dev(srel), dev(cb), dev(layer.s_channel)
+    lin = cr.W4A8Linear(q, s, c, ws)
+    for M in (1, 5, 8):
+        x = inputs.activations(M, K, seed + M)
+        ref = oracle.linear(x, layer.qdata, srel, cb, layer.s_channel, threads=8)
+        y = lin(bf16_dev(x))
+        xq, xs = cr.cr_rotate_quant_act(bf16_dev(x), cr.gemv_rows(M))
+        y2 = lin.gemv(xq, xs, m=M)
+        y3 = cr.cr_w4a8_gemv(xq, xs, q, s, c, ws, m=M)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(y), ref["y"]), (M, cb_kind, scales)
+        assert torch.equal(y2, y3) and torch.equal(y, y2)

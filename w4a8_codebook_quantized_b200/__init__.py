@@ -97,6 +97,7 @@ def lib() -> ctypes.CDLL:
             L.cr_w4a8_plan_create.argtypes = [P, P, P, P, P, i64, i64, i32, i32, ctypes.POINTER(P)]
             L.cr_w4a8_plan_forward.argtypes = [P, P, i64, P, P, P, P]
             L.cr_w4a8_plan_forward_host.argtypes = [P, P, i64, P, P, P, P, P, P]
+            L.cr_w4a8_plan_gemv.argtypes = [P, P, P, i64, P, P]
             L.cr_w4a8_plan_destroy.argtypes = [P]
             L.cr_w4a8_plan_bind_host.argtypes = [P, P, i64, P, P, P, P, P, ctypes.POINTER(P)]
             L.cr_w4a8_host_call_run.argtypes = [P, P]
@@ -564,6 +565,23 @@ class W4A8Linear:
         _need(out, "out", (self.out_dtype,), shape=(M, self.N))
         _check(self._fwd(self._plan, x.data_ptr(), M, out.data_ptr(), xq_work.data_ptr(), xs_work.data_ptr(),
                          _stream(stream)), "cr_w4a8_plan_forward")
+        return out
+
+    def gemv(self, xq, xs, m: Optional[int] = None, out=None, stream=None):
+        """The decode GEMV on already quantised activations (xq int8 [>= M, K],
+        xs fp32 [>= M], M <= 8): cr_w4a8_plan_gemv."""
+        torch = _torch()
+        _need(xq, "xq", (torch.int8,), 2)
+        _need(xs, "xs", (torch.float32,), 1)
+        M = xq.shape[0] if m is None else int(m)
+        if xq.shape[1] != self.K or xq.shape[0] < M or xs.shape[0] < M:
+            raise ValueError(f"xq {tuple(xq.shape)} / xs {tuple(xs.shape)} do not match M={M}, K={self.K}")
+        with self._device_ctx(xq, xs, out):
+            if out is None:
+                out = torch.empty(M, self.N, dtype=self.out_dtype, device=xq.device)
+            _need(out, "out", (self.out_dtype,), shape=(M, self.N))
+            _check(self._L.cr_w4a8_plan_gemv(self._plan, xq.data_ptr(), xs.data_ptr(), M, out.data_ptr(),
+                                             _stream(stream)), "cr_w4a8_plan_gemv")
         return out
 
     def forward_host(self, x_host, out_host, x_dev, out_dev, xq_work=None, xs_work=None, stream=None):

@@ -70,6 +70,39 @@ __device__ __forceinline__ uint4 lut_entry(uint32_t s, const float *cb /* 16, an
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// The split form of a level table (the fast decode of the decode GEMV): from
+// the 16 levels L of `e` (lut_entry), two 8-byte tables P (x, y) and Q (z, w)
+// with, for each j = 0..7, P[j] + sgn(Q[j]) = L[j] and sgn(P[j]) + Q[j] =
+// L[j + 8], where sgn(v) is -1 for a negative byte and 0 otherwise (what a
+// sign-replicating byte permute returns).  Taking P[j] = L[j] + a and
+// Q[j] = L[j + 8] + b with a = [Q[j] < 0], b = [P[j] < 0] always has an int8
+// solution unless one of the two levels is 127 and the other negative; ok is
+// cleared for such a table.
+__device__ __forceinline__ uint4 lut_entry_split(const uint4 &e, bool &ok)
+{
+    const uint32_t w[4] = {e.x, e.y, e.z, e.w};
+    uint32_t P[2] = {0u, 0u}, Q[2] = {0u, 0u};
+    ok = true;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int p = (int)(int8_t)(w[j >> 2] >> (8 * (j & 3)));
+        const int q = (int)(int8_t)(w[2 + (j >> 2)] >> (8 * (j & 3)));
+        int A = p, B = q + (p < 0 ? 1 : 0);  // a = 0: needs Q[j] = B >= 0
+        if (B < 0 || B > 127) {
+            A = p + 1;                        // a = 1: needs Q[j] < 0
+            B = q + (A < 0 ? 1 : 0);
+            if (p > 126 || B >= 0) {
+                ok = false;
+                A = 0;
+                B = 0;
+            }
+        }
+        P[j >> 2] |= ((uint32_t)A & 0xFFu) << (8 * (j & 3));
+        Q[j >> 2] |= ((uint32_t)B & 0xFFu) << (8 * (j & 3));
+    }
+    return make_uint4(P[0], P[1], Q[0], Q[1]);
+}
+
 // PTX prmt in its default mode: selector nibble i = {sign-replicate bit, 3-bit
 // source byte index} for output byte i; source bytes 0-3 from a, 4-7 from b.
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)

@@ -38,6 +38,7 @@ struct DeviceState {
     std::atomic<bool> gemm_attr_set{false};
     std::atomic<bool> gemm_pair_attr_set{false};
     std::atomic<bool> gemv_attr_set{false};
+    std::atomic<bool> gemv_split_attr_set{false};
     std::atomic<bool> gemv_grouped_attr_set{false};
     std::atomic<bool> gemm_bf16_attr_set{false};
     std::atomic<bool> gemm_pair_bf16_attr_set{false};
@@ -249,27 +250,34 @@ cr_status build_gemv_args(cr::gv::GemvArgs<L> &args, const float *codebook, int6
 
 // Launch the decode GEMV with complete arguments: a persistent grid of as
 // many CTAs as fit on the SMs, optionally as a programmatic dependent of the
-// previous kernel on the stream.
+// previous kernel on the stream.  split: the layer's tables all have a split
+// form (checked when it was prepared); the split variant of the kernel runs
+// where every CTA has at most two row tiles.  attr_set / split_attr_set: the
+// once-per-device shared-memory attribute of the plain and split variants.
 template <int L>
-cr_status launch_gemv_args(int num_sms, std::atomic<bool> &attr_set, const cr::gv::GemvArgs<L> &args, cudaStream_t stream,
-                           bool pdl)
+cr_status launch_gemv_args(int num_sms, std::atomic<bool> &attr_set, const cr::gv::GemvArgs<L> &args,
+                           cudaStream_t stream, bool pdl, bool split = false,
+                           std::atomic<bool> *split_attr_set = nullptr)
 {
     using namespace cr;
     using C = gv::Prod;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(gv::gemv_kernel<C, L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)C::kSmemBytes) != cudaSuccess) {
+    // persistent grid of several CTAs per SM, at most one wave
+    const int64_t slots = (int64_t)C::kMinBlocks * num_sms;
+    const int64_t grid = args.num_tiles < slots ? args.num_tiles : slots;
+    const bool use_split = split && split_attr_set != nullptr && args.num_tiles <= 2 * grid;
+    void (*kern)(const gv::GemvArgs<L>) = use_split ? gv::gemv_kernel<C, L, true> : gv::gemv_kernel<C, L, false>;
+    std::atomic<bool> &flag = use_split ? *split_attr_set : attr_set;
+    if (!flag) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmemBytes) !=
+            cudaSuccess) {
             cudaGetLastError();
             return CR_ERR_CUDA;
         }
-        attr_set = true;
+        flag = true;
     }
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    // persistent grid of several CTAs per SM, at most one wave
-    const int64_t slots = (int64_t)C::kMinBlocks * num_sms;
-    const int64_t grid = args.num_tiles < slots ? args.num_tiles : slots;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(gv::kThreads);
@@ -277,7 +285,7 @@ cr_status launch_gemv_args(int num_sms, std::atomic<bool> &attr_set, const cr::g
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return launched(cudaLaunchKernelEx(&cfg, gv::gemv_kernel<C, L>, args));
+    return launched(cudaLaunchKernelEx(&cfg, kern, args));
 }
 
 template <int L>
@@ -545,6 +553,45 @@ cr_status run_gemm(DeviceState &d, const int8_t *xq, const float *xs, const uint
 
 }  // namespace
 
+// The result word of split_check_kernel (one per device; checks are
+// serialised under g_mutex).
+static __device__ int g_split_bad = 0;
+
+namespace {
+// Whether every scale byte of a layer srel [N, K / 16] has a split table for
+// this codebook: split_check_kernel on the legacy default stream, waited for.
+cr_status check_split(DeviceState &d, const uint8_t *srel, const float *codebook, int64_t N, int64_t K, bool &ok)
+{
+    ok = false;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_split_bad, &zero, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return CR_ERR_CUDA;
+    }
+    void *flag = nullptr;
+    if (cudaGetSymbolAddress(&flag, g_split_bad) != cudaSuccess) {
+        cudaGetLastError();
+        return CR_ERR_CUDA;
+    }
+    const int64_t bytes = N * (K / 16);
+    const int64_t words = bytes / 16;
+    int64_t grid = (words + 255) / 256;
+    if (grid > 2 * (int64_t)d.num_sms)
+        grid = 2 * (int64_t)d.num_sms;
+    if (grid < 1)
+        grid = 1;
+    cr::gv::split_check_kernel<<<(unsigned)grid, 256>>>(srel, bytes, codebook, static_cast<int *>(flag));
+    int bad = 1;
+    if (cudaGetLastError() != cudaSuccess || cudaMemcpyFromSymbol(&bad, g_split_bad, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return CR_ERR_CUDA;
+    }
+    ok = bad == 0;
+    return CR_OK;
+}
+}  // namespace
+
 // A prepared layer (cr_w4a8_plan_*): the validated layer, its device, and
 // the decode GEMV's arguments with the weight maps encoded; tm_x holds the
 // activation map of (xmap_base, xmap_M) once a forward has set it.
@@ -558,6 +605,7 @@ struct cr_w4a8_plan_st {
     cr_out_dtype out_dtype = CR_OUT_BF16;
     cr::gv::GemvArgs<1> gemv;
     int64_t tiles = 0;
+    bool split_ok = false;  // every scale byte of the layer has a split table (split_check_kernel)
     const int8_t *xmap_base = nullptr;
     int64_t xmap_M = -1;
     std::mutex mu;
@@ -1107,6 +1155,8 @@ cr_status cr_w4a8_plan_create(const uint8_t *qdata, const uint8_t *srel, const f
     if (N > 0) {
         cr_w4a8_layer ly{qdata, srel, s_channel, bias, N, nullptr, nullptr};
         st = build_gemv_args<1>(p->gemv, codebook, K, &ly, 1, out_dtype, 0, p->tiles);
+        if (st == CR_OK)
+            st = check_split(*d, srel, codebook, N, K, p->split_ok);
         if (st != CR_OK) {
             delete p;
             return st;
@@ -1163,7 +1213,44 @@ cr_status cr_w4a8_plan_forward(cr_w4a8_plan plan, const uint16_t *x, int64_t M, 
     args.xs = xs_work;
     args.M = (int)M;
     args.layer[0].out = out;
-    return launch_gemv_args<1>(plan->d->num_sms, plan->d->gemv_attr_set, args, stream, /*pdl=*/true);
+    return launch_gemv_args<1>(plan->d->num_sms, plan->d->gemv_attr_set, args, stream, /*pdl=*/true,
+                               plan->split_ok, &plan->d->gemv_split_attr_set);
+}
+
+cr_status cr_w4a8_plan_gemv(cr_w4a8_plan plan, const int8_t *xq, const float *xs, int64_t M, void *out,
+                            cr_stream_t stream)
+{
+    if (!plan || M < 0)
+        return CR_ERR_INVALID_ARG;
+    if (M > CR_GEMV_MAX_M)
+        return CR_ERR_UNSUPPORTED;
+    if (M == 0 || plan->N == 0)
+        return CR_OK;
+    if (!xq || !xs || !out)
+        return CR_ERR_INVALID_ARG;
+    if (!aligned16(xq) || !aligned16(xs) || !aligned16(out))
+        return CR_ERR_ALIGNMENT;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != plan->device) {
+        cudaGetLastError();
+        return CR_ERR_INVALID_ARG;
+    }
+    cr::gv::GemvArgs<1> args;
+    {
+        std::lock_guard<std::mutex> lock(plan->mu);
+        if (plan->xmap_base != xq || plan->xmap_M != M) {
+            if (!encode_gemv_x_map(&plan->gemv.tm_x, xq, M, plan->K))
+                return CR_ERR_CUDA;
+            plan->xmap_base = xq;
+            plan->xmap_M = M;
+        }
+        args = plan->gemv;
+    }
+    args.xs = xs;
+    args.M = (int)M;
+    args.layer[0].out = out;
+    return launch_gemv_args<1>(plan->d->num_sms, plan->d->gemv_attr_set, args, stream, /*pdl=*/true,
+                               plan->split_ok, &plan->d->gemv_split_attr_set);
 }
 
 cr_status cr_w4a8_plan_forward_host(cr_w4a8_plan plan, const uint16_t *x_host, int64_t M, void *out_host,
@@ -1304,7 +1391,8 @@ cr_status cr_w4a8_host_call_run(cr_w4a8_host_call c, cr_stream_t stream)
     } else {
         st = launched(cr::rq::launch(c->x_dev, c->M, plan->K, c->MP, plan->act_qmax, c->xq, c->xs, stream));
         if (st == CR_OK)
-            st = launch_gemv_args<1>(d->num_sms, d->gemv_attr_set, c->gemv, stream, /*pdl=*/true);
+            st = launch_gemv_args<1>(d->num_sms, d->gemv_attr_set, c->gemv, stream, /*pdl=*/true, plan->split_ok,
+                                     &d->gemv_split_attr_set);
     }
     if (st != CR_OK)
         return st;
@@ -1459,7 +1547,7 @@ cr_status noalloc_scratch(NoallocState **out)
             return CR_ERR_CUDA;
         }
         s.scratch = static_cast<uint8_t *>(p);
-        if (cudaFuncSetAttribute(cr::gv::gemv_kernel<cr::gv::Prod, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(cr::gv::gemv_kernel<cr::gv::Prod, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)cr::gv::Prod::kSmemBytes) != cudaSuccess) {
             cudaGetLastError();
             return CR_ERR_CUDA;

@@ -151,6 +151,53 @@ __device__ __forceinline__ void slice_mma(const Ops &o, int32_t (&c)[4], int32_t
     mma_s8(d, e0, e1, e2, e3, o.X1.z, o.X1.w);
 }
 
+// Split decode.  The table entry of a scale byte may hold, instead of the 16
+// levels, two 8-byte tables P = T.x:T.y and Q = T.z:T.w (lut_entry_split)
+// built so that, for every code c,
+//   P-permute(c) + Q-permute(c ^ 8) = level(c)
+// where a byte permute with selector nibble c returns table byte c for c < 8
+// and, for c >= 8, the sign of table byte c - 8 replicated (0 or -1).  The two
+// permute results are two int8 weights whose sum is the decoded weight, and
+// the tensor core adds them: one MMA on each, with the same activations, into
+// the same accumulator (exact integer sums).  Per 8 codes that is 4 permutes,
+// one xor and two shifts against the 11 ALU operations of decode8, for one
+// more MMA per code word.  A launch uses it (the kernel's SPLIT variant) when
+// every table the layer reads has a split form, which the host establishes
+// once per prepared layer (split_check_kernel), and where a CTA has at most
+// two row tiles (there it was measured faster; with more tiles per CTA the
+// extra MMAs cost more than the decode saves).
+__device__ __forceinline__ void decode8_split(uint32_t c, const uint4 &T, uint32_t &p0, uint32_t &p1, uint32_t &q0,
+                                              uint32_t &q1)
+{
+    const uint32_t cx = c ^ 0x88888888u;
+    p0 = prmt(T.x, T.y, c);
+    q0 = prmt(T.z, T.w, cx);
+    p1 = prmt(T.x, T.y, c >> 16);
+    q1 = prmt(T.z, T.w, cx >> 16);
+}
+
+// slice_mma on split tables.
+__device__ __forceinline__ void slice_mma_split(const Ops &o, int32_t (&c)[4], int32_t (&d)[4])
+{
+    uint32_t pa0, pa2, qa0, qa2, pb1, pb3, qb1, qb3, ra0, ra2, sa0, sa2, rb1, rb3, sb1, sb3;
+    decode8_split(o.A.x, o.TA0, pa0, pa2, qa0, qa2);
+    decode8_split(o.B.x, o.TB0, pb1, pb3, qb1, qb3);
+    decode8_split(o.A.y, o.TA0, ra0, ra2, sa0, sa2);
+    decode8_split(o.B.y, o.TB0, rb1, rb3, sb1, sb3);
+    mma_s8(c, pa0, pb1, pa2, pb3, o.X0.x, o.X0.y);
+    mma_s8(d, ra0, rb1, ra2, rb3, o.X0.z, o.X0.w);
+    mma_s8(c, qa0, qb1, qa2, qb3, o.X0.x, o.X0.y);
+    mma_s8(d, sa0, sb1, sa2, sb3, o.X0.z, o.X0.w);
+    decode8_split(o.A.z, o.TA1, pa0, pa2, qa0, qa2);
+    decode8_split(o.B.z, o.TB1, pb1, pb3, qb1, qb3);
+    decode8_split(o.A.w, o.TA1, ra0, ra2, sa0, sa2);
+    decode8_split(o.B.w, o.TB1, rb1, rb3, sb1, sb3);
+    mma_s8(c, pa0, pb1, pa2, pb3, o.X1.x, o.X1.y);
+    mma_s8(d, ra0, rb1, ra2, rb3, o.X1.z, o.X1.w);
+    mma_s8(c, qa0, qb1, qa2, qb3, o.X1.x, o.X1.y);
+    mma_s8(d, sa0, sb1, sa2, sb3, o.X1.z, o.X1.w);
+}
+
 // The layers one launch covers: every layer is contracted with the same
 // activations (xq, xs) and was quantised with the same codebook; their row
 // tiles are numbered one after the other (layer l owns the tiles
@@ -213,7 +260,9 @@ __device__ __forceinline__ void locate(const GemvArgs<L> &a, int tile, int &l, i
     }
 }
 
-template <class C, int L>
+// SPLIT: the level tables in split form (slice_mma_split); only for layers
+// whose every scale byte has one (split_check_kernel).
+template <class C, int L, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __grid_constant__ GemvArgs<L> a)
 {
     constexpr int STAGES = C::kStages;
@@ -357,10 +406,13 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
             sh.cb[tid] = a.codebook[tid];
         asm volatile("bar.sync 2, %0;" ::"n"(kThreads) : "memory");
         {
+            // the plain level table of scale byte tid, or its split form
             const uint4 e = lut_entry((uint32_t)tid, sh.cb);
+            bool split_ok;
+            const uint4 t = SPLIT ? lut_entry_split(e, split_ok) : e;
 #pragma unroll
             for (int r = 0; r < C::kCopies; ++r)
-                sh.lut[tid * C::kCopies + ((r + tid) & (C::kCopies - 1))] = e;
+                sh.lut[tid * C::kCopies + ((r + tid) & (C::kCopies - 1))] = t;
         }
         consumer_sync();
         // (the consumers read only shared memory: the activation copies
@@ -410,7 +462,10 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
                         Ops o;
                         fetch_ops(o, sh.x[s] + off_x0, sh.x[s] + off_x1, sh.codes[s] + off_code,
                                   sh.srel[s] + off_srel, lutb, a.lut_step);
-                        slice_mma(o, c, d);
+                        if constexpr (SPLIT)
+                            slice_mma_split(o, c, d);
+                        else
+                            slice_mma(o, c, d);
                     }
                     __syncwarp();
                     if (ok && lane == 0)
@@ -528,6 +583,41 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
         }
     }
     __syncthreads();
+}
+
+// Whether every scale byte of a layer has a split table (lut_entry_split)
+// for this codebook: each CTA tabulates the 256 bytes' split forms, takes
+// tmin = the smallest magnitude (s & 0x7F) without one, and flags (in *bad,
+// which the host zeroed) any byte of its rows of srel [N, K / 16] with
+// s & 0x7F >= tmin.  Bytes below tmin all have a split form by its
+// definition; above it some may too (the check is conservative).  Per 4
+// bytes, bit 7 of each byte of (w & 0x7F7F7F7F) + (128 - tmin) * 0x01010101 is
+// set iff that byte's magnitude is >= tmin (no carry crosses a byte).
+__global__ void __launch_bounds__(256) split_check_kernel(const uint8_t *__restrict__ srel, int64_t bytes,
+                                                          const float *__restrict__ codebook, int *__restrict__ bad)
+{
+    __shared__ float cb[16];
+    __shared__ int tmin;
+    if (threadIdx.x < 16)
+        cb[threadIdx.x] = codebook[threadIdx.x];
+    if (threadIdx.x == 0)
+        tmin = 128;
+    __syncthreads();
+    bool ok;
+    lut_entry_split(lut_entry(threadIdx.x, cb), ok);
+    if (!ok)
+        atomicMin(&tmin, (int)(threadIdx.x & 0x7Fu));
+    __syncthreads();
+    const uint32_t addc = (uint32_t)(128 - tmin) * 0x01010101u;
+    uint32_t flags = 0u;
+    const int64_t words = bytes / 16;  // whole 16-byte pieces (K / 16 is a multiple of 16)
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < words; i += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(srel) + i);
+        flags |= (((v.x & 0x7F7F7F7Fu) + addc) | ((v.y & 0x7F7F7F7Fu) + addc) | ((v.z & 0x7F7F7F7Fu) + addc) |
+                  ((v.w & 0x7F7F7F7Fu) + addc)) & 0x80808080u;
+    }
+    if (__syncthreads_or(flags != 0u) && threadIdx.x == 0)
+        atomicOr(bad, 1);
 }
 
 }  // namespace gv

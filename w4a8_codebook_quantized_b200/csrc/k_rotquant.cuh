@@ -14,7 +14,8 @@
 // quadruple (v0, v1, v2, v3) along a digit becomes S - 2 v[3-a] with
 // S = (v0 + v1) + (v2 + v3); the result is scaled by 1/16.
 //
-// Layout: one CTA of 256 threads per row.  A half-warp (16 lanes) owns one
+// Layout: one CTA per row, of 256 threads (512 for short batches of long
+// rows, where the few CTAs would otherwise leave most SMs idle).  A half-warp (16 lanes) owns one
 // 256-element block, viewed as a 16 x 16 matrix with element 16a + b: lane L
 // first holds row a = L (16 contiguous bf16, two 16-byte loads), applies the
 // stride-1 and stride-4 digits in registers, transposes through shared memory
@@ -32,9 +33,10 @@
 namespace cr {
 namespace rq {
 
-constexpr int kThreads = 256;
-constexpr int kHalfWarps = kThreads / 16;  // blocks of 256 in flight per CTA
-constexpr int kMaxBlocksInRegs = 4;        // per half-warp: K <= 16384 stays in registers
+constexpr int kThreads = 256;              // the CTA size for batches of many rows
+constexpr int kWideThreads = 512;          // ... and for at most kWideRows rows of K >= 8192
+constexpr int kWideRows = 16;
+constexpr int kMaxBlocksInRegs = 4;        // per half-warp: K <= 16384 (32768 wide) stays in registers
 
 // One digit of the rotation on a quadruple (row a of h4 is all ones except
 // -1 at column 3 - a).  2v is exact, so fma(-2, v, S) is S - 2v rounded once.
@@ -176,16 +178,17 @@ __device__ __forceinline__ float max_abs16(const float (&v)[16])
     return fmaxf(fmaxf(m[0], m[2]), fmaxf(m[1], m[3]));
 }
 
-template <int J, bool kRecompute>
-__global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
+template <int J, bool kRecompute, int THREADS>
+__global__ void __launch_bounds__(THREADS) rotquant_kernel(const uint16_t *__restrict__ x, int64_t M, int64_t K,
                                                             int qmax, int8_t *__restrict__ xq,
                                                             float *__restrict__ xs)
 {
     // half-warp buffers 16 floats apart in bank space: the two halves of a warp
     // never touch the same bank in one transpose step
+    constexpr int kHalfWarps = THREADS / 16;  // blocks of 256 in flight per CTA
     __shared__ __align__(16) float tr_all[kHalfWarps][16 * 16 + 16];
     __shared__ __align__(16) uint8_t tb_all[kHalfWarps][272];
-    __shared__ float warp_max[kThreads / 32];
+    __shared__ float warp_max[THREADS / 32];
 
     // Let a programmatic dependent (the decode GEMV) start its weight stream
     // now; it waits for this grid's results before it reads them.
@@ -209,7 +212,7 @@ __global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__re
     int8_t *__restrict__ qrow = xq + m * K;
 
     if (m >= M) {  // padding row of the decode GEMV operand
-        for (int64_t c = tid; c < K / 16; c += kThreads)
+        for (int64_t c = tid; c < K / 16; c += THREADS)
             reinterpret_cast<uint4 *>(qrow)[c] = make_uint4(0u, 0u, 0u, 0u);
         if (tid == 0)
             xs[m] = 1.0f;
@@ -251,7 +254,7 @@ __global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__re
     __syncthreads();
     float rmax = warp_max[0];
 #pragma unroll
-    for (int w = 1; w < kThreads / 32; ++w)
+    for (int w = 1; w < THREADS / 32; ++w)
         rmax = fmaxf(rmax, warp_max[w]);
     // rmax is max |R| = 16 max |r|; the row maximum of r is rmax / 16 rounded
     // (rounding is monotonic, so that is also the max of the rounded r).
@@ -277,21 +280,23 @@ __global__ void __launch_bounds__(kThreads) rotquant_kernel(const uint16_t *__re
         xs[m] = scale;
 }
 
-inline cudaError_t launch(const uint16_t *x, int64_t M, int64_t K, int64_t MP, int qmax, int8_t *xq, float *xs,
-                          cudaStream_t stream)
+template <int THREADS>
+inline cudaError_t launch_t(const uint16_t *x, int64_t M, int64_t K, int64_t MP, int qmax, int8_t *xq, float *xs,
+                            cudaStream_t stream)
 {
+    constexpr int kHalfWarps = THREADS / 16;
     const int64_t per_hw = (K / 256 + kHalfWarps - 1) / kHalfWarps;  // blocks per half-warp
     void (*kern)(const uint16_t *, int64_t, int64_t, int, int8_t *, float *) =
-        per_hw <= 1   ? rotquant_kernel<1, false>
-        : per_hw == 2 ? rotquant_kernel<2, false>
-        : per_hw == 3 ? rotquant_kernel<3, false>
-        : per_hw == 4 ? rotquant_kernel<4, false>
-                      : rotquant_kernel<1, true>;
+        per_hw <= 1   ? rotquant_kernel<1, false, THREADS>
+        : per_hw == 2 ? rotquant_kernel<2, false, THREADS>
+        : per_hw == 3 ? rotquant_kernel<3, false, THREADS>
+        : per_hw == 4 ? rotquant_kernel<4, false, THREADS>
+                      : rotquant_kernel<1, true, THREADS>;
     // a programmatic dependent of the previous kernel on the stream: its
     // launch overlaps that kernel's tail, and the kernel waits for it
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)MP);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(THREADS);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -299,6 +304,16 @@ inline cudaError_t launch(const uint16_t *x, int64_t M, int64_t K, int64_t MP, i
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, x, M, K, qmax, xq, xs);
+}
+
+// One CTA per row: 512 threads when there are few rows of K >= 8192 (the
+// decode batches), 256 otherwise.
+inline cudaError_t launch(const uint16_t *x, int64_t M, int64_t K, int64_t MP, int qmax, int8_t *xq, float *xs,
+                          cudaStream_t stream)
+{
+    if (MP <= kWideRows && K >= 8192)
+        return launch_t<kWideThreads>(x, M, K, MP, qmax, xq, xs, stream);
+    return launch_t<kThreads>(x, M, K, MP, qmax, xq, xs, stream);
 }
 
 }  // namespace rq
