@@ -122,6 +122,10 @@ cr_status current_device(DeviceState **out)
         }
         if (d.usable && !have_encode_tiled())
             d.usable = false;
+        if (d.usable && cr::rq::set_attributes() != cudaSuccess) {
+            cudaGetLastError();
+            d.usable = false;
+        }
     }
     if (!d.usable)
         return CR_ERR_NO_DEVICE;
