@@ -44,6 +44,15 @@ namespace cr {
 namespace rq {
 
 constexpr int kShortRows = 16;  // batches of at most this many rows take the scalar form
+// Shared memory each short-batch CTA reserves beyond what it uses.  In a
+// decode step the rotation's few CTAs become resident while the previous
+// GEMV still fills the SMs, and the block scheduler may stack up to four of
+// them (512 threads each) on the first SM that frees up, where they share its
+// issue slots.  The reservation caps them at two per SM while a GEMV CTA can
+// still sit beside one.  Measured on B200: the M = 8, N = K = 8192 decode step
+// 15.4 -> 14.2 us, the others unchanged or slightly faster; 80 KB and more
+// slowed the M <= 4 steps.
+constexpr int kShortReserve = 60 * 1024;
 
 // ================================================================ scalar form (short batches)
 
@@ -309,6 +318,7 @@ inline cudaError_t launch_rows_t(const uint16_t *x, int64_t M, int64_t K, int64_
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)MP);
     cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = kShortReserve;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -648,19 +658,38 @@ __global__ void __launch_bounds__(THREADS) rotquant_pairs_kernel(const uint16_t 
 
 using KernelFn = void (*)(const uint16_t *, int64_t, int64_t, int, int8_t *, float *);
 
-// Opt the CTA sizes whose transpose buffers pass 48 KB into the larger
-// dynamic shared memory.  Once per device, before the first launch.
+// Opt the kernels whose dynamic shared memory passes 48 KB into the larger
+// size: the packed form's 384- and 512-thread CTAs (transpose buffers) and
+// every short-batch kernel (its reservation).  Once per device, before the
+// first launch.
 inline cudaError_t set_attributes()
 {
-    const KernelFn wide[3] = {rotquant_pairs_kernel<1, false, 512>, rotquant_pairs_kernel<2, false, 512>,
-                              rotquant_pairs_kernel<1, true, 512>};
-    for (KernelFn f : wide) {
-        const cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes<512>());
+    struct Need {
+        KernelFn f;
+        int bytes;
+    };
+    const Need need[] = {
+        {rotquant_pairs_kernel<1, false, 512>, smem_bytes<512>()},
+        {rotquant_pairs_kernel<2, false, 512>, smem_bytes<512>()},
+        {rotquant_pairs_kernel<1, true, 512>, smem_bytes<512>()},
+        {rotquant_pairs_kernel<1, false, 384>, smem_bytes<384>()},
+        {rotquant_rows_kernel<1, false, 256>, kShortReserve},
+        {rotquant_rows_kernel<2, false, 256>, kShortReserve},
+        {rotquant_rows_kernel<3, false, 256>, kShortReserve},
+        {rotquant_rows_kernel<4, false, 256>, kShortReserve},
+        {rotquant_rows_kernel<1, true, 256>, kShortReserve},
+        {rotquant_rows_kernel<1, false, 512>, kShortReserve},
+        {rotquant_rows_kernel<2, false, 512>, kShortReserve},
+        {rotquant_rows_kernel<3, false, 512>, kShortReserve},
+        {rotquant_rows_kernel<4, false, 512>, kShortReserve},
+        {rotquant_rows_kernel<1, true, 512>, kShortReserve},
+    };
+    for (const Need &n : need) {
+        const cudaError_t e = cudaFuncSetAttribute(n.f, cudaFuncAttributeMaxDynamicSharedMemorySize, n.bytes);
         if (e != cudaSuccess)
             return e;
     }
-    return cudaFuncSetAttribute(rotquant_pairs_kernel<1, false, 384>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                smem_bytes<384>());
+    return cudaSuccess;
 }
 
 template <int J, bool kRecompute, int THREADS>
