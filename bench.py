@@ -59,7 +59,7 @@ def parse():
     p.add_argument("--prefill-extra", default="c3_prefill_2k_4k,c4_mlp_up,c4_mlp_down",
                    help="comma-separated prefill workloads reported beside the prefill block (empty: none)")
     p.add_argument("--backward-workload", default="c3_prefill_2k_4k")
-    p.add_argument("--only", default=None, choices=["headline", "decode-transient", "quantiser", "int8-peak"],
+    p.add_argument("--only", default=None, choices=["headline", "decode-transient", "quantiser", "int8-peak", "rotate-quant"],
                    help="run one piece alone (profiling runs): the headline step and GEMV, the prefill weight "
                         "transient, the offline quantiser, or the INT8 rate kernel")
     p.add_argument("--no-prefill", action="store_true")
@@ -492,7 +492,7 @@ def run_ours(args):
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
     cr.lib()
-    if args.only in ("decode-transient", "quantiser", "int8-peak"):
+    if args.only in ("decode-transient", "quantiser", "int8-peak", "rotate-quant"):
         return run_only(args, world, rank, local)
     pk = peaks()
     case = inputs.CASES[args.workload]
@@ -663,6 +663,29 @@ def run_only(args, world, rank, local):
         t = e0.elapsed_time(e1) / 1000.0 / 20
         out.update({"N": N, "K": K, "us": round(t * 1e6, 2),
                     "gb_per_s": round(N * K * (0.5 + 1 / 16 + 1) / t / 1e9, 1)})
+    elif args.only == "rotate-quant":
+        # the rotate+quantise kernel alone on the activations of the prefill
+        # workload: two warm launches, then 20 back to back timed with CUDA
+        # events (each reads 2 bytes and writes 1 byte per element, plus the
+        # row scales)
+        case = inputs.CASES[args.prefill_workload]
+        M, K = case.M, case.K
+        x = torch.from_numpy(inputs.activations(M, K, case.seed, case.dist).view(np.int16)).cuda() \
+            .view(torch.bfloat16)
+        xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+        xs = torch.empty(M, dtype=torch.float32, device="cuda")
+        for _ in range(2):
+            cr.cr_rotate_quant_act(x, xq=xq, xs=xs)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(20):
+            cr.cr_rotate_quant_act(x, xq=xq, xs=xs)
+        e1.record()
+        torch.cuda.synchronize()
+        t = e0.elapsed_time(e1) / 1000.0 / 20
+        out.update({"workload": case.name, "M": M, "K": K, "us": round(t * 1e6, 2),
+                    "gb_per_s": round((3 * M * K + 4 * M) / t / 1e9, 1)})
     elif args.only == "quantiser":
         # the offline quantiser and the stochastic re-assignment on an
         # [8192, 4096] rotated weight

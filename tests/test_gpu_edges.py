@@ -292,14 +292,16 @@ def test_gemv_decodes_every_scale_byte(cb_kind, scales):
 
 @pytest.mark.parametrize("cb_kind", ["fixed", "arange", "unsorted"])
 @pytest.mark.parametrize("scales", ["all_bytes", "generator", "one_large"])
-@pytest.mark.parametrize("N", [4096 + 48, 12288])
+@pytest.mark.parametrize("N", [4096 + 48, 4752, 19200])
 def test_prepared_layer_decode_matches_oracle(cb_kind, scales, N):
     """A prepared layer (W4A8Linear) checks its scale bytes once and then
-    decodes with split tables when all of them have one (and each CTA has
-    at most two row tiles: N = 4144 here; N = 12288 has more).  Its forward
-    and its GEMV on quantised activations must equal the oracle and the
-    unprepared GEMV bit for bit, for layers whose bytes all allow the split
-    form, none do, or all but one."""
+    decodes with split tables when all of them have one and each CTA has at
+    most two row tiles: N = 4144 (16-row tiles) and N = 4752 (32-row tiles,
+    the last one ragged); at N = 19200 (600 tiles of 32 rows) CTAs have more
+    and the plain tables serve.  Its forward and its GEMV on quantised
+    activations must equal the oracle and the unprepared GEMV bit for bit,
+    for layers whose bytes all allow the split form, none do, or all but
+    one."""
     K, seed = 2048, 91
     layer = inputs.layer(N, K, seed)
     cb = _codebook(cb_kind)

@@ -153,10 +153,13 @@ def test_gemv(M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(8, 8192, 8192), (3, 6000, 2048), (1, 5000, 256), (8, 12288, 4096),
-                                   (5, 4752, 7936)])
+                                   (5, 4752, 7936), (4, 4739, 1280), (8, 4736, 2304), (2, 19200, 1024)])
 def test_gemv_several_tiles_per_cta(M, N, K):
-    """More row tiles than CTA slots: CTAs walk several tiles, their rings
-    running across tile boundaries (chunk counts 1 to 8)."""
+    """Layers of at least one 32-row tile per SM (N >= 32 x 148), which take
+    32-row tiles: ragged last tiles (N = 4752, 5000, 6000, and 4739, whose
+    outputs leave one by one), exactly one tile per SM (N = 4736), CTAs
+    walking several tiles with their rings running across tile boundaries
+    (chunk counts 1 to 8)."""
     _contraction_case(cr.cr_w4a8_gemv, M, N, K, seed=M + N + K)
 
 
@@ -458,7 +461,8 @@ def _swiglu_case(fn, M, N, K, seed, kind="bf16", with_bias=False):
 
 @pytest.mark.parametrize("M,N,K,kind,bias", [(1, 32, 256, "bf16", False), (8, 4096, 1024, "bf16", False),
                                              (3, 26, 512, "bf16", True), (5, 1000, 2048, "f32", True),
-                                             (7, 2048, 16384, "bf16", False)])
+                                             (7, 2048, 16384, "bf16", False), (3, 4800, 1024, "bf16", True),
+                                             (8, 9000, 2048, "f32", False)])
 def test_gemv_swiglu(M, N, K, kind, bias):
     _swiglu_case(cr.cr_w4a8_gemv_swiglu, M, N, K, M + N + K, kind, bias)
 

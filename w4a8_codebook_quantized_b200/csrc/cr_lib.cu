@@ -39,6 +39,8 @@ struct DeviceState {
     std::atomic<bool> gemm_pair_attr_set{false};
     std::atomic<bool> gemv_attr_set{false};
     std::atomic<bool> gemv_split_attr_set{false};
+    std::atomic<bool> gemv32_attr_set{false};
+    std::atomic<bool> gemv32_split_attr_set{false};
     std::atomic<bool> gemv_grouped_attr_set{false};
     std::atomic<bool> gemm_bf16_attr_set{false};
     std::atomic<bool> gemm_pair_bf16_attr_set{false};
@@ -210,14 +212,26 @@ bool encode_gemv_x_map(CUtensorMap *map, const int8_t *xq, int64_t M, int64_t K)
                         true);
 }
 
-// Everything of a GEMV launch's arguments but the activations (tm_x, xs, M).
-// `tiles` returns the row tiles of all layers (0: nothing to launch).
+// Row tile height of a single-layer decode GEMV: 32 rows (two MMA row
+// blocks per activation stage) when the layer has at least one such tile per
+// SM, 16 otherwise, so that small layers keep more SMs busy.
+int gemv_tile_rows(int64_t N, int num_sms)
+{
+    return (N + 31) / 32 >= num_sms ? 32 : 16;
+}
+
+// Everything of a GEMV launch's arguments but the activations (tm_x, xs, M),
+// for row tiles of `rows` rows (16, or 32 for a single layer).  `tiles`
+// returns the row tiles of all layers (0: nothing to launch).
 template <int L>
 cr_status build_gemv_args(cr::gv::GemvArgs<L> &args, const float *codebook, int64_t K, const cr_w4a8_layer *layers,
-                          int num_layers, cr_out_dtype out_dtype, int swiglu, int64_t &tiles)
+                          int num_layers, cr_out_dtype out_dtype, int swiglu, int64_t &tiles, int rows = 16)
 {
     using namespace cr;
-    using C = gv::Prod;
+    using C = gv::Prod;  // the level-table copies (the same in every configuration)
+    static_assert(gv::Prod::kCopies == gv::Prod32::kCopies, "one table stride for both configurations");
+    if (rows != 16 && !(rows == 32 && L == 1))
+        return CR_ERR_INVALID_ARG;
     memset(&args, 0, sizeof(args));
     const uint64_t uK = (uint64_t)K;
     tiles = 0;
@@ -228,9 +242,9 @@ cr_status build_gemv_args(cr::gv::GemvArgs<L> &args, const float *codebook, int6
             continue; // no tiles; its pointers may be null
         const uint64_t uN = (uint64_t)ly.N;
         if (!make_tmap_3d(&args.tm_codes[l], ly.qdata, CU_TENSOR_MAP_DATA_TYPE_UINT32, {16, uN, uK / gv::kSlice},
-                          {uK / 2, 64}, {16, (uint32_t)gv::kRows, (uint32_t)(gv::kChunk / gv::kSlice)}, false) ||
+                          {uK / 2, 64}, {16, (uint32_t)rows, (uint32_t)(gv::kChunk / gv::kSlice)}, false) ||
             !make_tmap_3d(&args.tm_srel[l], ly.srel, CU_TENSOR_MAP_DATA_TYPE_UINT8, {16, uN, uK / 256}, {uK / 16, 16},
-                          {16, (uint32_t)gv::kRows, (uint32_t)(gv::kChunk / 256)}, false))
+                          {16, (uint32_t)rows, (uint32_t)(gv::kChunk / 256)}, false))
             return CR_ERR_CUDA;
         args.layer[l].ws = ly.s_channel;
         args.layer[l].bias = ly.bias;
@@ -238,7 +252,7 @@ cr_status build_gemv_args(cr::gv::GemvArgs<L> &args, const float *codebook, int6
         args.layer[l].acc_out = ly.acc_out;
         args.layer[l].N = (int)ly.N;
         args.layer[l].swiglu = swiglu;
-        tiles += (ly.N + gv::kRows - 1) / gv::kRows;
+        tiles += (ly.N + rows - 1) / rows;
     }
     if (tiles > INT_MAX)
         return CR_ERR_UNSUPPORTED;
@@ -249,6 +263,7 @@ cr_status build_gemv_args(cr::gv::GemvArgs<L> &args, const float *codebook, int6
     args.out_f32 = out_dtype == CR_OUT_F32 ? 1 : 0;
     args.lut_step = (uint32_t)(C::kCopies * sizeof(uint4));
     args.ahead = gv::kPrefetchAhead;
+    args.tile_rows = rows;
     return CR_OK;
 }
 
@@ -257,14 +272,13 @@ cr_status build_gemv_args(cr::gv::GemvArgs<L> &args, const float *codebook, int6
 // previous kernel on the stream.  split: the layer's tables all have a split
 // form (checked when it was prepared); the split variant of the kernel runs
 // where every CTA has at most two row tiles.  attr_set / split_attr_set: the
-// once-per-device shared-memory attribute of the plain and split variants.
-template <int L>
-cr_status launch_gemv_args(int num_sms, std::atomic<bool> &attr_set, const cr::gv::GemvArgs<L> &args,
-                           cudaStream_t stream, bool pdl, bool split = false,
-                           std::atomic<bool> *split_attr_set = nullptr)
+// once-per-device shared-memory attribute of the plain and split variants of
+// configuration C.
+template <class C, int L>
+cr_status launch_gemv_cfg(int num_sms, std::atomic<bool> &attr_set, const cr::gv::GemvArgs<L> &args,
+                          cudaStream_t stream, bool pdl, bool split, std::atomic<bool> *split_attr_set)
 {
     using namespace cr;
-    using C = gv::Prod;
     // persistent grid of several CTAs per SM, at most one wave
     const int64_t slots = (int64_t)C::kMinBlocks * num_sms;
     const int64_t grid = args.num_tiles < slots ? args.num_tiles : slots;
@@ -292,21 +306,42 @@ cr_status launch_gemv_args(int num_sms, std::atomic<bool> &attr_set, const cr::g
     return launched(cudaLaunchKernelEx(&cfg, kern, args));
 }
 
+// The configuration the arguments were built for (args.tile_rows): 32-row
+// tiles need the flags of their own attributes (attr32_set, split32_set).
+template <int L>
+cr_status launch_gemv_args(int num_sms, std::atomic<bool> &attr_set, const cr::gv::GemvArgs<L> &args,
+                           cudaStream_t stream, bool pdl, bool split = false,
+                           std::atomic<bool> *split_attr_set = nullptr, std::atomic<bool> *attr32_set = nullptr,
+                           std::atomic<bool> *split32_set = nullptr)
+{
+    if constexpr (L == 1) {
+        if (args.tile_rows == 32) {
+            if (attr32_set == nullptr)
+                return CR_ERR_INVALID_ARG;
+            return launch_gemv_cfg<cr::gv::Prod32, 1>(num_sms, *attr32_set, args, stream, pdl, split, split32_set);
+        }
+    }
+    return launch_gemv_cfg<cr::gv::Prod, L>(num_sms, attr_set, args, stream, pdl, split, split_attr_set);
+}
+
+// attr32_set: the flag of the 32-row configuration's attribute, or null to
+// keep 16-row tiles.
 template <int L>
 cr_status launch_gemv(int num_sms, std::atomic<bool> &attr_set, const int8_t *xq, const float *xs, const float *codebook,
                       int64_t M, int64_t K, const cr_w4a8_layer *layers, int num_layers, cr_out_dtype out_dtype,
-                      cudaStream_t stream, bool pdl, int swiglu = 0)
+                      cudaStream_t stream, bool pdl, int swiglu = 0, std::atomic<bool> *attr32_set = nullptr)
 {
     cr::gv::GemvArgs<L> args;
     int64_t tiles = 0;
-    cr_status st = build_gemv_args<L>(args, codebook, K, layers, num_layers, out_dtype, swiglu, tiles);
+    const int rows = (L == 1 && attr32_set != nullptr) ? gemv_tile_rows(layers[0].N, num_sms) : 16;
+    cr_status st = build_gemv_args<L>(args, codebook, K, layers, num_layers, out_dtype, swiglu, tiles, rows);
     if (st != CR_OK || tiles == 0)
         return st;
     if (!encode_gemv_x_map(&args.tm_x, xq, M, K))
         return CR_ERR_CUDA;
     args.xs = xs;
     args.M = (int)M;
-    return launch_gemv_args<L>(num_sms, attr_set, args, stream, pdl);
+    return launch_gemv_args<L>(num_sms, attr_set, args, stream, pdl, false, nullptr, attr32_set);
 }
 
 
@@ -316,7 +351,7 @@ cr_status run_gemv_layers(DeviceState &d, const int8_t *xq, const float *xs, con
 {
     if (num_layers == 1)
         return launch_gemv<1>(d.num_sms, d.gemv_attr_set, xq, xs, codebook, M, K, layers, 1, out_dtype, stream,
-                              pdl);
+                              pdl, 0, &d.gemv32_attr_set);
     return launch_gemv<cr::gv::kMaxLayers>(d.num_sms, d.gemv_grouped_attr_set, xq, xs, codebook, M, K, layers,
                                            num_layers, out_dtype, stream, pdl);
 }
@@ -325,7 +360,7 @@ cr_status run_gemv_layers(DeviceState &d, const int8_t *xq, const float *xs, con
 cr_status run_gemv(int num_sms, std::atomic<bool> &attr_set, const int8_t *xq, const float *xs, const uint8_t *qdata,
                    const uint8_t *srel, const float *codebook, const float *s_channel, const float *bias, int64_t M,
                    int64_t N, int64_t K, cr_out_dtype out_dtype, void *out, int32_t *acc_out, cudaStream_t stream,
-                   bool pdl, int swiglu = 0)
+                   bool pdl, int swiglu = 0, std::atomic<bool> *attr32_set = nullptr)
 {
     cr_w4a8_layer ly;
     ly.qdata = qdata;
@@ -335,7 +370,8 @@ cr_status run_gemv(int num_sms, std::atomic<bool> &attr_set, const int8_t *xq, c
     ly.N = N;
     ly.out = out;
     ly.acc_out = acc_out;
-    return launch_gemv<1>(num_sms, attr_set, xq, xs, codebook, M, K, &ly, 1, out_dtype, stream, pdl, swiglu);
+    return launch_gemv<1>(num_sms, attr_set, xq, xs, codebook, M, K, &ly, 1, out_dtype, stream, pdl, swiglu,
+                          attr32_set);
 }
 
 // Shared validation of the contraction entry points.
@@ -743,7 +779,7 @@ cr_status cr_w4a8_gemv(const int8_t *xq, const float *xs, const uint8_t *qdata, 
     if (st != CR_OK)
         return st;
     return run_gemv(d->num_sms, d->gemv_attr_set, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K,
-                    out_dtype, out, acc_out, stream, /*pdl=*/true);
+                    out_dtype, out, acc_out, stream, /*pdl=*/true, 0, &d->gemv32_attr_set);
 }
 
 cr_status cr_epilogue(const int32_t *acc, const float *xs, const float *s_channel, const float *bias, int64_t M,
@@ -817,7 +853,7 @@ cr_status linear_impl(const uint16_t *x, const uint8_t *qdata, const uint8_t *sr
     if (st != CR_OK)
         return st;
     return run_gemv(d->num_sms, d->gemv_attr_set, xq_work, xs_work, qdata, srel, codebook, s_channel, bias, M, N, K,
-                    out_dtype, out, nullptr, stream, /*pdl=*/true, swiglu);
+                    out_dtype, out, nullptr, stream, /*pdl=*/true, swiglu, &d->gemv32_attr_set);
 }
 
 // cr_w4a8_gemm_swiglu and cr_w4a8_gemv_swiglu.
@@ -838,7 +874,7 @@ cr_status contraction_swiglu(bool gemv, const int8_t *xq, const float *xs, const
         return st;
     if (gemv)
         return run_gemv(d->num_sms, d->gemv_attr_set, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K,
-                        out_dtype, out, nullptr, stream, /*pdl=*/true, /*swiglu=*/1);
+                        out_dtype, out, nullptr, stream, /*pdl=*/true, /*swiglu=*/1, &d->gemv32_attr_set);
     return run_gemm(*d, xq, xs, qdata, srel, codebook, s_channel, bias, M, N, K, out_dtype, out, nullptr, stream,
                     nullptr, /*swiglu=*/1);
 }
@@ -1158,7 +1194,7 @@ cr_status cr_w4a8_plan_create(const uint8_t *qdata, const uint8_t *srel, const f
     p->out_dtype = out_dtype;
     if (N > 0) {
         cr_w4a8_layer ly{qdata, srel, s_channel, bias, N, nullptr, nullptr};
-        st = build_gemv_args<1>(p->gemv, codebook, K, &ly, 1, out_dtype, 0, p->tiles);
+        st = build_gemv_args<1>(p->gemv, codebook, K, &ly, 1, out_dtype, 0, p->tiles, gemv_tile_rows(N, d->num_sms));
         if (st == CR_OK)
             st = check_split(*d, srel, codebook, N, K, p->split_ok);
         if (st != CR_OK) {
@@ -1218,7 +1254,8 @@ cr_status cr_w4a8_plan_forward(cr_w4a8_plan plan, const uint16_t *x, int64_t M, 
     args.M = (int)M;
     args.layer[0].out = out;
     return launch_gemv_args<1>(plan->d->num_sms, plan->d->gemv_attr_set, args, stream, /*pdl=*/true,
-                               plan->split_ok, &plan->d->gemv_split_attr_set);
+                               plan->split_ok, &plan->d->gemv_split_attr_set, &plan->d->gemv32_attr_set,
+                               &plan->d->gemv32_split_attr_set);
 }
 
 cr_status cr_w4a8_plan_gemv(cr_w4a8_plan plan, const int8_t *xq, const float *xs, int64_t M, void *out,
@@ -1254,7 +1291,8 @@ cr_status cr_w4a8_plan_gemv(cr_w4a8_plan plan, const int8_t *xq, const float *xs
     args.M = (int)M;
     args.layer[0].out = out;
     return launch_gemv_args<1>(plan->d->num_sms, plan->d->gemv_attr_set, args, stream, /*pdl=*/true,
-                               plan->split_ok, &plan->d->gemv_split_attr_set);
+                               plan->split_ok, &plan->d->gemv_split_attr_set, &plan->d->gemv32_attr_set,
+                               &plan->d->gemv32_split_attr_set);
 }
 
 cr_status cr_w4a8_plan_forward_host(cr_w4a8_plan plan, const uint16_t *x_host, int64_t M, void *out_host,
@@ -1396,7 +1434,7 @@ cr_status cr_w4a8_host_call_run(cr_w4a8_host_call c, cr_stream_t stream)
         st = launched(cr::rq::launch(c->x_dev, c->M, plan->K, c->MP, plan->act_qmax, c->xq, c->xs, stream));
         if (st == CR_OK)
             st = launch_gemv_args<1>(d->num_sms, d->gemv_attr_set, c->gemv, stream, /*pdl=*/true, plan->split_ok,
-                                     &d->gemv_split_attr_set);
+                                     &d->gemv_split_attr_set, &d->gemv32_attr_set, &d->gemv32_split_attr_set);
     }
     if (st != CR_OK)
         return st;
@@ -1552,7 +1590,8 @@ cr_status noalloc_scratch(NoallocState **out)
         }
         s.scratch = static_cast<uint8_t *>(p);
         if (cudaFuncSetAttribute(cr::gv::gemv_kernel<cr::gv::Prod, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)cr::gv::Prod::kSmemBytes) != cudaSuccess) {
+                                 (int)cr::gv::Prod::kSmemBytes) != cudaSuccess ||
+            cr::rq::set_attributes() != cudaSuccess) {
             cudaGetLastError();
             return CR_ERR_CUDA;
         }

@@ -8,10 +8,10 @@
 //
 // B200 design.
 //  * Streaming: a persistent grid (two CTAs per SM).  In each CTA one
-//    producer warp moves, per stage, the packed codes (16 weight rows x 1024
-//    columns, 8 KB), their group scales (1 KB) and the matching 1024 columns
-//    of the M <= 8 activation rows (M KB) into a ring of shared-memory
-//    stages with 3-D TMA copies; eight consumer warps decode and contract each
+//    producer warp moves, per stage, the packed codes of a row tile (16 or
+//    32 weight rows x 1024 columns, 8 or 16 KB), their group scales (1 or
+//    2 KB) and the matching 1024 columns of the M <= 8 activation rows (M KB)
+//    into a ring of shared-memory stages with 3-D TMA copies; eight consumer warps decode and contract each
 //    stage while the following ones are in flight; an epilogue warp reduces
 //    the consumers' partial sums and writes the outputs of a tile while the
 //    consumers already work on the next one.  Bytes in flight are set by the
@@ -40,6 +40,15 @@
 //    slice w, and the matching 32 activation bytes of token g; code word i
 //    (columns 8i..8i+7) feeds MMA i, its first four columns in the fragment
 //    slots of logical k = 4t..4t+3 and its last four in 16+4t..16+4t+3.
+//  * Tile height: with 32-row tiles a stage's activation copy and each
+//    thread's activation fragments serve two MMA row blocks (rows 0-15 and
+//    16-31), which halves the activation traffic into shared memory and the
+//    per-stage ring overhead per weight.  Measured on B200, a stage's
+//    activation copy costs far more than its bytes (removing it entirely took
+//    an M = 8, N = K = 8192 GEMV from 11.1 to 9.3 us; spreading its reads over
+//    16 copies in L2 changed nothing), so the copies per weight are what
+//    matters.  Layers with fewer tiles than SMs keep 16-row tiles, which
+//    spread them over more SMs.
 //  * Launch overlap: the kernel lets the next kernel on the stream launch at
 //    once, and it may itself start before the previous kernel ends (weight
 //    stream and table build first); the activation copies and every read of
@@ -58,31 +67,36 @@ constexpr int kConsumerWarps = 8;
 constexpr int kProducerWarp = kConsumerWarps;       // TMA issue
 constexpr int kEpilogueWarp = kConsumerWarps + 1;   // reduction, split-tile hand-off, outputs
 constexpr int kThreads = (kConsumerWarps + 2) * 32;
-constexpr int kRows = 16;                            // weight rows of a tile (the MMA's M)
+constexpr int kMmaRows = 16;                         // weight rows of one MMA (its M)
 constexpr int kSlice = 128;                          // columns per consumer warp per stage
 constexpr int kChunk = kConsumerWarps * kSlice;      // columns per stage
 constexpr int kTokens = 8;                           // activation rows of a stage (the MMA's N)
-constexpr int kCodeBytes = kRows * kChunk / 2;
-constexpr int kSrelBytes = kRows * kChunk / 16;
 constexpr int kXBytes = kTokens * kChunk;  // room for M = 8; a stage carries M * kChunk
 constexpr int kPrefetchAhead = 3;  // L2 prefetch distance of the weight stream, in stages
 constexpr int kRedBufs = 1;  // partial-sum mailboxes between the consumers and the epilogue warp
 
 // Shape of the ring: STAGES stages, MINB CTAs per SM, COPIES copies of the
 // level table (8 copies make every quarter-warp lookup conflict-free, 4 leave
-// occasional two-way conflicts for half the shared memory).
-template <int STAGES, int MINB, int COPIES>
+// occasional two-way conflicts for half the shared memory), ROWS weight rows
+// per tile: 16 (one MMA row block), or 32 (two row blocks that share every
+// activation stage and every activation fragment, so that a stage's
+// activation copy serves twice the weights).
+template <int STAGES, int MINB, int COPIES, int ROWS>
 struct Cfg {
     static constexpr int kStages = STAGES;
     static constexpr int kMinBlocks = MINB;
     static constexpr int kCopies = COPIES;
+    static constexpr int kRows = ROWS;
+    static constexpr int kBlocks = ROWS / kMmaRows;  // MMA row blocks per tile
+    static constexpr int kCodeBytes = ROWS * kChunk / 2;
+    static constexpr int kSrelBytes = ROWS * kChunk / 16;
     struct __align__(1024) Smem {
         uint8_t x[STAGES][kXBytes];          // [slice][token < M][128 B], 128-byte swizzle (1024-aligned)
         uint8_t codes[STAGES][kCodeBytes];   // [slice][row][64 B]
         uint8_t srel[STAGES][kSrelBytes];    // [256-column block][row][16 B]
         uint4 lut[256 * COPIES];             // lut[s * COPIES + c]: copy c of the levels of scale byte s
-        int32_t red[kRedBufs][kConsumerWarps][kRows][8];  // per-warp partial sums
-        alignas(16) uint16_t ostage[kTokens][kRows];      // a tile's bf16 outputs, token-major
+        int32_t red[kRedBufs][kConsumerWarps][ROWS][8];  // per-warp partial sums
+        alignas(16) uint16_t ostage[kTokens][ROWS];      // a tile's bf16 outputs, token-major
         float cb[16];
         uint64_t full[STAGES];
         uint64_t empty[STAGES];
@@ -93,8 +107,10 @@ struct Cfg {
     static constexpr size_t kSmemBytes = sizeof(Smem) + 1024;
 };
 
-// The configuration the library launches.
-using Prod = Cfg<5, 2, 4>;
+// The configurations the library launches: 16-row tiles, and 32-row tiles
+// for single layers with enough rows to fill the SMs with them.
+using Prod = Cfg<5, 2, 4, 16>;
+using Prod32 = Cfg<3, 2, 4, 32>;
 
 __device__ __forceinline__ void mma_s8(int32_t (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                        uint32_t b0, uint32_t b1)
@@ -108,8 +124,9 @@ __device__ __forceinline__ void mma_s8(int32_t (&c)[4], uint32_t a0, uint32_t a1
 
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
-// The operands of one stage for one thread: its activation fragments, the
-// 32 codes of rows g and g + 8, and the level tables of their two groups.
+// The operands of one stage for one thread and one MMA row block: the
+// activation fragments (shared by the tile's row blocks), the 32 codes of
+// rows g and g + 8, and the level tables of their two groups.
 struct Ops {
     uint4 X0, X1, A, B, TA0, TA1, TB0, TB1;
 };
@@ -119,11 +136,9 @@ struct Ops {
 // further.  lut_step is a kernel argument rather than a constant so that the
 // address is one integer multiply-add, which issues on the FMA pipe and leaves
 // the ALU pipe, the decode's bottleneck, to the byte permutes.
-__device__ __forceinline__ void fetch_ops(Ops &o, const uint8_t *x0, const uint8_t *x1, const uint8_t *codes_g,
-                                          const uint8_t *srel_g, const uint8_t *lutb, uint32_t lut_step)
+__device__ __forceinline__ void fetch_w(Ops &o, const uint8_t *codes_g, const uint8_t *srel_g, const uint8_t *lutb,
+                                        uint32_t lut_step)
 {
-    o.X0 = *reinterpret_cast<const uint4 *>(x0);
-    o.X1 = *reinterpret_cast<const uint4 *>(x1);
     o.A = *reinterpret_cast<const uint4 *>(codes_g);
     o.B = *reinterpret_cast<const uint4 *>(codes_g + 8 * 64);
     o.TA0 = *reinterpret_cast<const uint4 *>(lutb + (uint32_t)srel_g[0] * lut_step);
@@ -233,6 +248,7 @@ struct GemvArgs {
     int M, K, num_layers, num_tiles, out_f32;
     uint32_t lut_step;
     int ahead;
+    int tile_rows;  // the configuration's row tile height (16 or 32), for the host's launch
 };
 
 // The layer that owns global row tile `tile`.
@@ -248,15 +264,15 @@ __device__ __forceinline__ int layer_of(const GemvArgs<L> &a, int tile)
 }
 
 // Layer and first row of global row tile `tile` (compile-time for one layer).
-template <int L>
+template <int ROWS, int L>
 __device__ __forceinline__ void locate(const GemvArgs<L> &a, int tile, int &l, int &row)
 {
     if constexpr (L == 1) {
         l = 0;
-        row = tile * kRows;
+        row = tile * ROWS;
     } else {
         l = layer_of(a, tile);
-        row = (tile - a.layer[l].tile0) * kRows;
+        row = (tile - a.layer[l].tile0) * ROWS;
     }
 }
 
@@ -270,7 +286,8 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
     extern __shared__ uint8_t smem_raw[];
     Smem &sh = smem_aligned_1024<Smem>(smem_raw);
     const int M = a.M, K = a.K;
-    const uint32_t stage_tx = (uint32_t)(kCodeBytes + kSrelBytes + M * kChunk);
+    constexpr int kRows = C::kRows, kBlocks = C::kBlocks;
+    const uint32_t stage_tx = (uint32_t)(C::kCodeBytes + C::kSrelBytes + M * kChunk);
 
     // The next kernel on the stream may launch now: a GEMV of the next layer
     // starts its weight stream in the SM slots this grid frees, and whatever
@@ -335,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
             };
             auto weights = [&](const Pos &p, int s) {
                 int l, row;
-                locate(a, p.tile, l, row);
+                locate<C::kRows>(a, p.tile, l, row);
                 tma_load_3d(sh.codes[s], &a.tm_codes[l], 0, row, p.c * (kChunk / kSlice), &sh.full[s]);
                 tma_load_3d(sh.srel[s], &a.tm_srel[l], 0, row, p.c * (kChunk / 256), &sh.full[s]);
             };
@@ -344,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
             // its data in L2
             auto prefetch = [&](const Pos &p) {
                 int l, row;
-                locate(a, p.tile, l, row);
+                locate<C::kRows>(a, p.tile, l, row);
                 tma_prefetch_3d(&a.tm_codes[l], 0, row, p.c * (kChunk / kSlice));
                 tma_prefetch_3d(&a.tm_srel[l], 0, row, p.c * (kChunk / 256));
             };
@@ -420,9 +437,10 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
 
         const int g = lane >> 2, t = lane & 3, sl = warp;
         const uint8_t *lutb = reinterpret_cast<const uint8_t *>(sh.lut + (lane & (C::kCopies - 1)));
-        // this thread's offsets inside a stage
-        const int off_code = sl * (kRows * 64) + g * 64 + 16 * t;                       // row g; g + 8 at +512
-        const int off_srel = (sl >> 1) * (kRows * 16) + g * 16 + 8 * (sl & 1) + 2 * t;  // row g; g + 8 at +128
+        // this thread's offsets inside a stage (row g; g + 8 at +512 and +128;
+        // MMA row block b at +1024 b and +256 b)
+        const int off_code = sl * (kRows * 64) + g * 64 + 16 * t;
+        const int off_srel = (sl >> 1) * (kRows * 16) + g * 16 + 8 * (sl & 1) + 2 * t;
         // 128-byte line of (slice sl, token g); the swizzle permutes the
         // 16-byte chunks of a line by its index mod 8
         const int xl = sl * M + g;
@@ -431,23 +449,34 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
         // chunks in which this warp's slice lies inside K (K is a multiple of 256)
         const int nvalid = (K - kSlice * sl + kChunk - 1) / kChunk;
         // hand a tile's partial sums to the epilogue warp and go on
-        auto hand_off = [&](int seg, int32_t (&c)[4], int32_t (&d)[4]) {
+        auto hand_off = [&](int seg, int32_t (&c)[kBlocks][4], int32_t (&d)[kBlocks][4]) {
             const int rb = seg % kRedBufs;
             const bool ok = mbar_wait_bounded_warp(&sh.red_empty[rb], ((uint32_t)(seg / kRedBufs) & 1u) ^ 1u, abort);
             // C fragment: c0 (row g, token 2t), c1 (g, 2t+1), c2 (g+8, 2t), c3 (g+8, 2t+1)
-            sh.red[rb][warp][g][2 * t] = c[0] + d[0];
-            sh.red[rb][warp][g][2 * t + 1] = c[1] + d[1];
-            sh.red[rb][warp][g + 8][2 * t] = c[2] + d[2];
-            sh.red[rb][warp][g + 8][2 * t + 1] = c[3] + d[3];
+#pragma unroll
+            for (int b = 0; b < kBlocks; ++b) {
+                const int r = kMmaRows * b + g;
+                sh.red[rb][warp][r][2 * t] = c[b][0] + d[b][0];
+                sh.red[rb][warp][r][2 * t + 1] = c[b][1] + d[b][1];
+                sh.red[rb][warp][r + 8][2 * t] = c[b][2] + d[b][2];
+                sh.red[rb][warp][r + 8][2 * t + 1] = c[b][3] + d[b][3];
+            }
             __syncwarp();
             if (ok && lane == 0)
                 mbar_arrive(&sh.red_full[rb]);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-                c[i] = d[i] = 0;
+            for (int b = 0; b < kBlocks; ++b)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    c[b][i] = d[b][i] = 0;
         };
-        // two accumulators break the dependency chain between MMAs
-        int32_t c[4] = {0, 0, 0, 0}, d[4] = {0, 0, 0, 0};
+        // two accumulators per row block break the dependency chain between MMAs
+        int32_t c[kBlocks][4], d[kBlocks][4];
+#pragma unroll
+        for (int b = 0; b < kBlocks; ++b)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                c[b][i] = d[b][i] = 0;
         int ch = 0, seg = 0;
         // The ring is walked STAGES stages at a time with the stage index a
         // compile-time constant, so every shared-memory address is a fixed
@@ -459,13 +488,25 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
                 if (q0 + s < total) {
                     const bool ok = mbar_wait_bounded_warp(&sh.full[s], ph, abort);
                     if (ok && ch < nvalid) {
-                        Ops o;
-                        fetch_ops(o, sh.x[s] + off_x0, sh.x[s] + off_x1, sh.codes[s] + off_code,
-                                  sh.srel[s] + off_srel, lutb, a.lut_step);
-                        if constexpr (SPLIT)
-                            slice_mma_split(o, c, d);
-                        else
-                            slice_mma(o, c, d);
+                        Ops o[kBlocks];
+                        o[0].X0 = *reinterpret_cast<const uint4 *>(sh.x[s] + off_x0);
+                        o[0].X1 = *reinterpret_cast<const uint4 *>(sh.x[s] + off_x1);
+#pragma unroll
+                        for (int b = 0; b < kBlocks; ++b) {
+                            if (b > 0) {
+                                o[b].X0 = o[0].X0;
+                                o[b].X1 = o[0].X1;
+                            }
+                            fetch_w(o[b], sh.codes[s] + off_code + 1024 * b, sh.srel[s] + off_srel + 256 * b, lutb,
+                                    a.lut_step);
+                        }
+#pragma unroll
+                        for (int b = 0; b < kBlocks; ++b) {
+                            if constexpr (SPLIT)
+                                slice_mma_split(o[b], c[b], d[b]);
+                            else
+                                slice_mma(o[b], c[b], d[b]);
+                        }
                     }
                     __syncwarp();
                     if (ok && lane == 0)
@@ -487,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
         for (int seg = 0; seg < my_tiles; ++seg) {
             const int tile = (int)blockIdx.x + seg * (int)gridDim.x;
             int l, row0;
-            locate(a, tile, l, row0);
+            locate<C::kRows>(a, tile, l, row0);
             const GemvLayer &ly = a.layer[l];
             const int N = ly.N;
             const float *__restrict__ ws = ly.ws;
@@ -497,10 +538,11 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
             int32_t *__restrict__ acc_out = ly.acc_out;
             const bool out_f32 = a.out_f32 != 0;
             // this lane's outputs: e = lane + 32 u -> row e / 8, token e % 8
-            float exs[4], ews[4], eb[4];
-            bool live[4];
+            constexpr int kOut = kRows * kTokens / 32;  // outputs per lane
+            float exs[kOut], ews[kOut], eb[kOut];
+            bool live[kOut];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < kOut; ++u) {
                 const int e = lane + 32 * u, r = e >> 3, m = e & 7, n = row0 + r;
                 live[u] = m < M && n < N;
                 exs[u] = live[u] ? xs[m] : 0.0f;
@@ -509,9 +551,9 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
             }
             const int rb = seg % kRedBufs;
             const bool ok = mbar_wait_bounded_warp(&sh.red_full[rb], (uint32_t)(seg / kRedBufs) & 1u, abort);
-            int32_t acc[4];
+            int32_t acc[kOut];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < kOut; ++u) {
                 const int e = lane + 32 * u;
                 int32_t v = 0;
 #pragma unroll
@@ -529,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
                 // of the same u (row0 is a multiple of 16)
                 const int F = N >> 1;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < kOut; ++u) {
                     const int e = lane + 32 * u, n = row0 + (e >> 3), m = e & 7;
                     float y = __fmul_rn(__int2float_rn(acc[u]), __fmul_rn(exs[u], ews[u]));
                     if (bias != nullptr)
@@ -546,9 +588,9 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
                 }
             } else if (go && !out_f32 && acc_out == nullptr && (N & 7) == 0 && row0 + kRows <= N) {
                 // a whole tile of bf16 outputs: staged token-major, then each
-                // token's 16 outputs leave as two 16-byte stores
+                // token's kRows outputs leave as kRows / 8 16-byte stores
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < kOut; ++u) {
                     const int e = lane + 32 * u;
                     float y = __fmul_rn(__int2float_rn(acc[u]), __fmul_rn(exs[u], ews[u]));
                     if (bias != nullptr)
@@ -556,15 +598,16 @@ __global__ void __launch_bounds__(kThreads, C::kMinBlocks) gemv_kernel(const __g
                     sh.ostage[e & 7][e >> 3] = to_bf16_bits(y);
                 }
                 __syncwarp();
-                if (lane < 2 * M) {
-                    const int m = lane >> 1, h = lane & 1;
+                constexpr int kPieces = kRows / 8;  // 16-byte pieces of a token's outputs
+                if (lane < kPieces * M) {
+                    const int m = lane / kPieces, h = lane % kPieces;
                     const uint4 v = *reinterpret_cast<const uint4 *>(&sh.ostage[m][8 * h]);
                     *reinterpret_cast<uint4 *>(reinterpret_cast<uint16_t *>(out) + (int64_t)m * N + row0 + 8 * h) = v;
                 }
                 __syncwarp();
             } else if (go) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
+                for (int u = 0; u < kOut; ++u) {
                     if (!live[u])
                         continue;
                     const int e = lane + 32 * u, n = row0 + (e >> 3), m = e & 7;
