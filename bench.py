@@ -59,9 +59,11 @@ def parse():
     p.add_argument("--prefill-extra", default="c3_prefill_2k_4k,c4_mlp_up,c4_mlp_down",
                    help="comma-separated prefill workloads reported beside the prefill block (empty: none)")
     p.add_argument("--backward-workload", default="c3_prefill_2k_4k")
-    p.add_argument("--only", default=None, choices=["headline", "decode-transient", "quantiser", "int8-peak", "rotate-quant"],
+    p.add_argument("--only", default=None,
+                   choices=["headline", "decode-transient", "quantiser", "int8-peak", "rotate-quant", "prefill"],
                    help="run one piece alone (profiling runs): the headline step and GEMV, the prefill weight "
-                        "transient, the offline quantiser, or the INT8 rate kernel")
+                        "transient, the offline quantiser, the INT8 rate kernel, the rotate+quantise kernel on "
+                        "the prefill workload's activations, or the prefill block of --prefill-workload")
     p.add_argument("--no-prefill", action="store_true")
     p.add_argument("--no-grouped", action="store_true")
     p.add_argument("--no-swiglu", action="store_true")
@@ -98,6 +100,7 @@ def gemv_launch_bytes(M, N, K):
 
 
 GEMV_SOURCES = ("k_gemv.cuh", "cr_device.cuh")
+KERNEL_LAUNCHES = 200  # chained launches over which a roofline kernel's duration is averaged
 
 
 def source_digest(files):
@@ -430,15 +433,19 @@ def gemv_block(case, args, world, rank, local, pk, sets=None):
     secs, clocks = graph_time(sets.step, args.steps, args.warmup, world, local)
     secs = max_over_ranks(secs, world)
     wb = weight_bytes(N, K)
-    ksecs, _ = graph_time(sets.contraction_only, args.steps, args.warmup, world, local)
+    # the kernel's own duration: a chain of at least KERNEL_LAUNCHES launches
+    # in one graph, so that the graph's start-up is not charged to a short
+    # chain's few launches
+    klaunches = max(args.steps, KERNEL_LAUNCHES)
+    ksecs, _ = graph_time(sets.contraction_only, klaunches, args.warmup, world, local)
     ksecs = max_over_ranks(ksecs, world)
-    per_launch = ksecs / args.steps
+    per_launch = ksecs / klaunches
     achieved = gemv_launch_bytes(M, N, K) / per_launch / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": prior_traffic(f"gemv_kernel_{case.name}"),
                 "kernel": "cr::gv::gemv_kernel", "peak_source": f"{pk['source']} (hbm_gbs)",
                 "algorithmic_bytes_per_launch": gemv_launch_bytes(M, N, K),
-                "us_per_launch": round(per_launch * 1e6, 3)}
+                "us_per_launch": round(per_launch * 1e6, 3), "launches_timed": klaunches}
     return {"workload": f"{case.name}: decode batch M={M}, N={N}, K={K}, rot 256, group 16, seed {case.seed}",
             "value": round(aggregate_value(wb, args.steps, world, secs), 2), "unit": "GB/s",
             "us_per_step": round(secs / args.steps * 1e6, 3),
@@ -495,6 +502,14 @@ def run_ours(args):
     if args.only in ("decode-transient", "quantiser", "int8-peak", "rotate-quant"):
         return run_only(args, world, rank, local)
     pk = peaks()
+    if args.only == "prefill":
+        # the prefill block of --prefill-workload alone (its INT8 fraction
+        # against the measured bf16 rate x the nominal ratio)
+        blk = run_prefill(args, world, rank, pk, None, args.prefill_workload)
+        cr.cr_check_device_error()
+        if rank == 0:
+            print(json.dumps({"only": "prefill", **blk}), flush=True)
+        return
     case = inputs.CASES[args.workload]
     if case.M > 8:
         raise SystemExit("the headline workload must be a decode batch (M <= 8)")
@@ -646,7 +661,8 @@ def run_only(args, world, rank, local):
         out.update(measure_int8_peak(world))
     elif args.only == "decode-transient":
         # the prefill's int8 weight transient on an [8192, 4096] layer: two
-        # warm launches, then 20 back to back timed with CUDA events
+        # warm launches, then 20 back to back in one CUDA graph, timed with
+        # CUDA events
         N, K = 8192, 4096
         layer = inputs.layer(N, K, 1)
         q, s, cb = (torch.from_numpy(a).cuda() for a in (layer.qdata, layer.srel, layer.codebook))
@@ -654,20 +670,15 @@ def run_only(args, world, rank, local):
         for _ in range(2):
             cr.cr_w4a8_decode_int8(q, s, cb, w8)
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(20):
-            cr.cr_w4a8_decode_int8(q, s, cb, w8)
-        e1.record()
-        torch.cuda.synchronize()
-        t = e0.elapsed_time(e1) / 1000.0 / 20
+        t = replay_time(lambda: cr.cr_w4a8_decode_int8(q, s, cb, w8, stream=torch.cuda.current_stream()), 20)
         out.update({"N": N, "K": K, "us": round(t * 1e6, 2),
                     "gb_per_s": round(N * K * (0.5 + 1 / 16 + 1) / t / 1e9, 1)})
     elif args.only == "rotate-quant":
         # the rotate+quantise kernel alone on the activations of the prefill
-        # workload: two warm launches, then 20 back to back timed with CUDA
-        # events (each reads 2 bytes and writes 1 byte per element, plus the
-        # row scales)
+        # workload: two warm launches, then 20 back to back in one CUDA
+        # graph, timed with CUDA events (each reads 2 bytes and writes 1 byte
+        # per element, plus the row scales; the 20 launches reuse one input,
+        # so it comes from L2 after the first)
         case = inputs.CASES[args.prefill_workload]
         M, K = case.M, case.K
         x = torch.from_numpy(inputs.activations(M, K, case.seed, case.dist).view(np.int16)).cuda() \
@@ -677,13 +688,7 @@ def run_only(args, world, rank, local):
         for _ in range(2):
             cr.cr_rotate_quant_act(x, xq=xq, xs=xs)
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for _ in range(20):
-            cr.cr_rotate_quant_act(x, xq=xq, xs=xs)
-        e1.record()
-        torch.cuda.synchronize()
-        t = e0.elapsed_time(e1) / 1000.0 / 20
+        t = replay_time(lambda: cr.cr_rotate_quant_act(x, xq=xq, xs=xs, stream=torch.cuda.current_stream()), 20)
         out.update({"workload": case.name, "M": M, "K": K, "us": round(t * 1e6, 2),
                     "gb_per_s": round((3 * M * K + 4 * M) / t / 1e9, 1)})
     elif args.only == "quantiser":
@@ -705,6 +710,31 @@ def run_only(args, world, rank, local):
     cr.cr_check_device_error()
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def replay_time(fn, n):
+    """fn() captured n times in one CUDA graph (uploaded first), replayed
+    once after a warm replay; seconds per call by CUDA events on the replay
+    stream."""
+    import torch
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(n):
+            fn()
+    upload_graph(g, stream)
+    with torch.cuda.stream(stream):
+        g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        g.replay()
+        e1.record(stream)
+    stream.synchronize()
+    del g
+    return e0.elapsed_time(e1) / 1000.0 / n
 
 
 def flushed_medians(fns, steps):

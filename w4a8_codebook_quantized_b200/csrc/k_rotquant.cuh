@@ -594,7 +594,10 @@ __global__ void __launch_bounds__(THREADS) rotquant_pairs_kernel(const uint16_t 
 
     const uint16_t *__restrict__ xrow = x + m * K;
     uint64_t *tr = rq_smem + 256 * hw;
-    uint8_t *tb = reinterpret_cast<uint8_t *>(tr);  // the same buffer serves the byte transpose
+    // the same buffer serves the byte transpose; the odd half-warp's byte
+    // tiles start 64 bytes in, so that the byte stores of a warp's two
+    // half-warps fall in different banks
+    uint8_t *tb = reinterpret_cast<uint8_t *>(tr) + 64 * (hw & 1);
     float amax = 0.0f;
     uint64_t v[kRecompute ? 1 : J][16];
     // the second block of pair p, or nullptr where the row ends with a lone block
