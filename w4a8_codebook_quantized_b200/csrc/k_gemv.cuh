@@ -72,7 +72,12 @@ constexpr int kSlice = 128;                          // columns per consumer war
 constexpr int kChunk = kConsumerWarps * kSlice;      // columns per stage
 constexpr int kTokens = 8;                           // activation rows of a stage (the MMA's N)
 constexpr int kXBytes = kTokens * kChunk;  // room for M = 8; a stage carries M * kChunk
-constexpr int kPrefetchAhead = 3;  // L2 prefetch distance of the weight stream, in stages
+// L2 prefetch distance of the weight stream beyond the ring, in stages.
+// Measured on B200 with the current rings (A/B in both build orders): 0 beats
+// 3 on the large layers (M = 8, N = K = 8192: 11.0 -> 10.5 us; 16384^2:
+// 37.7 -> 34.6 us) and ties elsewhere, so the prefetch is off; the mechanism
+// stays for other ring depths.
+constexpr int kPrefetchAhead = 0;
 constexpr int kRedBufs = 1;  // partial-sum mailboxes between the consumers and the epilogue warp
 
 // Shape of the ring: STAGES stages, MINB CTAs per SM, COPIES copies of the
