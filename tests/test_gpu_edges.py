@@ -49,13 +49,16 @@ def _x_for_rotated(r):
     return bits
 
 
+@pytest.mark.parametrize("reps", [1, 10])
 @pytest.mark.parametrize("qmax", [64, 127])
-def test_rotate_quant_exact_ties(qmax):
+def test_rotate_quant_exact_ties(qmax, reps):
     """Rotated rows with amax == qmax (scale exactly 1) and half-integer
     entries: every entry is an exact tie of rint, which goes to the even
     integer (ai-toolkit convrot_w4a8_quant.py, w4a8_act_quant_kernel,
     libdevice rint).  The device's division-free rounding must take its exact
-    path here and agree with the oracle bit for bit."""
+    path here and agree with the oracle bit for bit: as a short batch (4 rows)
+    and, with the rows repeated, as a 40-row batch (the packed form, where a
+    block pair's two halves carry the ties of blocks 0 and 1)."""
     K = 512
     r = np.zeros((4, K), np.float64)
     if qmax == 64:
@@ -79,12 +82,14 @@ def test_rotate_quant_exact_ties(qmax):
     # row 2: all zero (scale 1); row 3: row 0 doubled, so its scale is 2 and
     # r / scale gives row 0's ties again
     r[3] = 2 * r[0]
+    r = np.tile(r, (reps, 1))
     x = _x_for_rotated(r)
-    xq_r, xs_r = oracle.rotate_quant_act(x, 4, qmax)
-    for (m, k), q in expect.items():
-        assert int(xq_r[m, k]) == q, (m, k, int(xq_r[m, k]), q)
+    xq_r, xs_r = oracle.rotate_quant_act(x, 4 * reps, qmax)
+    for rep in range(reps):
+        for (m, k), q in expect.items():
+            assert int(xq_r[4 * rep + m, k]) == q, (rep, m, k, int(xq_r[4 * rep + m, k]), q)
     assert xs_r[0] == 1.0 and xs_r[1] == 1.0 and xs_r[2] == 1.0
-    xq, xs = cr.cr_rotate_quant_act(bf16_dev(x), 4, qmax)
+    xq, xs = cr.cr_rotate_quant_act(bf16_dev(x), 4 * reps, qmax)
     torch.cuda.synchronize()
     assert np.array_equal(host(xs).view(np.uint32), xs_r.view(np.uint32))
     assert np.array_equal(host(xq), xq_r)

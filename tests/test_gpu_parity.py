@@ -72,27 +72,40 @@ def _rq_case(M, K, seed, mp=None, qmax=127, dist="outliers"):
 
 
 @pytest.mark.parametrize("M,K,MP", [(1, 256, 1), (3, 1024, 4), (8, 4096, 8), (5, 4096, 8), (2, 8192, 2),
-                                    (4, 12288, 4), (2, 16384, 2), (2, 20480, 2), (1, 65536, 1), (33, 768, 33)])
+                                    (4, 12288, 4), (2, 16384, 2), (2, 20480, 2), (1, 65536, 1), (33, 768, 33),
+                                    (100, 256, 100), (40, 1280, 40), (24, 12288, 24), (17, 16384, 17),
+                                    (20, 24576, 20), (18, 32768, 18), (17, 40960, 17), (300, 4096, 300)])
 def test_rotate_quant_shapes(M, K, MP):
+    """Short batches (at most 16 rows: one block per half-warp) and longer
+    ones (a pair of blocks per half-warp in packed fp32x2), across every CTA
+    size and register-holding depth of both forms: a lone last block (odd
+    K / 256), 64 to 512 threads, two pairs per half-warp, the recomputing
+    second pass, and rows beyond one wave of CTAs."""
     _rq_case(M, K, seed=M * 1000 + K, mp=MP)
 
 
 def test_rotate_quant_other_qmax_and_gelu_inputs():
     _rq_case(6, 2048, 7, qmax=7)
     _rq_case(4, 12288, 8, dist="gelu")
+    _rq_case(40, 2048, 9, qmax=7)
+    _rq_case(64, 12288, 10, dist="gelu")
 
 
-def test_rotate_quant_degenerate_rows():
-    """Zero rows (scale 1), subnormal-only rows, huge rows, a one-hot row."""
-    K = 512
+@pytest.mark.parametrize("reps,K", [(1, 512), (4, 512), (4, 768)])
+def test_rotate_quant_degenerate_rows(reps, K):
+    """Zero rows (scale 1), subnormal-only rows, huge rows, a one-hot row; as a
+    short batch (5 rows, padded to 8) and as 20-row batches (the packed form,
+    with a lone last block when K = 768)."""
     rows = np.zeros((5, K), np.float64)
     rows[1, :7] = 2.0 ** -130
     rows[2] = np.linspace(-2.0 ** 100, 2.0 ** 100, K)
     rows[3, 300] = -1.0
     rows[4] = 1.0
+    rows = np.tile(rows, (reps, 1))
+    mp = 8 if reps == 1 else rows.shape[0]
     x = torch.from_numpy(rows).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
-    xq, xs = cr.cr_rotate_quant_act(bf16_dev(x), 8, 127)
-    xq_r, xs_r = oracle.rotate_quant_act(x, 8, 127)
+    xq, xs = cr.cr_rotate_quant_act(bf16_dev(x), mp, 127)
+    xq_r, xs_r = oracle.rotate_quant_act(x, mp, 127)
     assert np.array_equal(host(xs).view(np.uint32), xs_r.view(np.uint32))
     assert np.array_equal(host(xq), xq_r)
     assert host(xs)[0] == 1.0 and (host(xq)[0] == 0).all()
