@@ -95,6 +95,25 @@ def test_rotate_quant_exact_ties(qmax, reps):
     assert np.array_equal(host(xq), xq_r)
 
 
+@pytest.mark.parametrize("M,K", [(8, 4096), (64, 4096), (20, 768), (4, 16384), (40, 12288)])
+def test_rotate_quant_wide_exponents(M, K):
+    """bf16 rows whose values spread over 2^-24 .. 2^24, so that the fp32
+    partial sums of the butterfly round (on the configs' activations they are
+    mostly exact): the row scales (the rounded maximum of each rotated row
+    over qmax) and every quantised byte must equal the oracle's, in both
+    kernel forms (short batches and the packed pairs)."""
+    rng = np.random.default_rng(M * 7 + K)
+    vals = rng.choice([-1.0, 1.0], size=(M, K)) * np.exp2(rng.integers(-24, 25, size=(M, K))) * \
+        rng.uniform(1.0, 2.0, size=(M, K))
+    x = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    mp = cr.gemv_rows(M) if M <= 8 else M
+    xq, xs = cr.cr_rotate_quant_act(bf16_dev(x), mp, 127)
+    torch.cuda.synchronize()
+    xq_r, xs_r = oracle.rotate_quant_act(x, mp, 127)
+    assert np.array_equal(host(xs).view(np.uint32), xs_r.view(np.uint32))
+    assert np.array_equal(host(xq), xq_r)
+
+
 def _very_negative_gate_layer(F, K, seed):
     """An interleaved gate/up layer whose epilogue values are dominated by
     the bias: gates g in about [-90.5, -85] (e^-g overflows fp32 below -88.7,

@@ -220,6 +220,46 @@ def test_rotation_identity_in_exact_arithmetic():
         assert np.array_equal(lhs, 256 * (x.astype(np.int64) @ W.astype(np.int64).T))
 
 
+def test_rotation_follows_the_stated_fp32_order():
+    """Not a pin of the pages (they leave the fp32 order open): a regression
+    check that the oracle computes the order this library states for the
+    rotation -- the exact bf16 -> fp32 widening; the four base-4 digits of the
+    in-block index in the order stride 1, 4, 16, 64; per quadruple
+    S = (v0 + v1) + (v2 + v3) and out[a] = S - 2 v[3 - a], each operation
+    rounded to fp32; then the factor 1/16 -- restated with numpy float32
+    array operations (one reshape per digit) and compared bit for bit on
+    random data, where another digit order, pairing or sign placement rounds
+    differently."""
+    # bf16 values with widely spread exponents, so that the fp32 partial sums
+    # round (the activations of the configs are often summed exactly)
+    rng = np.random.default_rng(21)
+    M, K = 8, 768
+    vals = rng.choice([-1.0, 1.0], size=(M, K)) * np.exp2(rng.integers(-24, 25, size=(M, K))) * \
+        rng.uniform(1.0, 2.0, size=(M, K))
+    x_bits = _bf16(vals)
+    x = (x_bits.astype(np.uint32) << 16).view(np.float32)
+    v = x.reshape(M, K // 256, 256)
+    two = np.float32(2.0)
+    for stride in (1, 4, 16, 64):
+        w = v.reshape(M, K // 256, 256 // (4 * stride), 4, stride)
+        q0, q1, q2, q3 = (w[:, :, :, i, :] for i in range(4))
+        S = (q0 + q1) + (q2 + q3)
+        v = np.stack([S - two * q3, S - two * q2, S - two * q1, S - two * q0], axis=3).reshape(M, K // 256, 256)
+    ref = (v * np.float32(0.0625)).reshape(M, K).astype(np.float32)
+    got = oracle.rotate_rows(x_bits)
+    assert got.dtype == np.float32
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    # the same data in another digit order rounds differently somewhere
+    v = x.reshape(M, K // 256, 256)
+    for stride in (64, 16, 4, 1):
+        w = v.reshape(M, K // 256, 256 // (4 * stride), 4, stride)
+        q0, q1, q2, q3 = (w[:, :, :, i, :] for i in range(4))
+        S = (q0 + q1) + (q2 + q3)
+        v = np.stack([S - two * q3, S - two * q2, S - two * q1, S - two * q0], axis=3).reshape(M, K // 256, 256)
+    other = (v * np.float32(0.0625)).reshape(M, K).astype(np.float32)
+    assert not np.array_equal(got.view(np.uint32), other.view(np.uint32))
+
+
 def test_rotation_rejects_bad_k():
     with pytest.raises(ValueError):
         oracle.rotate_rows(np.zeros((1, 128), np.uint16))
