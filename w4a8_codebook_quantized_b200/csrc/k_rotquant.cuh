@@ -28,8 +28,8 @@
 //    computes both at once with the packed fp32x2 arithmetic of sm_100
 //    (add / sub / mul / fma .f32x2: each half of a 64-bit register is one fp32
 //    value, rounded exactly as the scalar instruction rounds it), so one
-//    instruction does the work of two; the kernel is bound by instruction
-//    issue, and this halves the arithmetic.
+//    instruction does the work of two; the scalar form was bound by
+//    instruction issue at these sizes, and this halves its arithmetic.
 //  - Short batches (decode, at most kShortRows rows): a half-warp owns ONE
 //    block in scalar fp32, so that twice as many threads share a row and each
 //    one's chain of dependent instructions is shortest: here few CTAs run and
