@@ -258,6 +258,14 @@ def test_plan_validation(L):
     assert L.cr_w4a8_plan_destroy(None) == cr.CR_OK
 
 
+def test_int8_peak_validation(L):
+    ops = ctypes.c_double(-1.0)
+    assert L.cr_mma_i8_peak(0, ctypes.byref(ops), None) == cr.CR_ERR_INVALID_ARG
+    assert L.cr_mma_i8_peak((1 << 20) + 1, ctypes.byref(ops), None) == cr.CR_ERR_INVALID_ARG
+    assert L.cr_mma_i8_peak(16, None, None) == cr.CR_ERR_INVALID_ARG
+    assert ops.value == -1.0
+
+
 def test_selftest_validation(L):
     assert L.cr_selftest_wait_timeout(10, None) == cr.CR_ERR_INVALID_ARG        # below 1 ms
     assert L.cr_selftest_wait_timeout(2 * 10 ** 9, None) == cr.CR_ERR_INVALID_ARG  # above 1 s

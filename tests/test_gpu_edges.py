@@ -347,3 +347,25 @@ def test_prepared_layer_decode_matches_oracle(cb_kind, scales, N):
         torch.cuda.synchronize()
         assert np.array_equal(host(y), ref["y"]), (M, cb_kind, scales)
         assert torch.equal(y2, y3) and torch.equal(y, y2)
+
+
+def test_int8_rate_kernel_runs_and_counts_its_operations():
+    """The INT8 tensor-core rate kernel (the prefill roofline's denominator):
+    one launch per SM pair of `iters` groups of four 256 x 256 x 32 MMAs on
+    resident operands; it reports 2 * 256 * 256 * 128 * iters operations per
+    pair, completes without a device error, and its rate is a plausible
+    fraction of the part's dense INT8 figure."""
+    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    stream = torch.cuda.current_stream()
+    ops = cr.cr_mma_i8_peak(64, stream=stream)
+    assert ops == 2.0 * 256 * 256 * 128 * 64 * pairs
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    ops = cr.cr_mma_i8_peak(2048, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    cr.cr_check_device_error()
+    tops = ops / (e0.elapsed_time(e1) * 1e-3) / 1e12
+    assert 500.0 < tops < 9000.0, tops
+

@@ -44,6 +44,7 @@ struct DeviceState {
     std::atomic<bool> gemv_grouped_attr_set{false};
     std::atomic<bool> gemm_bf16_attr_set{false};
     std::atomic<bool> gemm_pair_bf16_attr_set{false};
+    std::atomic<bool> peak_attr_set{false};
     // side stream and events on which cr_w4a8_linear's prefill path decodes
     // the weight while the activations are rotated and quantised
     cudaStream_t side = nullptr;
@@ -1680,14 +1681,13 @@ cr_status cr_mma_i8_peak(int64_t iters, double *ops_per_launch, cr_stream_t stre
     const cr_status st = current_device(&d);
     if (st != CR_OK)
         return st;
-    static std::atomic<bool> attr_set{false};
-    if (!attr_set) {
+    if (!d->peak_attr_set) {
         if (cudaFuncSetAttribute(cr::pk::mma_i8_peak_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)cr::pk::kSmemBytes) != cudaSuccess) {
             cudaGetLastError();
             return CR_ERR_CUDA;
         }
-        attr_set = true;
+        d->peak_attr_set = true;
     }
     const int pairs = d->num_sms / 2;
     cudaLaunchConfig_t cfg = {};
