@@ -531,7 +531,7 @@ def run_ours(args):
            "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N,
            "ms_per_step": round(esecs / args.steps * 1e3, 5),
            "path": "W4A8Linear.forward_host (bound call, cr_w4a8_host_call_run), eager: x from pinned host memory "
-                   "by a copy kernel, rotate+quant, GEMV, y to pinned host memory by a copy kernel (4 launches)"}
+                   "by a copy kernel, rotate+quant, GEMV storing y into pinned host memory (3 launches)"}
     del sets
 
     gemv_extra = []

@@ -487,7 +487,11 @@ cr_status cr_w4a8_ste_backward_ws(const uint16_t *grad, const uint8_t *qdata, co
  *   transfer between two kernels); other copies use cudaMemcpyAsync.  The
  *   kernel copying x_host reads it before the previous kernel on the stream
  *   has finished: x_host must not be written by a kernel that immediately
- *   precedes this call and allows early launch of its dependents.
+ *   precedes this call and allows early launch of its dependents.  For a
+ *   decode batch (M <= CR_GEMV_MAX_M) with bf16 outputs, N a multiple of 8,
+ *   and an out_host that qualifies for the kernel copy, the decode GEMV
+ *   stores y into out_host itself and out_dev is not written; otherwise
+ *   out_dev holds y after the call.
  * cr_w4a8_plan_gemv: the decode GEMV of (4) on the plan's layer and already
  *   quantised activations (ai-toolkit convrot_w4a8_quant.py, gemv_prepared):
  *   xq [>= M, K] int8, xs [M] fp32, 1 <= M <= 8 (CR_ERR_UNSUPPORTED above),

@@ -660,7 +660,7 @@ struct cr_w4a8_host_call_st {
     const uint16_t *x_host = nullptr;
     void *out_host = nullptr;
     const void *x_map = nullptr;  // device address of x_host (copied by a kernel), or null (copy engine)
-    void *out_map = nullptr;      // the same for out_host
+    void *out_map = nullptr;      // the same for out_host (a decode batch's GEMV stores into it directly)
     uint16_t *x_dev = nullptr;
     void *out_dev = nullptr;
     int8_t *xq = nullptr;
@@ -885,6 +885,15 @@ cr_status contraction_swiglu(bool gemv, const int8_t *xq, const float *xs, const
 // its first and last byte lie in page-locked host memory mapped for the
 // device at addresses `bytes - 1` apart; otherwise null.
 constexpr size_t kHostCopyMax = 1u << 20;
+
+// Whether a host-buffer forward's decode GEMV stores y into the mapped
+// out_host itself: a decode batch with bf16 outputs whose every full row tile
+// leaves as 16-byte stores (N a multiple of 8).  Other outputs would cross the
+// host link as scattered 2- or 4-byte stores, and the copy kernel moves them.
+bool gemv_stores_host(const cr_w4a8_plan_st *plan, int64_t M)
+{
+    return M <= CR_GEMV_MAX_M && plan->out_dtype == CR_OUT_BF16 && plan->N % 8 == 0;
+}
 
 const void *small_mapped_host(const void *p, size_t bytes)
 {
@@ -1337,6 +1346,11 @@ cr_status cr_w4a8_plan_forward_host(cr_w4a8_plan plan, const uint16_t *x_host, i
         cudaGetLastError();
         return CR_ERR_CUDA;
     }
+    // A decode batch's GEMV stores y into mapped host memory itself: its
+    // epilogue only stores the outputs, so the transfer is spread over the
+    // launch instead of following it as another kernel.
+    if (out_map && gemv_stores_host(plan, M))
+        return cr_w4a8_plan_forward(plan, x_dev, M, out_map, xq_work, xs_work, stream);
     st = cr_w4a8_plan_forward(plan, x_dev, M, out_dev, xq_work, xs_work, stream);
     if (st != CR_OK)
         return st;
@@ -1401,7 +1415,8 @@ cr_status cr_w4a8_plan_bind_host(cr_w4a8_plan plan, const uint16_t *x_host, int6
             c->MP <<= 1;
         c->gemv.xs = xs_work;
         c->gemv.M = (int)M;
-        c->gemv.layer[0].out = out_dev;
+        // as in cr_w4a8_plan_forward_host
+        c->gemv.layer[0].out = (c->out_map && gemv_stores_host(plan, M)) ? c->out_map : out_dev;
     }
     *call = c;
     return CR_OK;
@@ -1439,6 +1454,8 @@ cr_status cr_w4a8_host_call_run(cr_w4a8_host_call c, cr_stream_t stream)
     }
     if (st != CR_OK)
         return st;
+    if (c->out_map && gemv_stores_host(plan, c->M))
+        return CR_OK;  // the GEMV stored y into out_host
     if (c->out_map)
         return launched(cr::ew::launch_host_copy(c->out_map, c->out_dev, (int64_t)c->ob, false, d->num_sms, stream));
     if (cudaMemcpyAsync(c->out_host, c->out_dev, c->ob, cudaMemcpyDeviceToHost, stream) != cudaSuccess) {
