@@ -554,6 +554,20 @@ float or_group_scale_als(const float *gw, const float *codebook, int *q /* [16] 
     return gs;
 }
 
+/* [CR] _assign_grid on one group of 16 rotated weights: target = w / s_channel
+ * (an fp32 division), then the nearest level of the group's grid, or with
+ * rand != NULL the stochastic choice with rand[i] as the draw of weight i.
+ * The quantiser's final assignment and the code re-assignment both run it,
+ * as the page's _quantize_rotated_rows and requantize both call _assign_grid
+ * on w / s_channel and grid_levels(codebook, s_rel). */
+static void or_assign_group(const float *w, float s_channel, const float *levels, const float *rand, int *c)
+{
+    for (int i = 0; i < 16; ++i) {
+        const float t = w[i] / s_channel;
+        c[i] = rand ? or_stochastic_level(levels, 16, t, rand[i]) : or_nearest_level(levels, 16, t);
+    }
+}
+
 /* [CR] quantize_w4a8_rotated (row chunking does not change the result: rows
  * are independent).  w_rot [N, K] fp32 (already rotated), K a multiple of 16.
  * Per row: the group scales gs and codes of or_group_scale_als; s_channel =
@@ -589,11 +603,10 @@ int or_quantize_rotated(const float *w_rot, int64_t N, int64_t K, const float *c
             srel[n * G + g] = b;
             float levels[16];
             or_grid_levels(codebook, b, levels);
-            for (int i = 0; i < 16; i += 2) {
-                const int c0 = or_nearest_level(levels, 16, row[16 * g + i] / sch);
-                const int c1 = or_nearest_level(levels, 16, row[16 * g + i + 1] / sch);
-                qdata[n * (K / 2) + 8 * g + i / 2] = (uint8_t)(c0 | (c1 << 4));
-            }
+            int c[16];
+            or_assign_group(row + 16 * g, sch, levels, NULL, c);
+            for (int i = 0; i < 16; i += 2)
+                qdata[n * (K / 2) + 8 * g + i / 2] = (uint8_t)(c[i] | (c[i + 1] << 4));
         }
     }
     free(gs);
@@ -615,11 +628,7 @@ int or_assign_codes(const float *w_rot, const uint8_t *srel, const float *s_chan
             float levels[16];
             or_grid_levels(codebook, srel[n * G + g], levels);
             int c[16];
-            for (int i = 0; i < 16; ++i) {
-                const int64_t k = 16 * g + i;
-                const float t = w_rot[n * K + k] / s_channel[n];
-                c[i] = rand ? or_stochastic_level(levels, 16, t, rand[n * K + k]) : or_nearest_level(levels, 16, t);
-            }
+            or_assign_group(w_rot + n * K + 16 * g, s_channel[n], levels, rand ? rand + n * K + 16 * g : NULL, c);
             for (int i = 0; i < 16; i += 2)
                 qdata[n * (K / 2) + 8 * g + i / 2] = (uint8_t)(c[i] | (c[i + 1] << 4));
         }
