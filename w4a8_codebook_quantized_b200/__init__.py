@@ -588,7 +588,9 @@ class W4A8Linear:
         """x_host [M, K] bf16 and out_host [M, N] in host memory (pinned for
         asynchronous copies), x_dev / out_dev their device buffers: queues the
         copy in, the forward and the copy out on the stream; out_host is ready
-        once the stream has reached that point.  With caller-owned work
+        once the stream has reached that point.  A decode batch with bf16
+        outputs, N a multiple of 8 and a pinned out_host has its GEMV store y
+        into out_host directly, and out_dev is then not written.  With caller-owned work
         buffers the call is bound to its tensors (cr_w4a8_plan_bind_host),
         and a repeat with the same tensors, unchanged in storage and shape,
         only queues the launches."""
