@@ -558,8 +558,9 @@ float or_group_scale_als(const float *gw, const float *codebook, int *q /* [16] 
  * (an fp32 division), then the nearest level of the group's grid, or with
  * rand != NULL the stochastic choice with rand[i] as the draw of weight i.
  * The quantiser's final assignment and the code re-assignment both run it,
- * as the page's _quantize_rotated_rows and requantize both call _assign_grid
- * on w / s_channel and grid_levels(codebook, s_rel). */
+ * as the page's _quantize_rotated_rows and requantize_codes_ (and
+ * fake_quant_rotated_weight) all call _assign_grid on w / s_channel and
+ * grid_levels(codebook, s_rel). */
 static void or_assign_group(const float *w, float s_channel, const float *levels, const float *rand, int *c)
 {
     for (int i = 0; i < 16; ++i) {
